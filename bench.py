@@ -1,0 +1,357 @@
+#!/usr/bin/env python
+"""Benchmark: prefix-aware batched decode attention on B200.
+
+One step = the whole hot path over one decode batch: pack on the host
+(pa_plan_create: tree block table, profit model, split, tile selection), the
+async upload of the plan, forward and merge on the GPU.  The default workload is
+the Llama-3-8B-shaped decode layer (batch 64, 32/8 heads, head_dim 128, one
+shared 2048-token prefix plus suffixes uniform 128-1024, page 16).
+
+Metric: decode-attention queries/s (B / time per step), with the unique-KV bytes
+per second reported beside it as a fraction of the measured HBM bandwidth.
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and a device sync
+on both sides, timed with CUDA events on the launching stream; max over ranks.
+Between steps the KV pools rotate over several device copies whose total size
+exceeds L2, so no step finds its KV in L2.
+
+Under torchrun each rank runs its own batch (seed + rank): weak scaling, no
+collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+_ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, _ROOT)
+
+METRIC = "decode-attn queries/s; unique-KV HBM GB/s as % of B200 peak (1 GPU)"
+UNIT = "queries/s"
+L2_BYTES = 126 * 2 ** 20
+
+
+def peaks():
+    p = os.path.join(_ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.samples = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append([x.strip() for x in line.split(",")])
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm = [float(s[1]) for s in self.samples if len(s) >= 9 and s[1].replace(".", "").isdigit()]
+        smax = [float(s[2]) for s in self.samples if len(s) >= 9 and s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            if len(s) >= 9:
+                for n, v in zip(names, s[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reference_arm(args, rank, world):
+    """The fp64 CPU oracle timed on the host cores (bounded sample per step)."""
+    if rank != 0:
+        return
+    import oracle
+    from prefix_aware_decode_b200 import workload as wl
+
+    w = wl.make_config(args.config, seed=1000 + args.config)
+    cores = os.cpu_count() or 1
+    n = min(w.B, args.ref_queries)
+    qs = np.arange(n, dtype=np.int32)
+    for _ in range(args.warmup):
+        oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs[:1], nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs, nthreads=cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = n / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.CONFIG_NAMES[args.config], "queries_per_step": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"first {n} of {w.B} queries of the workload per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--copies", type=int, default=0, help="KV pool copies rotated between steps (0: enough to exceed L2)")
+    ap.add_argument("--ref-queries", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+
+    import torch
+
+    import prefix_aware_decode_b200 as pad
+    from prefix_aware_decode_b200 import workload as wl
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    hbm_peak, bf16_peak, peak_kind = peaks()
+    w = wl.make_config(args.config, seed=1000 + args.config + 7919 * rank)
+    unique_bytes = w.unique_kv_bytes
+    pool_bytes = w.k_pool.nbytes + w.v_pool.nbytes
+    copies = args.copies or max(2, int(np.ceil(3 * L2_BYTES / pool_bytes)) + 1)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+    q = dev(w.q)
+    k0, v0 = dev(w.k_pool), dev(w.v_pool)
+    pools = [(k0, v0)] + [(k0.clone(), v0.clone()) for _ in range(copies - 1)]
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    kv_lens, block_table = w.kv_lens, w.block_table
+
+    probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    pst = probe.stats()
+    ws_bytes = probe.workspace_bytes
+    probe.close()
+    workspaces = [torch.empty((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device="cuda") for _ in range(2)]
+
+    # per-step profiling events around each launch (recorded once so they exist)
+    def mk_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)
+        return evs
+
+    nsteps = args.warmup + args.steps
+    step_events = [mk_events(6) for _ in range(nsteps)]
+    plan_us = []
+
+    def step(i, prof=True):
+        t = time.perf_counter()
+        plan = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+        plan_us.append((time.perf_counter() - t) * 1e6)
+        if prof:
+            plan.set_profile_events(step_events[i])
+        ws = workspaces[i % 2]
+        kp, vp = pools[i % copies]
+        plan.upload(ws, stream)
+        plan.forward(q, kp, vp, ws, stream)
+        plan.merge(ws, out, lse, stream)
+        plan.close()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    probe.upload(workspaces[0], stream)
+    status = probe.device_status(workspaces[0], stream)
+    probe.close()
+    assert status == pad.PA_OK, status
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    plan_us.clear()
+    ev0.record(stream)
+    for i in range(args.warmup, nsteps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+
+    # per-kernel times inside the timed region
+    def avg(a, b):
+        xs = []
+        for i in range(args.warmup, nsteps):
+            e = step_events[i]
+            xs.append(e[a].elapsed_time(e[b]))
+        return sum(xs) / len(xs)
+
+    has_mma = pst["num_segments_mma"] > 0
+    simt_ms = avg(2, 3)
+    mma_ms = avg(0, 1) if has_mma else 0.0
+    merge_ms = avg(4, 5)
+    fwd_merge_ms = avg(0 if has_mma else 2, 5)
+
+    # algorithmic bytes of one CUDA-core forward launch: the KV of its (page, kv head)
+    # tiles, its q rows, and its fp32 partial rows
+    G = w.Hq // w.Hkv
+    probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    hdr = pad.PaImageHeader.from_buffer_copy(probe.host_image()[:256].tobytes())
+    probe.close()
+    simt_tiles = hdr.num_loads
+    tile_bytes = 2 * 16 * w.D * 2
+    simt_bytes = simt_tiles * tile_bytes + hdr.num_segments_simt * (G * w.D * 2 + G * (w.D + 1) * 4)
+    achieved = simt_bytes / (simt_ms * 1e-3) / 1e9
+
+    queries_per_s = w.B * world / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": queries_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.CONFIG_NAMES[args.config], "batch": w.B, "heads": f"{w.Hq}/{w.Hkv}",
+                   "head_dim": w.D, "page": w.P, "seed": w.seed, "unique_kv_bytes": unique_bytes,
+                   "prefix_ratio": round(w.prefix_ratio, 4), "l2": f"KV pools rotated over {copies} device copies "
+                   f"({copies * pool_bytes / 2**20:.0f} MiB > L2 {L2_BYTES // 2**20} MiB)",
+                   "step": "pack (host) + upload + forward + merge", "parallelism": f"replicas x{world}"},
+        "unique_kv_gbs": unique_bytes / (ms_step * 1e-3) / 1e9,
+        "unique_kv_frac_of_hbm": unique_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak,
+        "device_ms": {"mma_forward": mma_ms, "simt_forward": simt_ms, "merge": merge_ms,
+                      "forward_plus_merge": fwd_merge_ms},
+        "forward_merge_queries_per_s": w.B / (fwd_merge_ms * 1e-3),
+        "forward_merge_unique_kv_frac": unique_bytes / (fwd_merge_ms * 1e-3) / 1e9 / hbm_peak,
+        "plan_us_median": statistics.median(plan_us),
+        "plan": {k: pst[k] for k in ("num_segments_simt", "num_segments_mma", "simt_warps", "num_partial_rows",
+                                     "read_kv_bytes", "workspace_bytes", "image_bytes")},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "fwd_simt_kernel<128,4>",
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
+        "gpu_launches": args.steps * (3 if has_mma else 2),
+        "clocks": clk,
+    }
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).pin_memory()
+        hk = torch.from_numpy(np.ascontiguousarray(w.k_pool).view(np.int16)).pin_memory()
+        hv = torch.from_numpy(np.ascontiguousarray(w.v_pool).view(np.int16)).pin_memory()
+        ho = torch.empty((w.B, w.Hq, w.D), dtype=torch.int16).pin_memory()
+        hl = torch.empty((w.B, w.Hq), dtype=torch.float32).pin_memory()
+        dq = torch.empty_like(q)
+        dk, dv = torch.empty_like(k0), torch.empty_like(v0)
+
+        def e2e_step(copy_kv: bool):
+            dq.view(torch.int16).copy_(hq, non_blocking=True)
+            if copy_kv:
+                dk.view(torch.int16).copy_(hk, non_blocking=True)
+                dv.view(torch.int16).copy_(hv, non_blocking=True)
+            plan = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+            plan.upload(workspaces[0], stream)
+            plan.attend(dq, dk, dv, workspaces[0], out, lse, stream)
+            plan.close()
+            ho.copy_(out.view(torch.int16), non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        res = {}
+        for copy_kv in (True, False):
+            for _ in range(2):
+                e2e_step(copy_kv)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step(copy_kv)
+            b.record(stream)
+            torch.cuda.synchronize()
+            res[copy_kv] = a.elapsed_time(b) / args.e2e_steps
+        h2d = w.q.nbytes + w.k_pool.nbytes + w.v_pool.nbytes
+        d2h = out.numel() * 2 + lse.numel() * 4
+        line["e2e"] = {"value": w.B * world / (res[True] * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h,
+                       "note": "every input (q and both KV pools) copied from pinned host memory each step"}
+        line["e2e_kv_resident"] = {"value": w.B * world / (res[False] * 1e-3), "unit": UNIT,
+                                   "h2d_bytes_per_step": w.q.nbytes, "d2h_bytes_per_step": d2h,
+                                   "note": "q from pinned host memory, KV cache resident on the device"}
+
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        cores = os.cpu_count() or 1
+        n = min(w.B, args.ref_queries)
+        qs = np.arange(n, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs, nthreads=cores)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"first {n} of {w.B} queries of the same workload, one pass"}
+
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,244 @@
+/*
+ * pa.h -- C ABI of the prefix-aware decode-attention library (libpa.so).
+ *
+ * The library computes batched single-token decode attention
+ *     out[b][h] = softmax(q[b][h] . K_b^T / sqrt(d)) V_b
+ * for B requests over a paged bf16 KV cache whose requests share prefixes.
+ * Sources: the PAT review ("PAT: Accelerating LLM Decoding via Prefix-Aware
+ * Attention with Resource Efficient Multi-Tile Kernel", section 三 核心公式 for the
+ * formula, Pack-Forward-merge 范式 for the three stages), and the short-term
+ * memory page (技术原理: each request's own token is appended to its KV before
+ * it attends; PagedAttention for the paged cache).
+ *
+ * The three stages map to calls:
+ *   pack     pa_plan_create   host: tree-structured block table, profit model,
+ *                             split of long nodes, tile-class selection
+ *            pa_plan_upload   async H2D copy of the plan into the workspace
+ *   forward  pa_forward       device: partial attention per (node, kv head,
+ *                             query tile, key range) into fp32 partials
+ *   merge    pa_merge         device: log-sum-exp combine of each (request,
+ *                             head)'s partials into bf16 out and fp32 lse
+ *
+ * Memory ownership: the caller allocates and owns every device buffer (q, the
+ * pools, the workspace, out, lse).  The library owns only the host-side plan
+ * object; a plan keeps no device pointer past the call that received it.
+ * Device calls are asynchronous on the stream given.  Nothing throws across
+ * this ABI; every call returns a pa_status.
+ *
+ * Tensor layouts (row-major, contiguous, bf16 = IEEE bfloat16 bit patterns):
+ *   q       bf16 [B][Hq][D]
+ *   k_pool  bf16 [num_pages][Hkv][P][D]     (v_pool alike); 16-byte aligned
+ *   out     bf16 [B][Hq][D]                 round-to-nearest-even
+ *   lse     fp32 [B][Hq]                    natural log of sum exp(scaled logits)
+ *   block_table int32 [B][max_pages] (host); kv_lens int32 [B] (host)
+ * Query head h reads kv head h / (Hq / Hkv).  Token t of request b is slot
+ * t % P of page block_table[b][t / P]; entries past ceil(kv_len/P) are ignored.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,     /* bad argument: page id, kv_len, shape, partial shared page */
+  PA_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim, GQA ratio, page size */
+  PA_ERR_NOMEM = 3,       /* host allocation failed, or workspace too small */
+  PA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up (recorded in the workspace) */
+  PA_ERR_DEVICE = 6       /* a device-side check failed (recorded in the workspace) */
+} pa_status;
+
+/* pa_config.flags */
+#define PA_PLAN_NO_SHARING (1u << 0)   /* query-centric: inline every shared node (baseline mode) */
+#define PA_PLAN_ALWAYS_SHARE (1u << 1) /* keep every shared node shared, whatever the profit model says */
+#define PA_PLAN_DEBUG_CHECKS (1u << 2) /* device-side index checks; failures set PA_ERR_DEVICE */
+#define PA_PLAN_FAULT_DROP_LOAD (1u << 8) /* tests only: forward skips one KV load, so its bounded
+                                             wait must expire and record PA_ERR_TIMEOUT */
+
+typedef struct {
+  int32_t num_q_heads;      /* Hq */
+  int32_t num_kv_heads;     /* Hkv; Hq / Hkv must be 1, 2, 4 or 8 */
+  int32_t head_dim;         /* D: 64 or 128 */
+  int32_t page_size;        /* P: 16 */
+  float softmax_scale;      /* 0 selects 1/sqrt(head_dim) */
+  int32_t num_sms;          /* 0: query the current device (148 on B200 if none) */
+  int32_t max_chunk_tokens; /* 0: heuristic; else upper bound on tokens per forward work unit
+                               (rounded down to a multiple of page_size, at least one page) */
+  uint32_t flags;           /* PA_PLAN_* */
+  int32_t wait_timeout_us;  /* device bounded-wait limit; 0 selects 2,000,000 (2 s) */
+} pa_config;
+
+typedef struct pa_plan pa_plan; /* opaque, host-owned */
+
+typedef struct {
+  int32_t batch;
+  int32_t num_nodes;        /* non-empty nodes of the tree block table */
+  int32_t num_shared_nodes; /* nodes with two or more requests */
+  int32_t num_kept_shared;  /* shared nodes the profit model kept shared (not inlined) */
+  int32_t num_items;        /* node items (a node x query tile) */
+  int32_t num_segments;     /* forward work units (item x kv head x key range) */
+  int32_t num_segments_simt;/* units on the CUDA-core class (one request, G rows) */
+  int32_t num_segments_mma; /* units on the tensor-core class (two or more requests) */
+  int32_t num_partial_rows; /* partial result rows per kv head group (each holds G rows) */
+  int32_t simt_warps;       /* warps of the CUDA-core forward launch */
+  int64_t unique_tokens;    /* tokens of distinct tree nodes (each shared page once) */
+  int64_t naive_tokens;     /* sum of kv_lens (query-centric reads) */
+  int64_t read_tokens;      /* tokens the plan reads from the pools (per kv head) */
+  int64_t unique_kv_bytes;  /* unique_tokens * 2 * Hkv * D * 2 */
+  int64_t read_kv_bytes;    /* read_tokens * 2 * Hkv * D * 2 */
+  uint64_t workspace_bytes; /* device workspace the caller must provide */
+  uint64_t image_bytes;     /* bytes pa_plan_upload copies to the device */
+  double plan_us;           /* host time spent in pa_plan_create */
+} pa_plan_stats;
+
+/*
+ * Pack: build a plan for one decode batch (host only; no device call).
+ *   cfg               head configuration and planner options (copied)
+ *   batch             B >= 1
+ *   kv_lens           host int32[B], each in [1, max_pages * page_size]
+ *   block_table       host int32[B][max_pages], row-major; the first
+ *                     ceil(kv_lens[b] / page_size) entries of row b must be in
+ *                     [0, num_pages_in_pool)
+ *   num_pages_in_pool size of the pools' first dimension
+ *   out               receives the new plan (NULL on error)
+ * Two requests share a page when their rows hold the same page id at the same
+ * position after an identical prefix (prefix caching).  A shared page must be
+ * full for every request that shares it, else PA_ERR_INVALID.  Inputs are read
+ * during the call only.
+ */
+pa_status pa_plan_create(const pa_config *cfg, int32_t batch, const int32_t *kv_lens,
+                         const int32_t *block_table, int32_t max_pages, int32_t num_pages_in_pool,
+                         pa_plan **out);
+
+/* Device workspace size in bytes for this plan (256-byte aligned buffer required). */
+pa_status pa_plan_workspace_size(const pa_plan *plan, size_t *bytes);
+
+/*
+ * Copy the plan (item, segment and page tables, and a zeroed status word) into
+ * the caller's device workspace, asynchronously on `stream` (cudaStream_t).
+ * The image is first copied into a library-owned pinned staging buffer (a
+ * small pool reused once each copy has completed), so the call does not wait
+ * for earlier work on the stream and the plan may be destroyed right after it
+ * returns.  bytes must be at least pa_plan_workspace_size; the workspace must
+ * be 256-byte aligned.
+ */
+pa_status pa_plan_upload(const pa_plan *plan, void *d_workspace, size_t bytes, void *stream);
+
+/*
+ * Forward: partial attention of every planned work unit into the workspace's
+ * fp32 partial buffers.  q, k_pool, v_pool are device pointers in the layouts
+ * above; k_pool and v_pool must be 16-byte aligned.  Needs a prior
+ * pa_plan_upload to the same workspace (ordered before on the stream).
+ * Asynchronous on `stream`; launch failures return PA_ERR_CUDA.
+ */
+pa_status pa_forward(const pa_plan *plan, const void *q, const void *k_pool, const void *v_pool,
+                     void *d_workspace, void *stream);
+
+/*
+ * Merge: log-sum-exp combine of the partials of every (request, head) into
+ * out (bf16 [B][Hq][D], round-to-nearest-even) and lse (fp32 [B][Hq]; may be
+ * NULL).  Asynchronous on `stream`, ordered after pa_forward.
+ */
+pa_status pa_merge(const pa_plan *plan, void *d_workspace, void *out, float *lse, void *stream);
+
+/*
+ * pa_forward followed by pa_merge on the same stream (the whole device path of
+ * one decode step).
+ */
+pa_status pa_attend(const pa_plan *plan, const void *q, const void *k_pool, const void *v_pool,
+                    void *d_workspace, void *out, float *lse, void *stream);
+
+/*
+ * Read the device status word of the workspace (synchronises `stream`).
+ * *out = PA_OK, PA_ERR_TIMEOUT or PA_ERR_DEVICE.  The word is cleared by the
+ * next pa_plan_upload.
+ */
+pa_status pa_get_device_status(const pa_plan *plan, const void *d_workspace, void *stream, pa_status *out);
+
+/* Counters of the plan (host only). */
+pa_status pa_plan_get_stats(const pa_plan *plan, pa_plan_stats *out);
+
+/*
+ * Copy the host image that pa_plan_upload sends (stats.image_bytes bytes) into
+ * dst (host memory).  Its layout is described by pa_image_layout below; tests
+ * use it to execute a plan on the CPU.
+ */
+pa_status pa_plan_host_image(const pa_plan *plan, void *dst, size_t bytes);
+
+/*
+ * Profiling hook: up to six cudaEvent_t handles (owned by the caller) that
+ * pa_forward and pa_merge record on their stream around each launch:
+ *   events[0], events[1]  before / after the tensor-core (MMA) forward launch
+ *   events[2], events[3]  before / after the CUDA-core (SIMT) forward launch
+ *   events[4], events[5]  before / after the merge launch
+ * NULL entries are skipped; n = 0 turns the hook off.  Events of a class with no
+ * work are not recorded.  The events must stay valid while the plan uses them.
+ */
+pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t n);
+
+/* Release a plan (NULL is ignored). */
+void pa_plan_destroy(pa_plan *plan);
+
+/* Static description of a status code. */
+const char *pa_status_string(pa_status s);
+
+/*
+ * Layout of the uploaded image and the workspace.  All offsets are bytes from
+ * the workspace base and are multiples of 256.
+ *
+ *   header      pa_image_header
+ *   nodes       pa_item[num_items]            a node (or its query tile)
+ *   segs        pa_seg[num_segments]          SIMT segments first, then MMA
+ *   pages       int32[num_page_entries]       page ids, per item
+ *   queries     int32[num_query_entries]      request ids, per item
+ *   seg_prows   int32[num_query_entries_mma]  partial row of each (MMA seg, query)
+ *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
+ *   warp_loads  int32[simt_warps + 1]         SIMT warp w loads tiles [warp_loads[w], warp_loads[w+1])
+ *   tiles       int32[num_loads]              page * Hkv + kv_head of every SIMT tile load, in
+ *                                             the order the warps consume them
+ *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
+ *                                             [prow_off[b*Hkv+g], prow_off[b*Hkv+g+1])
+ *   partial_lse fp32[num_partial_rows][G]     (workspace only, not uploaded)
+ *   partial_o   fp32[num_partial_rows][G][D]  (workspace only, not uploaded)
+ */
+typedef struct {
+  int32_t page_off;  /* into pages: this item's page ids */
+  int32_t n_tokens;  /* valid tokens of the item, from slot 0 of its first page */
+  int32_t n_queries; /* requests in the item; rows = n_queries * G */
+  int32_t query_off; /* into queries */
+} pa_item;
+
+typedef struct {
+  int32_t item;       /* index into nodes */
+  int32_t kv_head;    /* kv head g */
+  int32_t page_begin; /* first page of the run, index within the item's pages */
+  int32_t n_tokens;   /* valid tokens of the run (its pages are ceil(n_tokens / P)) */
+  int32_t prow;       /* SIMT: the partial row written; MMA: index into seg_prows */
+  int32_t query;      /* SIMT: the request; MMA: first request of the item */
+  int32_t pad0, pad1; /* 32-byte records */
+} pa_seg;
+
+typedef struct {
+  uint32_t magic;   /* 0x50414231 */
+  int32_t status;   /* device status word (pa_status), 0 after upload */
+  int32_t fault_a;  /* where a device check or wait failed (diagnostics) */
+  int32_t fault_b;
+  int32_t batch, num_q_heads, num_kv_heads, head_dim, page_size;
+  int32_t num_items, num_segments, num_segments_simt, num_segments_mma, simt_warps;
+  int32_t num_partial_rows, num_loads;
+  uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_warp_segs, off_warp_loads, off_tiles,
+      off_prow_off;
+  uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;
+} pa_image_header;
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

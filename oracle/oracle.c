@@ -117,23 +117,34 @@ static void attend_one(paged_job *j, int qi, int h) {
   const int g = h / G;
   const int64_t n = j->kv_lens[b];
   double *qd = (double *)malloc(sizeof(double) * D);
-  double *K = (double *)malloc(sizeof(double) * (size_t)n * D);
-  double *V = (double *)malloc(sizeof(double) * (size_t)n * D);
+  double *score = (double *)malloc(sizeof(double) * (size_t)n);
+  double *out = j->out + ((size_t)qi * j->Hq + h) * D;
   for (int d = 0; d < D; ++d) qd[d] = bf16_to_f64(j->q[((size_t)b * j->Hq + h) * D + d]);
+  /* token t of request b: slot t % P of page block_table[b][t / P], kv head g */
+#define ORACLE_ROW(pool, t)                                                                  \
+  ((pool) + ((((size_t)j->block_table[(size_t)b * j->max_pages + (t) / P] * Hkv + g) * P + \
+              (size_t)((t) % P)) * D))
+  double m = -INFINITY;
   for (int64_t t = 0; t < n; ++t) {
-    int64_t page = j->block_table[(size_t)b * j->max_pages + t / P];
-    int64_t slot = t % P;
-    size_t base = (((size_t)page * Hkv + g) * P + slot) * D;
-    for (int d = 0; d < D; ++d) {
-      K[t * D + d] = bf16_to_f64(j->k_pool[base + d]);
-      V[t * D + d] = bf16_to_f64(j->v_pool[base + d]);
-    }
+    const uint16_t *krow = ORACLE_ROW(j->k_pool, t);
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += qd[d] * bf16_to_f64(krow[d]);
+    score[t] = j->scale * s;
+    if (score[t] > m) m = score[t];
   }
-  oracle_attend_dense(D, j->scale, qd, K, V, n, j->out + ((size_t)qi * j->Hq + h) * D,
-                      j->lse + (size_t)qi * j->Hq + h);
+  double l = 0.0;
+  for (int d = 0; d < D; ++d) out[d] = 0.0;
+  for (int64_t t = 0; t < n; ++t) {
+    const uint16_t *vrow = ORACLE_ROW(j->v_pool, t);
+    const double w = exp(score[t] - m);
+    l += w;
+    for (int d = 0; d < D; ++d) out[d] += w * bf16_to_f64(vrow[d]);
+  }
+#undef ORACLE_ROW
+  for (int d = 0; d < D; ++d) out[d] /= l;
+  j->lse[(size_t)qi * j->Hq + h] = m + log(l);
   free(qd);
-  free(K);
-  free(V);
+  free(score);
 }
 
 static void *paged_worker(void *arg) {

@@ -1,0 +1,183 @@
+// C ABI: device-side calls of libpa.so (upload, forward, merge, status).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "plan.h"
+
+namespace {
+
+PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
+  const pa_image_header& h = p.hdr;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  PaDevPtrs d{};
+  d.ws = b;
+  d.items = reinterpret_cast<const pa_item*>(b + h.off_nodes);
+  d.segs = reinterpret_cast<const pa_seg*>(b + h.off_segs);
+  d.pages = reinterpret_cast<const int32_t*>(b + h.off_pages);
+  d.queries = reinterpret_cast<const int32_t*>(b + h.off_queries);
+  d.seg_prows = reinterpret_cast<const int32_t*>(b + h.off_seg_prows);
+  d.warp_segs = reinterpret_cast<const int32_t*>(b + h.off_warp_segs);
+  d.warp_loads = reinterpret_cast<const int32_t*>(b + h.off_warp_loads);
+  d.tiles = reinterpret_cast<const int32_t*>(b + h.off_tiles);
+  d.prow_off = reinterpret_cast<const int32_t*>(b + h.off_prow_off);
+  d.partial_lse = reinterpret_cast<float*>(b + h.off_partial_lse);
+  d.partial_o = reinterpret_cast<float*>(b + h.off_partial_o);
+  d.status = reinterpret_cast<int32_t*>(b + offsetof(pa_image_header, status));
+  return d;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D view of a pool: rows = num_pages * Hkv * P, columns = D bf16; box 64 x 16
+// with 128-byte swizzle (one half of a (page, kv head) tile per copy).
+bool encode_pool(const pa_plan& p, const void* pool, void* out) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)p.D, (cuuint64_t)p.num_pages_in_pool * p.Hkv * p.P};
+  cuuint64_t strides[1] = {(cuuint64_t)p.D * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(reinterpret_cast<CUtensorMap*>(out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Pinned staging buffers for plan uploads.  A copy from pageable memory makes
+// the runtime wait for the stream first, which would serialise host planning
+// with the device work of the previous step; a copy from pinned memory does
+// not.  A slot is reused once the event recorded after its copy has completed.
+struct PinnedSlot {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+  int device = -1;
+  cudaEvent_t done = nullptr;
+};
+std::mutex g_pin_mu;
+std::vector<PinnedSlot> g_pin;
+
+// Returns a slot index whose buffer holds >= n bytes and is free, or -1.
+int pin_acquire(size_t n, int device) {
+  for (size_t i = 0; i < g_pin.size(); ++i) {
+    PinnedSlot& s = g_pin[i];
+    if (s.device != device || s.bytes < n) continue;
+    if (cudaEventQuery(s.done) == cudaSuccess) return (int)i;
+  }
+  PinnedSlot s;
+  size_t cap = 1 << 16;
+  while (cap < n) cap <<= 1;
+  if (cudaMallocHost(&s.ptr, cap) != cudaSuccess) return -1;
+  if (cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess) {
+    cudaFreeHost(s.ptr);
+    return -1;
+  }
+  s.bytes = cap;
+  s.device = device;
+  g_pin.push_back(s);
+  return (int)g_pin.size() - 1;
+}
+
+void record_profile(const pa_plan& p, int which, cudaStream_t st) {
+  if (p.prof[which]) cudaEventRecord(static_cast<cudaEvent_t>(p.prof[which]), st);
+}
+
+}  // namespace
+
+extern "C" pa_status pa_plan_upload(const pa_plan* plan, void* d_workspace, size_t bytes, void* stream) {
+  if (!plan || !d_workspace) return PA_ERR_INVALID;
+  if (bytes < plan->hdr.workspace_bytes) return PA_ERR_NOMEM;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return PA_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pin_mu);
+  const int slot = pin_acquire(plan->image.size(), device);
+  if (slot < 0) {
+    // no pinned memory: a pageable copy is still correct, only slower
+    cudaError_t e = cudaMemcpyAsync(d_workspace, plan->image.data(), plan->image.size(), cudaMemcpyHostToDevice, st);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
+  PinnedSlot& s = g_pin[slot];
+  std::memcpy(s.ptr, plan->image.data(), plan->image.size());
+  cudaError_t e = cudaMemcpyAsync(d_workspace, s.ptr, plan->image.size(), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaEventRecord(s.done, st) != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_plan_set_profile_events(pa_plan* plan, void* const* events, int32_t n) {
+  if (!plan || n < 0 || n > 6 || (n > 0 && !events)) return PA_ERR_INVALID;
+  for (int i = 0; i < 6; ++i) plan->prof[i] = i < n ? events[i] : nullptr;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_forward(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
+                                void* d_workspace, void* stream) {
+  if (!plan || !q || !k_pool || !v_pool || !d_workspace) return PA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool) |
+       reinterpret_cast<uintptr_t>(q)) & 15)
+    return PA_ERR_INVALID;
+  PaDevPtrs d = dev_ptrs(*plan, d_workspace);
+  d.q = static_cast<const uint16_t*>(q);
+  d.k_pool = static_cast<const uint16_t*>(k_pool);
+  d.v_pool = static_cast<const uint16_t*>(v_pool);
+  if (plan->hdr.num_segments_mma > 0) {
+    if (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool) {
+      if (!encode_pool(*plan, k_pool, plan->tma_k) || !encode_pool(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
+      plan->tma_k_ptr = k_pool;
+      plan->tma_v_ptr = v_pool;
+    }
+    record_profile(*plan, 0, static_cast<cudaStream_t>(stream));
+    if (pa_launch_mma(*plan, d, stream) != 0) return PA_ERR_CUDA;
+    record_profile(*plan, 1, static_cast<cudaStream_t>(stream));
+  }
+  record_profile(*plan, 2, static_cast<cudaStream_t>(stream));
+  if (pa_launch_simt(*plan, d, stream) != 0) return PA_ERR_CUDA;
+  record_profile(*plan, 3, static_cast<cudaStream_t>(stream));
+  return PA_OK;
+}
+
+extern "C" pa_status pa_merge(const pa_plan* plan, void* d_workspace, void* out, float* lse, void* stream) {
+  if (!plan || !d_workspace || !out) return PA_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(out) & 15) return PA_ERR_INVALID;
+  PaDevPtrs d = dev_ptrs(*plan, d_workspace);
+  record_profile(*plan, 4, static_cast<cudaStream_t>(stream));
+  const int e = pa_launch_merge(*plan, d, out, lse, stream);
+  record_profile(*plan, 5, static_cast<cudaStream_t>(stream));
+  return e == 0 ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" pa_status pa_attend(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
+                               void* d_workspace, void* out, float* lse, void* stream) {
+  pa_status s = pa_forward(plan, q, k_pool, v_pool, d_workspace, stream);
+  if (s != PA_OK) return s;
+  return pa_merge(plan, d_workspace, out, lse, stream);
+}
+
+extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_workspace, void* stream,
+                                          pa_status* out) {
+  if (!plan || !d_workspace || !out) return PA_ERR_INVALID;
+  int32_t word = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* src = static_cast<const uint8_t*>(d_workspace) + offsetof(pa_image_header, status);
+  if (cudaMemcpyAsync(&word, src, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
+  *out = static_cast<pa_status>(word);
+  return PA_OK;
+}

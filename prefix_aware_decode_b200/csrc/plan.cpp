@@ -1,0 +1,442 @@
+// Pack stage (host): tree-structured block table, profit model, split of long
+// nodes, tile-class selection, work ordering and partial-row assignment.
+//
+// Source: the PAT review, section 三 (Pack Scheduler 工作流, Figure 7: a decode
+// batch, its tree-structured block table, packing scheme 1 that keeps a parent
+// node separate from its leaves and packing scheme 2 that folds a leaf together
+// with its parent; Pack 阶段: group queries by shared prefix into CTA work with a
+// profit-model heuristic that weighs prefix length and query count; Forward 阶段:
+// a runtime tile selector, multi-stream execution and long-KV splitting).  The
+// page gives no formula for the profit model or the split; the rules used here
+// are stated at each step.
+//
+// Cost: every (request, page) entry of the block table is compared at most
+// once while the tree is built, and the work lists are written with one pass
+// over the items, so planning is linear in the number of pages.
+#include <algorithm>
+#include <chrono>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <numeric>
+#include <vector>
+
+#include "plan.h"
+
+namespace {
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+struct ItemRec {
+  int page_off, n_tokens, n_queries, query_off;
+  bool simt;
+};
+
+struct SegRec {
+  int item, kv_head, page_begin, n_tokens, prow, query;
+};
+
+struct Planner {
+  const int32_t* kv_lens;
+  const int32_t* bt;
+  int max_pages, P, G, Hq, Hkv, D;
+  uint32_t flags;
+  std::vector<int> order, npg;
+  // outputs of the tree walk
+  std::vector<ItemRec> items;
+  std::vector<int32_t> pages, queries;
+  int64_t unique_tokens = 0, read_tokens = 0;
+  int num_nodes = 0, num_shared = 0, num_kept = 0;
+  bool invalid = false;
+  std::vector<int> qbuf;
+
+  const int32_t* row(int b) const { return bt + (size_t)b * max_pages; }
+
+  void add_item(int rep, int page_lo, int page_hi, int64_t tokens, const int* qs, int nq, bool simt) {
+    const int off = (int)pages.size();
+    const int32_t* r = row(rep);
+    pages.insert(pages.end(), r + page_lo, r + page_hi);
+    if (simt) {
+      items.push_back({off, (int)tokens, 1, (int)queries.size(), true});
+      queries.push_back(qs[0]);
+      read_tokens += tokens;
+      return;
+    }
+    // tensor-core class: query tiles of at most kMmaRowsPerCta rows
+    const int qpt = std::max(1, kMmaRowsPerCta / G);
+    for (int t = 0; t < nq; t += qpt) {
+      const int n = std::min(qpt, nq - t);
+      items.push_back({off, (int)tokens, n, (int)queries.size(), false});
+      queries.insert(queries.end(), qs + t, qs + t + n);
+      read_tokens += tokens;
+    }
+  }
+
+  // Profit model (packing scheme 1 vs 2).  A node with n >= 2 requests whose
+  // item would cover L tokens stays shared iff
+  //     (n - 1) * L * Bt  >  n * Hq * (4D + 4) * 2 + C_item,
+  // Bt = K+V bytes per token over all kv heads: what sharing saves is the
+  // (n - 1) extra reads of the node; what it costs is one more fp32 partial row
+  // per request and head (written by forward, read by merge) and a fixed
+  // per-item overhead C_item.  Otherwise the node is folded into its children.
+  bool keep_shared(int n, int64_t L) const {
+    if (flags & PA_PLAN_NO_SHARING) return false;
+    if (flags & PA_PLAN_ALWAYS_SHARE) return true;
+    const double Bt = 2.0 * Hkv * D * 2, C_item = 64.0 * 1024;
+    return (n - 1) * (double)L * Bt > n * (double)Hq * (4.0 * D + 4.0) * 2.0 + C_item;
+  }
+
+  // Requests order[lo, hi) share logical pages [0, depth).  eff_lo is the first
+  // page not yet covered by an emitted ancestor (pages of folded ancestors are
+  // read again by this subtree's items).
+  void walk(int lo, int hi, int depth, int eff_lo) {
+    if (invalid) return;
+    if (hi - lo == 1) {
+      const int b = order[lo];
+      if (npg[b] > depth) {
+        ++num_nodes;
+        unique_tokens += kv_lens[b] - (int64_t)depth * P;
+      }
+      add_item(b, eff_lo, npg[b], kv_lens[b] - (int64_t)eff_lo * P, &b, 1, true);
+      return;
+    }
+    // extend the common prefix column by column
+    const int32_t* r0 = row(order[lo]);
+    int mn = npg[order[lo]];
+    for (int i = lo + 1; i < hi; ++i) mn = std::min(mn, npg[order[i]]);
+    int l = depth;
+    while (l < mn) {
+      const int32_t v = r0[l];
+      bool same = true;
+      for (int i = lo + 1; i < hi; ++i)
+        if (row(order[i])[l] != v) { same = false; break; }
+      if (!same) break;
+      ++l;
+    }
+    bool keep = false;
+    int next_eff = eff_lo;
+    const int nq = hi - lo;
+    if (l > depth) {
+      // a shared page must be full for every request that shares it
+      for (int i = lo; i < hi; ++i)
+        if (kv_lens[order[i]] / P < l) { invalid = true; return; }
+      ++num_nodes;
+      ++num_shared;
+      unique_tokens += (int64_t)(l - depth) * P;
+      keep = keep_shared(nq, (int64_t)(l - eff_lo) * P);
+      if (keep) {
+        ++num_kept;
+        qbuf.assign(order.begin() + lo, order.begin() + hi);
+        std::sort(qbuf.begin(), qbuf.end());
+        add_item(qbuf[0], eff_lo, l, (int64_t)(l - eff_lo) * P, qbuf.data(), nq, false);
+        next_eff = l;
+      }
+    }
+    // requests ending at page l come first; the rest are grouped by their page at l
+    auto mid = std::partition(order.begin() + lo, order.begin() + hi, [&](int b) { return npg[b] == l; });
+    const int e = (int)(mid - order.begin());
+    for (int i = lo; i < e; ++i)
+      if (!keep && l > eff_lo) {
+        const int b = order[i];
+        add_item(b, eff_lo, l, kv_lens[b] - (int64_t)eff_lo * P, &b, 1, true);
+      }
+    std::sort(order.begin() + e, order.begin() + hi, [&](int a, int b) {
+      const int32_t pa = row(a)[l], pb = row(b)[l];
+      return pa != pb ? pa < pb : a < b;
+    });
+    int start = e;
+    for (int i = e + 1; i <= hi; ++i) {
+      if (i == hi || row(order[i])[l] != row(order[start])[l]) {
+        walk(start, i, l, next_eff);
+        start = i;
+      }
+    }
+  }
+};
+
+}  // namespace
+
+extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const int32_t* kv_lens,
+                                    const int32_t* block_table, int32_t max_pages, int32_t num_pages_in_pool,
+                                    pa_plan** out) {
+  if (out) *out = nullptr;
+  if (!cfg || !kv_lens || !block_table || !out) return PA_ERR_INVALID;
+  auto t0 = std::chrono::steady_clock::now();
+  const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, D = cfg->head_dim, P = cfg->page_size;
+  if (batch < 1 || max_pages < 1 || num_pages_in_pool < 1 || Hq < 1 || Hkv < 1 || D < 1 || P < 1)
+    return PA_ERR_INVALID;
+  if (Hq % Hkv != 0) return PA_ERR_INVALID;
+  const int G = Hq / Hkv;
+  if (!(G == 1 || G == 2 || G == 4 || G == 8)) return PA_ERR_UNSUPPORTED;
+  if (!(D == 64 || D == 128)) return PA_ERR_UNSUPPORTED;
+  if (P != 16) return PA_ERR_UNSUPPORTED;
+  if (cfg->softmax_scale < 0.f || !std::isfinite(cfg->softmax_scale)) return PA_ERR_INVALID;
+  if (cfg->max_chunk_tokens < 0 || cfg->wait_timeout_us < 0 || cfg->num_sms < 0) return PA_ERR_INVALID;
+  const uint32_t flags = cfg->flags;
+  if ((flags & PA_PLAN_NO_SHARING) && (flags & PA_PLAN_ALWAYS_SHARE)) return PA_ERR_INVALID;
+  if ((int64_t)num_pages_in_pool * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
+
+  pa_plan* plan = new (std::nothrow) pa_plan();
+  if (!plan) return PA_ERR_NOMEM;
+  try {
+    plan->cfg = *cfg;
+    plan->B = batch;
+    plan->Hq = Hq;
+    plan->Hkv = Hkv;
+    plan->G = G;
+    plan->D = D;
+    plan->P = P;
+    plan->num_pages_in_pool = num_pages_in_pool;
+    plan->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / std::sqrt((float)D);
+    plan->num_sms = cfg->num_sms > 0 ? cfg->num_sms : 148;
+    plan->flags = flags;
+    plan->wait_timeout_us = cfg->wait_timeout_us > 0 ? cfg->wait_timeout_us : 2000000;
+
+    // ---- validation
+    Planner pl;
+    pl.kv_lens = kv_lens;
+    pl.bt = block_table;
+    pl.max_pages = max_pages;
+    pl.P = P;
+    pl.G = G;
+    pl.Hq = Hq;
+    pl.Hkv = Hkv;
+    pl.D = D;
+    pl.flags = flags;
+    pl.npg.resize(batch);
+    int64_t total_pages = 0;
+    for (int b = 0; b < batch; ++b) {
+      const int64_t n = kv_lens[b];
+      if (n < 1 || n > (int64_t)max_pages * P) { delete plan; return PA_ERR_INVALID; }
+      pl.npg[b] = (int)ceil_div(n, P);
+      total_pages += pl.npg[b];
+      const int32_t* r = block_table + (size_t)b * max_pages;
+      bool bad = false;
+      for (int j = 0; j < pl.npg[b]; ++j) bad |= (uint32_t)r[j] >= (uint32_t)num_pages_in_pool;
+      if (bad) { delete plan; return PA_ERR_INVALID; }
+    }
+
+    // ---- tree-structured block table + profit model + emission
+    pl.order.resize(batch);
+    std::iota(pl.order.begin(), pl.order.end(), 0);
+    pl.items.reserve(batch + 64);
+    pl.pages.reserve(total_pages);
+    pl.queries.reserve(2 * batch);
+    pl.walk(0, batch, 0, 0);
+    if (pl.invalid) { delete plan; return PA_ERR_INVALID; }
+    const std::vector<ItemRec>& items = pl.items;
+    const std::vector<int32_t>& pages = pl.pages;
+    const std::vector<int32_t>& queries = pl.queries;
+
+    // ---- split and tile selection
+    // Tile class by rows (requests x G): one request -> SIMT class (CUDA
+    // cores); two or more -> MMA class (tensor cores, query tiles of <= 64 rows).
+    // SIMT: stream-K split.  The (item, kv head) page runs are concatenated and
+    // cut into equal spans of `span` pages, one span per warp; a span may end
+    // inside an item, so every warp gets the same number of pages and partial
+    // rows appear only at span boundaries.
+    // MMA: each (item, kv head) is cut into chunks of `chunk` tokens, one CTA
+    // per chunk, launched longest first.
+    const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
+    int64_t simt_pages = 0, mma_tile_tokens = 0;
+    for (const auto& it : items) {
+      if (it.simt) simt_pages += ceil_div(it.n_tokens, P) * Hkv;
+      else mma_tile_tokens += (int64_t)it.n_tokens * Hkv;
+    }
+    std::vector<SegRec> simt_segs, mma_segs;
+    std::vector<int32_t> warp_segs{0}, warp_loads{0};
+    std::vector<int32_t> tiles((size_t)simt_pages);
+    if (simt_pages > 0) {
+      const int64_t W = (int64_t)plan->num_sms * kSimtWarpsPerCta;
+      int64_t span = ceil_div(simt_pages, W);
+      if (span < 4) span = 4;
+      if (max_chunk_pages) span = std::min(span, max_chunk_pages);
+      simt_segs.reserve(items.size() * Hkv + simt_pages / span + 8);
+      int64_t used = 0;  // pages in the current warp's span
+      size_t t = 0;      // tiles written
+      for (size_t i = 0; i < items.size(); ++i) {
+        const ItemRec& it = items[i];
+        if (!it.simt) continue;
+        const int npages = (int)ceil_div(it.n_tokens, P);
+        const int32_t* pp = pages.data() + it.page_off;
+        const int b = queries[it.query_off];
+        for (int g = 0; g < Hkv; ++g) {
+          for (int j = 0; j < npages; ++j) tiles[t + j] = pp[j] * Hkv + g;
+          t += npages;
+          int pb = 0;
+          while (pb < npages) {
+            const int take = (int)std::min<int64_t>(npages - pb, span - used);
+            const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
+            simt_segs.push_back({(int)i, g, pb, tok, -1, b});
+            pb += take;
+            used += take;
+            if (used == span) {
+              warp_segs.push_back((int32_t)simt_segs.size());
+              warp_loads.push_back((int32_t)(t - (npages - pb)));
+              used = 0;
+            }
+          }
+        }
+      }
+      if (used > 0) {
+        warp_segs.push_back((int32_t)simt_segs.size());
+        warp_loads.push_back((int32_t)t);
+      }
+    }
+    if (mma_tile_tokens > 0) {
+      const int64_t target = (int64_t)plan->num_sms * 4;
+      int64_t chunk = ceil_div(ceil_div(mma_tile_tokens, target), P) * P;
+      chunk = std::max<int64_t>(512, std::min<int64_t>(8192, chunk));
+      if (max_chunk_pages) chunk = std::min<int64_t>(chunk, max_chunk_pages * P);
+      for (size_t i = 0; i < items.size(); ++i) {
+        const ItemRec& it = items[i];
+        if (it.simt) continue;
+        const int npages = (int)ceil_div(it.n_tokens, P);
+        const int cp = (int)(chunk / P);
+        for (int pb = 0; pb < npages; pb += cp) {
+          const int pe = std::min(npages, pb + cp);
+          const int tok = std::min(it.n_tokens, pe * P) - pb * P;
+          for (int g = 0; g < Hkv; ++g) mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
+        }
+      }
+      std::stable_sort(mma_segs.begin(), mma_segs.end(),
+                       [](const SegRec& a, const SegRec& b) { return a.n_tokens > b.n_tokens; });
+    }
+
+    // ---- partial rows: contiguous per (request, kv head), in a fixed order
+    std::vector<int32_t> prow_off((size_t)batch * Hkv + 1, 0);
+    for (const auto& s : mma_segs) {
+      const ItemRec& it = items[s.item];
+      for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
+    }
+    for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
+    for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
+    std::vector<int32_t> cursor(prow_off.begin(), prow_off.end() - 1);
+    std::vector<int32_t> seg_prows;
+    for (auto& s : mma_segs) {
+      const ItemRec& it = items[s.item];
+      s.prow = (int)seg_prows.size();
+      for (int j = 0; j < it.n_queries; ++j)
+        seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
+    }
+    for (auto& s : simt_segs) s.prow = cursor[(size_t)s.query * Hkv + s.kv_head]++;
+    const int num_prows = prow_off.back();
+
+    // ---- image
+    pa_image_header& h = plan->hdr;
+    std::memset(&h, 0, sizeof(h));
+    h.magic = 0x50414231u;
+    h.batch = batch;
+    h.num_q_heads = Hq;
+    h.num_kv_heads = Hkv;
+    h.head_dim = D;
+    h.page_size = P;
+    h.num_items = (int32_t)items.size();
+    h.num_segments_simt = (int32_t)simt_segs.size();
+    h.num_segments_mma = (int32_t)mma_segs.size();
+    h.num_segments = h.num_segments_simt + h.num_segments_mma;
+    h.simt_warps = (int32_t)warp_segs.size() - 1;
+    h.num_partial_rows = num_prows;
+    h.num_loads = (int32_t)tiles.size();
+    uint64_t off = align256(sizeof(pa_image_header));
+    h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
+    h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
+    h.off_pages = off; off = align256(off + pages.size() * 4);
+    h.off_queries = off; off = align256(off + queries.size() * 4);
+    h.off_seg_prows = off; off = align256(off + seg_prows.size() * 4);
+    h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
+    h.off_warp_loads = off; off = align256(off + warp_loads.size() * 4);
+    h.off_tiles = off; off = align256(off + tiles.size() * 4);
+    h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
+    h.image_bytes = off;
+    h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
+    h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
+    h.workspace_bytes = off;
+
+    plan->image.resize(h.image_bytes);
+    uint8_t* img = plan->image.data();
+    std::memcpy(img, &h, sizeof(h));
+    pa_item* di = reinterpret_cast<pa_item*>(img + h.off_nodes);
+    for (size_t i = 0; i < items.size(); ++i)
+      di[i] = {items[i].page_off, items[i].n_tokens, items[i].n_queries, items[i].query_off};
+    pa_seg* ds = reinterpret_cast<pa_seg*>(img + h.off_segs);
+    size_t k = 0;
+    for (const auto& s : simt_segs) ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, 0};
+    for (const auto& s : mma_segs) ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, 0};
+    auto put = [&](uint64_t o, const std::vector<int32_t>& v) {
+      if (!v.empty()) std::memcpy(img + o, v.data(), v.size() * 4);
+    };
+    put(h.off_pages, pages);
+    put(h.off_queries, queries);
+    put(h.off_seg_prows, seg_prows);
+    put(h.off_warp_segs, warp_segs);
+    put(h.off_warp_loads, warp_loads);
+    put(h.off_tiles, tiles);
+    put(h.off_prow_off, prow_off);
+
+    pa_plan_stats& st = plan->stats;
+    st.batch = batch;
+    st.num_nodes = pl.num_nodes;
+    st.num_shared_nodes = pl.num_shared;
+    st.num_kept_shared = pl.num_kept;
+    st.num_items = (int32_t)items.size();
+    st.num_segments = h.num_segments;
+    st.num_segments_simt = h.num_segments_simt;
+    st.num_segments_mma = h.num_segments_mma;
+    st.num_partial_rows = num_prows;
+    st.simt_warps = h.simt_warps;
+    st.unique_tokens = pl.unique_tokens;
+    int64_t naive = 0;
+    for (int b = 0; b < batch; ++b) naive += kv_lens[b];
+    st.naive_tokens = naive;
+    st.read_tokens = pl.read_tokens;
+    st.unique_kv_bytes = pl.unique_tokens * (int64_t)(2 * Hkv * D * 2);
+    st.read_kv_bytes = pl.read_tokens * (int64_t)(2 * Hkv * D * 2);
+    st.workspace_bytes = h.workspace_bytes;
+    st.image_bytes = h.image_bytes;
+    st.plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+    *out = plan;
+    return PA_OK;
+  } catch (const std::bad_alloc&) {
+    delete plan;
+    return PA_ERR_NOMEM;
+  } catch (...) {
+    delete plan;
+    return PA_ERR_INVALID;
+  }
+}
+
+extern "C" pa_status pa_plan_workspace_size(const pa_plan* plan, size_t* bytes) {
+  if (!plan || !bytes) return PA_ERR_INVALID;
+  *bytes = plan->hdr.workspace_bytes;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_plan_get_stats(const pa_plan* plan, pa_plan_stats* out) {
+  if (!plan || !out) return PA_ERR_INVALID;
+  *out = plan->stats;
+  return PA_OK;
+}
+
+extern "C" pa_status pa_plan_host_image(const pa_plan* plan, void* dst, size_t bytes) {
+  if (!plan || !dst) return PA_ERR_INVALID;
+  if (bytes < plan->image.size()) return PA_ERR_NOMEM;
+  std::memcpy(dst, plan->image.data(), plan->image.size());
+  return PA_OK;
+}
+
+extern "C" void pa_plan_destroy(pa_plan* plan) { delete plan; }
+
+extern "C" const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_NOMEM: return "out of memory or workspace too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_TIMEOUT: return "device wait timed out";
+    case PA_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}

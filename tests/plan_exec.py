@@ -1,0 +1,121 @@
+"""CPU executor of a plan image (test utility; neither the oracle nor the product).
+
+It reads the bytes pa_plan_upload would send (layout in include/pa.h), runs
+every forward segment in fp64 with the oracle's dense attention, and merges each
+(request, head)'s partial rows with the oracle's log-sum-exp merge.  It also
+checks the plan's structure: every (request, kv head) reads each of its tokens
+exactly once, every partial row is written once, and the SIMT tile list matches
+the segments.
+"""
+import ctypes
+
+import numpy as np
+
+import oracle
+from prefix_aware_decode_b200 import PaImageHeader
+from prefix_aware_decode_b200 import workload as wl
+
+
+class Image:
+    def __init__(self, buf: np.ndarray):
+        h = PaImageHeader.from_buffer_copy(buf[: ctypes.sizeof(PaImageHeader)].tobytes())
+        assert h.magic == 0x50414231
+        self.h = h
+
+        def arr(off, n, dt=np.int32, cols=None):
+            a = np.frombuffer(buf, dtype=dt, count=n * (cols or 1), offset=off)
+            return a.reshape(n, cols) if cols else a
+
+        self.items = arr(h.off_nodes, h.num_items, cols=4)  # page_off, n_tokens, n_queries, query_off
+        self.segs = arr(h.off_segs, h.num_segments, cols=8)[:, :6]  # item, kv_head, page_begin, n_tokens, prow, query
+        n_pages = (h.off_queries - h.off_pages) // 4
+        self.pages = arr(h.off_pages, n_pages)
+        self.queries = arr(h.off_queries, (h.off_seg_prows - h.off_queries) // 4)
+        self.seg_prows = arr(h.off_seg_prows, (h.off_warp_segs - h.off_seg_prows) // 4)
+        self.warp_segs = arr(h.off_warp_segs, h.simt_warps + 1)
+        self.warp_loads = arr(h.off_warp_loads, h.simt_warps + 1)
+        self.tiles = arr(h.off_tiles, h.num_loads)
+        self.prow_off = arr(h.off_prow_off, h.batch * h.num_kv_heads + 1)
+
+
+def check_structure(img: Image, kv_lens, block_table, P=16):
+    h = img.h
+    B, Hkv, G = h.batch, h.num_kv_heads, h.num_q_heads // h.num_kv_heads
+    nseg_simt = h.num_segments_simt
+    # warp lists partition the SIMT segments and tiles, in order
+    assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
+    assert np.all(np.diff(img.warp_segs) > 0)
+    assert img.warp_loads[0] == 0 and img.warp_loads[-1] == h.num_loads
+    # the tile list equals the pages of the SIMT segments, in order
+    t = 0
+    for w in range(h.simt_warps):
+        assert img.warp_loads[w] == t
+        for si in range(img.warp_segs[w], img.warp_segs[w + 1]):
+            item, g, pb, nt, prow, q = img.segs[si]
+            po, itok, nq, qo = img.items[item]
+            assert nq == 1 and img.queries[qo] == q
+            npg = -(-nt // P)
+            want = img.pages[po + pb: po + pb + npg] * Hkv + g
+            assert np.array_equal(img.tiles[t:t + npg], want)
+            t += npg
+    assert t == h.num_loads
+    # coverage: each (request, kv head) reads each token (page, slot) exactly once
+    seen = {}
+    prows_written = np.zeros(h.num_partial_rows, dtype=np.int64)
+    for si in range(h.num_segments):
+        item, g, pb, nt, prow, q0 = img.segs[si]
+        po, itok, nq, qo = img.items[item]
+        assert 1 <= nt and pb * P + nt <= itok
+        qs = img.queries[qo: qo + nq]
+        if si < nseg_simt:
+            prs = [prow]
+        else:
+            prs = img.seg_prows[prow: prow + nq]
+        for b, pr in zip(qs, prs):
+            assert img.prow_off[b * Hkv + g] <= pr < img.prow_off[b * Hkv + g + 1]
+            prows_written[pr] += 1
+            for tok in range(pb * P, pb * P + nt):
+                key = (int(b), int(g), int(img.pages[po + tok // P]), tok % P)
+                seen[key] = seen.get(key, 0) + 1
+    assert np.all(prows_written == 1)
+    assert all(v == 1 for v in seen.values())
+    for b in range(B):
+        n = int(kv_lens[b])
+        for g in range(Hkv):
+            for tok in range(n):
+                assert seen.get((b, g, int(block_table[b, tok // P]), tok % P)) == 1, (b, g, tok)
+    assert len(seen) == int(np.sum(kv_lens)) * Hkv
+
+
+def execute(img: Image, q, k_pool, v_pool, scale=None, P=16):
+    """Run the plan in fp64: returns (out[B][Hq][D], lse[B][Hq])."""
+    h = img.h
+    B, Hq, Hkv, D = h.batch, h.num_q_heads, h.num_kv_heads, h.head_dim
+    G = Hq // Hkv
+    po_ = np.zeros((h.num_partial_rows, G, D))
+    pl_ = np.full((h.num_partial_rows, G), -np.inf)
+    kf = wl.bf16_bits_to_f32(k_pool).astype(np.float64)
+    vf = wl.bf16_bits_to_f32(v_pool).astype(np.float64)
+    qf = wl.bf16_bits_to_f32(q).astype(np.float64)
+    for si in range(h.num_segments):
+        item, g, pb, nt, prow, q0 = img.segs[si]
+        po, itok, nq, qo = img.items[item]
+        toks = np.arange(pb * P, pb * P + nt)
+        pg = img.pages[po + toks // P]
+        K = kf[pg, g, toks % P]
+        V = vf[pg, g, toks % P]
+        qs = img.queries[qo: qo + nq]
+        prs = [prow] if si < h.num_segments_simt else img.seg_prows[prow: prow + nq]
+        for b, pr in zip(qs, prs):
+            for r in range(G):
+                o, l = oracle.attend_dense(qf[b, g * G + r], K, V, scale)
+                po_[pr, r] = o
+                pl_[pr, r] = l
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        for hh in range(Hq):
+            g, r = hh // G, hh % G
+            a, e = img.prow_off[b * Hkv + g], img.prow_off[b * Hkv + g + 1]
+            out[b, hh], lse[b, hh] = oracle.merge(po_[a:e, r], pl_[a:e, r])
+    return out, lse

@@ -1,0 +1,155 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Inputs are the seeded synthetic workloads (NaN-poisoned spare pages and
+tails); tolerances: max abs 2e-3 and max relative 1e-2 (floored by the row rms)
+on bf16 outputs, 1e-4 on fp32 lse.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import prefix_aware_decode_b200 as pad
+from prefix_aware_decode_b200 import workload as wl
+
+from gpu_util import DevWorkload, assert_close, compare, run
+
+pytestmark = pytest.mark.gpu
+
+_cache = {}
+
+
+def dev_config(c, scale=1.0):
+    key = (c, scale)
+    if key not in _cache:
+        _cache.clear()
+        torch.cuda.empty_cache()
+        _cache[key] = DevWorkload(wl.make_config(c, scale=scale))
+    return _cache[key]
+
+
+def sample(B, n, seed=0):
+    if B <= n:
+        return np.arange(B, dtype=np.int32)
+    r = np.random.default_rng(seed)
+    s = np.sort(r.choice(B, size=n - 2, replace=False))
+    return np.unique(np.concatenate([[0, B - 1], s])).astype(np.int32)
+
+
+@pytest.mark.parametrize("config", [1, 2])
+def test_small_configs_full_parity(config):
+    dw = dev_config(config)
+    w = dw.w
+    out, lse, st, _ = run(dw)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    m = compare(out, lse, ref_o, ref_l)
+    assert_close(m, f"config {config}")
+
+
+@pytest.mark.parametrize("config", [3, 4])
+def test_large_configs_sampled_parity(config):
+    dw = dev_config(config)
+    w = dw.w
+    out, lse, st, _ = run(dw)
+    qs = sample(w.B, 40, seed=config)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs)
+    assert_close(compare(out, lse, ref_o, ref_l, queries=qs), f"config {config}")
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+def test_config5_sampled_parity():
+    dw = dev_config(5)
+    w = dw.w
+    out, lse, st, _ = run(dw)
+    assert st["num_segments_mma"] > 0
+    qs = np.array([0, 1, 15, 16, 255, 256, 500, 511], dtype=np.int32)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs)
+    assert_close(compare(out, lse, ref_o, ref_l, queries=qs), "config 5")
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("flags,chunk", [(pad.PA_PLAN_NO_SHARING, 0), (pad.PA_PLAN_ALWAYS_SHARE, 64),
+                                         (0, 16), (pad.PA_PLAN_ALWAYS_SHARE, 16)])
+def test_plan_modes_match_oracle(flags, chunk):
+    dw = dev_config(2, scale=0.25)
+    w = dw.w
+    out, lse, st, _ = run(dw, flags=flags, max_chunk_tokens=chunk)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    assert_close(compare(out, lse, ref_o, ref_l), f"flags {flags} chunk {chunk}")
+
+
+@pytest.mark.parametrize("G,D", [(1, 64), (2, 128), (4, 64), (4, 128), (8, 64), (8, 128), (1, 128), (2, 64)])
+def test_random_forests_gqa_and_head_dim(G, D):
+    roots = wl.random_tree(seed=G * 10 + D, n_queries=24, depth=3, shared_pages=(1, 12), leaf_tokens=(1, 300),
+                           fanout=(1, 6))
+    w = wl.build_workload("rand", roots, Hq=4 * G, Hkv=4, D=D, seed=G * 1000 + D)
+    dw = DevWorkload(w)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    for flags, chunk in [(0, 0), (pad.PA_PLAN_ALWAYS_SHARE, 32), (pad.PA_PLAN_NO_SHARING, 0)]:
+        out, lse, st, _ = run(dw, flags=flags, max_chunk_tokens=chunk)
+        assert_close(compare(out, lse, ref_o, ref_l), f"G={G} D={D} flags={flags}")
+
+
+def test_edge_lengths_and_ragged_tails():
+    lens = [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 255, 256, 257, 1000, 4099]
+    roots = [wl.Node(n) for n in lens]
+    # plus a shared prefix whose children end 0..17 tokens after it
+    roots.append(wl.Node(48, [wl.Node(n) for n in (1, 5, 16, 17)]))
+    w = wl.build_workload("edges", roots, Hq=32, Hkv=8, D=128, seed=4242)
+    dw = DevWorkload(w)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    for flags, chunk in [(0, 0), (pad.PA_PLAN_ALWAYS_SHARE, 16), (0, 32)]:
+        out, lse, st, _ = run(dw, flags=flags, max_chunk_tokens=chunk)
+        assert_close(compare(out, lse, ref_o, ref_l), f"edges flags={flags} chunk={chunk}")
+
+
+def test_single_key_returns_v_row_bit_exact():
+    roots = [wl.Node(1) for _ in range(16)]
+    w = wl.build_workload("one", roots, Hq=32, Hkv=8, D=128, seed=77)
+    dw = DevWorkload(w)
+    out, lse, st, _ = run(dw)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    G = w.Hq // w.Hkv
+    for b in range(w.B):
+        page = w.block_table[b, 0]
+        for h in range(w.Hq):
+            assert np.array_equal(got[b, h], w.v_pool[page, h // G, 0]), (b, h)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    assert np.abs(lse.cpu().numpy() - ref_l).max() <= 1e-4
+
+
+def test_results_are_bit_reproducible():
+    dw = dev_config(2, scale=0.25)
+    a, la, _, _ = run(dw)
+    b, lb, _, _ = run(dw)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)) and torch.equal(la, lb)
+
+
+@pytest.mark.parametrize("flags", [0, pad.PA_PLAN_ALWAYS_SHARE])
+def test_bounded_wait_reports_timeout_and_context_survives(flags):
+    """A forward that never receives one of its loads must give up after the
+    configured limit, record PA_ERR_TIMEOUT in the workspace, and leave the
+    context usable (a normal run right after it still matches the oracle)."""
+    w = wl.make_config(1)
+    dw = DevWorkload(w)
+    out, lse, st, status = run(dw, flags=flags | pad.PA_PLAN_FAULT_DROP_LOAD, wait_timeout_us=20000,
+                               check_status=False)
+    assert status == pad.PA_ERR_TIMEOUT
+    out, lse, st, status = run(dw, flags=flags)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    assert_close(compare(out, lse, ref_o, ref_l), "after timeout")
+
+
+def test_attend_convenience_and_validation():
+    dw = dev_config(1)
+    w = dw.w
+    out, lse = pad.attend(dw.q, dw.k, dw.v, w.block_table, w.kv_lens)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    assert_close(compare(out, lse, ref_o, ref_l), "attend()")
+    plan = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    ws = plan.alloc_workspace()
+    # a workspace that is too small, or misaligned pointers, are refused before anything is enqueued
+    assert plan._lib.pa_plan_upload(plan.handle, ws.data_ptr(), 16, None) == pad.PA_ERR_NOMEM
+    assert plan._lib.pa_forward(plan.handle, dw.q.data_ptr() + 2, dw.k.data_ptr(), dw.v.data_ptr(),
+                                ws.data_ptr(), None) == pad.PA_ERR_INVALID
+    plan.close()

@@ -1,0 +1,132 @@
+"""Pack stage on the host: tree structure, coverage, validation, and the plan
+executed on the CPU (fp64) against the oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import prefix_aware_decode_b200 as pad
+from prefix_aware_decode_b200 import workload as wl
+
+from plan_exec import Image, check_structure, execute
+
+
+def make_plan(w, **kw):
+    return pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D, **kw)
+
+
+def test_exports_match_header(repo_root):
+    import ctypes
+    import os
+    import re
+    hdr = open(os.path.join(repo_root, "include", "pa.h")).read()
+    declared = re.findall(r"^\s*(?:pa_status|void|const char \*)\s*(pa_\w+)\s*\(", hdr, re.M)
+    assert declared, "no declarations found"
+    L = pad.lib()
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) <= set(pad._binding.EXPORTS) | {"pa_plan_stats"}
+    assert ctypes.sizeof(pad._binding.PaConfig) == 36
+
+
+@pytest.mark.parametrize("config", [1, 2, 3, 4, 5])
+def test_config_plans_cover_every_token(config):
+    w = wl.make_config(config, with_values=False, scale=1.0 if config in (1, 2) else 0.125)
+    p = make_plan(w)
+    st = p.stats()
+    check_structure(Image(p.host_image()), w.kv_lens, w.block_table)
+    assert st["unique_tokens"] == w.unique_tokens
+    assert st["naive_tokens"] == w.naive_tokens
+    assert st["read_tokens"] >= st["unique_tokens"]
+
+
+def test_config2_tree_and_classes():
+    w = wl.make_config(2, with_values=False)
+    st = make_plan(w).stats()
+    assert st["num_nodes"] == 65 and st["num_shared_nodes"] == 1 and st["num_kept_shared"] == 1
+    # 256 rows of the shared root -> 4 query tiles of 64 rows on the tensor-core class
+    assert st["num_items"] == 64 + 4
+    assert st["num_segments_mma"] > 0 and st["num_segments_simt"] > 0
+
+
+def test_config4_has_no_tensor_core_work():
+    w = wl.make_config(4, with_values=False)
+    st = make_plan(w).stats()
+    assert st["num_segments_mma"] == 0 and st["num_shared_nodes"] == 0
+    assert st["read_tokens"] == st["unique_tokens"] == st["naive_tokens"]
+
+
+def test_no_sharing_mode_reads_naive_tokens():
+    w = wl.make_config(2, with_values=False)
+    st = make_plan(w, flags=pad.PA_PLAN_NO_SHARING).stats()
+    assert st["num_kept_shared"] == 0 and st["num_segments_mma"] == 0
+    assert st["read_tokens"] == st["naive_tokens"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_forests_execute_to_oracle(seed):
+    G = [1, 2, 4, 8][seed % 4]
+    D = [64, 128][seed % 2]
+    roots = wl.random_tree(seed=100 + seed, n_queries=7, depth=3, shared_pages=(1, 4), leaf_tokens=(1, 40))
+    w = wl.build_workload("rand", roots, Hq=2 * G, Hkv=2, D=D, seed=500 + seed)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    for flags, chunk in [(0, 0), (pad.PA_PLAN_ALWAYS_SHARE, 16), (pad.PA_PLAN_NO_SHARING, 32),
+                         (pad.PA_PLAN_ALWAYS_SHARE, 0)]:
+        p = make_plan(w, flags=flags, max_chunk_tokens=chunk)
+        img = Image(p.host_image())
+        check_structure(img, w.kv_lens, w.block_table)
+        out, lse = execute(img, w.q, w.k_pool, w.v_pool)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+
+
+def test_config1_executes_to_oracle():
+    w = wl.make_config(1)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    for chunk in (0, 16, 48):
+        img = Image(make_plan(w, max_chunk_tokens=chunk).host_image())
+        out, lse = execute(img, w.q, w.k_pool, w.v_pool)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+
+
+def test_requests_ending_inside_the_tree():
+    # request 0's KV is exactly the shared prefix of requests 1 and 2 (full pages)
+    P = 16
+    bt = np.array([[5, 6, -1, -1], [5, 6, 7, -1], [5, 6, 8, 9]], dtype=np.int32)
+    kv = np.array([32, 40, 50], dtype=np.int32)
+    for flags in (0, pad.PA_PLAN_ALWAYS_SHARE, pad.PA_PLAN_NO_SHARING):
+        p = pad.Plan(kv, bt, 10, 4, 1, 64, flags=flags)
+        check_structure(Image(p.host_image()), kv, bt, P)
+    # two identical full requests
+    bt2 = np.array([[3, 4], [3, 4]], dtype=np.int32)
+    p = pad.Plan(np.array([32, 32], dtype=np.int32), bt2, 5, 4, 1, 64, flags=pad.PA_PLAN_ALWAYS_SHARE)
+    check_structure(Image(p.host_image()), np.array([32, 32]), bt2, P)
+
+
+def test_validation_errors():
+    bt = np.array([[1, 2], [1, 3]], dtype=np.int32)
+    ok = np.array([20, 30], dtype=np.int32)
+    pad.Plan(ok, bt, 4, 8, 2, 64)
+    cases = [
+        (dict(kv_lens=np.array([0, 30], dtype=np.int32)), pad.PA_ERR_INVALID),      # empty request
+        (dict(kv_lens=np.array([20, 33], dtype=np.int32)), pad.PA_ERR_INVALID),     # beyond max_pages * P
+        (dict(num_pages=3), pad.PA_ERR_INVALID),                                     # page id 3 out of range
+        (dict(kv_lens=np.array([10, 30], dtype=np.int32)), pad.PA_ERR_INVALID),     # shared page 1 partial
+        (dict(num_q_heads=12, num_kv_heads=4), pad.PA_ERR_UNSUPPORTED),              # G = 3
+        (dict(num_q_heads=8, num_kv_heads=3), pad.PA_ERR_INVALID),                   # not a multiple
+        (dict(head_dim=96), pad.PA_ERR_UNSUPPORTED),
+        (dict(page_size=32), pad.PA_ERR_UNSUPPORTED),
+    ]
+    for kw, code in cases:
+        args = dict(kv_lens=ok, block_table=bt, num_pages=4, num_q_heads=8, num_kv_heads=2, head_dim=64)
+        args.update(kw)
+        with pytest.raises(pad.PaError) as e:
+            pad.Plan(**args)
+        assert e.value.status == code, kw
+
+
+def test_plan_is_deterministic():
+    w = wl.make_config(3, with_values=False, scale=0.25)
+    a = make_plan(w).host_image()
+    b = make_plan(w).host_image()
+    assert np.array_equal(a, b)
