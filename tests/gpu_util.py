@@ -6,8 +6,9 @@ import torch
 import prefix_aware_decode_b200 as pad
 
 # Tolerances on bf16 outputs and fp32 lse against the fp64 oracle.
-MAX_ABS = 2e-3   # absolute, where |o| <= 0.5; above that the bound is the bf16
-                 # half-ulp 2^-8 |o| (rounding to bf16 alone can exceed 2e-3 there)
+MAX_ABS = 2e-3   # absolute, where |o| <= 0.256; above that the bound is one bf16 ulp,
+                 # 2^-7 |o|: the output rounding (half an ulp) plus the bf16 rounding of
+                 # p in the tensor-core p.V product (2^-9 relative per weight)
 MAX_REL = 1e-2   # |g - o| / max(|o|, rms of the (request, head) row of o)
 MAX_LSE = 1e-4
 
@@ -52,7 +53,7 @@ def compare(out: torch.Tensor, lse: torch.Tensor, ref_o: np.ndarray, ref_l: np.n
     err = np.abs(g - ref_o)
     rms = np.sqrt(np.mean(ref_o ** 2, axis=-1, keepdims=True))
     rel = err / np.maximum(np.abs(ref_o), rms)
-    abs_bound = np.maximum(MAX_ABS, np.abs(ref_o) * 1.1 * 2.0 ** -8)  # + 10% for fp32 arithmetic
+    abs_bound = np.maximum(MAX_ABS, np.abs(ref_o) * 2.0 ** -7)
     return dict(max_abs=float(err.max()), max_rel=float(rel.max()), max_lse=float(np.abs(gl - ref_l).max()),
                 abs_over_bound=float((err / abs_bound).max()),
                 finite=bool(np.isfinite(g).all() and np.isfinite(gl).all()),
