@@ -196,7 +196,7 @@ def main():
         return evs
 
     nsteps = args.warmup + args.steps
-    step_events = [mk_events(6) for _ in range(nsteps)]
+    step_events = [mk_events(2) for _ in range(nsteps)]
     plan_us = []
 
     def step(i, prof=True):
@@ -208,8 +208,7 @@ def main():
         ws = workspaces[i % 2]
         kp, vp = pools[i % copies]
         plan.upload(ws, stream)
-        plan.forward(q, kp, vp, ws, stream)
-        plan.merge(ws, out, lse, stream)
+        plan.attend(q, kp, vp, ws, out, lse, stream)
         plan.close()
 
     for i in range(args.warmup):
@@ -242,30 +241,17 @@ def main():
         ms = float(t.item())
     ms_step = ms / args.steps
 
-    # per-kernel times inside the timed region
-    def avg(a, b):
-        xs = []
-        for i in range(args.warmup, nsteps):
-            e = step_events[i]
-            xs.append(e[a].elapsed_time(e[b]))
-        return sum(xs) / len(xs)
+    # forward (both classes, merge fused) time inside the timed region, per step
+    fwd_ms = statistics.mean(step_events[i][0].elapsed_time(step_events[i][1]) for i in range(args.warmup, nsteps))
 
-    has_mma = pst["num_segments_mma"] > 0
-    simt_ms = avg(2, 3)
-    mma_ms = avg(0, 1) if has_mma else 0.0
-    merge_ms = avg(4, 5)
-    fwd_merge_ms = avg(0 if has_mma else 2, 5)
-
-    # algorithmic bytes of one CUDA-core forward launch: the KV of its (page, kv head)
-    # tiles, its q rows, and its fp32 partial rows
+    # algorithmic bytes of one forward: the KV of its (page, kv head) tiles (each
+    # node read once per query tile), the q rows, the fp32 partial rows written
+    # and read back, and the bf16 output and fp32 lse
     G = w.Hq // w.Hkv
-    probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
-    hdr = pad.PaImageHeader.from_buffer_copy(probe.host_image()[:256].tobytes())
-    probe.close()
-    simt_tiles = hdr.num_loads
     tile_bytes = 2 * 16 * w.D * 2
-    simt_bytes = simt_tiles * tile_bytes + hdr.num_segments_simt * (G * w.D * 2 + G * (w.D + 1) * 4)
-    achieved = simt_bytes / (simt_ms * 1e-3) / 1e9
+    fwd_bytes = (pst["read_kv_bytes"] + w.q.nbytes + 2 * pst["num_partial_rows"] * G * (w.D + 1) * 4
+                 + w.B * w.Hq * (w.D * 2 + 4))
+    achieved = fwd_bytes / (fwd_ms * 1e-3) / 1e9
 
     queries_per_s = w.B * world / (ms_step * 1e-3)
     line = {
@@ -279,17 +265,17 @@ def main():
                    "step": "pack (host) + upload + forward + merge", "parallelism": f"replicas x{world}"},
         "unique_kv_gbs": unique_bytes / (ms_step * 1e-3) / 1e9,
         "unique_kv_frac_of_hbm": unique_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak,
-        "device_ms": {"mma_forward": mma_ms, "simt_forward": simt_ms, "merge": merge_ms,
-                      "forward_plus_merge": fwd_merge_ms},
-        "forward_merge_queries_per_s": w.B / (fwd_merge_ms * 1e-3),
-        "forward_merge_unique_kv_frac": unique_bytes / (fwd_merge_ms * 1e-3) / 1e9 / hbm_peak,
+        "device_ms": {"forward_merge_fused": fwd_ms},
+        "forward_queries_per_s": w.B / (fwd_ms * 1e-3),
+        "forward_unique_kv_frac": unique_bytes / (fwd_ms * 1e-3) / 1e9 / hbm_peak,
         "plan_us_median": statistics.median(plan_us),
-        "plan": {k: pst[k] for k in ("num_segments_simt", "num_segments_mma", "simt_warps", "num_partial_rows",
-                                     "read_kv_bytes", "workspace_bytes", "image_bytes")},
+        "plan": {k: pst[k] for k in ("num_segments_simt", "num_segments_mma", "simt_warps", "mma_ctas",
+                                     "num_partial_rows", "read_kv_bytes", "workspace_bytes", "image_bytes")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "fwd_simt_kernel<128,4>",
+                     "frac": achieved / hbm_peak, "traffic": None,
+                     "kernel": "forward (fwd_simt_kernel<128,4> + fwd_mma_kernel<128>, merge fused)",
                      "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
-        "gpu_launches": args.steps * (3 if has_mma else 2),
+        "gpu_launches": args.steps * ((pst["mma_ctas"] > 0) + (pst["simt_warps"] > 0)),
         "clocks": clk,
     }
 

@@ -86,7 +86,8 @@ typedef struct {
   int32_t num_segments_simt;/* units on the CUDA-core class (one request, G rows) */
   int32_t num_segments_mma; /* units on the tensor-core class (two or more requests) */
   int32_t num_partial_rows; /* partial result rows per kv head group (each holds G rows) */
-  int32_t simt_warps;       /* warps of the CUDA-core forward launch */
+  int32_t simt_warps;       /* CUDA-core class warps of the forward launch */
+  int32_t mma_ctas;         /* tensor-core class CTAs of the forward launch (one per SM) */
   int64_t unique_tokens;    /* tokens of distinct tree nodes (each shared page once) */
   int64_t naive_tokens;     /* sum of kv_lens (query-centric reads) */
   int64_t read_tokens;      /* tokens the plan reads from the pools (per kv head) */
@@ -148,8 +149,10 @@ pa_status pa_forward(const pa_plan *plan, const void *q, const void *k_pool, con
 pa_status pa_merge(const pa_plan *plan, void *d_workspace, void *out, float *lse, void *stream);
 
 /*
- * pa_forward followed by pa_merge on the same stream (the whole device path of
- * one decode step).
+ * Forward with the merge fused into it (one launch): the warp that writes the
+ * last partial row of a (request, kv head) pair merges that pair into out and
+ * lse.  Same results as pa_forward + pa_merge, bit for bit.  The arrival
+ * counters it uses are left at zero, so the uploaded plan can be run again.
  */
 pa_status pa_attend(const pa_plan *plan, const void *q, const void *k_pool, const void *v_pool,
                     void *d_workspace, void *out, float *lse, void *stream);
@@ -172,13 +175,12 @@ pa_status pa_plan_get_stats(const pa_plan *plan, pa_plan_stats *out);
 pa_status pa_plan_host_image(const pa_plan *plan, void *dst, size_t bytes);
 
 /*
- * Profiling hook: up to six cudaEvent_t handles (owned by the caller) that
- * pa_forward and pa_merge record on their stream around each launch:
- *   events[0], events[1]  before / after the tensor-core (MMA) forward launch
- *   events[2], events[3]  before / after the CUDA-core (SIMT) forward launch
- *   events[4], events[5]  before / after the merge launch
- * NULL entries are skipped; n = 0 turns the hook off.  Events of a class with no
- * work are not recorded.  The events must stay valid while the plan uses them.
+ * Profiling hook: up to four cudaEvent_t handles (owned by the caller) that
+ * the device calls record on their stream around each launch:
+ *   events[0], events[1]  before / after the forward launch (pa_forward, pa_attend)
+ *   events[2], events[3]  before / after the merge launch (pa_merge)
+ * NULL entries are skipped; n = 0 turns the hook off.  The events must stay
+ * valid while the plan uses them.
  */
 pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t n);
 
@@ -198,6 +200,9 @@ const char *pa_status_string(pa_status s);
  *   pages       int32[num_page_entries]       page ids, per item
  *   queries     int32[num_query_entries]      request ids, per item
  *   seg_prows   int32[num_query_entries_mma]  partial row of each (MMA seg, query)
+ *   mma_segs    int32[mma_ctas + 1]           MMA CTA c runs MMA segs [mma_segs[c], mma_segs[c+1])
+ *                                             (indices counted from the first MMA seg)
+ *   counters    int32[B * Hkv]                arrival counters of the fused merge (zero)
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
  *   warp_loads  int32[simt_warps + 1]         SIMT warp w loads tiles [warp_loads[w], warp_loads[w+1])
  *   tiles       int32[num_loads]              page * Hkv + kv_head of every SIMT tile load, in
@@ -232,8 +237,9 @@ typedef struct {
   int32_t batch, num_q_heads, num_kv_heads, head_dim, page_size;
   int32_t num_items, num_segments, num_segments_simt, num_segments_mma, simt_warps;
   int32_t num_partial_rows, num_loads;
-  uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_warp_segs, off_warp_loads, off_tiles,
-      off_prow_off;
+  int32_t mma_ctas, pad1;
+  uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_mma_segs, off_counters, off_warp_segs,
+      off_warp_loads, off_tiles, off_prow_off;
   uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;
 } pa_image_header;
 

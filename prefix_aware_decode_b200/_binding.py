@@ -41,7 +41,7 @@ class PaPlanStats(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_nodes", ctypes.c_int32), ("num_shared_nodes", ctypes.c_int32),
                 ("num_kept_shared", ctypes.c_int32), ("num_items", ctypes.c_int32), ("num_segments", ctypes.c_int32),
                 ("num_segments_simt", ctypes.c_int32), ("num_segments_mma", ctypes.c_int32),
-                ("num_partial_rows", ctypes.c_int32), ("simt_warps", ctypes.c_int32),
+                ("num_partial_rows", ctypes.c_int32), ("simt_warps", ctypes.c_int32), ("mma_ctas", ctypes.c_int32),
                 ("unique_tokens", ctypes.c_int64), ("naive_tokens", ctypes.c_int64), ("read_tokens", ctypes.c_int64),
                 ("unique_kv_bytes", ctypes.c_int64), ("read_kv_bytes", ctypes.c_int64),
                 ("workspace_bytes", ctypes.c_uint64), ("image_bytes", ctypes.c_uint64), ("plan_us", ctypes.c_double)]
@@ -52,9 +52,10 @@ class PaImageHeader(ctypes.Structure):
                  ("fault_b", ctypes.c_int32)]
                 + [(n, ctypes.c_int32) for n in ("batch", "num_q_heads", "num_kv_heads", "head_dim", "page_size",
                                                  "num_items", "num_segments", "num_segments_simt", "num_segments_mma",
-                                                 "simt_warps", "num_partial_rows", "num_loads")]
+                                                 "simt_warps", "num_partial_rows", "num_loads", "mma_ctas", "pad1")]
                 + [(n, ctypes.c_uint64) for n in ("off_nodes", "off_segs", "off_pages", "off_queries",
-                                                  "off_seg_prows", "off_warp_segs", "off_warp_loads", "off_tiles",
+                                                  "off_seg_prows", "off_mma_segs", "off_counters", "off_warp_segs",
+                                                  "off_warp_loads", "off_tiles",
                                                   "off_prow_off", "off_partial_lse", "off_partial_o", "image_bytes",
                                                   "workspace_bytes")])
 
@@ -207,9 +208,9 @@ class Plan:
                "pa_attend")
 
     def set_profile_events(self, events):
-        """events: up to six torch.cuda.Event (or None): MMA, SIMT, merge (begin, end) pairs."""
+        """events: up to four torch.cuda.Event (or None): forward (begin, end), merge (begin, end)."""
         self._prof_events = list(events)  # keep them alive
-        arr = (ctypes.c_void_p * 6)()
+        arr = (ctypes.c_void_p * 4)()
         for i, e in enumerate(self._prof_events):
             arr[i] = None if e is None else e.cuda_event
         _check(self._lib.pa_plan_set_profile_events(self._h, arr, len(self._prof_events)),

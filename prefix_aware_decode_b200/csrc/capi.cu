@@ -21,6 +21,8 @@ PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   d.pages = reinterpret_cast<const int32_t*>(b + h.off_pages);
   d.queries = reinterpret_cast<const int32_t*>(b + h.off_queries);
   d.seg_prows = reinterpret_cast<const int32_t*>(b + h.off_seg_prows);
+  d.mma_cta_segs = reinterpret_cast<const int32_t*>(b + h.off_mma_segs);
+  d.counters = reinterpret_cast<int32_t*>(b + h.off_counters);
   d.warp_segs = reinterpret_cast<const int32_t*>(b + h.off_warp_segs);
   d.warp_loads = reinterpret_cast<const int32_t*>(b + h.off_warp_loads);
   d.tiles = reinterpret_cast<const int32_t*>(b + h.off_tiles);
@@ -62,35 +64,65 @@ bool encode_pool(const pa_plan& p, const void* pool, void* out) {
 // Pinned staging buffers for plan uploads.  A copy from pageable memory makes
 // the runtime wait for the stream first, which would serialise host planning
 // with the device work of the previous step; a copy from pinned memory does
-// not.  A slot is reused once the event recorded after its copy has completed.
+// not.  Each device has a ring of kPinSlots buffers used round-robin; before a
+// slot is reused the host waits for the event recorded after its last copy, so
+// the host can run at most kPinSlots uploads ahead of the device.
+constexpr int kPinSlots = 8;
 struct PinnedSlot {
   void* ptr = nullptr;
   size_t bytes = 0;
-  int device = -1;
   cudaEvent_t done = nullptr;
 };
+struct PinnedRing {
+  PinnedSlot slot[kPinSlots];
+  int next = 0;
+};
 std::mutex g_pin_mu;
-std::vector<PinnedSlot> g_pin;
+PinnedRing g_pin[64];
 
-// Returns a slot index whose buffer holds >= n bytes and is free, or -1.
-int pin_acquire(size_t n, int device) {
-  for (size_t i = 0; i < g_pin.size(); ++i) {
-    PinnedSlot& s = g_pin[i];
-    if (s.device != device || s.bytes < n) continue;
-    if (cudaEventQuery(s.done) == cudaSuccess) return (int)i;
+// Returns a free pinned slot of >= n bytes for the current device, or nullptr.
+PinnedSlot* pin_acquire(size_t n, int device) {
+  if (device < 0 || device >= 64) return nullptr;
+  PinnedRing& r = g_pin[device];
+  PinnedSlot& s = r.slot[r.next];
+  r.next = (r.next + 1) % kPinSlots;
+  if (s.done && cudaEventSynchronize(s.done) != cudaSuccess) return nullptr;
+  if (s.bytes < n) {
+    if (s.ptr) cudaFreeHost(s.ptr);
+    s.ptr = nullptr;
+    s.bytes = 0;
+    size_t cap = 1 << 16;
+    while (cap < n) cap <<= 1;
+    if (cudaMallocHost(&s.ptr, cap) != cudaSuccess) {
+      s.ptr = nullptr;
+      return nullptr;
+    }
+    s.bytes = cap;
   }
-  PinnedSlot s;
-  size_t cap = 1 << 16;
-  while (cap < n) cap <<= 1;
-  if (cudaMallocHost(&s.ptr, cap) != cudaSuccess) return -1;
-  if (cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess) {
-    cudaFreeHost(s.ptr);
-    return -1;
+  if (!s.done && cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+  return &s;
+}
+
+// One side stream per device for the tensor-core class, with fork/join events.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+SideStream* side_stream() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream& s = g_side[dev];
+  if (!s.stream) {
+    if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess) return nullptr;
   }
-  s.bytes = cap;
-  s.device = device;
-  g_pin.push_back(s);
-  return (int)g_pin.size() - 1;
+  return &s;
 }
 
 void record_profile(const pa_plan& p, int which, cudaStream_t st) {
@@ -107,67 +139,88 @@ extern "C" pa_status pa_plan_upload(const pa_plan* plan, void* d_workspace, size
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_pin_mu);
-  const int slot = pin_acquire(plan->image.size(), device);
-  if (slot < 0) {
+  PinnedSlot* s = pin_acquire(plan->image.size(), device);
+  if (!s) {
     // no pinned memory: a pageable copy is still correct, only slower
     cudaError_t e = cudaMemcpyAsync(d_workspace, plan->image.data(), plan->image.size(), cudaMemcpyHostToDevice, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
-  PinnedSlot& s = g_pin[slot];
-  std::memcpy(s.ptr, plan->image.data(), plan->image.size());
-  cudaError_t e = cudaMemcpyAsync(d_workspace, s.ptr, plan->image.size(), cudaMemcpyHostToDevice, st);
+  std::memcpy(s->ptr, plan->image.data(), plan->image.size());
+  cudaError_t e = cudaMemcpyAsync(d_workspace, s->ptr, plan->image.size(), cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return PA_ERR_CUDA;
-  if (cudaEventRecord(s.done, st) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaEventRecord(s->done, st) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
 
 extern "C" pa_status pa_plan_set_profile_events(pa_plan* plan, void* const* events, int32_t n) {
-  if (!plan || n < 0 || n > 6 || (n > 0 && !events)) return PA_ERR_INVALID;
-  for (int i = 0; i < 6; ++i) plan->prof[i] = i < n ? events[i] : nullptr;
+  if (!plan || n < 0 || n > 4 || (n > 0 && !events)) return PA_ERR_INVALID;
+  for (int i = 0; i < 4; ++i) plan->prof[i] = i < n ? events[i] : nullptr;
   return PA_OK;
 }
 
-extern "C" pa_status pa_forward(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
-                                void* d_workspace, void* stream) {
+namespace {
+
+pa_status launch(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool, void* d_workspace,
+                 void* out, float* lse, void* stream) {
   if (!plan || !q || !k_pool || !v_pool || !d_workspace) return PA_ERR_INVALID;
   if ((reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool) |
-       reinterpret_cast<uintptr_t>(q)) & 15)
+       reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15)
     return PA_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return PA_ERR_INVALID;
   PaDevPtrs d = dev_ptrs(*plan, d_workspace);
   d.q = static_cast<const uint16_t*>(q);
   d.k_pool = static_cast<const uint16_t*>(k_pool);
   d.v_pool = static_cast<const uint16_t*>(v_pool);
-  if (plan->hdr.num_segments_mma > 0) {
-    if (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool) {
-      if (!encode_pool(*plan, k_pool, plan->tma_k) || !encode_pool(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
-      plan->tma_k_ptr = k_pool;
-      plan->tma_v_ptr = v_pool;
-    }
-    record_profile(*plan, 0, static_cast<cudaStream_t>(stream));
-    if (pa_launch_mma(*plan, d, stream) != 0) return PA_ERR_CUDA;
-    record_profile(*plan, 1, static_cast<cudaStream_t>(stream));
+  if (plan->hdr.mma_ctas > 0 && (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool)) {
+    if (!encode_pool(*plan, k_pool, plan->tma_k) || !encode_pool(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
+    plan->tma_k_ptr = k_pool;
+    plan->tma_v_ptr = v_pool;
   }
-  record_profile(*plan, 2, static_cast<cudaStream_t>(stream));
-  if (pa_launch_simt(*plan, d, stream) != 0) return PA_ERR_CUDA;
-  record_profile(*plan, 3, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  record_profile(*plan, 0, st);
+  if (plan->hdr.mma_ctas > 0 && plan->hdr.simt_warps > 0) {
+    // multi-stream forward: the MMA class runs on a side stream concurrently
+    // with the SIMT class on the caller's stream (fork / join by events)
+    SideStream* ss = side_stream();
+    if (!ss) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(ss->mu);
+    if (cudaEventRecord(ss->fork, st) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess) return PA_ERR_CUDA;
+    if (pa_launch_forward_mma(*plan, d, out, lse, ss->stream) != 0) return PA_ERR_CUDA;
+    if (pa_launch_forward_simt(*plan, d, out, lse, st) != 0) return PA_ERR_CUDA;
+    if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return PA_ERR_CUDA;
+  } else if (plan->hdr.mma_ctas > 0) {
+    if (pa_launch_forward_mma(*plan, d, out, lse, st) != 0) return PA_ERR_CUDA;
+  } else {
+    if (pa_launch_forward_simt(*plan, d, out, lse, st) != 0) return PA_ERR_CUDA;
+  }
+  record_profile(*plan, 1, st);
   return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_forward(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
+                                void* d_workspace, void* stream) {
+  return launch(plan, q, k_pool, v_pool, d_workspace, nullptr, nullptr, stream);
 }
 
 extern "C" pa_status pa_merge(const pa_plan* plan, void* d_workspace, void* out, float* lse, void* stream) {
   if (!plan || !d_workspace || !out) return PA_ERR_INVALID;
-  if (reinterpret_cast<uintptr_t>(out) & 15) return PA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(d_workspace) & 255))
+    return PA_ERR_INVALID;
   PaDevPtrs d = dev_ptrs(*plan, d_workspace);
-  record_profile(*plan, 4, static_cast<cudaStream_t>(stream));
+  record_profile(*plan, 2, static_cast<cudaStream_t>(stream));
   const int e = pa_launch_merge(*plan, d, out, lse, stream);
-  record_profile(*plan, 5, static_cast<cudaStream_t>(stream));
+  record_profile(*plan, 3, static_cast<cudaStream_t>(stream));
   return e == 0 ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" pa_status pa_attend(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
                                void* d_workspace, void* out, float* lse, void* stream) {
-  pa_status s = pa_forward(plan, q, k_pool, v_pool, d_workspace, stream);
-  if (s != PA_OK) return s;
-  return pa_merge(plan, d_workspace, out, lse, stream);
+  if (!out) return PA_ERR_INVALID;
+  return launch(plan, q, k_pool, v_pool, d_workspace, out, lse, stream);
 }
 
 extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_workspace, void* stream,

@@ -231,24 +231,51 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
 
     // ---- split and tile selection
     // Tile class by rows (requests x G): one request -> SIMT class (CUDA
-    // cores); two or more -> MMA class (tensor cores, query tiles of <= 64 rows).
-    // SIMT: stream-K split.  The (item, kv head) page runs are concatenated and
-    // cut into equal spans of `span` pages, one span per warp; a span may end
-    // inside an item, so every warp gets the same number of pages and partial
-    // rows appear only at span boundaries.
-    // MMA: each (item, kv head) is cut into chunks of `chunk` tokens, one CTA
-    // per chunk, launched longest first.
+    // cores); two or more -> MMA class (tensor cores, query tiles of <= 128 rows).
+    // The two classes run as two concurrent launches of one CTA per SM each; k
+    // SMs take the MMA class, the rest the SIMT class.  k balances the two
+    // classes' estimated times:
+    //   T_simt(k) = SIMT tile bytes / ((num_sms - k) * kSimtBytesPerSmUs)
+    //   T_mma(k)  = sum over MMA tiles of max(bytes / kMmaBytesPerSmUs,
+    //               flops / kMmaFlopsPerSmUs) / k
+    // Both classes split their work stream-K: the (item, kv head) page runs are
+    // concatenated and cut into equal spans, one span per SIMT warp or per MMA
+    // CTA; a span may end inside an item, so partial rows appear only at span
+    // boundaries (long-KV splitting without a fixed chunk size).
+    const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
+    const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
+    const double kMmaFlopsPerSmUs = 0.7e6;     // flop per us per SM, mma.sync with 8 warps (measured)
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
-    int64_t simt_pages = 0, mma_tile_tokens = 0;
+    const double tile_bytes = 2.0 * 16 * D * 2;
+    int64_t simt_pages = 0, mma_pages = 0;
+    double mma_cost = 0;  // SM-us
     for (const auto& it : items) {
-      if (it.simt) simt_pages += ceil_div(it.n_tokens, P) * Hkv;
-      else mma_tile_tokens += (int64_t)it.n_tokens * Hkv;
+      const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
+      if (it.simt) {
+        simt_pages += np;
+      } else {
+        mma_pages += np;
+        const double rows = 16.0 * ceil_div((int64_t)it.n_queries * G, 16);
+        const double flops = 16.0 * rows * D * 4;
+        mma_cost += np * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
+      }
+    }
+    const int S = plan->num_sms;
+    int n_mma = 0;  // SMs given to the MMA class
+    if (mma_pages > 0 && simt_pages == 0) {
+      n_mma = S;
+    } else if (mma_pages > 0) {
+      double best = 1e300;
+      for (int kk = 1; kk < S; ++kk) {
+        const double t = std::max(simt_pages * tile_bytes / ((S - kk) * kSimtBytesPerSmUs), mma_cost / kk);
+        if (t < best) { best = t; n_mma = kk; }
+      }
     }
     std::vector<SegRec> simt_segs, mma_segs;
-    std::vector<int32_t> warp_segs{0}, warp_loads{0};
+    std::vector<int32_t> warp_segs{0}, warp_loads{0}, mma_cta_segs{0};
     std::vector<int32_t> tiles((size_t)simt_pages);
     if (simt_pages > 0) {
-      const int64_t W = (int64_t)plan->num_sms * kSimtWarpsPerCta;
+      const int64_t W = (int64_t)(S - n_mma) * kSimtWarpsPerCta;
       int64_t span = ceil_div(simt_pages, W);
       if (span < 4) span = 4;
       if (max_chunk_pages) span = std::min(span, max_chunk_pages);
@@ -284,24 +311,31 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
         warp_loads.push_back((int32_t)t);
       }
     }
-    if (mma_tile_tokens > 0) {
-      const int64_t target = (int64_t)plan->num_sms * 4;
-      int64_t chunk = ceil_div(ceil_div(mma_tile_tokens, target), P) * P;
-      chunk = std::max<int64_t>(512, std::min<int64_t>(8192, chunk));
-      if (max_chunk_pages) chunk = std::min<int64_t>(chunk, max_chunk_pages * P);
+    if (mma_pages > 0) {
+      int64_t span = ceil_div(mma_pages, n_mma);
+      if (span < 16) span = 16;
+      if (max_chunk_pages) span = std::min(span, max_chunk_pages);
+      int64_t used = 0;
       for (size_t i = 0; i < items.size(); ++i) {
         const ItemRec& it = items[i];
         if (it.simt) continue;
         const int npages = (int)ceil_div(it.n_tokens, P);
-        const int cp = (int)(chunk / P);
-        for (int pb = 0; pb < npages; pb += cp) {
-          const int pe = std::min(npages, pb + cp);
-          const int tok = std::min(it.n_tokens, pe * P) - pb * P;
-          for (int g = 0; g < Hkv; ++g) mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
+        for (int g = 0; g < Hkv; ++g) {
+          int pb = 0;
+          while (pb < npages) {
+            const int take = (int)std::min<int64_t>(npages - pb, span - used);
+            const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
+            mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
+            pb += take;
+            used += take;
+            if (used == span) {
+              mma_cta_segs.push_back((int32_t)mma_segs.size());
+              used = 0;
+            }
+          }
         }
       }
-      std::stable_sort(mma_segs.begin(), mma_segs.end(),
-                       [](const SegRec& a, const SegRec& b) { return a.n_tokens > b.n_tokens; });
+      if (used > 0) mma_cta_segs.push_back((int32_t)mma_segs.size());
     }
 
     // ---- partial rows: contiguous per (request, kv head), in a fixed order
@@ -337,6 +371,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.num_segments_mma = (int32_t)mma_segs.size();
     h.num_segments = h.num_segments_simt + h.num_segments_mma;
     h.simt_warps = (int32_t)warp_segs.size() - 1;
+    h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
     h.num_partial_rows = num_prows;
     h.num_loads = (int32_t)tiles.size();
     uint64_t off = align256(sizeof(pa_image_header));
@@ -345,6 +380,8 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.off_pages = off; off = align256(off + pages.size() * 4);
     h.off_queries = off; off = align256(off + queries.size() * 4);
     h.off_seg_prows = off; off = align256(off + seg_prows.size() * 4);
+    h.off_mma_segs = off; off = align256(off + mma_cta_segs.size() * 4);
+    h.off_counters = off; off = align256(off + (size_t)batch * Hkv * 4);
     h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
     h.off_warp_loads = off; off = align256(off + warp_loads.size() * 4);
     h.off_tiles = off; off = align256(off + tiles.size() * 4);
@@ -354,7 +391,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
     h.workspace_bytes = off;
 
-    plan->image.resize(h.image_bytes);
+    plan->image.assign(h.image_bytes, 0);
     uint8_t* img = plan->image.data();
     std::memcpy(img, &h, sizeof(h));
     pa_item* di = reinterpret_cast<pa_item*>(img + h.off_nodes);
@@ -370,6 +407,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     put(h.off_pages, pages);
     put(h.off_queries, queries);
     put(h.off_seg_prows, seg_prows);
+    put(h.off_mma_segs, mma_cta_segs);
     put(h.off_warp_segs, warp_segs);
     put(h.off_warp_loads, warp_loads);
     put(h.off_tiles, tiles);
@@ -386,6 +424,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     st.num_segments_mma = h.num_segments_mma;
     st.num_partial_rows = num_prows;
     st.simt_warps = h.simt_warps;
+    st.mma_ctas = h.mma_ctas;
     st.unique_tokens = pl.unique_tokens;
     int64_t naive = 0;
     for (int b = 0; b < batch; ++b) naive += kv_lens[b];

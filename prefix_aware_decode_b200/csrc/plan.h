@@ -9,10 +9,11 @@
 static_assert(sizeof(pa_seg) == 32, "pa_seg must be 32 bytes (vector loads)");
 static_assert(sizeof(pa_item) == 16, "pa_item must be 16 bytes");
 
-// Warps of the CUDA-core (SIMT) forward class per CTA, and the shape of the
-// tensor-core (MMA) class: 4 consumer warps x 16 rows.
+// Forward launch shapes, one CTA per SM for both classes.  A CUDA-core (SIMT)
+// CTA runs 8 independent warps; a tensor-core (MMA) CTA runs 8 consumer warps
+// of 16 rows each (128 rows) and one producer warp.
 constexpr int kSimtWarpsPerCta = 8;
-constexpr int kMmaRowsPerCta = 64;
+constexpr int kMmaRowsPerCta = 128;
 
 struct pa_plan {
   pa_config cfg;
@@ -31,8 +32,8 @@ struct pa_plan {
   alignas(64) mutable uint8_t tma_k[128] = {};
   alignas(64) mutable uint8_t tma_v[128] = {};
   // optional cudaEvent_t handles recorded around the launches (profiling):
-  // [0,1] tensor-core forward, [2,3] CUDA-core forward, [4,5] merge
-  void* prof[6] = {};
+  // [0,1] forward launch (pa_forward / pa_attend), [2,3] merge launch
+  void* prof[4] = {};
 };
 
 // Kernel launchers (kernels.cu).  Return 0 or a cudaError_t value.
@@ -46,6 +47,8 @@ struct PaDevPtrs {
   const int32_t* pages;
   const int32_t* queries;
   const int32_t* seg_prows;
+  const int32_t* mma_cta_segs;
+  int32_t* counters;
   const int32_t* warp_segs;
   const int32_t* warp_loads;
   const int32_t* tiles;
@@ -55,6 +58,9 @@ struct PaDevPtrs {
   int32_t* status;
 };
 
-int pa_launch_simt(const pa_plan& p, const PaDevPtrs& d, void* stream);
-int pa_launch_mma(const pa_plan& p, const PaDevPtrs& d, void* stream);
+// out == nullptr: partial rows only; else the merge is fused into the launches.
+// The two classes run as two kernels; `side` is a second stream that the
+// caller has made wait for `stream` (the MMA kernel goes there).
+int pa_launch_forward_mma(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* side);
+int pa_launch_forward_simt(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);

@@ -31,7 +31,9 @@ class Image:
         n_pages = (h.off_queries - h.off_pages) // 4
         self.pages = arr(h.off_pages, n_pages)
         self.queries = arr(h.off_queries, (h.off_seg_prows - h.off_queries) // 4)
-        self.seg_prows = arr(h.off_seg_prows, (h.off_warp_segs - h.off_seg_prows) // 4)
+        self.seg_prows = arr(h.off_seg_prows, (h.off_mma_segs - h.off_seg_prows) // 4)
+        self.mma_segs = arr(h.off_mma_segs, h.mma_ctas + 1)
+        self.counters = arr(h.off_counters, h.batch * h.num_kv_heads)
         self.warp_segs = arr(h.off_warp_segs, h.simt_warps + 1)
         self.warp_loads = arr(h.off_warp_loads, h.simt_warps + 1)
         self.tiles = arr(h.off_tiles, h.num_loads)
@@ -42,9 +44,16 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
     h = img.h
     B, Hkv, G = h.batch, h.num_kv_heads, h.num_q_heads // h.num_kv_heads
     nseg_simt = h.num_segments_simt
+    # MMA CTA lists partition the MMA segments; arrival counters start at zero
+    if h.num_segments_mma:
+        assert img.mma_segs[0] == 0 and img.mma_segs[-1] == h.num_segments_mma
+        assert np.all(np.diff(img.mma_segs) > 0)
+    else:
+        assert h.mma_ctas == 0
+    assert np.all(img.counters == 0)
     # warp lists partition the SIMT segments and tiles, in order
     assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
-    assert np.all(np.diff(img.warp_segs) > 0)
+    assert np.all(np.diff(img.warp_segs) > 0) or nseg_simt == 0
     assert img.warp_loads[0] == 0 and img.warp_loads[-1] == h.num_loads
     # the tile list equals the pages of the SIMT segments, in order
     t = 0

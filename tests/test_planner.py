@@ -43,8 +43,9 @@ def test_config2_tree_and_classes():
     w = wl.make_config(2, with_values=False)
     st = make_plan(w).stats()
     assert st["num_nodes"] == 65 and st["num_shared_nodes"] == 1 and st["num_kept_shared"] == 1
-    # 256 rows of the shared root -> 4 query tiles of 64 rows on the tensor-core class
-    assert st["num_items"] == 64 + 4
+    # 256 rows of the shared root -> 2 query tiles of 128 rows on the tensor-core class
+    assert st["num_items"] == 64 + 2
+    assert 0 < st["mma_ctas"] < 148 and st["simt_warps"] <= (148 - st["mma_ctas"]) * 8
     assert st["num_segments_mma"] > 0 and st["num_segments_simt"] > 0
 
 
