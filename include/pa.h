@@ -226,7 +226,8 @@ typedef struct {
   int32_t n_tokens;   /* valid tokens of the run (its pages are ceil(n_tokens / P)) */
   int32_t prow;       /* SIMT: the partial row written; MMA: index into seg_prows */
   int32_t query;      /* SIMT: the request; MMA: first request of the item */
-  int32_t pad0, pad1; /* 32-byte records */
+  int32_t sole;       /* SIMT: 1 if this is the only partial row of (query, kv_head) */
+  int32_t pad;        /* 32-byte records */
 } pa_seg;
 
 typedef struct {

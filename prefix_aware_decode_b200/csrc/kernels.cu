@@ -6,10 +6,10 @@
 // tile selector; multi-stream execution; long KV is split).  Two tile classes,
 // chosen by the planner from the rows of each work unit (requests x G query
 // heads), run as two concurrent launches of one persistent CTA per SM:
-//   - MMA class: work units with two or more requests, up to 128 rows.  A
-//     producer warp streams 64-key stages with 2-D TMA copies (128-byte
-//     swizzle); 8 consumer warps each run bf16 mma.sync with fp32 accumulation
-//     on 16 rows.
+//   - MMA class: work units with two or more requests, up to 128 rows, on the
+//     5th-generation tensor cores: a producer warp streams 64-key stages with
+//     2-D TMA copies (128-byte swizzle), one thread issues tcgen05.mma with the
+//     accumulators in tensor memory, and 4 warps run the softmax.
 //   - SIMT class: work units of one request (G <= 8 rows).  Each of 8 warps
 //     streams its own run of (page, kv head) tiles with 1-D bulk copies into a
 //     private shared-memory ring and computes on the CUDA cores with packed
@@ -66,65 +66,78 @@ struct FwdArgs {
 // ---------------------------------------------------------------- merge of one (request, kv head)
 
 // One warp merges the partial rows of (b, g) into out[b][g*G .. g*G+G-1][:] and
-// lse[b][...].  Partial rows are read through L2 (they may have been written by
+// lse[b][...], in one online pass: lane l handles row l / (32/G) and a run of
+// D*G/32 head dims, so every load of the loop is independent of the running
+// state.  Partial rows are read through L2 (they may have been written by
 // other SMs in the same launch).
-template <int D>
+template <int D, int G>
 __device__ __forceinline__ void merge_pair(const int32_t* prow_off, const float* partial_lse, const float* partial_o,
-                                           __nv_bfloat16* out, float* lse, int Hq, int Hkv, int G, int b, int g,
-                                           int lane) {
-  constexpr int VD = D / 32;
+                                           __nv_bfloat16* out, float* lse, int Hq, int Hkv, int b, int g, int lane) {
+  constexpr int LPR = 32 / G;   // lanes per row
+  constexpr int VPL = D / LPR;  // head dims per lane
+  const int r = lane / LPR, d0 = (lane % LPR) * VPL;
   const int p0 = prow_off[b * Hkv + g], p1 = prow_off[b * Hkv + g + 1];
-  for (int r = 0; r < G; ++r) {
-    float mx = -INFINITY;
-    for (int p = p0; p < p1; ++p) mx = fmaxf(mx, __ldcg(partial_lse + (size_t)p * G + r));
-    float z = 0.f;
-    for (int p = p0; p < p1; ++p) z += expf(__ldcg(partial_lse + (size_t)p * G + r) - mx);
-    const float L = mx + logf(z);
-    float acc[VD];
+  float m = -INFINITY, z = 0.f, acc[VPL];
 #pragma unroll
-    for (int i = 0; i < VD; ++i) acc[i] = 0.f;
-    for (int p = p0; p < p1; ++p) {
-      const float wgt = expf(__ldcg(partial_lse + (size_t)p * G + r) - L);
-      const float* src = partial_o + ((size_t)p * G + r) * D + lane * VD;
-      if constexpr (VD == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-        acc[0] += wgt * v.x;
-        acc[1] += wgt * v.y;
-        acc[2] += wgt * v.z;
-        acc[3] += wgt * v.w;
-      } else {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
-        acc[0] += wgt * v.x;
-        acc[1] += wgt * v.y;
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+#pragma unroll 2
+  for (int p = p0; p < p1; ++p) {
+    const float lp = __ldcg(partial_lse + (size_t)p * G + r);
+    float o[VPL];
+    const float* src = partial_o + ((size_t)p * G + r) * D + d0;
+    if constexpr (VPL % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < VPL / 4; ++i) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + i);
+        o[4 * i] = v.x;
+        o[4 * i + 1] = v.y;
+        o[4 * i + 2] = v.z;
+        o[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL / 2; ++i) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(src) + i);
+        o[2 * i] = v.x;
+        o[2 * i + 1] = v.y;
       }
     }
-    const int h = g * G + r;
-    __nv_bfloat16* dst = out + ((size_t)b * Hq + h) * D + lane * VD;
+    const float mn = fmaxf(m, lp);
+    const float sa = m == -INFINITY ? 0.f : expf(m - mn), sb = expf(lp - mn);
+    z = z * sa + sb;
 #pragma unroll
-    for (int i = 0; i < VD; i += 2)
-      *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i], acc[i + 1]);
-    if (lse && lane == 0) lse[(size_t)b * Hq + h] = L;
+    for (int i = 0; i < VPL; ++i) acc[i] = acc[i] * sa + o[i] * sb;
+    m = mn;
   }
+  const float inv = 1.f / z;
+  __nv_bfloat16* dst = out + ((size_t)b * Hq + g * G + r) * D + d0;
+#pragma unroll
+  for (int i = 0; i < VPL; i += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+  if (lse && lane % LPR == 0) lse[(size_t)b * Hq + g * G + r] = m + logf(z);
 }
 
-// Called by a whole warp after it wrote partial rows of (b, g): counts the
-// arrival and merges the pair if this was the last of its partial rows.
-template <int D>
-__device__ __forceinline__ void arrive_and_merge(const FwdArgs& a, int b, int g, int lane) {
+// Called by a whole warp after it wrote partial rows of up to 32 (request, kv
+// head g) pairs, lane j holding request bj for j < n: counts the arrivals (in
+// parallel) and merges every pair for which this was the last partial row.
+template <int D, int G>
+__device__ __forceinline__ void arrive_and_merge(const FwdArgs& a, int bj, int n, int g, int lane) {
   __threadfence();
   __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    const int bg = b * a.Hkv + g;
-    const int n = a.prow_off[bg + 1] - a.prow_off[bg];
-    last = atomicAdd(&a.counters[bg], 1) == n - 1;
+  bool last = false;
+  if (lane < n) {
+    const int bg = bj * a.Hkv + g;
+    last = atomicAdd(&a.counters[bg], 1) == a.prow_off[bg + 1] - a.prow_off[bg] - 1;
   }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (last) {
-    __threadfence();
-    merge_pair<D>(a.prow_off, a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, a.Hkv, a.G, b, g, lane);
-    __syncwarp();
-    if (lane == 0) a.counters[b * a.Hkv + g] = 0;  // ready for the next launch
+  unsigned todo = __ballot_sync(0xffffffffu, last);
+  if (!todo) return;
+  __threadfence();
+  while (todo) {
+    const int j = __ffs(todo) - 1;
+    todo &= todo - 1;
+    const int b = __shfl_sync(0xffffffffu, bj, j);
+    merge_pair<D, G>(a.prow_off, a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, a.Hkv, b, g, lane);
+    if (lane == j) a.counters[b * a.Hkv + g] = 0;  // ready for the next launch
   }
 }
 
@@ -151,17 +164,19 @@ struct SimtShape {
 
 struct SegInfo {
   int n_tokens, prow, query, kv_head;
+  bool sole;
 };
 
 __device__ __forceinline__ SegInfo load_seg(const pa_seg* segs, int i, int end) {
-  SegInfo r{0, 0, 0, 0};
+  SegInfo r{0, 0, 0, 0, false};
   if (i < end) {
     const int4 x = *reinterpret_cast<const int4*>(segs + i);        // item, kv_head, page_begin, n_tokens
-    const int2 y = *reinterpret_cast<const int2*>(&segs[i].prow);  // prow, query
+    const int4 y = *reinterpret_cast<const int4*>(&segs[i].prow);  // prow, query, sole, pad
     r.n_tokens = x.w;
     r.kv_head = x.y;
     r.prow = y.x;
     r.query = y.y;
+    r.sole = y.z != 0;
   }
   return r;
 }
@@ -425,21 +440,38 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
           }
       }
     }
-    // write: group k writes rows r with r % NG == k
+    // write: group k writes rows r with r % NG == k; a (request, kv head) with a
+    // single partial row goes straight to the output when the merge is fused
+    const bool direct = a.out && cur.sole;
 #pragma unroll
     for (int r = 0; r < G; ++r) {
       if (r % S::NG != grp) continue;
       const float inv = 1.f / l[r];
-      float* dst = a.partial_o + ((size_t)cur.prow * G + r) * D;
+      const float lse_r = (m[r] + lg2(l[r])) * kLn2;
+      if (direct) {
+        __nv_bfloat16* dst = a.out + ((size_t)cur.query * a.Hq + cur.kv_head * G + r) * D;
 #pragma unroll
-      for (int j = 0; j < CPL; ++j) {
-        float4* d4 = reinterpret_cast<float4*>(dst + (li + LPG * j) * 8);
-        d4[0] = make_float4(o[r][j][0].x * inv, o[r][j][0].y * inv, o[r][j][1].x * inv, o[r][j][1].y * inv);
-        d4[1] = make_float4(o[r][j][2].x * inv, o[r][j][2].y * inv, o[r][j][3].x * inv, o[r][j][3].y * inv);
+        for (int j = 0; j < CPL; ++j) {
+          uint4 w;
+          w.x = pack_bf16x2(o[r][j][0].x * inv, o[r][j][0].y * inv);
+          w.y = pack_bf16x2(o[r][j][1].x * inv, o[r][j][1].y * inv);
+          w.z = pack_bf16x2(o[r][j][2].x * inv, o[r][j][2].y * inv);
+          w.w = pack_bf16x2(o[r][j][3].x * inv, o[r][j][3].y * inv);
+          *reinterpret_cast<uint4*>(dst + (li + LPG * j) * 8) = w;
+        }
+        if (li == 0 && a.lse) a.lse[(size_t)cur.query * a.Hq + cur.kv_head * G + r] = lse_r;
+      } else {
+        float* dst = a.partial_o + ((size_t)cur.prow * G + r) * D;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+          float4* d4 = reinterpret_cast<float4*>(dst + (li + LPG * j) * 8);
+          d4[0] = make_float4(o[r][j][0].x * inv, o[r][j][0].y * inv, o[r][j][1].x * inv, o[r][j][1].y * inv);
+          d4[1] = make_float4(o[r][j][2].x * inv, o[r][j][2].y * inv, o[r][j][3].x * inv, o[r][j][3].y * inv);
+        }
+        if (li == 0) a.partial_lse[(size_t)cur.prow * G + r] = lse_r;
       }
-      if (li == 0) a.partial_lse[(size_t)cur.prow * G + r] = (m[r] + lg2(l[r])) * kLn2;
     }
-    if (a.out) arrive_and_merge<D>(a, cur.query, cur.kv_head, lane);
+    if (a.out && !direct) arrive_and_merge<D, G>(a, cur.query, 1, cur.kv_head, lane);
     cur = nx;
     nx = nxx;
     nxx = load_seg(a.segs, si + 3, seg_end);
@@ -451,56 +483,94 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   }
 }
 
-// ---------------------------------------------------------------- MMA class
+// ---------------------------------------------------------------- MMA class (tcgen05 + TMEM)
+//
+// One CTA per SM runs a list of segments (item of <= 128 rows, kv head g, key
+// range).  Warp 0: TMA producer of 64-key K/V stages.  Warp 1: TMEM owner and
+// single-thread tcgen05.mma issuer.  Warps 2-5: softmax, one tile row (TMEM
+// lane) per thread.  Per 64-key stage i:
+//   S(i) = Q K^T          -> TMEM (double-buffered, 64 columns each)
+//   p = exp2(s - m)       -> P = P_hi + P_lo, two bf16 matrices in swizzled
+//                            shared memory (P_lo = bf16(p - P_hi), so P keeps
+//                            about 16 significant bits instead of 8)
+//   O += P_hi V + P_lo V  -> TMEM (D columns)
+// S(i+1) is issued before P(i) is ready, so the tensor core overlaps the
+// softmax.  The running maximum is only raised (and O rescaled in TMEM) when a
+// row's maximum grows by more than 2^8; the final normalisation uses the same
+// maximum for numerator and denominator, so the result is unchanged.
 
-constexpr int kMmaKT = 64;  // keys per stage (4 pages)
-constexpr int kMmaNST = 4;  // stages
-constexpr int kMmaConsumers = kMmaRowsPerCta / 16;
-constexpr int kMmaThreads = (kMmaConsumers + 1) * 32;  // + producer warp
+constexpr int kMmaKT = 64;          // keys per stage (4 pages)
+constexpr int kMmaNST = 4;          // K/V stages in flight
+constexpr int kMmaThreads = 192;    // 6 warps
+constexpr uint32_t kTmemCols = 256; // S x 2 (64 columns each) + O (<= 128 columns)
+constexpr float kRescaleThreshold = 8.f;  // log2 units
 
 template <int D>
 struct MmaShape {
   static constexpr int HALVES = D / 64;
-  static constexpr int KBYTES = HALVES * kMmaKT * 128;  // one operand of one stage
-  static constexpr int STAGE = 2 * KBYTES;
-  static constexpr int SMEM = kMmaNST * STAGE + 2 * kMmaNST * 8 + 1024;  // + alignment slack
+  static constexpr int KBLK = kMmaKT * 128;        // one 64-key x 64-dim swizzled block (8 KB)
+  static constexpr int STAGE = 2 * HALVES * KBLK;  // K and V of one stage
+  static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
+  static constexpr int OFF_Q = kMmaNST * STAGE;
+  static constexpr int OFF_P = OFF_Q + HALVES * QBLK;  // P_hi, then P_lo at + PBLK
+  static constexpr int PBLK = 128 * 128;
+  static constexpr int OFF_BAR = OFF_P + 2 * PBLK;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
   static_assert(SMEM <= kSmemMax, "MMA ring does not fit");
 };
 
-// byte offset of (row, 16-byte chunk) in a 128-byte-swizzled [rows][64] bf16 block
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+enum : int { kBarFull = 0, kBarEmpty = 4, kBarSFull = 8, kBarSFree = 10, kBarPFull = 12, kBarOFull = 13,
+             kBarQFull = 14, kBarOFree = 15, kBarDone = 16, kNumBars = 17 };
+
+// All lanes wait; the warp fails together if any lane timed out.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  const bool ok = mbar_wait_bounded(bar, parity, timeout_ns);
+  return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
+template <int D, int G>
 __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
                                          uint8_t* smem_raw) {
   using S = MmaShape<D>;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kMmaNST * S::STAGE);
-  uint64_t* empty = full + kMmaNST;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = a.G;
   const int s_begin = a.n_segs_simt + a.mma_cta_segs[blockIdx.x];
   const int s_end = a.n_segs_simt + a.mma_cta_segs[blockIdx.x + 1];
+  const uint32_t q_base = smem_u32(smem + S::OFF_Q), p_base = smem_u32(smem + S::OFF_P);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMmaNST; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), kMmaConsumers);
+      mbar_init(bar(kBarFull + s), 1);
+      mbar_init(bar(kBarEmpty + s), 1);
     }
+    mbar_init(bar(kBarSFull), 1);
+    mbar_init(bar(kBarSFull + 1), 1);
+    mbar_init(bar(kBarSFree), 128);
+    mbar_init(bar(kBarSFree + 1), 128);
+    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarQFull), 128);
+    mbar_init(bar(kBarOFree), 128);
+    mbar_init(bar(kBarDone), 1);
     fence_mbar_init();
   }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem + 128;
 
-  if (warp == kMmaConsumers) {
-    // ---------------- producer: every stage of every segment of this CTA, in order
+  if (warp == 0) {
+    // ---------------- TMA producer: every stage of every segment of this CTA, in order
     if (lane == 0) {
       prefetch_tmap(tk);
       prefetch_tmap(tv);
-      uint32_t lastpar = 0;  // bit s: parity of the last phase loaded on stage s
-      uint32_t any = 0;      // bit s: stage s has been loaded at least once
-      int i = 0;             // stages issued so far
+      uint32_t lastpar = 0, any = 0;
+      int i = 0;
       bool ok = true;
       for (int si = s_begin; si < s_end && ok; ++si) {
         const pa_seg seg = a.segs[si];
@@ -508,197 +578,240 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         const int npages = (seg.n_tokens + 15) >> 4;
         for (int st = 0; st < npages; st += 4, ++i) {
           const int s = i % kMmaNST;
-          if (i >= kMmaNST && !mbar_wait_bounded(smem_u32(&empty[s]), ((i / kMmaNST) - 1) & 1, a.timeout_ns)) {
+          if (i >= kMmaNST && !mbar_wait_bounded(bar(kBarEmpty + s), ((i / kMmaNST) - 1) & 1, a.timeout_ns)) {
             record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -2);
             ok = false;
             break;
           }
-          const int np = min(4, npages - st);
-          const uint32_t fb = smem_u32(&full[s]);
           if (a.fault_drop && blockIdx.x == 0 && i == 0) continue;  // test: this stage never arrives
+          const int np = min(4, npages - st);
+          const uint32_t fb = bar(kBarFull + s);
           mbar_arrive_expect_tx(fb, (uint32_t)np * 2 * 16 * D * 2);
           uint8_t* kst = smem + s * S::STAGE;
-          uint8_t* vst = kst + S::KBYTES;
+          uint8_t* vst = kst + S::HALVES * S::KBLK;
           for (int pp = 0; pp < np; ++pp) {
             const int row = (a.pages[page_base + st + pp] * a.Hkv + seg.kv_head) * 16;
 #pragma unroll
             for (int h = 0; h < S::HALVES; ++h) {
-              tma_load_2d(smem_u32(kst + h * kMmaKT * 128 + pp * 2048), tk, 64 * h, row, fb);
-              tma_load_2d(smem_u32(vst + h * kMmaKT * 128 + pp * 2048), tv, 64 * h, row, fb);
+              tma_load_2d(smem_u32(kst + h * S::KBLK + pp * 2048), tk, 64 * h, row, fb);
+              tma_load_2d(smem_u32(vst + h * S::KBLK + pp * 2048), tv, 64 * h, row, fb);
             }
           }
           lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / kMmaNST) & 1) << s);
           any |= 1u << s;
         }
       }
-      // drain: the last load of every stage used must have landed before exit
       for (int s = 0; s < kMmaNST; ++s)
-        if (any & (1u << s)) mbar_wait_bounded(smem_u32(&full[s]), (lastpar >> s) & 1u, a.timeout_ns);
+        if (any & (1u << s)) mbar_wait_bounded(bar(kBarFull + s), (lastpar >> s) & 1u, a.timeout_ns);
     }
-    return;
-  }
-
-  // ---------------- consumers: warp w owns rows 16w .. 16w+15 of each segment
-  const int t4 = lane >> 2, c4 = lane & 3;
-  const int mi = lane >> 3, rr = lane & 7;
-  constexpr int KS = D / 16;  // k-steps over the head dim
-  int i = 0;                  // stages consumed so far
-  for (int si = s_begin; si < s_end; ++si) {
-    const pa_seg seg = a.segs[si];
-    const pa_item item = a.items[seg.item];
-    const int g = seg.kv_head;
-    const int npages = (seg.n_tokens + 15) >> 4;
-    const int R = item.n_queries * G;
-    const bool active = warp * 16 < R;
-    const int r0 = warp * 16 + t4, r1 = r0 + 8;
-    uint32_t qa[KS][4];
-    if (active) {
-      auto qrow = [&](int r) -> const uint16_t* {
-        if (r >= R) return nullptr;
-        const int b = a.queries[item.query_off + r / G];
-        return a.q + ((size_t)b * a.Hq + g * G + (r % G)) * D;
+  } else if (warp == 1) {
+    // ---------------- tcgen05.mma issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc_bf16(128, kMmaKT, false, false);
+      constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, false, true);
+      struct Prev { int s, np, segord; bool first; };
+      Prev prev{0, 0, 0, false};
+      bool have_prev = false, ok = true;
+      int i = 0, segord = 0;
+      auto do_pv = [&](const Prev& pv, int j) -> bool {
+        if (!mbar_wait_bounded(bar(kBarPFull), j & 1, a.timeout_ns)) return false;
+        if (pv.first && pv.segord >= 1 && !mbar_wait_bounded(bar(kBarOFree), (pv.segord - 1) & 1, a.timeout_ns))
+          return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(smem + pv.s * S::STAGE + S::HALVES * S::KBLK);
+        for (int kk = 0; kk < pv.np; ++kk) {
+          // P: K-major, 64 keys = one 128-byte swizzle atom per row; V: MN-major
+          // (64-dim atoms at +KBLK, 8-key groups at +1 KB), 16 keys per MMA
+          const uint64_t bd = umma_sdesc_sw128(v_base + kk * 2048, S::KBLK >> 4, 64);
+          umma_bf16(tO, umma_sdesc_sw128(p_base + kk * 32, 1, 64), bd, idesc_o, (pv.first && kk == 0) ? 0u : 1u);
+          umma_bf16(tO, umma_sdesc_sw128(p_base + S::PBLK + kk * 32, 1, 64), bd, idesc_o, 1u);
+        }
+        umma_commit(bar(kBarOFull));
+        umma_commit(bar(kBarEmpty + pv.s));
+        return true;
       };
-      const uint16_t* q0 = qrow(r0);
-      const uint16_t* q1 = qrow(r1);
+      for (int si = s_begin; si < s_end && ok; ++si) {
+        const int npages = (a.segs[si].n_tokens + 15) >> 4;
+        for (int st = 0; st < npages; st += 4, ++i) {
+          const int s = i % kMmaNST;
+          const bool first = st == 0;
+          if (!mbar_wait_bounded(bar(kBarFull + s), (i / kMmaNST) & 1, a.timeout_ns) ||
+              (first && !mbar_wait_bounded(bar(kBarQFull), segord & 1, a.timeout_ns)) ||
+              (i >= 2 && !mbar_wait_bounded(bar(kBarSFree + (i & 1)), ((i >> 1) - 1) & 1, a.timeout_ns))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(smem + s * S::STAGE);
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        const int d0 = kk * 16 + 2 * c4;
-        qa[kk][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + d0) : 0u;
-        qa[kk][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + d0) : 0u;
-        qa[kk][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + d0 + 8) : 0u;
-        qa[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + d0 + 8) : 0u;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // Q and K: K-major 128-byte swizzle, 64-dim blocks, 8-row groups at +1 KB
+            const uint64_t ad = umma_sdesc_sw128(q_base + (kk >> 2) * S::QBLK + (kk & 3) * 32, 1, 64);
+            const uint64_t bd = umma_sdesc_sw128(k_base + (kk >> 2) * S::KBLK + (kk & 3) * 32, 1, 64);
+            umma_bf16(tmem + (i & 1) * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(kBarSFull + (i & 1)));
+          if (have_prev && !do_pv(prev, i - 1)) {
+            ok = false;
+            break;
+          }
+          prev = Prev{s, min(4, npages - st), segord, first};
+          have_prev = true;
+        }
+        ++segord;
       }
+      if (ok && have_prev) ok = do_pv(prev, i - 1);
+      if (!ok) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -3);
+      // every MMA issued by this thread has completed before TMEM is released
+      umma_commit(bar(kBarDone));
+      mbar_wait_bounded(bar(kBarDone), 0, a.timeout_ns);
     }
-    float oacc[D / 8][4];
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-    for (int st = 0; st < npages; st += 4, ++i) {
-      const int s = i % kMmaNST;
-      if (!mbar_wait_bounded(smem_u32(&full[s]), (i / kMmaNST) & 1, a.timeout_ns)) {
-        if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, warp);
-        return;
+  } else {
+    // ---------------- softmax: thread = tile row = TMEM lane
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    bool ok = true;
+    int i = 0, segord = 0;
+    auto load_q = [&](int si) {
+      const pa_seg seg = a.segs[si];
+      const pa_item item = a.items[seg.item];
+      const int R = item.n_queries * G;
+      const uint16_t* src = nullptr;
+      if (r < R) {
+        const int b = a.queries[item.query_off + r / G];
+        src = a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
       }
-      const int np = min(4, npages - st);
-      const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
-      const bool partial = kvalid < np * 16;
-      if (active) {
-        const uint32_t kb = smem_u32(smem + s * S::STAGE), vb = kb + S::KBYTES;
-        float sacc[8][4];
 #pragma unroll
-        for (int n = 0; n < 8; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = src ? *reinterpret_cast<const uint4*>(src + 8 * c) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + S::OFF_Q + (c >> 3) * S::QBLK + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarQFull));
+    };
+    if (s_begin < s_end) load_q(s_begin);
+    for (int si = s_begin; si < s_end && ok; ++si) {
+      const pa_seg seg = a.segs[si];
+      const pa_item item = a.items[seg.item];
+      const int R = item.n_queries * G;
+      const int npages = (seg.n_tokens + 15) >> 4;
+      float m_used = -INFINITY, l = 0.f;
+      for (int st = 0; st < npages; st += 4, ++i) {
+        const int s = i % kMmaNST;
+        const int np = min(4, npages - st);
+        const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
+        if (!warp_wait(bar(kBarSFull + (i & 1)), (i >> 1) & 1, a.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        float sv[kMmaKT];
+        tmem_ld32(tmem + (i & 1) * kMmaKT + lane_off, *reinterpret_cast<float(*)[32]>(&sv[0]));
+        tmem_ld32(tmem + (i & 1) * kMmaKT + 32 + lane_off, *reinterpret_cast<float(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(kBarSFree + (i & 1)));
+        // all S products of this segment are done: Q may be replaced by the next segment's
+        if (st + 4 >= npages && si + 1 < s_end) load_q(si + 1);
+        float mx = -INFINITY;
 #pragma unroll
-        for (int ntp = 0; ntp < 4; ++ntp) {
-          if (ntp < np) {
+        for (int j = 0; j < kMmaKT; ++j) {
+          sv[j] = j < kvalid ? sv[j] * a.qscale : -INFINITY;
+          mx = fmaxf(mx, sv[j]);
+        }
+        const float mnew = fmaxf(m_used, mx);
+        // the previous p.V product must be done before P and O are touched
+        if (i >= 1) {
+          if (!warp_wait(bar(kBarOFull), (i - 1) & 1, a.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (st == 0) {
+          m_used = mnew;
+        } else {
+          const bool need = mnew > m_used + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2(m_used - mnew) : 1.f;
 #pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-              const int key = (2 * ntp + (mi >> 1)) * 8 + rr;
-              const int dof = kk * 16 + 8 * (mi & 1);
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4(kb + (dof >> 6) * (kMmaKT * 128) + swz(key, (dof & 63) >> 3), b0, b1, b2, b3);
-              mma_bf16_16816(sacc[2 * ntp], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
-              mma_bf16_16816(sacc[2 * ntp + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+            for (int c = 0; c < D / 32; ++c) {
+              float ov[32];
+              tmem_ld32(tO + lane_off + 32 * c, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ov[j] *= alpha;
+              tmem_st32(tO + lane_off + 32 * c, ov);
+            }
+            tmem_wait_st();
+            if (need) {
+              l *= alpha;
+              m_used = mnew;
             }
           }
         }
-        // scale, mask, row max
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        const float ms = m_used == -INFINITY ? 0.f : m_used;
+        uint32_t ph[kMmaKT / 2], pl[kMmaKT / 2];
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = n * 8 + 2 * c4 + (e & 1);
-            sacc[n][e] = key < kvalid ? sacc[n][e] * a.qscale : -INFINITY;
-          }
-          mx0 = fmaxf(mx0, fmaxf(sacc[n][0], sacc[n][1]));
-          mx1 = fmaxf(mx1, fmaxf(sacc[n][2], sacc[n][3]));
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float al0 = mn0 == -INFINITY ? 1.f : ex2(m0 - mn0);
-        const float al1 = mn1 == -INFINITY ? 1.f : ex2(m1 - mn1);
-        m0 = mn0;
-        m1 = mn1;
-        const float ms0 = m0 == -INFINITY ? 0.f : m0, ms1 = m1 == -INFINITY ? 0.f : m1;
-        l0 *= al0;
-        l1 *= al1;
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-          oacc[n][0] *= al0;
-          oacc[n][1] *= al0;
-          oacc[n][2] *= al1;
-          oacc[n][3] *= al1;
-        }
-        uint32_t pf[8][2];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          const float p0 = ex2(sacc[n][0] - ms0), p1 = ex2(sacc[n][1] - ms0);
-          const float p2 = ex2(sacc[n][2] - ms1), p3 = ex2(sacc[n][3] - ms1);
-          l0 += p0 + p1;
-          l1 += p2 + p3;
-          pf[n][0] = pack_bf16x2(p0, p1);
-          pf[n][1] = pack_bf16x2(p2, p3);
+        for (int j = 0; j < kMmaKT / 2; ++j) {
+          const float p0 = ex2(sv[2 * j] - ms), p1 = ex2(sv[2 * j + 1] - ms);
+          l += p0 + p1;
+          ph[j] = pack_bf16x2(p0, p1);
+          const float2 h = bf16x2_to_f2(ph[j]);
+          pl[j] = pack_bf16x2(p0 - h.x, p1 - h.y);
         }
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          if (kk < np) {
-            const uint32_t a0 = pf[2 * kk][0], a1 = pf[2 * kk][1], a2 = pf[2 * kk + 1][0], a3 = pf[2 * kk + 1][1];
-            uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-            if (partial) {
-              // V rows past the last valid key may hold NaN; p = 0 there, but 0 * NaN
-              // would still poison the product, so the fragments are zeroed instead
-              const int k0 = kk * 16 + 2 * c4;
-              mlo = (k0 < kvalid ? 0x0000FFFFu : 0u) | (k0 + 1 < kvalid ? 0xFFFF0000u : 0u);
-              mhi = (k0 + 8 < kvalid ? 0x0000FFFFu : 0u) | (k0 + 9 < kvalid ? 0xFFFF0000u : 0u);
-            }
-#pragma unroll
-            for (int ntp = 0; ntp < D / 16; ++ntp) {
-              const int key = kk * 16 + 8 * (mi & 1) + rr;
-              const int d = (2 * ntp + (mi >> 1)) * 8;
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4_t(vb + (d >> 6) * (kMmaKT * 128) + swz(key, (d & 63) >> 3), b0, b1, b2, b3);
-              mma_bf16_16816(oacc[2 * ntp], a0, a1, a2, a3, b0 & mlo, b1 & mhi);
-              mma_bf16_16816(oacc[2 * ntp + 1], a0, a1, a2, a3, b2 & mlo, b3 & mhi);
-            }
+        for (int c = 0; c < 8; ++c) {
+          const int off = S::OFF_P + r * 128 + ((c ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(smem + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+          *reinterpret_cast<uint4*>(smem + off + S::PBLK) =
+              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+        }
+        if (kvalid < np * 16) {
+          // V rows past the last valid key may hold NaN; p = 0 there but 0 * NaN
+          // would still poison the product, so those rows are zeroed
+          uint8_t* vst = smem + s * S::STAGE + S::HALVES * S::KBLK;
+          const int nz = np * 16 - kvalid;
+          for (int idx = r; idx < nz * S::HALVES * 8; idx += 128) {
+            const int row = kvalid + idx / (S::HALVES * 8);
+            const int h = (idx >> 3) % S::HALVES, c = idx & 7;
+            *reinterpret_cast<uint4*>(vst + h * S::KBLK + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
           }
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-    }
-    if (!active) continue;
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-    if (r0 < R) {
-      const int prow = a.seg_prows[seg.prow + r0 / G];
-      float* dst = a.partial_o + ((size_t)prow * G + (r0 % G)) * D;
+      if (!ok) break;
+      // epilogue: O row from TMEM, normalised, as this segment's partial row
+      if (!warp_wait(bar(kBarOFull), (i - 1) & 1, a.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      float ov[D];
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n)
-        *reinterpret_cast<float2*>(dst + n * 8 + 2 * c4) = make_float2(oacc[n][0] * inv0, oacc[n][1] * inv0);
-      if (c4 == 0) a.partial_lse[(size_t)prow * G + (r0 % G)] = (m0 + lg2(l0)) * kLn2;
-    }
-    if (r1 < R) {
-      const int prow = a.seg_prows[seg.prow + r1 / G];
-      float* dst = a.partial_o + ((size_t)prow * G + (r1 % G)) * D;
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + lane_off + 32 * c, *reinterpret_cast<float(*)[32]>(&ov[32 * c]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kBarOFree));
+      if (r < R) {
+        const int prow = a.seg_prows[seg.prow + r / G];
+        float* dst = a.partial_o + ((size_t)prow * G + (r % G)) * D;
+        const float inv = 1.f / l;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n)
-        *reinterpret_cast<float2*>(dst + n * 8 + 2 * c4) = make_float2(oacc[n][2] * inv1, oacc[n][3] * inv1);
-      if (c4 == 0) a.partial_lse[(size_t)prow * G + (r1 % G)] = (m1 + lg2(l1)) * kLn2;
+        for (int c = 0; c < D / 4; ++c)
+          *reinterpret_cast<float4*>(dst + 4 * c) =
+              make_float4(ov[4 * c] * inv, ov[4 * c + 1] * inv, ov[4 * c + 2] * inv, ov[4 * c + 3] * inv);
+        a.partial_lse[(size_t)prow * G + (r % G)] = (m_used + lg2(l)) * kLn2;
+      }
+      if (a.out) {
+        // this warp's 32 rows hold whole (request, kv head) row groups (32 % G == 0)
+        const int qpw = 32 / G;
+        const int n = max(0, min(qpw, item.n_queries - quad * qpw));
+        const int bj = lane < n ? a.queries[item.query_off + quad * qpw + lane] : 0;
+        arrive_and_merge<D, G>(a, bj, n, seg.kv_head, lane);
+      }
+      ++segord;
     }
-    if (a.out) {
-      // this warp's 16 rows hold whole (request, kv head) row groups (16 % G == 0)
-      const int qpw = 16 / G;
-      for (int j = warp * qpw; j < min((warp + 1) * qpw, item.n_queries); ++j)
-        arrive_and_merge<D>(a, a.queries[item.query_off + j], g, lane);
-    }
+    if (!ok && lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, warp);
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, kTmemCols);
 }
 
 template <int D, int G>
@@ -707,11 +820,11 @@ __global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1) fwd_simt_kernel(cons
   simt_role<D, G>(a, smem);
 }
 
-template <int D>
+template <int D, int G>
 __global__ void __launch_bounds__(kMmaThreads, 1)
     fwd_mma_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  mma_role<D>(a, &tk, &tv, smem);
+  mma_role<D, G>(a, &tk, &tv, smem);
 }
 
 struct MergeArgs {
@@ -723,11 +836,11 @@ struct MergeArgs {
   int B, Hq, Hkv, G;
 };
 
-template <int D>
+template <int D, int G>
 __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (w >= a.B * a.Hkv) return;
-  merge_pair<D>(a.prow_off, a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, a.Hkv, a.G, w / a.Hkv, w % a.Hkv, lane);
+  merge_pair<D, G>(a.prow_off, a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, a.Hkv, w / a.Hkv, w % a.Hkv, lane);
 }
 
 FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse) {
@@ -775,16 +888,22 @@ int launch_simt_t(const FwdArgs& a, cudaStream_t st) {
   return (int)cudaGetLastError();
 }
 
-template <int D>
+template <int D, int G>
 int launch_mma_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
   constexpr int smem = MmaShape<D>::SMEM;
-  auto k = fwd_mma_kernel<D>;
+  auto k = fwd_mma_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
   if (a.n_mma_ctas <= 0) return 0;
   const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
   const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
   k<<<a.n_mma_ctas, kMmaThreads, smem, st>>>(a, *tk, *tv);
+  return (int)cudaGetLastError();
+}
+
+template <int D, int G>
+int launch_merge_t(const MergeArgs& a, int grid, cudaStream_t st) {
+  merge_kernel<D, G><<<grid, 256, 0, st>>>(a);
   return (int)cudaGetLastError();
 }
 
@@ -812,7 +931,18 @@ int pa_launch_forward_simt(const pa_plan& p, const PaDevPtrs& d, void* out, floa
 int pa_launch_forward_mma(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* side) {
   const FwdArgs a = make_fwd_args(p, d, out, lse);
   cudaStream_t st = static_cast<cudaStream_t>(side);
-  return p.D == 128 ? launch_mma_t<128>(p, a, st) : launch_mma_t<64>(p, a, st);
+#define PA_MMA_CASE(DD, GG) \
+  if (p.D == DD && p.G == GG) return launch_mma_t<DD, GG>(p, a, st);
+  PA_MMA_CASE(128, 4)
+  PA_MMA_CASE(128, 1)
+  PA_MMA_CASE(128, 2)
+  PA_MMA_CASE(128, 8)
+  PA_MMA_CASE(64, 4)
+  PA_MMA_CASE(64, 1)
+  PA_MMA_CASE(64, 2)
+  PA_MMA_CASE(64, 8)
+#undef PA_MMA_CASE
+  return (int)cudaErrorInvalidValue;
 }
 
 int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
@@ -826,10 +956,18 @@ int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse,
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.G = p.G;
-  const int warps = p.B * p.Hkv;
-  const int grid = (warps + 7) / 8;
+  const int grid = (p.B * p.Hkv + 7) / 8;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (p.D == 128) merge_kernel<128><<<grid, 256, 0, st>>>(a);
-  else merge_kernel<64><<<grid, 256, 0, st>>>(a);
-  return (int)cudaGetLastError();
+#define PA_MERGE_CASE(DD, GG) \
+  if (p.D == DD && p.G == GG) return launch_merge_t<DD, GG>(a, grid, st);
+  PA_MERGE_CASE(128, 4)
+  PA_MERGE_CASE(128, 1)
+  PA_MERGE_CASE(128, 2)
+  PA_MERGE_CASE(128, 8)
+  PA_MERGE_CASE(64, 4)
+  PA_MERGE_CASE(64, 1)
+  PA_MERGE_CASE(64, 2)
+  PA_MERGE_CASE(64, 8)
+#undef PA_MERGE_CASE
+  return (int)cudaErrorInvalidValue;
 }

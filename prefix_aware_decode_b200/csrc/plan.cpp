@@ -244,7 +244,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     // boundaries (long-KV splitting without a fixed chunk size).
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 0.7e6;     // flop per us per SM, mma.sync with 8 warps (measured)
+    const double kMmaFlopsPerSmUs = 4.0e6;     // flop per us per SM, tcgen05 class (split p: 1.5x the flops)
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
     int64_t simt_pages = 0, mma_pages = 0;
@@ -399,7 +399,11 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       di[i] = {items[i].page_off, items[i].n_tokens, items[i].n_queries, items[i].query_off};
     pa_seg* ds = reinterpret_cast<pa_seg*>(img + h.off_segs);
     size_t k = 0;
-    for (const auto& s : simt_segs) ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, 0};
+    for (const auto& s : simt_segs) {
+      const size_t bg = (size_t)s.query * Hkv + s.kv_head;
+      const int sole = prow_off[bg + 1] - prow_off[bg] == 1 ? 1 : 0;
+      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole, 0};
+    }
     for (const auto& s : mma_segs) ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, 0};
     auto put = [&](uint64_t o, const std::vector<int32_t>& v) {
       if (!v.empty()) std::memcpy(img + o, v.data(), v.size() * 4);
