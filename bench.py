@@ -196,20 +196,16 @@ def main():
         return evs
 
     nsteps = args.warmup + args.steps
-    step_events = [mk_events(2) for _ in range(nsteps)]
-    plan_us = []
+    prof_every = 4  # profiling events on every 4th step of the timed region
+    step_events = [mk_events(4) if i % prof_every == 0 else None for i in range(nsteps)]
+    host_us = []
+    stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, q, k0, v0, workspaces[0], out, lse, stream=stream)
 
-    def step(i, prof=True):
+    def step(i):
         t = time.perf_counter()
-        plan = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
-        plan_us.append((time.perf_counter() - t) * 1e6)
-        if prof:
-            plan.set_profile_events(step_events[i])
-        ws = workspaces[i % 2]
-        kp, vp = pools[i % copies]
-        plan.upload(ws, stream)
-        plan.attend(q, kp, vp, ws, out, lse, stream)
-        plan.close()
+        stepper.set_pools(*pools[i % copies])
+        stepper(kv_lens, block_table, events=step_events[i])
+        host_us.append((time.perf_counter() - t) * 1e6)
 
     for i in range(args.warmup):
         step(i)
@@ -226,7 +222,7 @@ def main():
     barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    plan_us.clear()
+    host_us.clear()
     ev0.record(stream)
     for i in range(args.warmup, nsteps):
         step(i)
@@ -242,7 +238,11 @@ def main():
     ms_step = ms / args.steps
 
     # forward (both classes, merge fused) time inside the timed region, per step
-    fwd_ms = statistics.mean(step_events[i][0].elapsed_time(step_events[i][1]) for i in range(args.warmup, nsteps))
+    def ev_ms(a_, b_):
+        return statistics.mean(step_events[i][a_].elapsed_time(step_events[i][b_])
+                               for i in range(args.warmup, nsteps) if step_events[i] is not None)
+
+    fwd_ms = ev_ms(0, 1)
 
     # algorithmic bytes of one forward: the KV of its (page, kv head) tiles (each
     # node read once per query tile), the q rows, the fp32 partial rows written
@@ -265,17 +265,18 @@ def main():
                    "step": "pack (host) + upload + forward + merge", "parallelism": f"replicas x{world}"},
         "unique_kv_gbs": unique_bytes / (ms_step * 1e-3) / 1e9,
         "unique_kv_frac_of_hbm": unique_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak,
-        "device_ms": {"forward_merge_fused": fwd_ms},
+        "device_ms": {"forward_merge_fused": fwd_ms, "profiled_steps": sum(e is not None for e in step_events[args.warmup:])},
         "forward_queries_per_s": w.B / (fwd_ms * 1e-3),
         "forward_unique_kv_frac": unique_bytes / (fwd_ms * 1e-3) / 1e9 / hbm_peak,
-        "plan_us_median": statistics.median(plan_us),
+        "plan_us": pst["plan_us"],
+        "host_us_per_step_median": statistics.median(host_us),
         "plan": {k: pst[k] for k in ("num_segments_simt", "num_segments_mma", "simt_warps", "mma_ctas",
                                      "num_partial_rows", "read_kv_bytes", "workspace_bytes", "image_bytes")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": None,
-                     "kernel": "forward (fwd_simt_kernel<128,4> + fwd_mma_kernel<128>, merge fused)",
+                     "kernel": "fwd_kernel<128,4> (both tile classes, merge fused)",
                      "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
-        "gpu_launches": args.steps * ((pst["mma_ctas"] > 0) + (pst["simt_warps"] > 0)),
+        "gpu_launches": args.steps,
         "clocks": clk,
     }
 
@@ -289,15 +290,15 @@ def main():
         dq = torch.empty_like(q)
         dk, dv = torch.empty_like(k0), torch.empty_like(v0)
 
+        e2e_stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, dq, dk, dv, workspaces[1], out, lse,
+                                     stream=stream)
+
         def e2e_step(copy_kv: bool):
             dq.view(torch.int16).copy_(hq, non_blocking=True)
             if copy_kv:
                 dk.view(torch.int16).copy_(hk, non_blocking=True)
                 dv.view(torch.int16).copy_(hv, non_blocking=True)
-            plan = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
-            plan.upload(workspaces[0], stream)
-            plan.attend(dq, dk, dv, workspaces[0], out, lse, stream)
-            plan.close()
+            e2e_stepper(kv_lens, block_table)
             ho.copy_(out.view(torch.int16), non_blocking=True)
             hl.copy_(lse, non_blocking=True)
 

@@ -184,6 +184,19 @@ pa_status pa_plan_host_image(const pa_plan *plan, void *dst, size_t bytes);
  */
 pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t n);
 
+/*
+ * One decode step in one call: pa_plan_create, pa_plan_upload and pa_attend
+ * (forward with the merge fused) on `stream`.  workspace_bytes must cover the
+ * plan's workspace (pa_plan_workspace_size of a plan of the same batch).
+ * profile_events: NULL, or four cudaEvent_t as for pa_plan_set_profile_events.
+ * plan_out: NULL (the plan is released before returning; its upload has
+ * already been staged) or receives the plan, which the caller then releases.
+ */
+pa_status pa_decode_step(const pa_config *cfg, int32_t batch, const int32_t *kv_lens, const int32_t *block_table,
+                         int32_t max_pages, int32_t num_pages_in_pool, const void *q, const void *k_pool,
+                         const void *v_pool, void *d_workspace, size_t workspace_bytes, void *out, float *lse,
+                         void *const *profile_events, void *stream, pa_plan **plan_out);
+
 /* Release a plan (NULL is ignored). */
 void pa_plan_destroy(pa_plan *plan);
 

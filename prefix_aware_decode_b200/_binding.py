@@ -63,7 +63,7 @@ class PaImageHeader(ctypes.Structure):
 # exported names, in the order pa.h declares them
 EXPORTS = ["pa_plan_create", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
            "pa_get_device_status", "pa_plan_get_stats", "pa_plan_host_image", "pa_plan_set_profile_events",
-           "pa_plan_destroy", "pa_status_string"]
+           "pa_decode_step", "pa_plan_destroy", "pa_status_string"]
 
 _lib = None
 
@@ -98,6 +98,9 @@ def lib() -> ctypes.CDLL:
     L.pa_plan_host_image.restype = st
     L.pa_plan_set_profile_events.argtypes = [vp, ctypes.POINTER(vp), i32]
     L.pa_plan_set_profile_events.restype = st
+    L.pa_decode_step.argtypes = [ctypes.POINTER(PaConfig), i32, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp,
+                                 ctypes.POINTER(vp), vp, ctypes.POINTER(vp)]
+    L.pa_decode_step.restype = st
     L.pa_plan_destroy.argtypes = [vp]
     L.pa_plan_destroy.restype = None
     L.pa_status_string.argtypes = [st]
@@ -208,7 +211,7 @@ class Plan:
                "pa_attend")
 
     def set_profile_events(self, events):
-        """events: up to four torch.cuda.Event (or None): forward (begin, end), merge (begin, end)."""
+        """events: up to four torch.cuda.Event (or None), see pa_plan_set_profile_events."""
         self._prof_events = list(events)  # keep them alive
         arr = (ctypes.c_void_p * 4)()
         for i, e in enumerate(self._prof_events):
@@ -246,3 +249,38 @@ def attend(q, k_pool, v_pool, block_table, kv_lens, softmax_scale: float = 0.0, 
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
     plan.close()
     return out, lse
+
+
+class DecodeStep:
+    """Repeated decode steps through pa_decode_step (one C call per step).
+
+    The fixed arguments (shapes, pools, workspace, outputs) are marshalled
+    once; each call passes the step's kv_lens / block_table (host arrays).
+    """
+
+    def __init__(self, num_pages, num_q_heads, num_kv_heads, head_dim, q, k_pool, v_pool, workspace, out, lse=None,
+                 page_size=16, softmax_scale=0.0, flags=0, max_chunk_tokens=0, stream=None):
+        self._lib = lib()
+        self.cfg = PaConfig(num_q_heads, num_kv_heads, head_dim, page_size, softmax_scale, 0, max_chunk_tokens,
+                            flags, 0)
+        self.num_pages = int(num_pages)
+        self.args = (_dptr(q, "q"), _dptr(k_pool, "k_pool"), _dptr(v_pool, "v_pool"),
+                     _dptr(workspace, "workspace", 256), workspace.numel() * workspace.element_size(),
+                     _dptr(out, "out"), _dptr(lse, "lse", 4) if lse is not None else None)
+        self.stream = _stream_ptr(stream)
+        self._events = None
+
+    def set_pools(self, k_pool, v_pool):
+        a = list(self.args)
+        a[1], a[2] = _dptr(k_pool, "k_pool"), _dptr(v_pool, "v_pool")
+        self.args = tuple(a)
+
+    def __call__(self, kv_lens: np.ndarray, block_table: np.ndarray, events=None):
+        ev = None
+        if events is not None:
+            self._events = (ctypes.c_void_p * 4)(*[e.cuda_event if e is not None else None for e in events])
+            ev = self._events
+        q, k, v, ws, wsb, out, lse = self.args
+        _check(self._lib.pa_decode_step(ctypes.byref(self.cfg), kv_lens.shape[0], kv_lens.ctypes.data,
+                                        block_table.ctypes.data, block_table.shape[1], self.num_pages, q, k, v,
+                                        ws, wsb, out, lse, ev, self.stream, None), "pa_decode_step")

@@ -103,30 +103,38 @@ PinnedSlot* pin_acquire(size_t n, int device) {
   return &s;
 }
 
-// One side stream per device for the tensor-core class, with fork/join events.
-struct SideStream {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-  std::mutex mu;
-};
-std::mutex g_side_mu;
-SideStream g_side[64];
-
-SideStream* side_stream() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(g_side_mu);
-  SideStream& s = g_side[dev];
-  if (!s.stream) {
-    if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-    if (cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-    if (cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-  }
-  return &s;
-}
-
 void record_profile(const pa_plan& p, int which, cudaStream_t st) {
   if (p.prof[which]) cudaEventRecord(static_cast<cudaEvent_t>(p.prof[which]), st);
+}
+
+// Encoded tensor maps, cached process-wide by (pool pointer, rows, head dim):
+// a pool keeps its map for every plan that reads it.
+struct TmapEntry {
+  const void* ptr = nullptr;
+  uint64_t rows = 0;
+  int D = 0;
+  alignas(64) uint8_t map[128];
+};
+std::mutex g_tmap_mu;
+TmapEntry g_tmap[32];
+int g_tmap_next = 0;
+
+bool tmap_get(const pa_plan& p, const void* pool, void* out) {
+  const uint64_t rows = (uint64_t)p.num_pages_in_pool * p.Hkv * p.P;
+  std::lock_guard<std::mutex> lock(g_tmap_mu);
+  for (const TmapEntry& e : g_tmap)
+    if (e.ptr == pool && e.rows == rows && e.D == p.D) {
+      std::memcpy(out, e.map, 128);
+      return true;
+    }
+  TmapEntry& e = g_tmap[g_tmap_next];
+  if (!encode_pool(p, pool, e.map)) return false;
+  e.ptr = pool;
+  e.rows = rows;
+  e.D = p.D;
+  g_tmap_next = (g_tmap_next + 1) % 32;
+  std::memcpy(out, e.map, 128);
+  return true;
 }
 
 }  // namespace
@@ -139,14 +147,14 @@ extern "C" pa_status pa_plan_upload(const pa_plan* plan, void* d_workspace, size
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_pin_mu);
-  PinnedSlot* s = pin_acquire(plan->image.size(), device);
+  PinnedSlot* s = pin_acquire(plan->image.size, device);
   if (!s) {
     // no pinned memory: a pageable copy is still correct, only slower
-    cudaError_t e = cudaMemcpyAsync(d_workspace, plan->image.data(), plan->image.size(), cudaMemcpyHostToDevice, st);
+    cudaError_t e = cudaMemcpyAsync(d_workspace, plan->image.data(), plan->image.size, cudaMemcpyHostToDevice, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
-  std::memcpy(s->ptr, plan->image.data(), plan->image.size());
-  cudaError_t e = cudaMemcpyAsync(d_workspace, s->ptr, plan->image.size(), cudaMemcpyHostToDevice, st);
+  std::memcpy(s->ptr, plan->image.data(), plan->image.size);
+  cudaError_t e = cudaMemcpyAsync(d_workspace, s->ptr, plan->image.size, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   if (cudaEventRecord(s->done, st) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
@@ -172,29 +180,13 @@ pa_status launch(const pa_plan* plan, const void* q, const void* k_pool, const v
   d.k_pool = static_cast<const uint16_t*>(k_pool);
   d.v_pool = static_cast<const uint16_t*>(v_pool);
   if (plan->hdr.mma_ctas > 0 && (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool)) {
-    if (!encode_pool(*plan, k_pool, plan->tma_k) || !encode_pool(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
+    if (!tmap_get(*plan, k_pool, plan->tma_k) || !tmap_get(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
     plan->tma_k_ptr = k_pool;
     plan->tma_v_ptr = v_pool;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   record_profile(*plan, 0, st);
-  if (plan->hdr.mma_ctas > 0 && plan->hdr.simt_warps > 0) {
-    // multi-stream forward: the MMA class runs on a side stream concurrently
-    // with the SIMT class on the caller's stream (fork / join by events)
-    SideStream* ss = side_stream();
-    if (!ss) return PA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(ss->mu);
-    if (cudaEventRecord(ss->fork, st) != cudaSuccess) return PA_ERR_CUDA;
-    if (cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess) return PA_ERR_CUDA;
-    if (pa_launch_forward_mma(*plan, d, out, lse, ss->stream) != 0) return PA_ERR_CUDA;
-    if (pa_launch_forward_simt(*plan, d, out, lse, st) != 0) return PA_ERR_CUDA;
-    if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return PA_ERR_CUDA;
-    if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return PA_ERR_CUDA;
-  } else if (plan->hdr.mma_ctas > 0) {
-    if (pa_launch_forward_mma(*plan, d, out, lse, st) != 0) return PA_ERR_CUDA;
-  } else {
-    if (pa_launch_forward_simt(*plan, d, out, lse, st) != 0) return PA_ERR_CUDA;
-  }
+  if (pa_launch_forward(*plan, d, out, lse, stream) != 0) return PA_ERR_CUDA;
   record_profile(*plan, 1, st);
   return PA_OK;
 }
@@ -233,4 +225,21 @@ extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_wor
   if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
   *out = static_cast<pa_status>(word);
   return PA_OK;
+}
+
+extern "C" pa_status pa_decode_step(const pa_config* cfg, int32_t batch, const int32_t* kv_lens,
+                                    const int32_t* block_table, int32_t max_pages, int32_t num_pages_in_pool,
+                                    const void* q, const void* k_pool, const void* v_pool, void* d_workspace,
+                                    size_t workspace_bytes, void* out, float* lse, void* const* profile_events,
+                                    void* stream, pa_plan** plan_out) {
+  if (plan_out) *plan_out = nullptr;
+  pa_plan* plan = nullptr;
+  pa_status st = pa_plan_create(cfg, batch, kv_lens, block_table, max_pages, num_pages_in_pool, &plan);
+  if (st != PA_OK) return st;
+  if (profile_events) pa_plan_set_profile_events(plan, profile_events, 4);
+  st = pa_plan_upload(plan, d_workspace, workspace_bytes, stream);
+  if (st == PA_OK) st = pa_attend(plan, q, k_pool, v_pool, d_workspace, out, lse, stream);
+  if (st == PA_OK && plan_out) *plan_out = plan;
+  else pa_plan_destroy(plan);
+  return st;
 }

@@ -3,9 +3,11 @@
 // Forward (the PAT review, section 三, Forward 阶段 and Figure 3: decode attention
 // is two GEMVs, q.K^T then p.V, fed by a tiling pipeline that streams KV tiles
 // from global memory through on-chip memory; multi-tile kernels with a runtime
-// tile selector; multi-stream execution; long KV is split).  Two tile classes,
-// chosen by the planner from the rows of each work unit (requests x G query
-// heads), run as two concurrent launches of one persistent CTA per SM:
+// tile selector; long KV is split).  One persistent launch with one CTA per
+// SM; the planner gives every CTA one of two tile classes, chosen by the rows
+// of its work units (requests x G query heads), and splits the SMs between the
+// classes so that both finish together (the pages' multi-stream execution,
+// done here as concurrent CTA roles inside one launch):
 //   - MMA class: work units with two or more requests, up to 128 rows, on the
 //     5th-generation tensor cores: a producer warp streams 64-key stages with
 //     2-D TMA copies (128-byte swizzle), one thread issues tcgen05.mma with the
@@ -297,7 +299,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   constexpr int NST = S::NST, LPG = S::LPG, CPL = S::CPL;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp >= kSimtWarpsPerCta) return;
-  const int gw = blockIdx.x * kSimtWarpsPerCta + warp;
+  const int gw = (blockIdx.x - a.n_mma_ctas) * kSimtWarpsPerCta + warp;
   if (gw >= a.n_simt_warps) return;  // no block-wide barrier in this role
   uint8_t* wbase = smem + warp * S::WARP_BYTES;
   uint8_t* qslot = wbase + NST * S::STAGE;  // two q-row slots
@@ -501,7 +503,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
 
 constexpr int kMmaKT = 64;          // keys per stage (4 pages)
 constexpr int kMmaNST = 4;          // K/V stages in flight
-constexpr int kMmaThreads = 192;    // 6 warps
+constexpr int kMmaWarps = 6;        // producer, MMA issuer, 4 softmax warps
 constexpr uint32_t kTmemCols = 256; // S x 2 (64 columns each) + O (<= 128 columns)
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -512,15 +514,18 @@ struct MmaShape {
   static constexpr int STAGE = 2 * HALVES * KBLK;  // K and V of one stage
   static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
   static constexpr int OFF_Q = kMmaNST * STAGE;
-  static constexpr int OFF_P = OFF_Q + HALVES * QBLK;  // P_hi, then P_lo at + PBLK
+  static constexpr int OFF_P = OFF_Q + HALVES * QBLK;  // 2 buffers x (P_hi, P_lo at + PBLK)
   static constexpr int PBLK = 128 * 128;
-  static constexpr int OFF_BAR = OFF_P + 2 * PBLK;
+  static constexpr int OFF_BAR = OFF_P + 4 * PBLK;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
   static_assert(SMEM <= kSmemMax, "MMA ring does not fit");
 };
 
-enum : int { kBarFull = 0, kBarEmpty = 4, kBarSFull = 8, kBarSFree = 10, kBarPFull = 12, kBarOFull = 13,
-             kBarQFull = 14, kBarOFree = 15, kBarDone = 16, kNumBars = 17 };
+// Barriers: K/V stage full / empty; S buffer full / free (x2); P buffer full
+// and p.V done (x2, one per P buffer, so no wait can fall two phases behind);
+// Q loaded; O read out; all MMAs retired.
+enum : int { kBarFull = 0, kBarEmpty = 4, kBarSFull = 8, kBarSFree = 10, kBarPFull = 12, kBarOFull = 14,
+             kBarQFull = 16, kBarOFree = 17, kBarDone = 18, kNumBars = 19 };
 
 // All lanes wait; the warp fails together if any lane timed out.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -551,7 +556,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     mbar_init(bar(kBarSFree), 128);
     mbar_init(bar(kBarSFree + 1), 128);
     mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarPFull + 1), 128);
     mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOFull + 1), 1);
     mbar_init(bar(kBarQFull), 128);
     mbar_init(bar(kBarOFree), 128);
     mbar_init(bar(kBarDone), 1);
@@ -565,45 +572,61 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
   const uint32_t tO = tmem + 128;
 
   if (warp == 0) {
-    // ---------------- TMA producer: every stage of every segment of this CTA, in order
+    // ---------------- TMA producer: every stage of every segment of this CTA, in
+    // order.  The warp holds the segment's page ids in a sliding window of 32
+    // lanes (plus the next window, prefetched), so no issue waits on a load.
     if (lane == 0) {
       prefetch_tmap(tk);
       prefetch_tmap(tv);
-      uint32_t lastpar = 0, any = 0;
-      int i = 0;
-      bool ok = true;
-      for (int si = s_begin; si < s_end && ok; ++si) {
-        const pa_seg seg = a.segs[si];
-        const int page_base = a.items[seg.item].page_off + seg.page_begin;
-        const int npages = (seg.n_tokens + 15) >> 4;
-        for (int st = 0; st < npages; st += 4, ++i) {
-          const int s = i % kMmaNST;
-          if (i >= kMmaNST && !mbar_wait_bounded(bar(kBarEmpty + s), ((i / kMmaNST) - 1) & 1, a.timeout_ns)) {
-            record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -2);
-            ok = false;
-            break;
-          }
-          if (a.fault_drop && blockIdx.x == 0 && i == 0) continue;  // test: this stage never arrives
-          const int np = min(4, npages - st);
+    }
+    uint32_t lastpar = 0, any = 0;
+    int i = 0;
+    bool ok = true;
+    for (int si = s_begin; si < s_end && ok; ++si) {
+      const pa_seg seg = a.segs[si];
+      const int32_t* pg = a.pages + a.items[seg.item].page_off + seg.page_begin;
+      const int npages = (seg.n_tokens + 15) >> 4;
+      int wbase = 0;
+      int wcur = lane < npages ? pg[lane] : 0;
+      int wnxt = 32 + lane < npages ? pg[32 + lane] : 0;
+      for (int st = 0; st < npages; st += 4, ++i) {
+        if (st - wbase >= 32) {
+          wbase += 32;
+          wcur = wnxt;
+          wnxt = wbase + 32 + lane < npages ? pg[wbase + 32 + lane] : 0;
+        }
+        const int s = i % kMmaNST;
+        if (i >= kMmaNST && !warp_wait(bar(kBarEmpty + s), ((i / kMmaNST) - 1) & 1, a.timeout_ns)) {
+          if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -2);
+          ok = false;
+          break;
+        }
+        const int np = min(4, npages - st);
+        int rows[4];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp)
+          rows[pp] = (__shfl_sync(0xffffffffu, wcur, (st - wbase + pp) & 31) * a.Hkv + seg.kv_head) * 16;
+        if (a.fault_drop && blockIdx.x == 0 && i == 0) continue;  // test: this stage never arrives
+        if (lane == 0) {
           const uint32_t fb = bar(kBarFull + s);
           mbar_arrive_expect_tx(fb, (uint32_t)np * 2 * 16 * D * 2);
           uint8_t* kst = smem + s * S::STAGE;
           uint8_t* vst = kst + S::HALVES * S::KBLK;
           for (int pp = 0; pp < np; ++pp) {
-            const int row = (a.pages[page_base + st + pp] * a.Hkv + seg.kv_head) * 16;
 #pragma unroll
             for (int h = 0; h < S::HALVES; ++h) {
-              tma_load_2d(smem_u32(kst + h * S::KBLK + pp * 2048), tk, 64 * h, row, fb);
-              tma_load_2d(smem_u32(vst + h * S::KBLK + pp * 2048), tv, 64 * h, row, fb);
+              tma_load_2d(smem_u32(kst + h * S::KBLK + pp * 2048), tk, 64 * h, rows[pp], fb);
+              tma_load_2d(smem_u32(vst + h * S::KBLK + pp * 2048), tv, 64 * h, rows[pp], fb);
             }
           }
-          lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / kMmaNST) & 1) << s);
-          any |= 1u << s;
         }
+        lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / kMmaNST) & 1) << s);
+        any |= 1u << s;
       }
+    }
+    if (lane == 0)
       for (int s = 0; s < kMmaNST; ++s)
         if (any & (1u << s)) mbar_wait_bounded(bar(kBarFull + s), (lastpar >> s) & 1u, a.timeout_ns);
-    }
   } else if (warp == 1) {
     // ---------------- tcgen05.mma issuer (one thread)
     if (lane == 0) {
@@ -614,19 +637,20 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       bool have_prev = false, ok = true;
       int i = 0, segord = 0;
       auto do_pv = [&](const Prev& pv, int j) -> bool {
-        if (!mbar_wait_bounded(bar(kBarPFull), j & 1, a.timeout_ns)) return false;
+        if (!mbar_wait_bounded(bar(kBarPFull + (j & 1)), (j >> 1) & 1, a.timeout_ns)) return false;
         if (pv.first && pv.segord >= 1 && !mbar_wait_bounded(bar(kBarOFree), (pv.segord - 1) & 1, a.timeout_ns))
           return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(smem + pv.s * S::STAGE + S::HALVES * S::KBLK);
+        const uint32_t pb = p_base + (j & 1) * 2 * S::PBLK;
         for (int kk = 0; kk < pv.np; ++kk) {
           // P: K-major, 64 keys = one 128-byte swizzle atom per row; V: MN-major
           // (64-dim atoms at +KBLK, 8-key groups at +1 KB), 16 keys per MMA
           const uint64_t bd = umma_sdesc_sw128(v_base + kk * 2048, S::KBLK >> 4, 64);
-          umma_bf16(tO, umma_sdesc_sw128(p_base + kk * 32, 1, 64), bd, idesc_o, (pv.first && kk == 0) ? 0u : 1u);
-          umma_bf16(tO, umma_sdesc_sw128(p_base + S::PBLK + kk * 32, 1, 64), bd, idesc_o, 1u);
+          umma_bf16(tO, umma_sdesc_sw128(pb + kk * 32, 1, 64), bd, idesc_o, (pv.first && kk == 0) ? 0u : 1u);
+          umma_bf16(tO, umma_sdesc_sw128(pb + S::PBLK + kk * 32, 1, 64), bd, idesc_o, 1u);
         }
-        umma_commit(bar(kBarOFull));
+        umma_commit(bar(kBarOFull + (j & 1)));
         umma_commit(bar(kBarEmpty + pv.s));
         return true;
       };
@@ -666,7 +690,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       umma_commit(bar(kBarDone));
       mbar_wait_bounded(bar(kBarDone), 0, a.timeout_ns);
     }
-  } else {
+  } else if (warp < kMmaWarps) {
     // ---------------- softmax: thread = tile row = TMEM lane
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
@@ -711,16 +735,20 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         mbar_arrive(bar(kBarSFree + (i & 1)));
         // all S products of this segment are done: Q may be replaced by the next segment's
         if (st + 4 >= npages && si + 1 < s_end) load_q(si + 1);
-        float mx = -INFINITY;
+        float mx8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) mx8[t] = -INFINITY;
 #pragma unroll
         for (int j = 0; j < kMmaKT; ++j) {
           sv[j] = j < kvalid ? sv[j] * a.qscale : -INFINITY;
-          mx = fmaxf(mx, sv[j]);
+          mx8[j & 7] = fmaxf(mx8[j & 7], sv[j]);
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mnew = fmaxf(m_used, mx);
-        // the previous p.V product must be done before P and O are touched
-        if (i >= 1) {
-          if (!warp_wait(bar(kBarOFull), (i - 1) & 1, a.timeout_ns)) { ok = false; break; }
+        // P buffer i%2 is free once p.V of stage i-2 is done
+        if (i >= 2) {
+          if (!warp_wait(bar(kBarOFull + (i & 1)), ((i >> 1) - 1) & 1, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
         }
         if (st == 0) {
@@ -728,6 +756,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         } else {
           const bool need = mnew > m_used + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
+            // O must hold every earlier p.V product before it is rescaled
+            if (!warp_wait(bar(kBarOFull + ((i - 1) & 1)), ((i - 1) >> 1) & 1, a.timeout_ns)) { ok = false; break; }
+            tc_fence_after();
             const float alpha = need ? ex2(m_used - mnew) : 1.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -747,17 +778,21 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         }
         const float ms = m_used == -INFINITY ? 0.f : m_used;
         uint32_t ph[kMmaKT / 2], pl[kMmaKT / 2];
+        float l8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) l8[t] = 0.f;
 #pragma unroll
         for (int j = 0; j < kMmaKT / 2; ++j) {
           const float p0 = ex2(sv[2 * j] - ms), p1 = ex2(sv[2 * j + 1] - ms);
-          l += p0 + p1;
+          l8[j & 7] += p0 + p1;
           ph[j] = pack_bf16x2(p0, p1);
           const float2 h = bf16x2_to_f2(ph[j]);
           pl[j] = pack_bf16x2(p0 - h.x, p1 - h.y);
         }
+        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const int off = S::OFF_P + r * 128 + ((c ^ (r & 7)) << 4);
+          const int off = S::OFF_P + (i & 1) * 2 * S::PBLK + r * 128 + ((c ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(smem + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
           *reinterpret_cast<uint4*>(smem + off + S::PBLK) =
               make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
@@ -775,11 +810,11 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull));
+        mbar_arrive(bar(kBarPFull + (i & 1)));
       }
       if (!ok) break;
       // epilogue: O row from TMEM, normalised, as this segment's partial row
-      if (!warp_wait(bar(kBarOFull), (i - 1) & 1, a.timeout_ns)) { ok = false; break; }
+      if (!warp_wait(bar(kBarOFull + ((i - 1) & 1)), ((i - 1) >> 1) & 1, a.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       float ov[D];
 #pragma unroll
@@ -814,17 +849,15 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
   if (warp == 1) tmem_free(tmem, kTmemCols);
 }
 
+// One persistent launch, one CTA per SM: CTAs [0, n_mma_ctas) run the
+// tensor-core class (warps 0-5; warps 6-7 only join the CTA barriers), the
+// others the CUDA-core class (8 warps).
 template <int D, int G>
-__global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1) fwd_simt_kernel(const FwdArgs a) {
+__global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1)
+    fwd_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  simt_role<D, G>(a, smem);
-}
-
-template <int D, int G>
-__global__ void __launch_bounds__(kMmaThreads, 1)
-    fwd_mma_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  mma_role<D, G>(a, &tk, &tv, smem);
+  if ((int)blockIdx.x < a.n_mma_ctas) mma_role<D, G>(a, &tk, &tv, smem);
+  else simt_role<D, G>(a, smem);
 }
 
 struct MergeArgs {
@@ -877,27 +910,17 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
 }
 
 template <int D, int G>
-int launch_simt_t(const FwdArgs& a, cudaStream_t st) {
-  constexpr int smem = SimtShape<D, G>::SMEM;
-  auto k = fwd_simt_kernel<D, G>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
+  constexpr int smem_simt = SimtShape<D, G>::SMEM, smem_mma = MmaShape<D>::SMEM;
+  const int smem = a.n_mma_ctas > 0 ? (smem_simt > smem_mma ? smem_simt : smem_mma) : smem_simt;
+  auto k = fwd_kernel<D, G>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
   if (e != cudaSuccess) return (int)e;
-  const int grid = (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
+  const int grid = a.n_mma_ctas + (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
   if (grid <= 0) return 0;
-  k<<<grid, kSimtWarpsPerCta * 32, smem, st>>>(a);
-  return (int)cudaGetLastError();
-}
-
-template <int D, int G>
-int launch_mma_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
-  constexpr int smem = MmaShape<D>::SMEM;
-  auto k = fwd_mma_kernel<D, G>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return (int)e;
-  if (a.n_mma_ctas <= 0) return 0;
   const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
   const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
-  k<<<a.n_mma_ctas, kMmaThreads, smem, st>>>(a, *tk, *tv);
+  k<<<grid, kSimtWarpsPerCta * 32, smem, st>>>(a, *tk, *tv);
   return (int)cudaGetLastError();
 }
 
@@ -911,11 +934,11 @@ int launch_merge_t(const MergeArgs& a, int grid, cudaStream_t st) {
 
 using namespace pa;
 
-int pa_launch_forward_simt(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
+int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
   const FwdArgs a = make_fwd_args(p, d, out, lse);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 #define PA_FWD_CASE(DD, GG) \
-  if (p.D == DD && p.G == GG) return launch_simt_t<DD, GG>(a, st);
+  if (p.D == DD && p.G == GG) return launch_fwd_t<DD, GG>(p, a, st);
   PA_FWD_CASE(128, 4)
   PA_FWD_CASE(128, 1)
   PA_FWD_CASE(128, 2)
@@ -925,23 +948,6 @@ int pa_launch_forward_simt(const pa_plan& p, const PaDevPtrs& d, void* out, floa
   PA_FWD_CASE(64, 2)
   PA_FWD_CASE(64, 8)
 #undef PA_FWD_CASE
-  return (int)cudaErrorInvalidValue;
-}
-
-int pa_launch_forward_mma(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* side) {
-  const FwdArgs a = make_fwd_args(p, d, out, lse);
-  cudaStream_t st = static_cast<cudaStream_t>(side);
-#define PA_MMA_CASE(DD, GG) \
-  if (p.D == DD && p.G == GG) return launch_mma_t<DD, GG>(p, a, st);
-  PA_MMA_CASE(128, 4)
-  PA_MMA_CASE(128, 1)
-  PA_MMA_CASE(128, 2)
-  PA_MMA_CASE(128, 8)
-  PA_MMA_CASE(64, 4)
-  PA_MMA_CASE(64, 1)
-  PA_MMA_CASE(64, 2)
-  PA_MMA_CASE(64, 8)
-#undef PA_MMA_CASE
   return (int)cudaErrorInvalidValue;
 }
 

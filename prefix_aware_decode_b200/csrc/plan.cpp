@@ -17,6 +17,8 @@
 #include <chrono>
 #include <cmath>
 #include <cstring>
+#include <cstdlib>
+#include <mutex>
 #include <new>
 #include <numeric>
 #include <vector>
@@ -24,6 +26,9 @@
 #include "plan.h"
 
 namespace {
+
+std::mutex g_buf_mu;
+std::vector<HostBuf> g_buf_free;  // at most kMaxFreeBufs kept
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
@@ -42,14 +47,16 @@ struct Planner {
   const int32_t* bt;
   int max_pages, P, G, Hq, Hkv, D;
   uint32_t flags;
-  std::vector<int> order, npg;
+  std::vector<int>& order;
+  std::vector<int>& npg;
   // outputs of the tree walk
-  std::vector<ItemRec> items;
-  std::vector<int32_t> pages, queries;
+  std::vector<ItemRec>& items;
+  std::vector<int32_t>& pages;
+  std::vector<int32_t>& queries;
+  std::vector<int>& qbuf;
   int64_t unique_tokens = 0, read_tokens = 0;
   int num_nodes = 0, num_shared = 0, num_kept = 0;
   bool invalid = false;
-  std::vector<int> qbuf;
 
   const int32_t* row(int b) const { return bt + (size_t)b * max_pages; }
 
@@ -155,7 +162,48 @@ struct Planner {
   }
 };
 
+// Reusable scratch of the planner (one per host thread), so a plan costs no
+// allocation once the sizes have been seen.
+struct Scratch {
+  std::vector<int> order, npg, qbuf;
+  std::vector<ItemRec> items;
+  std::vector<int32_t> pages, queries, warp_segs, warp_loads, mma_cta_segs, tiles, prow_off, cursor, seg_prows;
+  std::vector<SegRec> simt_segs, mma_segs;
+};
+
 }  // namespace
+
+HostBuf hostbuf_acquire(size_t n) {
+  {
+    std::lock_guard<std::mutex> lock(g_buf_mu);
+    size_t best = g_buf_free.size();
+    for (size_t i = 0; i < g_buf_free.size(); ++i)
+      if (g_buf_free[i].cap >= n && (best == g_buf_free.size() || g_buf_free[i].cap < g_buf_free[best].cap)) best = i;
+    if (best < g_buf_free.size()) {
+      HostBuf b = g_buf_free[best];
+      g_buf_free.erase(g_buf_free.begin() + best);
+      b.size = n;
+      return b;
+    }
+  }
+  HostBuf b;
+  size_t cap = 4096;
+  while (cap < n) cap <<= 1;
+  b.ptr = static_cast<uint8_t*>(std::malloc(cap));
+  if (!b.ptr) throw std::bad_alloc();
+  b.cap = cap;
+  b.size = n;
+  return b;
+}
+
+void hostbuf_release(HostBuf& b) {
+  if (!b.ptr) return;
+  constexpr size_t kMaxFreeBufs = 16;
+  std::lock_guard<std::mutex> lock(g_buf_mu);
+  if (g_buf_free.size() < kMaxFreeBufs) g_buf_free.push_back(b);
+  else std::free(b.ptr);
+  b = HostBuf{};
+}
 
 extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const int32_t* kv_lens,
                                     const int32_t* block_table, int32_t max_pages, int32_t num_pages_in_pool,
@@ -194,7 +242,12 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     plan->wait_timeout_us = cfg->wait_timeout_us > 0 ? cfg->wait_timeout_us : 2000000;
 
     // ---- validation
-    Planner pl;
+    static thread_local Scratch sc;
+    sc.items.clear();
+    sc.pages.clear();
+    sc.queries.clear();
+    Planner pl{kv_lens, block_table, max_pages, P, G, Hq, Hkv, D, flags, sc.order, sc.npg,
+               sc.items, sc.pages, sc.queries, sc.qbuf};
     pl.kv_lens = kv_lens;
     pl.bt = block_table;
     pl.max_pages = max_pages;
@@ -244,7 +297,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     // boundaries (long-KV splitting without a fixed chunk size).
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 4.0e6;     // flop per us per SM, tcgen05 class (split p: 1.5x the flops)
+    const double kMmaFlopsPerSmUs = 2.5e6;     // flop per us per SM, tcgen05 class (measured; split p: 1.5x the flops)
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
     int64_t simt_pages = 0, mma_pages = 0;
@@ -256,7 +309,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       } else {
         mma_pages += np;
         const double rows = 16.0 * ceil_div((int64_t)it.n_queries * G, 16);
-        const double flops = 16.0 * rows * D * 4;
+        const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
         mma_cost += np * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
       }
     }
@@ -271,9 +324,18 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
         if (t < best) { best = t; n_mma = kk; }
       }
     }
-    std::vector<SegRec> simt_segs, mma_segs;
-    std::vector<int32_t> warp_segs{0}, warp_loads{0}, mma_cta_segs{0};
-    std::vector<int32_t> tiles((size_t)simt_pages);
+    std::vector<SegRec>& simt_segs = sc.simt_segs;
+    std::vector<SegRec>& mma_segs = sc.mma_segs;
+    std::vector<int32_t>& warp_segs = sc.warp_segs;
+    std::vector<int32_t>& warp_loads = sc.warp_loads;
+    std::vector<int32_t>& mma_cta_segs = sc.mma_cta_segs;
+    std::vector<int32_t>& tiles = sc.tiles;
+    simt_segs.clear();
+    mma_segs.clear();
+    warp_segs.assign(1, 0);
+    warp_loads.assign(1, 0);
+    mma_cta_segs.assign(1, 0);
+    if (tiles.size() < (size_t)simt_pages) tiles.resize((size_t)simt_pages);
     if (simt_pages > 0) {
       const int64_t W = (int64_t)(S - n_mma) * kSimtWarpsPerCta;
       int64_t span = ceil_div(simt_pages, W);
@@ -339,15 +401,18 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     }
 
     // ---- partial rows: contiguous per (request, kv head), in a fixed order
-    std::vector<int32_t> prow_off((size_t)batch * Hkv + 1, 0);
+    std::vector<int32_t>& prow_off = sc.prow_off;
+    prow_off.assign((size_t)batch * Hkv + 1, 0);
     for (const auto& s : mma_segs) {
       const ItemRec& it = items[s.item];
       for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
     }
     for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
     for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
-    std::vector<int32_t> cursor(prow_off.begin(), prow_off.end() - 1);
-    std::vector<int32_t> seg_prows;
+    std::vector<int32_t>& cursor = sc.cursor;
+    cursor.assign(prow_off.begin(), prow_off.end() - 1);
+    std::vector<int32_t>& seg_prows = sc.seg_prows;
+    seg_prows.clear();
     for (auto& s : mma_segs) {
       const ItemRec& it = items[s.item];
       s.prow = (int)seg_prows.size();
@@ -373,7 +438,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.simt_warps = (int32_t)warp_segs.size() - 1;
     h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
     h.num_partial_rows = num_prows;
-    h.num_loads = (int32_t)tiles.size();
+    h.num_loads = (int32_t)simt_pages;
     uint64_t off = align256(sizeof(pa_image_header));
     h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
     h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
@@ -384,16 +449,17 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.off_counters = off; off = align256(off + (size_t)batch * Hkv * 4);
     h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
     h.off_warp_loads = off; off = align256(off + warp_loads.size() * 4);
-    h.off_tiles = off; off = align256(off + tiles.size() * 4);
+    h.off_tiles = off; off = align256(off + (size_t)simt_pages * 4);
     h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
     h.image_bytes = off;
     h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
     h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
     h.workspace_bytes = off;
 
-    plan->image.assign(h.image_bytes, 0);
+    plan->image = hostbuf_acquire(h.image_bytes);
     uint8_t* img = plan->image.data();
     std::memcpy(img, &h, sizeof(h));
+    std::memset(img + h.off_counters, 0, (size_t)batch * Hkv * 4);
     pa_item* di = reinterpret_cast<pa_item*>(img + h.off_nodes);
     for (size_t i = 0; i < items.size(); ++i)
       di[i] = {items[i].page_off, items[i].n_tokens, items[i].n_queries, items[i].query_off};
@@ -414,7 +480,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     put(h.off_mma_segs, mma_cta_segs);
     put(h.off_warp_segs, warp_segs);
     put(h.off_warp_loads, warp_loads);
-    put(h.off_tiles, tiles);
+    if (simt_pages) std::memcpy(img + h.off_tiles, tiles.data(), (size_t)simt_pages * 4);
     put(h.off_prow_off, prow_off);
 
     pa_plan_stats& st = plan->stats;
@@ -464,8 +530,8 @@ extern "C" pa_status pa_plan_get_stats(const pa_plan* plan, pa_plan_stats* out) 
 
 extern "C" pa_status pa_plan_host_image(const pa_plan* plan, void* dst, size_t bytes) {
   if (!plan || !dst) return PA_ERR_INVALID;
-  if (bytes < plan->image.size()) return PA_ERR_NOMEM;
-  std::memcpy(dst, plan->image.data(), plan->image.size());
+  if (bytes < plan->image.size) return PA_ERR_NOMEM;
+  std::memcpy(dst, plan->image.data(), plan->image.size);
   return PA_OK;
 }
 

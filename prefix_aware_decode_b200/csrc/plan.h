@@ -9,11 +9,21 @@
 static_assert(sizeof(pa_seg) == 32, "pa_seg must be 32 bytes (vector loads)");
 static_assert(sizeof(pa_item) == 16, "pa_item must be 16 bytes");
 
-// Forward launch shapes, one CTA per SM for both classes.  A CUDA-core (SIMT)
-// CTA runs 8 independent warps; a tensor-core (MMA) CTA runs 8 consumer warps
-// of 16 rows each (128 rows) and one producer warp.
+// Forward launch shape: 8 warps per CTA, one CTA per SM.  A CUDA-core (SIMT)
+// CTA runs 8 independent warps; a tensor-core (MMA) CTA works on tiles of up
+// to 128 rows with 6 warps (TMA producer, tcgen05 issuer, 4 softmax warps).
 constexpr int kSimtWarpsPerCta = 8;
 constexpr int kMmaRowsPerCta = 128;
+
+// Host buffer for plan images, taken from and returned to a small process-wide
+// pool so that building a plan does not page-fault fresh memory every time.
+struct HostBuf {
+  uint8_t* ptr = nullptr;
+  size_t size = 0, cap = 0;
+  uint8_t* data() const { return ptr; }
+};
+HostBuf hostbuf_acquire(size_t n);
+void hostbuf_release(HostBuf& b);
 
 struct pa_plan {
   pa_config cfg;
@@ -25,7 +35,8 @@ struct pa_plan {
   int32_t wait_timeout_us = 0;
   pa_plan_stats stats{};
   pa_image_header hdr{};
-  std::vector<uint8_t> image;  // exactly what pa_plan_upload sends
+  HostBuf image;  // exactly what pa_plan_upload sends (image.size bytes)
+  ~pa_plan() { hostbuf_release(image); }
   // cached TMA descriptors (encoded for the last pool pointers seen)
   mutable const void* tma_k_ptr = nullptr;
   mutable const void* tma_v_ptr = nullptr;
@@ -58,9 +69,6 @@ struct PaDevPtrs {
   int32_t* status;
 };
 
-// out == nullptr: partial rows only; else the merge is fused into the launches.
-// The two classes run as two kernels; `side` is a second stream that the
-// caller has made wait for `stream` (the MMA kernel goes there).
-int pa_launch_forward_mma(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* side);
-int pa_launch_forward_simt(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
+// out == nullptr: partial rows only; else the merge is fused into the launch.
+int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
