@@ -1,0 +1,90 @@
+"""World-size-2 data-parallel path on CPU (gloo): each rank plans its root
+subtrees with the C planner, executes the plan image in fp64, and the gathered
+result equals the oracle over the whole batch."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    import torch
+
+    import prefix_aware_decode_b200 as pad
+    from plan_exec import Image, check_structure, execute
+    from prefix_aware_decode_b200 import workload as wl
+    from prefix_aware_decode_b200.shard import local_batch, shard_by_root
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        roots = wl.random_tree(seed=31, n_queries=12, depth=2, shared_pages=(1, 3), leaf_tokens=(1, 40))
+        w = wl.build_workload("dp", roots, Hq=8, Hkv=2, D=64, seed=9)
+        owned = shard_by_root(w.block_table, w.kv_lens, world)
+        assert sum(len(o) for o in owned) == w.B
+        mine = owned[rank]
+        bt, kl, qq = local_batch(w.block_table, w.kv_lens, w.q, mine)
+        out = np.zeros((w.B, w.Hq, w.D))
+        lse = np.zeros((w.B, w.Hq))
+        if len(mine):
+            plan = pad.Plan(kl, bt, w.num_pages, w.Hq, w.Hkv, w.D)
+            img = Image(plan.host_image())
+            check_structure(img, kl, bt)
+            o, l = execute(img, qq, w.k_pool, w.v_pool)
+            out[mine], lse[mine] = o, l
+        t_out, t_lse = torch.from_numpy(out), torch.from_numpy(lse)
+        dist.all_reduce(t_out)
+        dist.all_reduce(t_lse)
+        if rank == 0:
+            import oracle
+            ro, rl = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+            q.put((float(np.abs(t_out.numpy() - ro).max()), float(np.abs(t_lse.numpy() - rl).max()),
+                   [len(o) for o in owned]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_sharded_batch_matches_oracle():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=240)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    err_o, err_l, sizes = q.get(timeout=5)
+    assert err_o < 1e-12 and err_l < 1e-12
+    assert all(s > 0 for s in sizes)
+
+
+def test_shard_by_root_keeps_subtrees_whole():
+    from prefix_aware_decode_b200 import workload as wl
+    from prefix_aware_decode_b200.shard import shard_by_root
+    w = wl.make_config(3, with_values=False, scale=0.25)
+    owned = shard_by_root(w.block_table, w.kv_lens, 4)
+    roots = [set(w.block_table[o, 0].tolist()) for o in owned if len(o)]
+    for i in range(len(roots)):
+        for j in range(i + 1, len(roots)):
+            assert not (roots[i] & roots[j])
+    assert sorted(np.concatenate(owned).tolist()) == list(range(w.B))
+    w5 = wl.make_config(5, with_values=False, scale=0.25)
+    owned5 = shard_by_root(w5.block_table, w5.kv_lens, 4)
+    loads = [int(w5.kv_lens[o].sum()) for o in owned5]
+    assert max(loads) <= 2 * min(loads)
