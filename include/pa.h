@@ -217,9 +217,6 @@ const char *pa_status_string(pa_status s);
  *                                             (indices counted from the first MMA seg)
  *   counters    int32[B * Hkv]                arrival counters of the fused merge (zero)
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
- *   warp_loads  int32[simt_warps + 1]         SIMT warp w loads tiles [warp_loads[w], warp_loads[w+1])
- *   tiles       int32[num_loads]              page * Hkv + kv_head of every SIMT tile load, in
- *                                             the order the warps consume them
  *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
  *                                             [prow_off[b*Hkv+g], prow_off[b*Hkv+g+1])
  *   partial_lse fp32[num_partial_rows][G]     (workspace only, not uploaded)
@@ -240,7 +237,7 @@ typedef struct {
   int32_t prow;       /* SIMT: the partial row written; MMA: index into seg_prows */
   int32_t query;      /* SIMT: the request; MMA: first request of the item */
   int32_t sole;       /* SIMT: 1 if this is the only partial row of (query, kv_head) */
-  int32_t pad;        /* 32-byte records */
+  int32_t page_start; /* index into pages of the run's first page (item page_off + page_begin) */
 } pa_seg;
 
 typedef struct {
@@ -250,10 +247,9 @@ typedef struct {
   int32_t fault_b;
   int32_t batch, num_q_heads, num_kv_heads, head_dim, page_size;
   int32_t num_items, num_segments, num_segments_simt, num_segments_mma, simt_warps;
-  int32_t num_partial_rows, num_loads;
-  int32_t mma_ctas, pad1;
+  int32_t num_partial_rows, mma_ctas;
   uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_mma_segs, off_counters, off_warp_segs,
-      off_warp_loads, off_tiles, off_prow_off;
+      off_prow_off;
   uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;
 } pa_image_header;
 

@@ -24,8 +24,6 @@ PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   d.mma_cta_segs = reinterpret_cast<const int32_t*>(b + h.off_mma_segs);
   d.counters = reinterpret_cast<int32_t*>(b + h.off_counters);
   d.warp_segs = reinterpret_cast<const int32_t*>(b + h.off_warp_segs);
-  d.warp_loads = reinterpret_cast<const int32_t*>(b + h.off_warp_loads);
-  d.tiles = reinterpret_cast<const int32_t*>(b + h.off_tiles);
   d.prow_off = reinterpret_cast<const int32_t*>(b + h.off_prow_off);
   d.partial_lse = reinterpret_cast<float*>(b + h.off_partial_lse);
   d.partial_o = reinterpret_cast<float*>(b + h.off_partial_o);

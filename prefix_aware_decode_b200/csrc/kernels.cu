@@ -49,8 +49,6 @@ struct FwdArgs {
   const int32_t* queries;
   const int32_t* seg_prows;
   const int32_t* warp_segs;
-  const int32_t* warp_loads;
-  const int32_t* tiles;
   const int32_t* mma_cta_segs;
   const int32_t* prow_off;
   int32_t* counters;
@@ -301,8 +299,8 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   if (warp >= kSimtWarpsPerCta) return;
   const int gw = (blockIdx.x - a.n_mma_ctas) * kSimtWarpsPerCta + warp;
   if (gw >= a.n_simt_warps) return;  // no block-wide barrier in this role
-  uint8_t* wbase = smem + warp * S::WARP_BYTES;
-  uint8_t* qslot = wbase + NST * S::STAGE;  // two q-row slots
+  uint8_t* wbase_smem = smem + warp * S::WARP_BYTES;
+  uint8_t* qslot = wbase_smem + NST * S::STAGE;  // two q-row slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSimtWarpsPerCta * S::WARP_BYTES) + warp * (NST + 2);
   uint64_t* qbars = bars + NST;
   if (lane == 0) {
@@ -313,28 +311,85 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
 
   const int grp = lane / LPG, li = lane % LPG;
   const int seg_begin = a.warp_segs[gw], seg_end = a.warp_segs[gw + 1];
-  const int ld_begin = a.warp_loads[gw], ld_end = a.warp_loads[gw + 1];
   const bool drop_first = a.fault_drop && gw == 0;
 
-  // ---- load side: lane 0 issues; lanes hold a sliding window of 32 tile ids
-  int ld = ld_begin;
-  int win_base = ld_begin;
-  int win_cur = ld_begin + lane < ld_end ? a.tiles[ld_begin + lane] : 0;
-  int win_nxt = ld_begin + 32 + lane < ld_end ? a.tiles[ld_begin + 32 + lane] : 0;
+  // ---- load side (lane 0 issues).  The warp's loads are the pages of its
+  // segments, in order.  Lanes hold the descriptors of a group of up to 32
+  // segments (first page index, page count, kv head) and their exclusive
+  // prefix sums; a window of 32 tile ids (page * Hkv + kv head) is filled by a
+  // per-lane binary search over the group plus one page-id load, and the next
+  // window is fetched one window ahead.
+  int sg_base = seg_begin;          // first segment of the current group
+  int sg_pstart = 0, sg_npg = 0, sg_g = 0, sg_off = 0, sg_tot = 0, sg_n = 0;
+  auto load_group = [&]() {
+    sg_n = min(32, seg_end - sg_base);
+    sg_pstart = 0;
+    sg_npg = 0;
+    sg_g = 0;
+    if (lane < sg_n) {
+      const pa_seg& sd = a.segs[sg_base + lane];
+      sg_pstart = sd.page_start;
+      sg_npg = (sd.n_tokens + 15) >> 4;
+      sg_g = sd.kv_head;
+    }
+    int incl = sg_npg;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    sg_off = incl - sg_npg;
+    sg_tot = __shfl_sync(0xffffffffu, incl, 31);
+  };
+  auto tile_for = [&](int x) -> int {  // x: page index within the group
+    int lo = 0;
+#pragma unroll
+    for (int step = 16; step > 0; step >>= 1) {
+      const int cand = lo + step;
+      const int oc = __shfl_sync(0xffffffffu, sg_off, cand & 31);
+      if (cand < sg_n && oc <= x) lo = cand;
+    }
+    const int ps = __shfl_sync(0xffffffffu, sg_pstart, lo);
+    const int o0 = __shfl_sync(0xffffffffu, sg_off, lo);
+    const int g = __shfl_sync(0xffffffffu, sg_g, lo);
+    return x < sg_tot ? a.pages[ps + (x - o0)] * a.Hkv + g : 0;
+  };
+  int ld_x = 0, wbase = 0;          // next load (within the group), current window base
+  bool ld_more = seg_begin < seg_end;
+  int win_cur = 0, win_nxt = 0;
+  if (ld_more) {
+    load_group();
+    win_cur = tile_for(lane);
+    win_nxt = tile_for(32 + lane);
+  }
   uint32_t inflight = 0;  // bit s: a copy into stage s (or q slot s - NST) is outstanding
   uint32_t parity = 0;    // bit s: parity of the next phase to wait for on barrier s
+  bool first_load = true;
 
   auto issue = [&](int stage) {
-    if (ld >= ld_end) return;
-    if (ld - win_base >= 32) {  // slide the window (warp-uniform)
-      win_base += 32;
-      win_cur = win_nxt;
-      win_nxt = win_base + 32 + lane < ld_end ? a.tiles[win_base + 32 + lane] : 0;
+    if (!ld_more) return;
+    if (ld_x >= sg_tot) {  // next group of segments (warp-uniform; only warps with > 32 segments)
+      sg_base += 32;
+      if (sg_base >= seg_end) {
+        ld_more = false;
+        return;
+      }
+      load_group();
+      ld_x = 0;
+      wbase = 0;
+      win_cur = tile_for(lane);
+      win_nxt = tile_for(32 + lane);
     }
-    const int tile = __shfl_sync(0xffffffffu, win_cur, ld - win_base);
-    const bool drop = drop_first && ld == ld_begin;
+    if (ld_x - wbase >= 32) {  // slide the window (warp-uniform)
+      wbase += 32;
+      win_cur = win_nxt;
+      win_nxt = tile_for(wbase + 32 + lane);
+    }
+    const int tile = __shfl_sync(0xffffffffu, win_cur, ld_x - wbase);
+    const bool drop = drop_first && first_load;
+    first_load = false;
     if (lane == 0 && !drop) {
-      uint8_t* st = wbase + stage * S::STAGE;
+      uint8_t* st = wbase_smem + stage * S::STAGE;
       const uint32_t bar = smem_u32(&bars[stage]);
       mbar_arrive_expect_tx(bar, 2 * S::TILE);
       const size_t off = (size_t)tile * (16 * D);
@@ -342,7 +397,8 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
       bulk_g2s(smem_u32(st + S::TILE), a.v_pool + off, S::TILE, bar);
     }
     if (!drop) inflight |= 1u << stage;
-    ++ld;
+    ++ld_x;
+    if (ld_x >= sg_tot && sg_base + 32 >= seg_end) ld_more = false;
   };
   // q rows (b, g*G .. g*G+G-1) are contiguous: q + (b*Hq + g*G)*D
   auto issue_q = [&](int slot, const SegInfo& si) {
@@ -408,7 +464,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
       }
       inflight &= ~(1u << stage);
       parity ^= 1u << stage;
-      const uint8_t* kt = wbase + stage * S::STAGE;
+      const uint8_t* kt = wbase_smem + stage * S::STAGE;
       const int nvalid = cur.n_tokens - pg * 16;
       if (nvalid >= 16) simt_page<D, G, false>(kt, kt + S::TILE, 16, grp, li, qf, o, m, l);
       else simt_page<D, G, true>(kt, kt + S::TILE, nvalid, grp, li, qf, o, m, l);
@@ -887,8 +943,6 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.queries = d.queries;
   a.seg_prows = d.seg_prows;
   a.warp_segs = d.warp_segs;
-  a.warp_loads = d.warp_loads;
-  a.tiles = d.tiles;
   a.mma_cta_segs = d.mma_cta_segs;
   a.prow_off = d.prow_off;
   a.counters = d.counters;

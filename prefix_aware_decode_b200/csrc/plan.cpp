@@ -167,7 +167,7 @@ struct Planner {
 struct Scratch {
   std::vector<int> order, npg, qbuf;
   std::vector<ItemRec> items;
-  std::vector<int32_t> pages, queries, warp_segs, warp_loads, mma_cta_segs, tiles, prow_off, cursor, seg_prows;
+  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows;
   std::vector<SegRec> simt_segs, mma_segs;
 };
 
@@ -297,7 +297,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     // boundaries (long-KV splitting without a fixed chunk size).
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 2.5e6;     // flop per us per SM, tcgen05 class (measured; split p: 1.5x the flops)
+    const double kMmaFlopsPerSmUs = 4.2e6;     // flop per us per SM, tcgen05 class (measured: ~1.47 us per 64-key stage of 128 rows)
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
     int64_t simt_pages = 0, mma_pages = 0;
@@ -327,15 +327,11 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     std::vector<SegRec>& simt_segs = sc.simt_segs;
     std::vector<SegRec>& mma_segs = sc.mma_segs;
     std::vector<int32_t>& warp_segs = sc.warp_segs;
-    std::vector<int32_t>& warp_loads = sc.warp_loads;
     std::vector<int32_t>& mma_cta_segs = sc.mma_cta_segs;
-    std::vector<int32_t>& tiles = sc.tiles;
     simt_segs.clear();
     mma_segs.clear();
     warp_segs.assign(1, 0);
-    warp_loads.assign(1, 0);
     mma_cta_segs.assign(1, 0);
-    if (tiles.size() < (size_t)simt_pages) tiles.resize((size_t)simt_pages);
     if (simt_pages > 0) {
       const int64_t W = (int64_t)(S - n_mma) * kSimtWarpsPerCta;
       int64_t span = ceil_div(simt_pages, W);
@@ -343,16 +339,12 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       if (max_chunk_pages) span = std::min(span, max_chunk_pages);
       simt_segs.reserve(items.size() * Hkv + simt_pages / span + 8);
       int64_t used = 0;  // pages in the current warp's span
-      size_t t = 0;      // tiles written
       for (size_t i = 0; i < items.size(); ++i) {
         const ItemRec& it = items[i];
         if (!it.simt) continue;
         const int npages = (int)ceil_div(it.n_tokens, P);
-        const int32_t* pp = pages.data() + it.page_off;
         const int b = queries[it.query_off];
         for (int g = 0; g < Hkv; ++g) {
-          for (int j = 0; j < npages; ++j) tiles[t + j] = pp[j] * Hkv + g;
-          t += npages;
           int pb = 0;
           while (pb < npages) {
             const int take = (int)std::min<int64_t>(npages - pb, span - used);
@@ -362,16 +354,12 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
             used += take;
             if (used == span) {
               warp_segs.push_back((int32_t)simt_segs.size());
-              warp_loads.push_back((int32_t)(t - (npages - pb)));
               used = 0;
             }
           }
         }
       }
-      if (used > 0) {
-        warp_segs.push_back((int32_t)simt_segs.size());
-        warp_loads.push_back((int32_t)t);
-      }
+      if (used > 0) warp_segs.push_back((int32_t)simt_segs.size());
     }
     if (mma_pages > 0) {
       int64_t span = ceil_div(mma_pages, n_mma);
@@ -438,7 +426,6 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.simt_warps = (int32_t)warp_segs.size() - 1;
     h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
     h.num_partial_rows = num_prows;
-    h.num_loads = (int32_t)simt_pages;
     uint64_t off = align256(sizeof(pa_image_header));
     h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
     h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
@@ -448,8 +435,6 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.off_mma_segs = off; off = align256(off + mma_cta_segs.size() * 4);
     h.off_counters = off; off = align256(off + (size_t)batch * Hkv * 4);
     h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
-    h.off_warp_loads = off; off = align256(off + warp_loads.size() * 4);
-    h.off_tiles = off; off = align256(off + (size_t)simt_pages * 4);
     h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
     h.image_bytes = off;
     h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
@@ -468,9 +453,11 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     for (const auto& s : simt_segs) {
       const size_t bg = (size_t)s.query * Hkv + s.kv_head;
       const int sole = prow_off[bg + 1] - prow_off[bg] == 1 ? 1 : 0;
-      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole, 0};
+      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
+                 items[s.item].page_off + s.page_begin};
     }
-    for (const auto& s : mma_segs) ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, 0};
+    for (const auto& s : mma_segs)
+      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, items[s.item].page_off + s.page_begin};
     auto put = [&](uint64_t o, const std::vector<int32_t>& v) {
       if (!v.empty()) std::memcpy(img + o, v.data(), v.size() * 4);
     };
@@ -479,8 +466,6 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     put(h.off_seg_prows, seg_prows);
     put(h.off_mma_segs, mma_cta_segs);
     put(h.off_warp_segs, warp_segs);
-    put(h.off_warp_loads, warp_loads);
-    if (simt_pages) std::memcpy(img + h.off_tiles, tiles.data(), (size_t)simt_pages * 4);
     put(h.off_prow_off, prow_off);
 
     pa_plan_stats& st = plan->stats;

@@ -61,8 +61,6 @@ struct PaDevPtrs {
   const int32_t* mma_cta_segs;
   int32_t* counters;
   const int32_t* warp_segs;
-  const int32_t* warp_loads;
-  const int32_t* tiles;
   const int32_t* prow_off;
   float* partial_lse;
   float* partial_o;

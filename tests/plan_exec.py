@@ -27,7 +27,10 @@ class Image:
             return a.reshape(n, cols) if cols else a
 
         self.items = arr(h.off_nodes, h.num_items, cols=4)  # page_off, n_tokens, n_queries, query_off
-        self.segs = arr(h.off_segs, h.num_segments, cols=8)[:, :6]  # item, kv_head, page_begin, n_tokens, prow, query
+        segs8 = arr(h.off_segs, h.num_segments, cols=8)
+        self.segs = segs8[:, :6]  # item, kv_head, page_begin, n_tokens, prow, query
+        self.seg_sole = segs8[:, 6]
+        self.seg_page_start = segs8[:, 7]
         n_pages = (h.off_queries - h.off_pages) // 4
         self.pages = arr(h.off_pages, n_pages)
         self.queries = arr(h.off_queries, (h.off_seg_prows - h.off_queries) // 4)
@@ -35,8 +38,6 @@ class Image:
         self.mma_segs = arr(h.off_mma_segs, h.mma_ctas + 1)
         self.counters = arr(h.off_counters, h.batch * h.num_kv_heads)
         self.warp_segs = arr(h.off_warp_segs, h.simt_warps + 1)
-        self.warp_loads = arr(h.off_warp_loads, h.simt_warps + 1)
-        self.tiles = arr(h.off_tiles, h.num_loads)
         self.prow_off = arr(h.off_prow_off, h.batch * h.num_kv_heads + 1)
 
 
@@ -51,23 +52,15 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
     else:
         assert h.mma_ctas == 0
     assert np.all(img.counters == 0)
-    # warp lists partition the SIMT segments and tiles, in order
+    # warp lists partition the SIMT segments, in order; page_start and sole are consistent
     assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
     assert np.all(np.diff(img.warp_segs) > 0) or nseg_simt == 0
-    assert img.warp_loads[0] == 0 and img.warp_loads[-1] == h.num_loads
-    # the tile list equals the pages of the SIMT segments, in order
-    t = 0
-    for w in range(h.simt_warps):
-        assert img.warp_loads[w] == t
-        for si in range(img.warp_segs[w], img.warp_segs[w + 1]):
-            item, g, pb, nt, prow, q = img.segs[si]
-            po, itok, nq, qo = img.items[item]
-            assert nq == 1 and img.queries[qo] == q
-            npg = -(-nt // P)
-            want = img.pages[po + pb: po + pb + npg] * Hkv + g
-            assert np.array_equal(img.tiles[t:t + npg], want)
-            t += npg
-    assert t == h.num_loads
+    for si in range(h.num_segments):
+        item, g, pb, nt, prow, q = img.segs[si]
+        assert img.seg_page_start[si] == img.items[item][0] + pb
+        if si < nseg_simt:
+            n_rows = img.prow_off[q * Hkv + g + 1] - img.prow_off[q * Hkv + g]
+            assert img.seg_sole[si] == (1 if n_rows == 1 else 0)
     # coverage: each (request, kv head) reads each token (page, slot) exactly once
     seen = {}
     prows_written = np.zeros(h.num_partial_rows, dtype=np.int64)
