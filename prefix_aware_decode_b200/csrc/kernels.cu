@@ -968,8 +968,14 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
   constexpr int smem_simt = SimtShape<D, G>::SMEM, smem_mma = MmaShape<D>::SMEM;
   const int smem = a.n_mma_ctas > 0 ? (smem_simt > smem_mma ? smem_simt : smem_mma) : smem_simt;
   auto k = fwd_kernel<D, G>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
-  if (e != cudaSuccess) return (int)e;
+  static bool attr_set[64] = {};  // per instantiation and device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+    if (e != cudaSuccess) return (int)e;
+    attr_set[dev] = true;
+  }
   const int grid = a.n_mma_ctas + (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
   if (grid <= 0) return 0;
   const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);

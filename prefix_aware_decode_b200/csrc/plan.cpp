@@ -318,9 +318,13 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     if (mma_pages > 0 && simt_pages == 0) {
       n_mma = S;
     } else if (mma_pages > 0) {
+      // T_simt = A / (S - k) and T_mma = C / k are equal at k = S C / (A + C);
+      // take the better of the two integers around it
+      const double A = simt_pages * tile_bytes / kSimtBytesPerSmUs, C = mma_cost;
+      const int k0 = std::max(1, std::min(S - 1, (int)(S * C / (A + C))));
       double best = 1e300;
-      for (int kk = 1; kk < S; ++kk) {
-        const double t = std::max(simt_pages * tile_bytes / ((S - kk) * kSimtBytesPerSmUs), mma_cost / kk);
+      for (int kk = k0; kk <= std::min(S - 1, k0 + 1); ++kk) {
+        const double t = std::max(A / (S - kk), C / kk);
         if (t < best) { best = t; n_mma = kk; }
       }
     }
