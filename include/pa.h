@@ -197,6 +197,31 @@ pa_status pa_decode_step(const pa_config *cfg, int32_t batch, const int32_t *kv_
                          const void *v_pool, void *d_workspace, size_t workspace_bytes, void *out, float *lse,
                          void *const *profile_events, void *stream, pa_plan **plan_out);
 
+/*
+ * pa_attend without a caller workspace, for callers that cannot allocate
+ * device memory where they run attention (inside a memory pool that forbids
+ * further allocation, an allocator-free runtime, a hook that must not touch
+ * the caching allocator).  The pages this library implements have no
+ * counterpart of this call; it is a deployment convenience.
+ *   The workspace is one static device array of 24 MiB, held by every GPU
+ *   that loads the library until the process exits.  A plan whose
+ *   pa_plan_workspace_size exceeds 24 MiB is refused with PA_ERR_NOMEM before
+ *   anything is enqueued.
+ *   Each call copies the plan image (status word and arrival counters at zero)
+ *   into the array with cudaMemcpyAsync from the plan's host memory, then runs
+ *   the fused forward there.  It calls no cudaMalloc, cudaFree, pinned-memory
+ *   allocator or other allocating routine.
+ *   Every call shares the one array and leaves the last call's contents in it:
+ *   calls that overlap on the GPU (other streams, other threads) race and
+ *   must be ordered by the caller.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ * Returns as pa_attend; the device status word is in the shared array and is
+ * not readable through pa_get_device_status.
+ */
+pa_status pa_attend_noalloc(const pa_plan *plan, const void *q, const void *k_pool, const void *v_pool, void *out,
+                            float *lse, void *stream);
+
 /* Release a plan (NULL is ignored). */
 void pa_plan_destroy(pa_plan *plan);
 

@@ -62,7 +62,7 @@ class PaImageHeader(ctypes.Structure):
 # exported names, in the order pa.h declares them
 EXPORTS = ["pa_plan_create", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
            "pa_get_device_status", "pa_plan_get_stats", "pa_plan_host_image", "pa_plan_set_profile_events",
-           "pa_decode_step", "pa_plan_destroy", "pa_status_string"]
+           "pa_decode_step", "pa_attend_noalloc", "pa_plan_destroy", "pa_status_string"]
 
 _lib = None
 
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
     L.pa_decode_step.argtypes = [ctypes.POINTER(PaConfig), i32, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp,
                                  ctypes.POINTER(vp), vp, ctypes.POINTER(vp)]
     L.pa_decode_step.restype = st
+    L.pa_attend_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+    L.pa_attend_noalloc.restype = st
     L.pa_plan_destroy.argtypes = [vp]
     L.pa_plan_destroy.restype = None
     L.pa_status_string.argtypes = [st]
@@ -217,6 +219,12 @@ class Plan:
             arr[i] = None if e is None else e.cuda_event
         _check(self._lib.pa_plan_set_profile_events(self._h, arr, len(self._prof_events)),
                "pa_plan_set_profile_events")
+
+    def attend_noalloc(self, q, k_pool, v_pool, out, lse=None, stream=None):
+        """pa_attend with the library's static device workspace (no allocation)."""
+        _check(self._lib.pa_attend_noalloc(self._h, _dptr(q, "q"), _dptr(k_pool, "k_pool"), _dptr(v_pool, "v_pool"),
+                                           _dptr(out, "out"), _dptr(lse, "lse", 4) if lse is not None else None,
+                                           _stream_ptr(stream)), "pa_attend_noalloc")
 
     def device_status(self, ws, stream=None) -> int:
         out = ctypes.c_int()

@@ -20,7 +20,7 @@ BUILD = os.path.join(REPO, "_build")
 LIB = os.path.join(HERE, "libpa.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-CU_SOURCES = ["kernels.cu", "capi.cu"]
+CU_SOURCES = ["kernels.cu", "capi.cu", "noalloc.cu"]
 CPP_SOURCES = ["plan.cpp"]
 HEADERS = ["plan.h", "ptx.cuh"]
 

@@ -213,6 +213,11 @@ extern "C" pa_status pa_attend(const pa_plan* plan, const void* q, const void* k
   return launch(plan, q, k_pool, v_pool, d_workspace, out, lse, stream);
 }
 
+pa_status pa_attend_ws(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool, void* ws,
+                       void* out, float* lse, void* stream) {
+  return pa_attend(plan, q, k_pool, v_pool, ws, out, lse, stream);
+}
+
 extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_workspace, void* stream,
                                           pa_status* out) {
   if (!plan || !d_workspace || !out) return PA_ERR_INVALID;

@@ -70,3 +70,7 @@ struct PaDevPtrs {
 // out == nullptr: partial rows only; else the merge is fused into the launch.
 int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
+
+// pa_attend on a workspace whose plan image is already (being) uploaded.
+pa_status pa_attend_ws(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool, void* ws,
+                       void* out, float* lse, void* stream);
