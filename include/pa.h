@@ -244,6 +244,8 @@ const char *pa_status_string(pa_status s);
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
  *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
  *                                             [prow_off[b*Hkv+g], prow_off[b*Hkv+g+1])
+ *   tail_pairs  int32[num_tail_pairs]         b*Hkv+g of every pair with a tensor-core
+ *                                             partial row, ascending
  *   partial_lse fp32[num_partial_rows][G]     (workspace only, not uploaded)
  *   partial_o   fp32[num_partial_rows][G][D]  (workspace only, not uploaded)
  */
@@ -261,7 +263,11 @@ typedef struct {
   int32_t n_tokens;   /* valid tokens of the run (its pages are ceil(n_tokens / P)) */
   int32_t prow;       /* SIMT: the partial row written; MMA: index into seg_prows */
   int32_t query;      /* SIMT: the request; MMA: first request of the item */
-  int32_t sole;       /* SIMT: 1 if this is the only partial row of (query, kv_head) */
+  int32_t sole;       /* SIMT, how the fused path combines this partial row of (query, kv_head):
+                       * 0: arrival counter, the last of the pair's writers merges it;
+                       * 1: it is the pair's only partial row and goes straight to the output;
+                       * 2: the pair also has tensor-core partial rows and is merged by the
+                       *    tail merge launch (tail_pairs).  MMA segments: 0. */
   int32_t page_start; /* index into pages of the run's first page (item page_off + page_begin) */
 } pa_seg;
 
@@ -273,8 +279,10 @@ typedef struct {
   int32_t batch, num_q_heads, num_kv_heads, head_dim, page_size;
   int32_t num_items, num_segments, num_segments_simt, num_segments_mma, simt_warps;
   int32_t num_partial_rows, mma_ctas;
+  int32_t num_tail_pairs; /* pairs merged by the tail launch of pa_attend / pa_decode_step */
+  int32_t reserved;
   uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_mma_segs, off_counters, off_warp_segs,
-      off_prow_off;
+      off_prow_off, off_tail_pairs;
   uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;
 } pa_image_header;
 

@@ -53,7 +53,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             if src.endswith(".cu"):
                 cmd = [cc] + ARCH + common + ["-lineinfo", "-Xptxas", "-v" if verbose else "-O3", "-c", path, "-o", obj]
             else:
-                cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-Wall", "-I", INCLUDE, "-I", CSRC,
+                cmd = ["g++", "-O3", "-std=c++17", "-fPIC", "-Wall", "-I", INCLUDE, "-I", CSRC,
                        "-I", "/usr/local/cuda/include", "-c", path, "-o", obj]
             if verbose:
                 print(" ".join(cmd), file=sys.stderr)

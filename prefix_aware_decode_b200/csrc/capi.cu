@@ -25,6 +25,7 @@ PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   d.counters = reinterpret_cast<int32_t*>(b + h.off_counters);
   d.warp_segs = reinterpret_cast<const int32_t*>(b + h.off_warp_segs);
   d.prow_off = reinterpret_cast<const int32_t*>(b + h.off_prow_off);
+  d.tail_pairs = reinterpret_cast<const int32_t*>(b + h.off_tail_pairs);
   d.partial_lse = reinterpret_cast<float*>(b + h.off_partial_lse);
   d.partial_o = reinterpret_cast<float*>(b + h.off_partial_o);
   d.status = reinterpret_cast<int32_t*>(b + offsetof(pa_image_header, status));
@@ -185,6 +186,7 @@ pa_status launch(const pa_plan* plan, const void* q, const void* k_pool, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   record_profile(*plan, 0, st);
   if (pa_launch_forward(*plan, d, out, lse, stream) != 0) return PA_ERR_CUDA;
+  if (out && plan->hdr.num_tail_pairs > 0 && pa_launch_tail_merge(*plan, d, out, lse, stream) != 0) return PA_ERR_CUDA;
   record_profile(*plan, 1, st);
   return PA_OK;
 }

@@ -65,48 +65,62 @@ struct FwdArgs {
 
 // ---------------------------------------------------------------- merge of one (request, kv head)
 
-// One warp merges the partial rows of (b, g) into out[b][g*G .. g*G+G-1][:] and
-// lse[b][...], in one online pass: lane l handles row l / (32/G) and a run of
-// D*G/32 head dims, so every load of the loop is independent of the running
-// state.  Partial rows are read through L2 (they may have been written by
-// other SMs in the same launch).
+// One warp merges the partial rows [p0, p1) of (b, g) into
+// out[b][g*G .. g*G+G-1][:] and lse[b][...]: lane l handles row l / (32/G) and
+// a run of D*G/32 head dims.  The partial rows are taken in batches of NB
+// whose loads are all issued before any is used, so a pair costs about one
+// memory round trip per NB partial rows.  Partial rows are read through L2
+// (they may have been written by other SMs in the same launch).
 template <int D, int G>
-__device__ __forceinline__ void merge_pair(const int32_t* prow_off, const float* partial_lse, const float* partial_o,
-                                           __nv_bfloat16* out, float* lse, int Hq, int Hkv, int b, int g, int lane) {
+__device__ __forceinline__ void merge_pair(const float* partial_lse, const float* partial_o, __nv_bfloat16* out,
+                                           float* lse, int Hq, int b, int g, int p0, int p1, int lane) {
   constexpr int LPR = 32 / G;   // lanes per row
   constexpr int VPL = D / LPR;  // head dims per lane
+  constexpr int NB = VPL >= 32 ? 2 : 4;
   const int r = lane / LPR, d0 = (lane % LPR) * VPL;
-  const int p0 = prow_off[b * Hkv + g], p1 = prow_off[b * Hkv + g + 1];
   float m = -INFINITY, z = 0.f, acc[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
-#pragma unroll 2
-  for (int p = p0; p < p1; ++p) {
-    const float lp = __ldcg(partial_lse + (size_t)p * G + r);
-    float o[VPL];
-    const float* src = partial_o + ((size_t)p * G + r) * D + d0;
-    if constexpr (VPL % 4 == 0) {
+  for (int pb = p0; pb < p1; pb += NB) {
+    float lp[NB], o[NB][VPL];
 #pragma unroll
-      for (int i = 0; i < VPL / 4; ++i) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + i);
-        o[4 * i] = v.x;
-        o[4 * i + 1] = v.y;
-        o[4 * i + 2] = v.z;
-        o[4 * i + 3] = v.w;
-      }
-    } else {
+    for (int k = 0; k < NB; ++k) {
+      const int p = pb + k < p1 ? pb + k : p1 - 1;  // past the end: reload the last row, weight 0
+      lp[k] = __ldcg(partial_lse + (size_t)p * G + r);
+      const float* src = partial_o + ((size_t)p * G + r) * D + d0;
+      if constexpr (VPL % 4 == 0) {
 #pragma unroll
-      for (int i = 0; i < VPL / 2; ++i) {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(src) + i);
-        o[2 * i] = v.x;
-        o[2 * i + 1] = v.y;
+        for (int i = 0; i < VPL / 4; ++i) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src) + i);
+          o[k][4 * i] = v.x;
+          o[k][4 * i + 1] = v.y;
+          o[k][4 * i + 2] = v.z;
+          o[k][4 * i + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < VPL / 2; ++i) {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(src) + i);
+          o[k][2 * i] = v.x;
+          o[k][2 * i + 1] = v.y;
+        }
       }
     }
-    const float mn = fmaxf(m, lp);
-    const float sa = m == -INFINITY ? 0.f : expf(m - mn), sb = expf(lp - mn);
-    z = z * sa + sb;
+    float mn = m;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) acc[i] = acc[i] * sa + o[i] * sb;
+    for (int k = 0; k < NB; ++k)
+      if (pb + k < p1) mn = fmaxf(mn, lp[k]);
+    const float sa = m == -INFINITY ? 0.f : expf(m - mn);
+    z *= sa;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] *= sa;
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      const float w = pb + k < p1 ? expf(lp[k] - mn) : 0.f;
+      z += w;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc[i] = fmaf(o[k][i], w, acc[i]);
+    }
     m = mn;
   }
   const float inv = 1.f / z;
@@ -125,9 +139,12 @@ __device__ __forceinline__ void arrive_and_merge(const FwdArgs& a, int bj, int n
   __threadfence();
   __syncwarp();
   bool last = false;
+  int p0 = 0, p1 = 0;
   if (lane < n) {
     const int bg = bj * a.Hkv + g;
-    last = atomicAdd(&a.counters[bg], 1) == a.prow_off[bg + 1] - a.prow_off[bg] - 1;
+    p0 = a.prow_off[bg];
+    p1 = a.prow_off[bg + 1];
+    last = atomicAdd(&a.counters[bg], 1) == p1 - p0 - 1;
   }
   unsigned todo = __ballot_sync(0xffffffffu, last);
   if (!todo) return;
@@ -136,7 +153,8 @@ __device__ __forceinline__ void arrive_and_merge(const FwdArgs& a, int bj, int n
     const int j = __ffs(todo) - 1;
     todo &= todo - 1;
     const int b = __shfl_sync(0xffffffffu, bj, j);
-    merge_pair<D, G>(a.prow_off, a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, a.Hkv, b, g, lane);
+    const int q0 = __shfl_sync(0xffffffffu, p0, j), q1 = __shfl_sync(0xffffffffu, p1, j);
+    merge_pair<D, G>(a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, b, g, q0, q1, lane);
     if (lane == j) a.counters[b * a.Hkv + g] = 0;  // ready for the next launch
   }
 }
@@ -164,11 +182,11 @@ struct SimtShape {
 
 struct SegInfo {
   int n_tokens, prow, query, kv_head;
-  bool sole;
+  int mode;  // how the fused path combines the partial row (pa_seg.sole)
 };
 
 __device__ __forceinline__ SegInfo load_seg(const pa_seg* segs, int i, int end) {
-  SegInfo r{0, 0, 0, 0, false};
+  SegInfo r{0, 0, 0, 0, 0};
   if (i < end) {
     const int4 x = *reinterpret_cast<const int4*>(segs + i);        // item, kv_head, page_begin, n_tokens
     const int4 y = *reinterpret_cast<const int4*>(&segs[i].prow);  // prow, query, sole, pad
@@ -176,7 +194,7 @@ __device__ __forceinline__ SegInfo load_seg(const pa_seg* segs, int i, int end) 
     r.kv_head = x.y;
     r.prow = y.x;
     r.query = y.y;
-    r.sole = y.z != 0;
+    r.mode = y.z;
   }
   return r;
 }
@@ -500,7 +518,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
     }
     // write: group k writes rows r with r % NG == k; a (request, kv head) with a
     // single partial row goes straight to the output when the merge is fused
-    const bool direct = a.out && cur.sole;
+    const bool direct = a.out && cur.mode == 1;
 #pragma unroll
     for (int r = 0; r < G; ++r) {
       if (r % S::NG != grp) continue;
@@ -529,7 +547,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
         if (li == 0) a.partial_lse[(size_t)cur.prow * G + r] = lse_r;
       }
     }
-    if (a.out && !direct) arrive_and_merge<D, G>(a, cur.query, 1, cur.kv_head, lane);
+    if (a.out && cur.mode == 0) arrive_and_merge<D, G>(a, cur.query, 1, cur.kv_head, lane);
     cur = nx;
     nx = nxx;
     nxx = load_seg(a.segs, si + 3, seg_end);
@@ -888,13 +906,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
               make_float4(ov[4 * c] * inv, ov[4 * c + 1] * inv, ov[4 * c + 2] * inv, ov[4 * c + 3] * inv);
         a.partial_lse[(size_t)prow * G + (r % G)] = (m_used + lg2(l)) * kLn2;
       }
-      if (a.out) {
-        // this warp's 32 rows hold whole (request, kv head) row groups (32 % G == 0)
-        const int qpw = 32 / G;
-        const int n = max(0, min(qpw, item.n_queries - quad * qpw));
-        const int bj = lane < n ? a.queries[item.query_off + quad * qpw + lane] : 0;
-        arrive_and_merge<D, G>(a, bj, n, seg.kv_head, lane);
-      }
+      // the pairs of these rows are merged by the tail merge launch
       ++segord;
     }
     if (!ok && lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, warp);
@@ -925,11 +937,15 @@ struct MergeArgs {
   int B, Hq, Hkv, G;
 };
 
+// One warp per (request, kv head) pair: every pair (list == nullptr), or the
+// n pairs b*Hkv+g listed.
 template <int D, int G>
-__global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
+__global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a, const int32_t* list, int n) {
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (w >= a.B * a.Hkv) return;
-  merge_pair<D, G>(a.prow_off, a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, a.Hkv, w / a.Hkv, w % a.Hkv, lane);
+  if (w >= n) return;
+  const int bg = list ? list[w] : w;
+  merge_pair<D, G>(a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, bg / a.Hkv, bg % a.Hkv, a.prow_off[bg],
+                   a.prow_off[bg + 1], lane);
 }
 
 FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse) {
@@ -985,8 +1001,8 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
 }
 
 template <int D, int G>
-int launch_merge_t(const MergeArgs& a, int grid, cudaStream_t st) {
-  merge_kernel<D, G><<<grid, 256, 0, st>>>(a);
+int launch_merge_t(const MergeArgs& a, const int32_t* list, int n, cudaStream_t st) {
+  merge_kernel<D, G><<<(n + 7) / 8, 256, 0, st>>>(a, list, n);
   return (int)cudaGetLastError();
 }
 
@@ -1011,7 +1027,11 @@ int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   return (int)cudaErrorInvalidValue;
 }
 
-int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
+namespace {
+
+int launch_merge_list(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, const int32_t* list, int n,
+                      void* stream) {
+  if (n <= 0) return 0;
   MergeArgs a;
   a.prow_off = d.prow_off;
   a.partial_lse = d.partial_lse;
@@ -1022,10 +1042,9 @@ int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse,
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.G = p.G;
-  const int grid = (p.B * p.Hkv + 7) / 8;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 #define PA_MERGE_CASE(DD, GG) \
-  if (p.D == DD && p.G == GG) return launch_merge_t<DD, GG>(a, grid, st);
+  if (p.D == DD && p.G == GG) return launch_merge_t<DD, GG>(a, list, n, st);
   PA_MERGE_CASE(128, 4)
   PA_MERGE_CASE(128, 1)
   PA_MERGE_CASE(128, 2)
@@ -1036,4 +1055,14 @@ int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse,
   PA_MERGE_CASE(64, 8)
 #undef PA_MERGE_CASE
   return (int)cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
+  return launch_merge_list(p, d, out, lse, nullptr, p.B * p.Hkv, stream);
+}
+
+int pa_launch_tail_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
+  return launch_merge_list(p, d, out, lse, d.tail_pairs, p.hdr.num_tail_pairs, stream);
 }

@@ -33,6 +33,16 @@ std::vector<HostBuf> g_buf_free;  // at most kMaxFreeBufs kept
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
+// First index in [from, to) where rows a and b differ (to if none): 64-byte
+// chunks compared with memcmp, then the differing chunk element by element.
+inline int first_diff(const int32_t* a, const int32_t* b, int from, int to) {
+  int i = from;
+  while (i + 16 <= to && std::memcmp(a + i, b + i, 64) == 0) i += 16;
+  for (; i < to; ++i)
+    if (a[i] != b[i]) return i;
+  return to;
+}
+
 struct ItemRec {
   int page_off, n_tokens, n_queries, query_off;
   bool simt;
@@ -108,19 +118,11 @@ struct Planner {
       add_item(b, eff_lo, npg[b], kv_lens[b] - (int64_t)eff_lo * P, &b, 1, true);
       return;
     }
-    // extend the common prefix column by column
+    // extend the common prefix: the shortest agreement of any row with the first
     const int32_t* r0 = row(order[lo]);
-    int mn = npg[order[lo]];
-    for (int i = lo + 1; i < hi; ++i) mn = std::min(mn, npg[order[i]]);
-    int l = depth;
-    while (l < mn) {
-      const int32_t v = r0[l];
-      bool same = true;
-      for (int i = lo + 1; i < hi; ++i)
-        if (row(order[i])[l] != v) { same = false; break; }
-      if (!same) break;
-      ++l;
-    }
+    int l = npg[order[lo]];
+    for (int i = lo + 1; i < hi; ++i) l = std::min(l, npg[order[i]]);
+    for (int i = lo + 1; i < hi && l > depth; ++i) l = first_diff(r0, row(order[i]), depth, l);
     bool keep = false;
     int next_eff = eff_lo;
     const int nq = hi - lo;
@@ -167,8 +169,9 @@ struct Planner {
 struct Scratch {
   std::vector<int> order, npg, qbuf;
   std::vector<ItemRec> items;
-  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows;
+  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows, tail_pairs;
   std::vector<SegRec> simt_segs, mma_segs;
+  std::vector<uint8_t> is_tail;
 };
 
 }  // namespace
@@ -264,9 +267,9 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       if (n < 1 || n > (int64_t)max_pages * P) { delete plan; return PA_ERR_INVALID; }
       pl.npg[b] = (int)ceil_div(n, P);
       total_pages += pl.npg[b];
-      const int32_t* r = block_table + (size_t)b * max_pages;
-      bool bad = false;
-      for (int j = 0; j < pl.npg[b]; ++j) bad |= (uint32_t)r[j] >= (uint32_t)num_pages_in_pool;
+      const uint32_t* r = reinterpret_cast<const uint32_t*>(block_table + (size_t)b * max_pages);
+      uint32_t bad = 0;
+      for (int j = 0; j < pl.npg[b]; ++j) bad |= r[j] >= (uint32_t)num_pages_in_pool ? 1u : 0u;
       if (bad) { delete plan; return PA_ERR_INVALID; }
     }
 
@@ -399,6 +402,17 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       const ItemRec& it = items[s.item];
       for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
     }
+    // pairs with a tensor-core partial row are merged by the tail launch (they
+    // are the MMA rows' pairs, already counted above)
+    std::vector<int32_t>& tail_pairs = sc.tail_pairs;
+    std::vector<uint8_t>& is_tail = sc.is_tail;
+    tail_pairs.clear();
+    is_tail.assign(prow_off.size() - 1, 0);
+    for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
+      if (prow_off[bg + 1] > 0) {
+        tail_pairs.push_back((int32_t)bg);
+        is_tail[bg] = 1;
+      }
     for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
     for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
     std::vector<int32_t>& cursor = sc.cursor;
@@ -430,6 +444,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.simt_warps = (int32_t)warp_segs.size() - 1;
     h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
     h.num_partial_rows = num_prows;
+    h.num_tail_pairs = (int32_t)tail_pairs.size();
     uint64_t off = align256(sizeof(pa_image_header));
     h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
     h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
@@ -440,6 +455,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.off_counters = off; off = align256(off + (size_t)batch * Hkv * 4);
     h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
     h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
+    h.off_tail_pairs = off; off = align256(off + tail_pairs.size() * 4);
     h.image_bytes = off;
     h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
     h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
@@ -456,7 +472,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     size_t k = 0;
     for (const auto& s : simt_segs) {
       const size_t bg = (size_t)s.query * Hkv + s.kv_head;
-      const int sole = prow_off[bg + 1] - prow_off[bg] == 1 ? 1 : 0;
+      const int sole = is_tail[bg] ? 2 : prow_off[bg + 1] - prow_off[bg] == 1 ? 1 : 0;
       ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
                  items[s.item].page_off + s.page_begin};
     }
@@ -471,6 +487,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     put(h.off_mma_segs, mma_cta_segs);
     put(h.off_warp_segs, warp_segs);
     put(h.off_prow_off, prow_off);
+    put(h.off_tail_pairs, tail_pairs);
 
     pa_plan_stats& st = plan->stats;
     st.batch = batch;

@@ -62,6 +62,7 @@ struct PaDevPtrs {
   int32_t* counters;
   const int32_t* warp_segs;
   const int32_t* prow_off;
+  const int32_t* tail_pairs;
   float* partial_lse;
   float* partial_o;
   int32_t* status;
@@ -70,6 +71,8 @@ struct PaDevPtrs {
 // out == nullptr: partial rows only; else the merge is fused into the launch.
 int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
+// Merge of the pairs in the plan's tail list (after a fused forward launch).
+int pa_launch_tail_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 
 // pa_attend on a workspace whose plan image is already (being) uploaded.
 pa_status pa_attend_ws(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool, void* ws,

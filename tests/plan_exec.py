@@ -39,6 +39,7 @@ class Image:
         self.counters = arr(h.off_counters, h.batch * h.num_kv_heads)
         self.warp_segs = arr(h.off_warp_segs, h.simt_warps + 1)
         self.prow_off = arr(h.off_prow_off, h.batch * h.num_kv_heads + 1)
+        self.tail_pairs = arr(h.off_tail_pairs, h.num_tail_pairs)
 
 
 def check_structure(img: Image, kv_lens, block_table, P=16):
@@ -52,7 +53,15 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
     else:
         assert h.mma_ctas == 0
     assert np.all(img.counters == 0)
-    # warp lists partition the SIMT segments, in order; page_start and sole are consistent
+    # the tail list holds exactly the pairs with a tensor-core partial row, ascending
+    mma_pairs = set()
+    for si in range(nseg_simt, h.num_segments):
+        item, g, pb, nt, prow, q = img.segs[si]
+        po, itok, nq, qo = img.items[item]
+        mma_pairs.update(int(b) * Hkv + int(g) for b in img.queries[qo: qo + nq])
+    assert list(img.tail_pairs) == sorted(mma_pairs)
+    # warp lists partition the SIMT segments, in order; page_start and the
+    # combine mode (tail merge, sole row or arrival counted) are consistent
     assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
     assert np.all(np.diff(img.warp_segs) > 0) or nseg_simt == 0
     for si in range(h.num_segments):
@@ -60,7 +69,10 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
         assert img.seg_page_start[si] == img.items[item][0] + pb
         if si < nseg_simt:
             n_rows = img.prow_off[q * Hkv + g + 1] - img.prow_off[q * Hkv + g]
-            assert img.seg_sole[si] == (1 if n_rows == 1 else 0)
+            want = 2 if int(q) * Hkv + int(g) in mma_pairs else (1 if n_rows == 1 else 0)
+            assert img.seg_sole[si] == want
+        else:
+            assert img.seg_sole[si] == 0
     # coverage: each (request, kv head) reads each token (page, slot) exactly once
     seen = {}
     prows_written = np.zeros(h.num_partial_rows, dtype=np.int64)
