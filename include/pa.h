@@ -88,6 +88,7 @@ typedef struct {
   int32_t num_partial_rows; /* partial result rows per kv head group (each holds G rows) */
   int32_t simt_warps;       /* CUDA-core class warps of the forward launch */
   int32_t mma_ctas;         /* tensor-core class CTAs of the forward launch (one per SM) */
+  int32_t num_tail_pairs;   /* (request, kv head) pairs merged by the tail merge launch */
   int64_t unique_tokens;    /* tokens of distinct tree nodes (each shared page once) */
   int64_t naive_tokens;     /* sum of kv_lens (query-centric reads) */
   int64_t read_tokens;      /* tokens the plan reads from the pools (per kv head) */

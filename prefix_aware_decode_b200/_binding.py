@@ -42,7 +42,7 @@ class PaPlanStats(ctypes.Structure):
                 ("num_kept_shared", ctypes.c_int32), ("num_items", ctypes.c_int32), ("num_segments", ctypes.c_int32),
                 ("num_segments_simt", ctypes.c_int32), ("num_segments_mma", ctypes.c_int32),
                 ("num_partial_rows", ctypes.c_int32), ("simt_warps", ctypes.c_int32), ("mma_ctas", ctypes.c_int32),
-                ("unique_tokens", ctypes.c_int64), ("naive_tokens", ctypes.c_int64), ("read_tokens", ctypes.c_int64),
+                ("num_tail_pairs", ctypes.c_int32), ("unique_tokens", ctypes.c_int64), ("naive_tokens", ctypes.c_int64), ("read_tokens", ctypes.c_int64),
                 ("unique_kv_bytes", ctypes.c_int64), ("read_kv_bytes", ctypes.c_int64),
                 ("workspace_bytes", ctypes.c_uint64), ("image_bytes", ctypes.c_uint64), ("plan_us", ctypes.c_double)]
 

@@ -3,15 +3,15 @@
 // Forward (the PAT review, section 三, Forward 阶段 and Figure 3: decode attention
 // is two GEMVs, q.K^T then p.V, fed by a tiling pipeline that streams KV tiles
 // from global memory through on-chip memory; multi-tile kernels with a runtime
-// tile selector; long KV is split).  One persistent launch with one CTA per
-// SM; the planner gives every CTA one of two tile classes, chosen by the rows
-// of its work units (requests x G query heads), and splits the SMs between the
-// classes so that both finish together (the pages' multi-stream execution,
-// done here as concurrent CTA roles inside one launch):
+// tile selector; long KV is split).  The planner gives every work unit one of
+// two tile classes, chosen by its rows (requests x G query heads), and splits
+// the SMs between the classes so that both finish together; the two classes
+// are two launches of one CTA per SM that run side by side (the pages'
+// multi-stream execution, done here with programmatic dependent launch):
 //   - MMA class: work units with two or more requests, up to 128 rows, on the
 //     5th-generation tensor cores: a producer warp streams 64-key stages with
-//     2-D TMA copies (128-byte swizzle), one thread issues tcgen05.mma with the
-//     accumulators in tensor memory, and 4 warps run the softmax.
+//     2-D TMA copies (128-byte swizzle), one thread issues tcgen05.mma with S,
+//     P and the accumulators in tensor memory, and 8 warps run the softmax.
 //   - SIMT class: work units of one request (G <= 8 rows).  Each of 8 warps
 //     streams its own run of (page, kv head) tiles with 1-D bulk copies into a
 //     private shared-memory ring and computes on the CUDA cores with packed
@@ -315,7 +315,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   constexpr int NST = S::NST, LPG = S::LPG, CPL = S::CPL;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp >= kSimtWarpsPerCta) return;
-  const int gw = (blockIdx.x - a.n_mma_ctas) * kSimtWarpsPerCta + warp;
+  const int gw = blockIdx.x * kSimtWarpsPerCta + warp;
   if (gw >= a.n_simt_warps) return;  // no block-wide barrier in this role
   uint8_t* wbase_smem = smem + warp * S::WARP_BYTES;
   uint8_t* qslot = wbase_smem + NST * S::STAGE;  // two q-row slots
@@ -561,24 +561,31 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
 
 // ---------------------------------------------------------------- MMA class (tcgen05 + TMEM)
 //
-// One CTA per SM runs a list of segments (item of <= 128 rows, kv head g, key
-// range).  Warp 0: TMA producer of 64-key K/V stages.  Warp 1: TMEM owner and
-// single-thread tcgen05.mma issuer.  Warps 2-5: softmax, one tile row (TMEM
-// lane) per thread.  Per 64-key stage i:
-//   S(i) = Q K^T          -> TMEM (double-buffered, 64 columns each)
-//   p = exp2(s - m)       -> P = P_hi + P_lo, two bf16 matrices in swizzled
-//                            shared memory (P_lo = bf16(p - P_hi), so P keeps
-//                            about 16 significant bits instead of 8)
-//   O += P_hi V + P_lo V  -> TMEM (D columns)
-// S(i+1) is issued before P(i) is ready, so the tensor core overlaps the
-// softmax.  The running maximum is only raised (and O rescaled in TMEM) when a
-// row's maximum grows by more than 2^8; the final normalisation uses the same
-// maximum for numerator and denominator, so the result is unchanged.
+// Its own launch of one CTA per SM, each running a list of segments (item of
+// <= 128 rows, kv head g, key range).  Warp 0: TMA producer of 64-key K/V
+// stages.  Warp 1: TMEM owner and single-thread tcgen05.mma issuer.  Warps
+// 2-9: softmax, two threads per tile row (TMEM lane): warps 2-5 take keys
+// 0-31 of every stage, warps 6-9 keys 32-63, each half with its own running
+// maximum, sum and accumulator, so the halves never wait on each other inside
+// a segment; the two partial results are combined once per segment.  Per
+// 64-key stage i (S/P buffer i % 3 in TMEM):
+//   S(i) = Q K^T                  -> TMEM, 64 columns
+//   p = exp2(s - m)               -> P = P_hi + P_lo, two bf16 matrices written
+//                                    over S(i) in TMEM (P_lo = p - P_hi, both
+//                                    truncated, so P keeps about 15 bits)
+//   O_h += P_hi,h V_h + P_lo,h V_h  (A operand read from TMEM)
+// S(i+1) is issued before p.V(i), so the tensor core overlaps the softmax; a
+// buffer is reused for S(i+3) only after p.V(i) has completed.  A half's
+// running maximum is only raised (and O_h rescaled in TMEM) when it grows by
+// more than 2^8; numerator and denominator use the same maximum, so the result
+// is unchanged.
 
-constexpr int kMmaKT = 64;          // keys per stage (4 pages)
-constexpr int kMmaNST = 4;          // K/V stages in flight
-constexpr int kMmaWarps = 6;        // producer, MMA issuer, 4 softmax warps
-constexpr uint32_t kTmemCols = 256; // S x 2 (64 columns each) + O (<= 128 columns)
+constexpr int kMmaKT = 64;           // keys per stage (4 pages)
+constexpr int kMmaWarps = 10;        // producer, MMA issuer, 8 softmax warps
+constexpr int kMmaThreads = kMmaWarps * 32;
+constexpr int kSmaxThreads = 256;    // softmax threads (two per tile row)
+constexpr int kSBufs = 3;            // S/P buffers in TMEM
+constexpr uint32_t kTmemCols = 512;  // the whole tensor memory of the SM (one CTA per SM)
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
 template <int D>
@@ -587,19 +594,24 @@ struct MmaShape {
   static constexpr int KBLK = kMmaKT * 128;        // one 64-key x 64-dim swizzled block (8 KB)
   static constexpr int STAGE = 2 * HALVES * KBLK;  // K and V of one stage
   static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
-  static constexpr int OFF_Q = kMmaNST * STAGE;
-  static constexpr int OFF_P = OFF_Q + HALVES * QBLK;  // 2 buffers x (P_hi, P_lo at + PBLK)
-  static constexpr int PBLK = 128 * 128;
-  static constexpr int OFF_BAR = OFF_P + 4 * PBLK;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
-  static_assert(SMEM <= kSmemMax, "MMA ring does not fit");
+  static constexpr int FIXED = HALVES * QBLK + 512 + 1024;  // Q, barriers, alignment slack
+  static constexpr int NST_FIT = (kSmemMax - FIXED) / STAGE;
+  static constexpr int NST = NST_FIT < 8 ? NST_FIT : 8;  // K/V stages in flight
+  static constexpr int OFF_Q = NST * STAGE;
+  static constexpr int OFF_BAR = OFF_Q + HALVES * QBLK;
+  static constexpr int SMEM = OFF_BAR + 512 + 1024;
+  // barriers: K/V full / empty per stage; S full, P full, p.V done per buffer;
+  // Q loaded; O read out; all MMAs retired; the two halves of each lane
+  // quarter have exchanged (m, l)
+  static constexpr int B_FULL = 0, B_EMPTY = NST, B_SFULL = 2 * NST, B_PFULL = B_SFULL + kSBufs,
+                       B_PV = B_PFULL + kSBufs, B_QFULL = B_PV + kSBufs, B_OFREE = B_QFULL + 1, B_DONE = B_OFREE + 1,
+                       B_XCH = B_DONE + 1, NBARS = B_XCH + 4;
+  // tensor memory columns: S/P buffers, the two half accumulators, (m, l) exchange
+  static constexpr uint32_t T_S = 0, T_O = kSBufs * kMmaKT, T_X = T_O + 2 * D;
+  static_assert(NST >= 3 && SMEM <= kSmemMax, "MMA ring does not fit");
+  static_assert(NBARS * 8 + 8 <= 512, "barrier area");
+  static_assert(T_X + 4 <= kTmemCols, "tensor memory plan does not fit");
 };
-
-// Barriers: K/V stage full / empty; S buffer full / free (x2); P buffer full
-// and p.V done (x2, one per P buffer, so no wait can fall two phases behind);
-// Q loaded; O read out; all MMAs retired.
-enum : int { kBarFull = 0, kBarEmpty = 4, kBarSFull = 8, kBarSFree = 10, kBarPFull = 12, kBarOFull = 14,
-             kBarQFull = 16, kBarOFree = 17, kBarDone = 18, kNumBars = 19 };
 
 // All lanes wait; the warp fails together if any lane timed out.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -611,31 +623,30 @@ template <int D, int G>
 __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
                                          uint8_t* smem_raw) {
   using S = MmaShape<D>;
+  constexpr int NST = S::NST;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::NBARS);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s_begin = a.n_segs_simt + a.mma_cta_segs[blockIdx.x];
   const int s_end = a.n_segs_simt + a.mma_cta_segs[blockIdx.x + 1];
-  const uint32_t q_base = smem_u32(smem + S::OFF_Q), p_base = smem_u32(smem + S::OFF_P);
+  const uint32_t q_base = smem_u32(smem + S::OFF_Q);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kMmaNST; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar(S::B_FULL + s), 1);
+      mbar_init(bar(S::B_EMPTY + s), 1);
     }
-    mbar_init(bar(kBarSFull), 1);
-    mbar_init(bar(kBarSFull + 1), 1);
-    mbar_init(bar(kBarSFree), 128);
-    mbar_init(bar(kBarSFree + 1), 128);
-    mbar_init(bar(kBarPFull), 128);
-    mbar_init(bar(kBarPFull + 1), 128);
-    mbar_init(bar(kBarOFull), 1);
-    mbar_init(bar(kBarOFull + 1), 1);
-    mbar_init(bar(kBarQFull), 128);
-    mbar_init(bar(kBarOFree), 128);
-    mbar_init(bar(kBarDone), 1);
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(bar(S::B_SFULL + b), 1);
+      mbar_init(bar(S::B_PFULL + b), kSmaxThreads);
+      mbar_init(bar(S::B_PV + b), 1);
+    }
+    mbar_init(bar(S::B_QFULL), kSmaxThreads);
+    mbar_init(bar(S::B_OFREE), kSmaxThreads);
+    mbar_init(bar(S::B_DONE), 1);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(S::B_XCH + q), 64);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -643,7 +654,6 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 128;
 
   if (warp == 0) {
     // ---------------- TMA producer: every stage of every segment of this CTA, in
@@ -669,8 +679,8 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           wcur = wnxt;
           wnxt = wbase + 32 + lane < npages ? pg[wbase + 32 + lane] : 0;
         }
-        const int s = i % kMmaNST;
-        if (i >= kMmaNST && !warp_wait(bar(kBarEmpty + s), ((i / kMmaNST) - 1) & 1, a.timeout_ns)) {
+        const int s = i % NST;
+        if (i >= NST && !warp_wait(bar(S::B_EMPTY + s), ((i / NST) - 1) & 1, a.timeout_ns)) {
           if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -2);
           ok = false;
           break;
@@ -682,7 +692,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           rows[pp] = (__shfl_sync(0xffffffffu, wcur, (st - wbase + pp) & 31) * a.Hkv + seg.kv_head) * 16;
         if (a.fault_drop && blockIdx.x == 0 && i == 0) continue;  // test: this stage never arrives
         if (lane == 0) {
-          const uint32_t fb = bar(kBarFull + s);
+          const uint32_t fb = bar(S::B_FULL + s);
           mbar_arrive_expect_tx(fb, (uint32_t)np * 2 * 16 * D * 2);
           uint8_t* kst = smem + s * S::STAGE;
           uint8_t* vst = kst + S::HALVES * S::KBLK;
@@ -694,13 +704,13 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             }
           }
         }
-        lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / kMmaNST) & 1) << s);
+        lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / NST) & 1) << s);
         any |= 1u << s;
       }
     }
     if (lane == 0)
-      for (int s = 0; s < kMmaNST; ++s)
-        if (any & (1u << s)) mbar_wait_bounded(bar(kBarFull + s), (lastpar >> s) & 1u, a.timeout_ns);
+      for (int s = 0; s < NST; ++s)
+        if (any & (1u << s)) mbar_wait_bounded(bar(S::B_FULL + s), (lastpar >> s) & 1u, a.timeout_ns);
   } else if (warp == 1) {
     // ---------------- tcgen05.mma issuer (one thread)
     if (lane == 0) {
@@ -711,31 +721,35 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       bool have_prev = false, ok = true;
       int i = 0, segord = 0;
       auto do_pv = [&](const Prev& pv, int j) -> bool {
-        if (!mbar_wait_bounded(bar(kBarPFull + (j & 1)), (j >> 1) & 1, a.timeout_ns)) return false;
-        if (pv.first && pv.segord >= 1 && !mbar_wait_bounded(bar(kBarOFree), (pv.segord - 1) & 1, a.timeout_ns))
+        const int b = j % kSBufs;
+        if (!mbar_wait_bounded(bar(S::B_PFULL + b), (j / kSBufs) & 1, a.timeout_ns)) return false;
+        // the first p.V of a segment overwrites O: the previous epilogue must have read it
+        if (pv.first && pv.segord >= 1 && !mbar_wait_bounded(bar(S::B_OFREE), (pv.segord - 1) & 1, a.timeout_ns))
           return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(smem + pv.s * S::STAGE + S::HALVES * S::KBLK);
-        const uint32_t pb = p_base + (j & 1) * 2 * S::PBLK;
-        for (int kk = 0; kk < pv.np; ++kk) {
-          // P: K-major, 64 keys = one 128-byte swizzle atom per row; V: MN-major
-          // (64-dim atoms at +KBLK, 8-key groups at +1 KB), 16 keys per MMA
-          const uint64_t bd = umma_sdesc_sw128(v_base + kk * 2048, S::KBLK >> 4, 64);
-          umma_bf16(tO, umma_sdesc_sw128(pb + kk * 32, 1, 64), bd, idesc_o, (pv.first && kk == 0) ? 0u : 1u);
-          umma_bf16(tO, umma_sdesc_sw128(pb + S::PBLK + kk * 32, 1, 64), bd, idesc_o, 1u);
+        for (int c = 0; c < pv.np; ++c) {
+          // 16-key chunk c (page c of the stage) belongs to key half c / 2.  P
+          // chunk c: P_hi in columns [16c, 16c + 8), P_lo in [16c + 8, 16c + 16)
+          // of the buffer; V: MN-major (64-dim atoms at +KBLK, 8-key groups at +1 KB)
+          const uint32_t d_o = tmem + S::T_O + (c >> 1) * D;
+          const uint32_t a_p = tmem + S::T_S + b * kMmaKT + 16 * c;
+          const uint64_t bd = umma_sdesc_sw128(v_base + c * 2048, S::KBLK >> 4, 64);
+          umma_bf16_ts(d_o, a_p, bd, idesc_o, (pv.first && (c & 1) == 0) ? 0u : 1u);
+          umma_bf16_ts(d_o, a_p + 8, bd, idesc_o, 1u);
         }
-        umma_commit(bar(kBarOFull + (j & 1)));
-        umma_commit(bar(kBarEmpty + pv.s));
+        umma_commit(bar(S::B_PV + b));
+        umma_commit(bar(S::B_EMPTY + pv.s));
         return true;
       };
       for (int si = s_begin; si < s_end && ok; ++si) {
         const int npages = (a.segs[si].n_tokens + 15) >> 4;
         for (int st = 0; st < npages; st += 4, ++i) {
-          const int s = i % kMmaNST;
+          const int s = i % NST, b = i % kSBufs;
           const bool first = st == 0;
-          if (!mbar_wait_bounded(bar(kBarFull + s), (i / kMmaNST) & 1, a.timeout_ns) ||
-              (first && !mbar_wait_bounded(bar(kBarQFull), segord & 1, a.timeout_ns)) ||
-              (i >= 2 && !mbar_wait_bounded(bar(kBarSFree + (i & 1)), ((i >> 1) - 1) & 1, a.timeout_ns))) {
+          if (!mbar_wait_bounded(bar(S::B_FULL + s), (i / NST) & 1, a.timeout_ns) ||
+              (first && !mbar_wait_bounded(bar(S::B_QFULL), segord & 1, a.timeout_ns)) ||
+              (i >= kSBufs && !mbar_wait_bounded(bar(S::B_PV + b), ((i / kSBufs) - 1) & 1, a.timeout_ns))) {
             ok = false;
             break;
           }
@@ -746,9 +760,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             // Q and K: K-major 128-byte swizzle, 64-dim blocks, 8-row groups at +1 KB
             const uint64_t ad = umma_sdesc_sw128(q_base + (kk >> 2) * S::QBLK + (kk & 3) * 32, 1, 64);
             const uint64_t bd = umma_sdesc_sw128(k_base + (kk >> 2) * S::KBLK + (kk & 3) * 32, 1, 64);
-            umma_bf16(tmem + (i & 1) * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem + S::T_S + b * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
-          umma_commit(bar(kBarSFull + (i & 1)));
+          umma_commit(bar(S::B_SFULL + b));
           if (have_prev && !do_pv(prev, i - 1)) {
             ok = false;
             break;
@@ -761,14 +775,17 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       if (ok && have_prev) ok = do_pv(prev, i - 1);
       if (!ok) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -3);
       // every MMA issued by this thread has completed before TMEM is released
-      umma_commit(bar(kBarDone));
-      mbar_wait_bounded(bar(kBarDone), 0, a.timeout_ns);
+      umma_commit(bar(S::B_DONE));
+      mbar_wait_bounded(bar(S::B_DONE), 0, a.timeout_ns);
     }
-  } else if (warp < kMmaWarps) {
-    // ---------------- softmax: thread = tile row = TMEM lane
+  } else {
+    // ---------------- softmax: thread = (tile row = TMEM lane, key half)
+    const int h = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
+    const int tid = (warp - 2) * 32 + lane;  // 0 .. 255
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    constexpr int QCH = D / 16;  // 16-byte q chunks per row loaded by each half
     bool ok = true;
     int i = 0, segord = 0;
     auto load_q = [&](int si) {
@@ -781,12 +798,13 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         src = a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
       }
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
+      for (int cc = 0; cc < QCH; ++cc) {
+        const int c = h * QCH + cc;
         const uint4 v = src ? *reinterpret_cast<const uint4*>(src + 8 * c) : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(smem + S::OFF_Q + (c >> 3) * S::QBLK + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
-      mbar_arrive(bar(kBarQFull));
+      mbar_arrive(bar(S::B_QFULL));
     };
     if (s_begin < s_end) load_q(s_begin);
     for (int si = s_begin; si < s_end && ok; ++si) {
@@ -796,52 +814,47 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const int npages = (seg.n_tokens + 15) >> 4;
       float m_used = -INFINITY, l = 0.f;
       for (int st = 0; st < npages; st += 4, ++i) {
-        const int s = i % kMmaNST;
+        const int s = i % NST, b = i % kSBufs;
         const int np = min(4, npages - st);
         const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
-        if (!warp_wait(bar(kBarSFull + (i & 1)), (i >> 1) & 1, a.timeout_ns)) { ok = false; break; }
+        const int kv_h = max(0, min(32, kvalid - 32 * h));  // valid keys of this half
+        if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        float sv[kMmaKT];
-        tmem_ld32(tmem + (i & 1) * kMmaKT + lane_off, *reinterpret_cast<float(*)[32]>(&sv[0]));
-        tmem_ld32(tmem + (i & 1) * kMmaKT + 32 + lane_off, *reinterpret_cast<float(*)[32]>(&sv[32]));
+        const uint32_t t_s = tmem + S::T_S + b * kMmaKT + 32 * h + lane_off;
+        float sv[32];
+        tmem_ld32(t_s, sv);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(kBarSFree + (i & 1)));
         // all S products of this segment are done: Q may be replaced by the next segment's
         if (st + 4 >= npages && si + 1 < s_end) load_q(si + 1);
-        float mx8[8];
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (kv_h == 32) {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) mx8[t] = -INFINITY;
+          for (int j = 0; j < 32; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < kMmaKT; ++j) {
-          sv[j] = j < kvalid ? sv[j] * a.qscale : -INFINITY;
-          mx8[j & 7] = fmaxf(mx8[j & 7], sv[j]);
+          for (int j = 0; j < 32; ++j)
+            if (j < kv_h) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float mnew = fmaxf(m_used, mx);
-        // P buffer i%2 is free once p.V of stage i-2 is done
-        if (i >= 2) {
-          if (!warp_wait(bar(kBarOFull + (i & 1)), ((i >> 1) - 1) & 1, a.timeout_ns)) { ok = false; break; }
-          tc_fence_after();
-        }
+        const float mraw = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float mnew = fmaxf(m_used, mraw == -INFINITY ? -INFINITY : mraw * a.qscale);
         if (st == 0) {
           m_used = mnew;
         } else {
           const bool need = mnew > m_used + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
-            // O must hold every earlier p.V product before it is rescaled
-            if (!warp_wait(bar(kBarOFull + ((i - 1) & 1)), ((i - 1) >> 1) & 1, a.timeout_ns)) { ok = false; break; }
+            // O_h must hold every earlier p.V product before it is rescaled
+            const int j = i - 1;
+            if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
             tc_fence_after();
             const float alpha = need ? ex2(m_used - mnew) : 1.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               float ov[32];
-              tmem_ld32(tO + lane_off + 32 * c, ov);
+              tmem_ld32(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) ov[j] *= alpha;
-              tmem_st32(tO + lane_off + 32 * c, ov);
+              for (int jj = 0; jj < 32; ++jj) ov[jj] *= alpha;
+              tmem_st32(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
             }
             tmem_wait_st();
             if (need) {
@@ -851,61 +864,92 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           }
         }
         const float ms = m_used == -INFINITY ? 0.f : m_used;
-        uint32_t ph[kMmaKT / 2], pl[kMmaKT / 2];
-        float l8[8];
+        // p, and its split P_hi + P_lo: P_hi keeps the top 16 bits of p (a
+        // truncated bf16), P_lo the top 16 bits of the exact remainder p - P_hi
+        float pw[32];
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int t = 0; t < 8; ++t) l8[t] = 0.f;
-#pragma unroll
-        for (int j = 0; j < kMmaKT / 2; ++j) {
-          const float p0 = ex2(sv[2 * j] - ms), p1 = ex2(sv[2 * j + 1] - ms);
-          l8[j & 7] += p0 + p1;
-          ph[j] = pack_bf16x2(p0, p1);
-          const float2 h = bf16x2_to_f2(ph[j]);
-          pl[j] = pack_bf16x2(p0 - h.x, p1 - h.y);
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = (2 * j < kv_h) ? ex2(fmaf(sv[2 * j], a.qscale, -ms)) : 0.f;
+          const float p1 = (2 * j + 1 < kv_h) ? ex2(fmaf(sv[2 * j + 1], a.qscale, -ms)) : 0.f;
+          l4[j & 3] += p0 + p1;
+          const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+          const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
+          const int w = (j >> 3) * 16 + (j & 7);
+          pw[w] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
+          pw[w + 8] = __uint_as_float(__byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632));
         }
-        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int off = S::OFF_P + (i & 1) * 2 * S::PBLK + r * 128 + ((c ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(smem + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-          *reinterpret_cast<uint4*>(smem + off + S::PBLK) =
-              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-        }
+        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        tmem_st32(t_s, pw);
         if (kvalid < np * 16) {
           // V rows past the last valid key may hold NaN; p = 0 there but 0 * NaN
           // would still poison the product, so those rows are zeroed
           uint8_t* vst = smem + s * S::STAGE + S::HALVES * S::KBLK;
           const int nz = np * 16 - kvalid;
-          for (int idx = r; idx < nz * S::HALVES * 8; idx += 128) {
+          for (int idx = tid; idx < nz * S::HALVES * 8; idx += kSmaxThreads) {
             const int row = kvalid + idx / (S::HALVES * 8);
-            const int h = (idx >> 3) % S::HALVES, c = idx & 7;
-            *reinterpret_cast<uint4*>(vst + h * S::KBLK + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            const int hh = (idx >> 3) % S::HALVES, c = idx & 7;
+            *reinterpret_cast<uint4*>(vst + hh * S::KBLK + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull + (i & 1)));
+        mbar_arrive(bar(S::B_PFULL + b));
       }
       if (!ok) break;
-      // epilogue: O row from TMEM, normalised, as this segment's partial row
-      if (!warp_wait(bar(kBarOFull + ((i - 1) & 1)), ((i - 1) >> 1) & 1, a.timeout_ns)) { ok = false; break; }
+      // ---- epilogue: combine the two key halves of each row; this thread
+      // writes head dims [h * D/2, (h + 1) * D/2) of the row's partial result
+      {
+        const int j = i - 1;
+        if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
+      }
       tc_fence_after();
-      float ov[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + lane_off + 32 * c, *reinterpret_cast<float(*)[32]>(&ov[32 * c]));
-      tmem_wait_ld();
+      {
+        const uint32_t mine[2] = {__float_as_uint(m_used), __float_as_uint(l)};
+        tmem_st2(tmem + S::T_X + 2 * h + lane_off, mine);
+        tmem_wait_st();
+      }
       tc_fence_before();
-      mbar_arrive(bar(kBarOFree));
+      mbar_arrive(bar(S::B_XCH + quad));
+      if (!warp_wait(bar(S::B_XCH + quad), segord & 1, a.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t other[2];
+      tmem_ld2(tmem + S::T_X + 2 * (1 - h) + lane_off, other);
+      tmem_wait_ld();
+      const float m0 = h == 0 ? m_used : __uint_as_float(other[0]), l0 = h == 0 ? l : __uint_as_float(other[1]);
+      const float m1 = h == 0 ? __uint_as_float(other[0]) : m_used, l1 = h == 0 ? __uint_as_float(other[1]) : l;
+      const float mm = fmaxf(m0, m1);
+      const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
+      const float L = w0 * l0 + w1 * l1;
+      const float c0 = w0 / L, c1 = w1 / L;
+      float* dst = nullptr;
       if (r < R) {
         const int prow = a.seg_prows[seg.prow + r / G];
-        float* dst = a.partial_o + ((size_t)prow * G + (r % G)) * D;
-        const float inv = 1.f / l;
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c)
-          *reinterpret_cast<float4*>(dst + 4 * c) =
-              make_float4(ov[4 * c] * inv, ov[4 * c + 1] * inv, ov[4 * c + 2] * inv, ov[4 * c + 3] * inv);
-        a.partial_lse[(size_t)prow * G + (r % G)] = (m_used + lg2(l)) * kLn2;
+        dst = a.partial_o + ((size_t)prow * G + (r % G)) * D + h * (D / 2);
+        if (h == 0) a.partial_lse[(size_t)prow * G + (r % G)] = (mm + lg2(L)) * kLn2;
       }
+#pragma unroll
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const uint32_t col = h * (D / 2) + 32 * cc;
+        float o0[32], o1[32];
+        tmem_ld32(tmem + S::T_O + col + lane_off, o0);
+        tmem_ld32(tmem + S::T_O + D + col + lane_off, o1);
+        tmem_wait_ld();
+        if (dst) {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float4 v;
+            v.x = c0 * o0[4 * q4] + (w1 > 0.f ? c1 * o1[4 * q4] : 0.f);
+            v.y = c0 * o0[4 * q4 + 1] + (w1 > 0.f ? c1 * o1[4 * q4 + 1] : 0.f);
+            v.z = c0 * o0[4 * q4 + 2] + (w1 > 0.f ? c1 * o1[4 * q4 + 2] : 0.f);
+            v.w = c0 * o0[4 * q4 + 3] + (w1 > 0.f ? c1 * o1[4 * q4 + 3] : 0.f);
+            *reinterpret_cast<float4*>(dst + 32 * cc + 4 * q4) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(S::B_OFREE));
       // the pairs of these rows are merged by the tail merge launch
       ++segord;
     }
@@ -917,15 +961,24 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
   if (warp == 1) tmem_free(tmem, kTmemCols);
 }
 
-// One persistent launch, one CTA per SM: CTAs [0, n_mma_ctas) run the
-// tensor-core class (warps 0-5; warps 6-7 only join the CTA barriers), the
-// others the CUDA-core class (8 warps).
+// Tensor-core class: CTA c runs MMA CTA list c.  It lets the CUDA-core launch
+// that follows it in the stream start at once (programmatic dependent launch).
 template <int D, int G>
-__global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1)
-    fwd_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    mma_fwd_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+  griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem[];
-  if ((int)blockIdx.x < a.n_mma_ctas) mma_role<D, G>(a, &tk, &tv, smem);
-  else simt_role<D, G>(a, smem);
+  mma_role<D, G>(a, &tk, &tv, smem);
+}
+
+// CUDA-core class: block c runs SIMT warps [8c, 8c + 8).  When it runs beside
+// a tensor-core launch it does not end before that launch has, so work later
+// in the stream sees both.
+template <int D, int G>
+__global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1) simt_fwd_kernel(const FwdArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  simt_role<D, G>(a, smem);
+  griddep_wait();
 }
 
 struct MergeArgs {
@@ -979,25 +1032,50 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   return a;
 }
 
-template <int D, int G>
-int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
-  constexpr int smem_simt = SimtShape<D, G>::SMEM, smem_mma = MmaShape<D>::SMEM;
-  const int smem = a.n_mma_ctas > 0 ? (smem_simt > smem_mma ? smem_simt : smem_mma) : smem_simt;
-  auto k = fwd_kernel<D, G>;
-  static bool attr_set[64] = {};  // per instantiation and device
+// Max dynamic shared memory is set once per kernel and device.
+template <typename K>
+int set_smem_attr(K kernel, bool (&done)[64]) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+  if (!done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
     if (e != cudaSuccess) return (int)e;
-    attr_set[dev] = true;
+    done[dev] = true;
   }
-  const int grid = a.n_mma_ctas + (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
-  if (grid <= 0) return 0;
-  const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
-  const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
-  k<<<grid, kSimtWarpsPerCta * 32, smem, st>>>(a, *tk, *tv);
-  return (int)cudaGetLastError();
+  return 0;
+}
+
+// The tensor-core launch (if any) first, then the CUDA-core launch, which may
+// start while the first still runs (programmatic stream serialization); the
+// two occupy disjoint SMs (one CTA per SM each, n_mma + n_simt <= SMs).
+template <int D, int G>
+int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
+  static bool attr_mma[64] = {}, attr_simt[64] = {};
+  const int n_simt_ctas = (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
+  if (a.n_mma_ctas > 0) {
+    auto k = mma_fwd_kernel<D, G>;
+    if (int e = set_smem_attr(k, attr_mma)) return e;
+    const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
+    const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
+    k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D>::SMEM, st>>>(a, *tk, *tv);
+    if (cudaError_t e = cudaGetLastError()) return (int)e;
+  }
+  if (n_simt_ctas > 0) {
+    auto k = simt_fwd_kernel<D, G>;
+    if (int e = set_smem_attr(k, attr_simt)) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_simt_ctas);
+    cfg.blockDim = dim3(kSimtWarpsPerCta * 32);
+    cfg.dynamicSmemBytes = SimtShape<D, G>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.n_mma_ctas > 0 ? 1 : 0;
+    if (cudaError_t e = cudaLaunchKernelEx(&cfg, k, a)) return (int)e;
+  }
+  return 0;
 }
 
 template <int D, int G>

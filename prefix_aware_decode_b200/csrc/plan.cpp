@@ -501,6 +501,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     st.num_partial_rows = num_prows;
     st.simt_warps = h.simt_warps;
     st.mma_ctas = h.mma_ctas;
+    st.num_tail_pairs = h.num_tail_pairs;
     st.unique_tokens = pl.unique_tokens;
     int64_t naive = 0;
     for (int b = 0; b < batch; ++b) naive += kv_lens[b];
