@@ -186,9 +186,17 @@ pa_status pa_plan_host_image(const pa_plan *plan, void *dst, size_t bytes);
 pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t n);
 
 /*
- * One decode step in one call: pa_plan_create, pa_plan_upload and pa_attend
- * (forward with the merge fused) on `stream`.  workspace_bytes must cover the
- * plan's workspace (pa_plan_workspace_size of a plan of the same batch).
+ * One decode step in one call: pa_plan_create, the upload of the plan image and
+ * pa_attend (forward with the merge fused) on `stream`.  workspace_bytes must
+ * cover the plan's workspace (pa_plan_workspace_size of a plan of the same
+ * batch); the workspace holds the partial rows.  The image itself goes to one
+ * of two device slots that the library owns per device (allocated on first use
+ * and grown when a larger image comes, the only device allocation of this
+ * call), copied on a stream of the library's own: the copy for step k+1 runs
+ * while the kernels of step k do, and `stream` waits for it (an event) before
+ * its launches.  A slot is refilled only after the launches that read it have
+ * completed.  The device status word of the step is in its slot: read it with
+ * pa_get_device_status on the plan returned through plan_out.
  * profile_events: NULL, or four cudaEvent_t as for pa_plan_set_profile_events.
  * plan_out: NULL (the plan is released before returning; its upload has
  * already been staged) or receives the plan, which the caller then releases.
@@ -245,8 +253,8 @@ const char *pa_status_string(pa_status s);
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
  *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
  *                                             [prow_off[b*Hkv+g], prow_off[b*Hkv+g+1])
- *   tail_pairs  int32[num_tail_pairs]         b*Hkv+g of every pair with a tensor-core
- *                                             partial row, ascending
+ *   tail_pairs  int32[num_tail_pairs]         b*Hkv+g of every pair whose partial rows are
+ *                                             all tensor-core rows, ascending
  *   partial_lse fp32[num_partial_rows][G]     (workspace only, not uploaded)
  *   partial_o   fp32[num_partial_rows][G][D]  (workspace only, not uploaded)
  */
@@ -264,11 +272,12 @@ typedef struct {
   int32_t n_tokens;   /* valid tokens of the run (its pages are ceil(n_tokens / P)) */
   int32_t prow;       /* SIMT: the partial row written; MMA: index into seg_prows */
   int32_t query;      /* SIMT: the request; MMA: first request of the item */
-  int32_t sole;       /* SIMT, how the fused path combines this partial row of (query, kv_head):
-                       * 0: arrival counter, the last of the pair's writers merges it;
-                       * 1: it is the pair's only partial row and goes straight to the output;
-                       * 2: the pair also has tensor-core partial rows and is merged by the
-                       *    tail merge launch (tail_pairs).  MMA segments: 0. */
+  int32_t sole;       /* SIMT: how the fused path combines this partial row of (query, kv_head).
+                       * Bits 0-1, the mode: 0: arrival counter, the last of the pair's SIMT
+                       * rows merges the pair; 1: it is the pair's only partial row and goes
+                       * straight to the output; 2: as 0, but the pair also has tensor-core
+                       * rows, so the merging warp first waits for the tensor-core launch.
+                       * Bits 2-31: the pair's number of SIMT partial rows.  MMA segments: 0. */
   int32_t page_start; /* index into pages of the run's first page (item page_off + page_begin) */
 } pa_seg;
 

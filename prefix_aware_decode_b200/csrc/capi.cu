@@ -11,11 +11,14 @@
 
 namespace {
 
+// Image tables at `image` (the workspace base unless the image was placed
+// elsewhere), partial rows in the workspace.
 PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   const pa_image_header& h = p.hdr;
-  uint8_t* b = static_cast<uint8_t*>(ws);
+  uint8_t* b = static_cast<uint8_t*>(p.dev_image ? p.dev_image : ws);
+  uint8_t* w = static_cast<uint8_t*>(ws);
   PaDevPtrs d{};
-  d.ws = b;
+  d.ws = w;
   d.items = reinterpret_cast<const pa_item*>(b + h.off_nodes);
   d.segs = reinterpret_cast<const pa_seg*>(b + h.off_segs);
   d.pages = reinterpret_cast<const int32_t*>(b + h.off_pages);
@@ -26,8 +29,8 @@ PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   d.warp_segs = reinterpret_cast<const int32_t*>(b + h.off_warp_segs);
   d.prow_off = reinterpret_cast<const int32_t*>(b + h.off_prow_off);
   d.tail_pairs = reinterpret_cast<const int32_t*>(b + h.off_tail_pairs);
-  d.partial_lse = reinterpret_cast<float*>(b + h.off_partial_lse);
-  d.partial_o = reinterpret_cast<float*>(b + h.off_partial_o);
+  d.partial_lse = reinterpret_cast<float*>(w + h.off_partial_lse);
+  d.partial_o = reinterpret_cast<float*>(w + h.off_partial_o);
   d.status = reinterpret_cast<int32_t*>(b + offsetof(pa_image_header, status));
   return d;
 }
@@ -225,12 +228,100 @@ extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_wor
   if (!plan || !d_workspace || !out) return PA_ERR_INVALID;
   int32_t word = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const uint8_t* src = static_cast<const uint8_t*>(d_workspace) + offsetof(pa_image_header, status);
+  const uint8_t* base = static_cast<const uint8_t*>(plan->dev_image ? plan->dev_image : d_workspace);
+  const uint8_t* src = base + offsetof(pa_image_header, status);
   if (cudaMemcpyAsync(&word, src, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
   *out = static_cast<pa_status>(word);
   return PA_OK;
 }
+
+namespace {
+
+// Per-step plan images of pa_decode_step: two device slots per device used
+// alternately, uploaded on a stream of the library's own so that the upload of
+// step k+1 runs while the kernels of step k do.  The compute stream waits for
+// the upload (an event) before its launches, and records when it has finished
+// reading the slot; the upload that next fills the slot waits for that.
+struct StepRing {
+  cudaStream_t upload = nullptr;
+  void* slot[2] = {nullptr, nullptr};
+  size_t cap[2] = {0, 0};
+  cudaEvent_t uploaded[2] = {nullptr, nullptr}, consumed[2] = {nullptr, nullptr};
+  bool consumed_set[2] = {false, false};
+  int next = 0;
+};
+std::mutex g_step_mu;
+StepRing g_step[64];
+
+StepRing* step_ring(int& device) {
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= 64) return nullptr;
+  StepRing& r = g_step[device];
+  if (!r.upload) {
+    if (cudaStreamCreateWithFlags(&r.upload, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (int j = 0; j < 2; ++j)
+      if (cudaEventCreateWithFlags(&r.uploaded[j], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&r.consumed[j], cudaEventDisableTiming) != cudaSuccess)
+        return nullptr;
+  }
+  return &r;
+}
+
+// Uploads the plan image into the next slot and makes `stream` wait for it;
+// the plan's kernels then read their tables there.
+pa_status step_upload(pa_plan* plan, cudaStream_t stream, int* slot_out) {
+  std::lock_guard<std::mutex> lock(g_step_mu);
+  int device = 0;
+  StepRing* r = step_ring(device);
+  if (!r) return PA_ERR_CUDA;
+  const int j = r->next;
+  const size_t n = plan->image.size;
+  if (r->cap[j] < n) {
+    // grow (rare): the slot's previous readers must be done before it is freed
+    if (r->consumed_set[j] && cudaEventSynchronize(r->consumed[j]) != cudaSuccess) return PA_ERR_CUDA;
+    if (r->slot[j]) cudaFree(r->slot[j]);
+    r->slot[j] = nullptr;
+    r->cap[j] = 0;
+    size_t cap = 1 << 20;
+    while (cap < n) cap <<= 1;
+    if (cudaMalloc(&r->slot[j], cap) != cudaSuccess) return PA_ERR_NOMEM;
+    r->cap[j] = cap;
+  }
+  if (r->consumed_set[j] && cudaStreamWaitEvent(r->upload, r->consumed[j], 0) != cudaSuccess) return PA_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> pin_lock(g_pin_mu);
+    PinnedSlot* s = pin_acquire(n, device);
+    if (s) {
+      std::memcpy(s->ptr, plan->image.data(), n);
+      if (cudaMemcpyAsync(r->slot[j], s->ptr, n, cudaMemcpyHostToDevice, r->upload) != cudaSuccess ||
+          cudaEventRecord(s->done, r->upload) != cudaSuccess)
+        return PA_ERR_CUDA;
+    } else if (cudaMemcpyAsync(r->slot[j], plan->image.data(), n, cudaMemcpyHostToDevice, r->upload) !=
+               cudaSuccess) {
+      return PA_ERR_CUDA;
+    }
+  }
+  if (cudaEventRecord(r->uploaded[j], r->upload) != cudaSuccess ||
+      cudaStreamWaitEvent(stream, r->uploaded[j], 0) != cudaSuccess)
+    return PA_ERR_CUDA;
+  plan->dev_image = r->slot[j];
+  r->next = j ^ 1;
+  *slot_out = j;
+  return PA_OK;
+}
+
+// After the launches of the step: the slot may be refilled once `stream` gets here.
+pa_status step_release(int j, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_step_mu);
+  int device = 0;
+  StepRing* r = step_ring(device);
+  if (!r) return PA_ERR_CUDA;
+  if (cudaEventRecord(r->consumed[j], stream) != cudaSuccess) return PA_ERR_CUDA;
+  r->consumed_set[j] = true;
+  return PA_OK;
+}
+
+}  // namespace
 
 extern "C" pa_status pa_decode_step(const pa_config* cfg, int32_t batch, const int32_t* kv_lens,
                                     const int32_t* block_table, int32_t max_pages, int32_t num_pages_in_pool,
@@ -242,8 +333,14 @@ extern "C" pa_status pa_decode_step(const pa_config* cfg, int32_t batch, const i
   pa_status st = pa_plan_create(cfg, batch, kv_lens, block_table, max_pages, num_pages_in_pool, &plan);
   if (st != PA_OK) return st;
   if (profile_events) pa_plan_set_profile_events(plan, profile_events, 4);
-  st = pa_plan_upload(plan, d_workspace, workspace_bytes, stream);
+  if (workspace_bytes < plan->hdr.workspace_bytes) st = PA_ERR_NOMEM;
+  int slot = -1;
+  if (st == PA_OK) st = step_upload(plan, static_cast<cudaStream_t>(stream), &slot);
   if (st == PA_OK) st = pa_attend(plan, q, k_pool, v_pool, d_workspace, out, lse, stream);
+  if (slot >= 0) {
+    const pa_status rs = step_release(slot, static_cast<cudaStream_t>(stream));
+    if (st == PA_OK) st = rs;
+  }
   if (st == PA_OK && plan_out) *plan_out = plan;
   else pa_plan_destroy(plan);
   return st;

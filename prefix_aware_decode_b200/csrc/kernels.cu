@@ -21,9 +21,11 @@
 //
 // Merge (Merge 阶段: an online-softmax combine of each query's partial results
 // across CTAs): LSE = log sum_j e^{lse_j}, out = sum_j e^{lse_j - LSE} o_j.  In
-// the fused path the warp that writes the last partial row of a (request, kv
-// head) merges it (arrival counter per pair); the same warp-level routine also
-// runs as a stand-alone merge launch.
+// the fused path the SIMT warp that writes the last SIMT partial row of a
+// (request, kv head) merges it (arrival counter per pair), waiting for the
+// tensor-core launch first when the pair also has tensor-core rows; pairs with
+// tensor-core rows only are merged by a short merge launch.  The same
+// warp-level routine also runs as the stand-alone merge launch.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -131,32 +133,23 @@ __device__ __forceinline__ void merge_pair(const float* partial_lse, const float
   if (lse && lane % LPR == 0) lse[(size_t)b * Hq + g * G + r] = m + logf(z);
 }
 
-// Called by a whole warp after it wrote partial rows of up to 32 (request, kv
-// head g) pairs, lane j holding request bj for j < n: counts the arrivals (in
-// parallel) and merges every pair for which this was the last partial row.
-template <int D, int G>
-__device__ __forceinline__ void arrive_and_merge(const FwdArgs& a, int bj, int n, int g, int lane) {
+// Called by a whole SIMT warp after it wrote a partial row of pair bg = b*Hkv+g:
+// counts the arrival; true if this was the last of the pair's n_simt SIMT rows.
+__device__ __forceinline__ bool simt_arrive(const FwdArgs& a, int bg, int n_simt, int lane) {
   __threadfence();
   __syncwarp();
-  bool last = false;
-  int p0 = 0, p1 = 0;
-  if (lane < n) {
-    const int bg = bj * a.Hkv + g;
-    p0 = a.prow_off[bg];
-    p1 = a.prow_off[bg + 1];
-    last = atomicAdd(&a.counters[bg], 1) == p1 - p0 - 1;
-  }
-  unsigned todo = __ballot_sync(0xffffffffu, last);
-  if (!todo) return;
+  int last = 0;
+  if (lane == 0) last = atomicAdd(&a.counters[bg], 1) == n_simt - 1;
+  if (!__shfl_sync(0xffffffffu, last, 0)) return false;
   __threadfence();
-  while (todo) {
-    const int j = __ffs(todo) - 1;
-    todo &= todo - 1;
-    const int b = __shfl_sync(0xffffffffu, bj, j);
-    const int q0 = __shfl_sync(0xffffffffu, p0, j), q1 = __shfl_sync(0xffffffffu, p1, j);
-    merge_pair<D, G>(a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, b, g, q0, q1, lane);
-    if (lane == j) a.counters[b * a.Hkv + g] = 0;  // ready for the next launch
-  }
+  return true;
+}
+
+template <int D, int G>
+__device__ __forceinline__ void merge_and_reset(const FwdArgs& a, int bg, int lane) {
+  merge_pair<D, G>(a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, bg / a.Hkv, bg % a.Hkv, a.prow_off[bg],
+                   a.prow_off[bg + 1], lane);
+  if (lane == 0) a.counters[bg] = 0;  // ready for the next launch
 }
 
 // ---------------------------------------------------------------- SIMT class
@@ -182,11 +175,11 @@ struct SimtShape {
 
 struct SegInfo {
   int n_tokens, prow, query, kv_head;
-  int mode;  // how the fused path combines the partial row (pa_seg.sole)
+  int mode, n_simt;  // how the fused path combines the partial row (pa_seg.sole)
 };
 
 __device__ __forceinline__ SegInfo load_seg(const pa_seg* segs, int i, int end) {
-  SegInfo r{0, 0, 0, 0, 0};
+  SegInfo r{0, 0, 0, 0, 0, 0};
   if (i < end) {
     const int4 x = *reinterpret_cast<const int4*>(segs + i);        // item, kv_head, page_begin, n_tokens
     const int4 y = *reinterpret_cast<const int4*>(&segs[i].prow);  // prow, query, sole, pad
@@ -194,7 +187,8 @@ __device__ __forceinline__ SegInfo load_seg(const pa_seg* segs, int i, int end) 
     r.kv_head = x.y;
     r.prow = y.x;
     r.query = y.y;
-    r.mode = y.z;
+    r.mode = y.z & 3;
+    r.n_simt = y.z >> 2;
   }
   return r;
 }
@@ -428,6 +422,11 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
     inflight |= 1u << (NST + slot);
   };
 
+  // pairs this warp merges once the tensor-core launch has completed
+  constexpr int kMaxDeferred = 16;
+  int deferred[kMaxDeferred];
+  int n_def = 0;
+
   SegInfo cur = load_seg(a.segs, seg_begin, seg_end);
   SegInfo nx = load_seg(a.segs, seg_begin + 1, seg_end);
   SegInfo nxx = load_seg(a.segs, seg_begin + 2, seg_end);
@@ -547,10 +546,26 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
         if (li == 0) a.partial_lse[(size_t)cur.prow * G + r] = lse_r;
       }
     }
-    if (a.out && cur.mode == 0) arrive_and_merge<D, G>(a, cur.query, 1, cur.kv_head, lane);
+    if (a.out && cur.mode != 1) {
+      const int bg = cur.query * a.Hkv + cur.kv_head;
+      if (simt_arrive(a, bg, cur.n_simt, lane)) {
+        if (cur.mode == 0) {
+          merge_and_reset<D, G>(a, bg, lane);
+        } else if (n_def < kMaxDeferred) {
+          deferred[n_def++] = bg;  // also has tensor-core rows: merged after this warp's own work
+        } else {
+          griddep_wait();
+          merge_and_reset<D, G>(a, bg, lane);
+        }
+      }
+    }
     cur = nx;
     nx = nxx;
     nxx = load_seg(a.segs, si + 3, seg_end);
+  }
+  if (n_def > 0 && !failed) {
+    griddep_wait();
+    for (int j = 0; j < n_def; ++j) merge_and_reset<D, G>(a, deferred[j], lane);
   }
   if (failed) {
     // wait (bounded) for this warp's copies still in flight before leaving
@@ -950,7 +965,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       }
       tc_fence_before();
       mbar_arrive(bar(S::B_OFREE));
-      // the pairs of these rows are merged by the tail merge launch
+      // these rows' pairs are merged by their last SIMT writer or the tail merge launch
       ++segord;
     }
     if (!ok && lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, warp);

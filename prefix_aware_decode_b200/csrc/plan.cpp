@@ -171,7 +171,7 @@ struct Scratch {
   std::vector<ItemRec> items;
   std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows, tail_pairs;
   std::vector<SegRec> simt_segs, mma_segs;
-  std::vector<uint8_t> is_tail;
+  std::vector<int32_t> n_mma_rows;
 };
 
 }  // namespace
@@ -300,7 +300,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     // boundaries (long-KV splitting without a fixed chunk size).
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 4.2e6;     // flop per us per SM, tcgen05 class (measured: ~1.47 us per 64-key stage of 128 rows)
+    const double kMmaFlopsPerSmUs = 2.7e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
     int64_t simt_pages = 0, mma_pages = 0;
@@ -402,18 +402,17 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       const ItemRec& it = items[s.item];
       for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
     }
-    // pairs with a tensor-core partial row are merged by the tail launch (they
-    // are the MMA rows' pairs, already counted above)
-    std::vector<int32_t>& tail_pairs = sc.tail_pairs;
-    std::vector<uint8_t>& is_tail = sc.is_tail;
-    tail_pairs.clear();
-    is_tail.assign(prow_off.size() - 1, 0);
-    for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
-      if (prow_off[bg + 1] > 0) {
-        tail_pairs.push_back((int32_t)bg);
-        is_tail[bg] = 1;
-      }
+    // fused merge: the last SIMT partial row of a pair to be written merges the
+    // pair (after the tensor-core launch has finished if the pair also has
+    // tensor-core rows); pairs with tensor-core rows only are merged by the
+    // tail merge launch
+    std::vector<int32_t>& n_mma_rows = sc.n_mma_rows;
+    n_mma_rows.assign(prow_off.begin() + 1, prow_off.end());
     for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
+    std::vector<int32_t>& tail_pairs = sc.tail_pairs;
+    tail_pairs.clear();
+    for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
+      if (n_mma_rows[bg] > 0 && prow_off[bg + 1] == n_mma_rows[bg]) tail_pairs.push_back((int32_t)bg);
     for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
     std::vector<int32_t>& cursor = sc.cursor;
     cursor.assign(prow_off.begin(), prow_off.end() - 1);
@@ -472,7 +471,9 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     size_t k = 0;
     for (const auto& s : simt_segs) {
       const size_t bg = (size_t)s.query * Hkv + s.kv_head;
-      const int sole = is_tail[bg] ? 2 : prow_off[bg + 1] - prow_off[bg] == 1 ? 1 : 0;
+      const int n_rows = prow_off[bg + 1] - prow_off[bg], n_simt = n_rows - n_mma_rows[bg];
+      const int mode = n_mma_rows[bg] > 0 ? 2 : n_rows == 1 ? 1 : 0;
+      const int sole = mode | (n_simt << 2);
       ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
                  items[s.item].page_off + s.page_begin};
     }

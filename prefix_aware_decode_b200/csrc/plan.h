@@ -45,6 +45,9 @@ struct pa_plan {
   // optional cudaEvent_t handles recorded around the launches (profiling):
   // [0,1] forward launch (pa_forward / pa_attend), [2,3] merge launch
   void* prof[4] = {};
+  // device copy of the image when it lives outside the caller's workspace
+  // (pa_decode_step's image ring); nullptr: at the workspace base
+  void* dev_image = nullptr;
 };
 
 // Kernel launchers (kernels.cu).  Return 0 or a cudaError_t value.

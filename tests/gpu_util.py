@@ -25,8 +25,11 @@ class DevWorkload:
         self.v = bf16_dev(w.v_pool)
 
 
-def run(dw: DevWorkload, flags=0, max_chunk_tokens=0, wait_timeout_us=0, check_status=True):
-    """Plan + upload + forward + merge through the C ABI; returns (out, lse, plan stats, status)."""
+def run(dw: DevWorkload, flags=0, max_chunk_tokens=0, wait_timeout_us=0, check_status=True, fused=False):
+    """Plan + upload + forward + merge through the C ABI; returns (out, lse, plan stats, status).
+
+    fused: pa_attend (merge inside the forward launches, plus the tail merge
+    launch) instead of pa_forward followed by pa_merge."""
     w = dw.w
     plan = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D, flags=flags,
                     max_chunk_tokens=max_chunk_tokens, wait_timeout_us=wait_timeout_us)
@@ -34,8 +37,11 @@ def run(dw: DevWorkload, flags=0, max_chunk_tokens=0, wait_timeout_us=0, check_s
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
     plan.upload(ws)
-    plan.forward(dw.q, dw.k, dw.v, ws)
-    plan.merge(ws, out, lse)
+    if fused:
+        plan.attend(dw.q, dw.k, dw.v, ws, out, lse)
+    else:
+        plan.forward(dw.q, dw.k, dw.v, ws)
+        plan.merge(ws, out, lse)
     status = plan.device_status(ws)
     torch.cuda.synchronize()
     if check_status:

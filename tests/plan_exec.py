@@ -53,13 +53,17 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
     else:
         assert h.mma_ctas == 0
     assert np.all(img.counters == 0)
-    # the tail list holds exactly the pairs with a tensor-core partial row, ascending
-    mma_pairs = set()
+    # pairs with tensor-core rows; the tail list holds those without SIMT rows, ascending
+    mma_pairs, simt_rows = set(), {}
     for si in range(nseg_simt, h.num_segments):
         item, g, pb, nt, prow, q = img.segs[si]
         po, itok, nq, qo = img.items[item]
         mma_pairs.update(int(b) * Hkv + int(g) for b in img.queries[qo: qo + nq])
-    assert list(img.tail_pairs) == sorted(mma_pairs)
+    for si in range(nseg_simt):
+        item, g, pb, nt, prow, q = img.segs[si]
+        bg = int(q) * Hkv + int(g)
+        simt_rows[bg] = simt_rows.get(bg, 0) + 1
+    assert list(img.tail_pairs) == sorted(bg for bg in mma_pairs if bg not in simt_rows)
     # warp lists partition the SIMT segments, in order; page_start and the
     # combine mode (tail merge, sole row or arrival counted) are consistent
     assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
@@ -69,8 +73,10 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
         assert img.seg_page_start[si] == img.items[item][0] + pb
         if si < nseg_simt:
             n_rows = img.prow_off[q * Hkv + g + 1] - img.prow_off[q * Hkv + g]
-            want = 2 if int(q) * Hkv + int(g) in mma_pairs else (1 if n_rows == 1 else 0)
-            assert img.seg_sole[si] == want
+            bg = int(q) * Hkv + int(g)
+            want = 2 if bg in mma_pairs else (1 if n_rows == 1 else 0)
+            assert img.seg_sole[si] & 3 == want
+            assert img.seg_sole[si] >> 2 == simt_rows[bg]
         else:
             assert img.seg_sole[si] == 0
     # coverage: each (request, kv head) reads each token (page, slot) exactly once

@@ -36,21 +36,23 @@ def sample(B, n, seed=0):
     return np.unique(np.concatenate([[0, B - 1], s])).astype(np.int32)
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("config", [1, 2])
-def test_small_configs_full_parity(config):
+def test_small_configs_full_parity(config, fused):
     dw = dev_config(config)
     w = dw.w
-    out, lse, st, _ = run(dw)
+    out, lse, st, _ = run(dw, fused=fused)
     ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
     m = compare(out, lse, ref_o, ref_l)
     assert_close(m, f"config {config}")
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("config", [3, 4])
-def test_large_configs_sampled_parity(config):
+def test_large_configs_sampled_parity(config, fused):
     dw = dev_config(config)
     w = dw.w
-    out, lse, st, _ = run(dw)
+    out, lse, st, _ = run(dw, fused=fused)
     qs = sample(w.B, 40, seed=config)
     ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs)
     assert_close(compare(out, lse, ref_o, ref_l, queries=qs), f"config {config}")
@@ -90,7 +92,8 @@ def test_random_forests_gqa_and_head_dim(G, D):
         assert_close(compare(out, lse, ref_o, ref_l), f"G={G} D={D} flags={flags}")
 
 
-def test_edge_lengths_and_ragged_tails():
+@pytest.mark.parametrize("fused", [False, True])
+def test_edge_lengths_and_ragged_tails(fused):
     lens = [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 255, 256, 257, 1000, 4099]
     roots = [wl.Node(n) for n in lens]
     # plus a shared prefix whose children end 0..17 tokens after it
@@ -99,8 +102,27 @@ def test_edge_lengths_and_ragged_tails():
     dw = DevWorkload(w)
     ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
     for flags, chunk in [(0, 0), (pad.PA_PLAN_ALWAYS_SHARE, 16), (0, 32)]:
-        out, lse, st, _ = run(dw, flags=flags, max_chunk_tokens=chunk)
+        out, lse, st, _ = run(dw, flags=flags, max_chunk_tokens=chunk, fused=fused)
         assert_close(compare(out, lse, ref_o, ref_l), f"edges flags={flags} chunk={chunk}")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_pairs_with_tensor_core_rows_only(fused):
+    # requests 0 and 1 hold the same four full pages and nothing else, so their
+    # (request, kv head) pairs have tensor-core partial rows only (merged by the
+    # tail merge launch in the fused path); requests 2 and 3 share those pages
+    # too and go on, so theirs mix tensor-core and SIMT rows
+    base = wl.make_config(1)
+    bt = base.block_table.copy()
+    kv = base.kv_lens.copy()
+    bt[1, :4] = bt[0, :4]
+    kv[0] = kv[1] = 64
+    w = wl.Workload(**{**base.__dict__, "block_table": bt, "kv_lens": kv})
+    dw = DevWorkload(w)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    out, lse, st, _ = run(dw, flags=pad.PA_PLAN_ALWAYS_SHARE, fused=fused)
+    assert st["num_tail_pairs"] == 2 * w.Hkv and st["mma_ctas"] >= 1
+    assert_close(compare(out, lse, ref_o, ref_l), "tensor-core-only pairs")
 
 
 def test_single_key_returns_v_row_bit_exact():
