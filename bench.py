@@ -95,6 +95,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
+def measured_traffic(config: int):
+    """DRAM bytes per step of the forward launches from the committed ncu capture,
+    or None when the kernels have changed since it was taken."""
+    import hashlib
+    try:
+        t = json.load(open(os.path.join(_ROOT, "profiles", "traffic.json")))
+        src = open(os.path.join(_ROOT, "prefix_aware_decode_b200", "csrc", "kernels.cu"), "rb").read()
+    except OSError:
+        return None
+    if hashlib.sha256(src).hexdigest()[:16] != t.get("kernels_cu_sha256_16"):
+        return None
+    w = t.get("workloads", {}).get(str(config))
+    return sum(w.values()) if w else None
+
+
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
@@ -243,7 +258,8 @@ def main():
                                for i in range(args.warmup, nsteps) if step_events[i] is not None)
 
     fwd_ms = ev_ms(0, 1)
-    launches_per_step = 1 + (pst["num_tail_pairs"] > 0)
+    # the tensor-core and CUDA-core forward launches (concurrent), the tail merge launch
+    launches_per_step = (pst["mma_ctas"] > 0) + (pst["simt_warps"] > 0) + (pst["num_tail_pairs"] > 0)
 
     # algorithmic bytes of one forward: the KV of its (page, kv head) tiles (each
     # node read once per query tile), the q rows, the fp32 partial rows written
@@ -275,9 +291,10 @@ def main():
                                      "num_tail_pairs", "num_partial_rows", "read_kv_bytes", "workspace_bytes",
                                      "image_bytes")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
-                     "kernel": "fwd_kernel (both tile classes; SIMT-only pairs merged in it) + merge_kernel over "
-                               "the pairs with tensor-core rows, timed together",
+                     "frac": achieved / hbm_peak, "traffic": measured_traffic(args.config),
+                     "traffic_unit": "bytes per step (DRAM read + write of the forward launches, ncu)",
+                     "kernel": "mma_fwd_kernel + simt_fwd_kernel (concurrent launches, merge fused into the "
+                               "SIMT launch) + merge_kernel over tensor-core-only pairs if any, timed together",
                      "launches_per_step": launches_per_step,
                      "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
         "gpu_launches": args.steps * launches_per_step,
