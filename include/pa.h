@@ -253,8 +253,8 @@ const char *pa_status_string(pa_status s);
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
  *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
  *                                             [prow_off[b*Hkv+g], prow_off[b*Hkv+g+1])
- *   tail_pairs  int32[num_tail_pairs]         b*Hkv+g of every pair whose partial rows are
- *                                             all tensor-core rows, ascending
+ *   tail_pairs  int32[num_tail_pairs]         b*Hkv+g of every pair merged by the tail merge
+ *                                             launch (tensor-core rows only, or mode 3), ascending
  *   partial_lse fp32[num_partial_rows][G]     (workspace only, not uploaded)
  *   partial_o   fp32[num_partial_rows][G][D]  (workspace only, not uploaded)
  */
@@ -276,8 +276,11 @@ typedef struct {
                        * Bits 0-1, the mode: 0: arrival counter, the last of the pair's SIMT
                        * rows merges the pair; 1: it is the pair's only partial row and goes
                        * straight to the output; 2: as 0, but the pair also has tensor-core
-                       * rows, so the merging warp first waits for the tensor-core launch.
-                       * Bits 2-31: the pair's number of SIMT partial rows.  MMA segments: 0. */
+                       * rows, so the merging warp first waits for the tensor-core launch;
+                       * 3: the pair also has tensor-core rows and is merged by the tail
+                       * merge launch (plans where a warp would otherwise defer more than
+                       * 16 such merges).  Bits 2-31: the pair's number of SIMT partial
+                       * rows.  MMA segments: 0. */
   int32_t page_start; /* index into pages of the run's first page (item page_off + page_begin) */
 } pa_seg;
 

@@ -546,7 +546,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
         if (li == 0) a.partial_lse[(size_t)cur.prow * G + r] = lse_r;
       }
     }
-    if (a.out && cur.mode != 1) {
+    if (a.out && (cur.mode == 0 || cur.mode == 2)) {
       const int bg = cur.query * a.Hkv + cur.kv_head;
       if (simt_arrive(a, bg, cur.n_simt, lane)) {
         if (cur.mode == 0) {

@@ -299,6 +299,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     // CTA; a span may end inside an item, so partial rows appear only at span
     // boundaries (long-KV splitting without a fixed chunk size).
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
+    const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
     const double kMmaFlopsPerSmUs = 2.7e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
@@ -308,10 +309,13 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     for (const auto& it : items) {
       const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
       if (it.simt) {
-        simt_pages += np;
+        // a SIMT work unit also pays a fixed latency (q rows, partial row,
+        // arrival): counted as kSimtSegPages more pages
+        simt_pages += np + kSimtSegPages * Hkv;
       } else {
         mma_pages += np;
-        const double rows = 16.0 * ceil_div((int64_t)it.n_queries * G, 16);
+        // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
+        const double rows = kMmaRowsPerCta;
         const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
         mma_cost += np * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
       }
@@ -353,13 +357,14 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
         const int b = queries[it.query_off];
         for (int g = 0; g < Hkv; ++g) {
           int pb = 0;
+          used += kSimtSegPages;  // the unit's fixed cost
           while (pb < npages) {
-            const int take = (int)std::min<int64_t>(npages - pb, span - used);
+            const int take = (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
             const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
             simt_segs.push_back({(int)i, g, pb, tok, -1, b});
             pb += take;
             used += take;
-            if (used == span) {
+            if (used >= span && (int64_t)warp_segs.size() < W) {  // never more than W warps
               warp_segs.push_back((int32_t)simt_segs.size());
               used = 0;
             }
@@ -409,10 +414,23 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     std::vector<int32_t>& n_mma_rows = sc.n_mma_rows;
     n_mma_rows.assign(prow_off.begin() + 1, prow_off.end());
     for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
+    // a SIMT warp defers the merges of its mixed pairs to the end of its work;
+    // if some warp would defer more than kSimtMaxDeferred, every mixed pair
+    // goes to the tail merge launch instead
+    bool mixed_to_tail = false;
+    if (!mma_segs.empty()) {
+      for (size_t w = 0; w + 1 < warp_segs.size() && !mixed_to_tail; ++w) {
+        int n = 0;
+        for (int si = warp_segs[w]; si < warp_segs[w + 1]; ++si)
+          n += n_mma_rows[(size_t)simt_segs[si].query * Hkv + simt_segs[si].kv_head] > 0;
+        mixed_to_tail = n > kSimtMaxDeferred;
+      }
+    }
     std::vector<int32_t>& tail_pairs = sc.tail_pairs;
     tail_pairs.clear();
     for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
-      if (n_mma_rows[bg] > 0 && prow_off[bg + 1] == n_mma_rows[bg]) tail_pairs.push_back((int32_t)bg);
+      if (n_mma_rows[bg] > 0 && (mixed_to_tail || prow_off[bg + 1] == n_mma_rows[bg]))
+        tail_pairs.push_back((int32_t)bg);
     for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
     std::vector<int32_t>& cursor = sc.cursor;
     cursor.assign(prow_off.begin(), prow_off.end() - 1);
@@ -472,7 +490,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     for (const auto& s : simt_segs) {
       const size_t bg = (size_t)s.query * Hkv + s.kv_head;
       const int n_rows = prow_off[bg + 1] - prow_off[bg], n_simt = n_rows - n_mma_rows[bg];
-      const int mode = n_mma_rows[bg] > 0 ? 2 : n_rows == 1 ? 1 : 0;
+      const int mode = n_mma_rows[bg] > 0 ? (mixed_to_tail ? 3 : 2) : n_rows == 1 ? 1 : 0;
       const int sole = mode | (n_simt << 2);
       ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
                  items[s.item].page_off + s.page_begin};

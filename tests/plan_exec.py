@@ -63,7 +63,14 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
         item, g, pb, nt, prow, q = img.segs[si]
         bg = int(q) * Hkv + int(g)
         simt_rows[bg] = simt_rows.get(bg, 0) + 1
-    assert list(img.tail_pairs) == sorted(bg for bg in mma_pairs if bg not in simt_rows)
+    modes = {int(m) & 3 for m in img.seg_sole[:nseg_simt]}
+    mixed_to_tail = 3 in modes
+    assert not (mixed_to_tail and 2 in modes)
+    assert list(img.tail_pairs) == sorted(bg for bg in mma_pairs if mixed_to_tail or bg not in simt_rows)
+    # a warp defers at most 16 mixed-pair merges
+    for w in range(len(img.warp_segs) - 1):
+        segs = range(img.warp_segs[w], img.warp_segs[w + 1])
+        assert sum(int(img.seg_sole[s]) & 3 == 2 for s in segs) <= 16
     # warp lists partition the SIMT segments, in order; page_start and the
     # combine mode (tail merge, sole row or arrival counted) are consistent
     assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
@@ -74,7 +81,7 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
         if si < nseg_simt:
             n_rows = img.prow_off[q * Hkv + g + 1] - img.prow_off[q * Hkv + g]
             bg = int(q) * Hkv + int(g)
-            want = 2 if bg in mma_pairs else (1 if n_rows == 1 else 0)
+            want = (3 if mixed_to_tail else 2) if bg in mma_pairs else (1 if n_rows == 1 else 0)
             assert img.seg_sole[si] & 3 == want
             assert img.seg_sole[si] >> 2 == simt_rows[bg]
         else:
