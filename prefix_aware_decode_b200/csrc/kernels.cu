@@ -596,7 +596,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
 // is unchanged.
 
 constexpr int kMmaKT = 64;           // keys per stage (4 pages)
-constexpr int kMmaWarps = 10;        // producer, MMA issuer, 8 softmax warps
+constexpr int kMmaWarps = 11;        // K producer, MMA issuer, 8 softmax warps, V producer
 constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kSmaxThreads = 256;    // softmax threads (two per tile row)
 constexpr int kSBufs = 3;            // S/P buffers in TMEM
@@ -607,18 +607,21 @@ template <int D>
 struct MmaShape {
   static constexpr int HALVES = D / 64;
   static constexpr int KBLK = kMmaKT * 128;        // one 64-key x 64-dim swizzled block (8 KB)
-  static constexpr int STAGE = 2 * HALVES * KBLK;  // K and V of one stage
+  static constexpr int KSTAGE = HALVES * KBLK;     // K (or V) of one stage
+  static constexpr int STAGE = 2 * KSTAGE;         // K and V of one stage
   static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
   static constexpr int FIXED = HALVES * QBLK + 512 + 1024;  // Q, barriers, alignment slack
   static constexpr int NST_FIT = (kSmemMax - FIXED) / STAGE;
-  static constexpr int NST = NST_FIT < 8 ? NST_FIT : 8;  // K/V stages in flight
+  static constexpr int NST = NST_FIT < 8 ? NST_FIT : 8;  // slots of the K ring and of the V ring
+  static constexpr int OFF_K = 0, OFF_V = NST * KSTAGE;
   static constexpr int OFF_Q = NST * STAGE;
   static constexpr int OFF_BAR = OFF_Q + HALVES * QBLK;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;
-  // barriers: K/V full / empty per stage; S full, P full, p.V done per buffer;
-  // Q loaded; O read out; all MMAs retired; the two halves of each lane
-  // quarter have exchanged (m, l)
-  static constexpr int B_FULL = 0, B_EMPTY = NST, B_SFULL = 2 * NST, B_PFULL = B_SFULL + kSBufs,
+  // barriers: K full / empty and V full / empty per ring slot; S full, P full,
+  // p.V done per buffer; Q loaded; O read out; all MMAs retired; the two halves
+  // of each lane quarter have exchanged (m, l)
+  static constexpr int B_FULL = 0, B_EMPTY = NST, B_VFULL = 2 * NST, B_VEMPTY = 3 * NST,
+                       B_SFULL = 4 * NST, B_PFULL = B_SFULL + kSBufs,
                        B_PV = B_PFULL + kSBufs, B_QFULL = B_PV + kSBufs, B_OFREE = B_QFULL + 1, B_DONE = B_OFREE + 1,
                        B_XCH = B_DONE + 1, NBARS = B_XCH + 4;
   // tensor memory columns: S/P buffers, the two half accumulators, (m, l) exchange
@@ -652,6 +655,8 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar(S::B_FULL + s), 1);
       mbar_init(bar(S::B_EMPTY + s), 1);
+      mbar_init(bar(S::B_VFULL + s), 1);
+      mbar_init(bar(S::B_VEMPTY + s), 1);
     }
     for (int b = 0; b < kSBufs; ++b) {
       mbar_init(bar(S::B_SFULL + b), 1);
@@ -670,14 +675,18 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------- TMA producer: every stage of every segment of this CTA, in
-    // order.  The warp holds the segment's page ids in a sliding window of 32
-    // lanes (plus the next window, prefetched), so no issue waits on a load.
-    if (lane == 0) {
-      prefetch_tmap(tk);
-      prefetch_tmap(tv);
-    }
+  if (warp == 0 || warp == kMmaWarps - 1) {
+    // ---------------- TMA producers: warp 0 streams the K stages, the last warp
+    // the V stages, of every segment of this CTA in order, each into its own
+    // ring.  A K slot is free again once S of its stage is done, a V slot once
+    // p.V is; so K runs ahead of V and neither ring holds a tile longer than
+    // it is needed.  The warp holds the segment's page ids in a sliding window
+    // of 32 lanes (plus the next window, prefetched), so no issue waits on a load.
+    const bool is_v = warp != 0;
+    const CUtensorMap* tm = is_v ? tv : tk;
+    const int b_full = is_v ? S::B_VFULL : S::B_FULL, b_empty = is_v ? S::B_VEMPTY : S::B_EMPTY;
+    uint8_t* ring = smem + (is_v ? S::OFF_V : S::OFF_K);
+    if (lane == 0) prefetch_tmap(tm);
     uint32_t lastpar = 0, any = 0;
     int i = 0;
     bool ok = true;
@@ -695,8 +704,8 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           wnxt = wbase + 32 + lane < npages ? pg[wbase + 32 + lane] : 0;
         }
         const int s = i % NST;
-        if (i >= NST && !warp_wait(bar(S::B_EMPTY + s), ((i / NST) - 1) & 1, a.timeout_ns)) {
-          if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -2);
+        if (i >= NST && !warp_wait(bar(b_empty + s), ((i / NST) - 1) & 1, a.timeout_ns)) {
+          if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, is_v ? -4 : -2);
           ok = false;
           break;
         }
@@ -705,18 +714,15 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp)
           rows[pp] = (__shfl_sync(0xffffffffu, wcur, (st - wbase + pp) & 31) * a.Hkv + seg.kv_head) * 16;
-        if (a.fault_drop && blockIdx.x == 0 && i == 0) continue;  // test: this stage never arrives
+        if (!is_v && a.fault_drop && blockIdx.x == 0 && i == 0) continue;  // test: this K stage never arrives
         if (lane == 0) {
-          const uint32_t fb = bar(S::B_FULL + s);
-          mbar_arrive_expect_tx(fb, (uint32_t)np * 2 * 16 * D * 2);
-          uint8_t* kst = smem + s * S::STAGE;
-          uint8_t* vst = kst + S::HALVES * S::KBLK;
+          const uint32_t fb = bar(b_full + s);
+          mbar_arrive_expect_tx(fb, (uint32_t)np * 16 * D * 2);
+          uint8_t* dst = ring + s * S::KSTAGE;
           for (int pp = 0; pp < np; ++pp) {
 #pragma unroll
-            for (int h = 0; h < S::HALVES; ++h) {
-              tma_load_2d(smem_u32(kst + h * S::KBLK + pp * 2048), tk, 64 * h, rows[pp], fb);
-              tma_load_2d(smem_u32(vst + h * S::KBLK + pp * 2048), tv, 64 * h, rows[pp], fb);
-            }
+            for (int h = 0; h < S::HALVES; ++h)
+              tma_load_2d(smem_u32(dst + h * S::KBLK + pp * 2048), tm, 64 * h, rows[pp], fb);
           }
         }
         lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / NST) & 1) << s);
@@ -725,7 +731,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     }
     if (lane == 0)
       for (int s = 0; s < NST; ++s)
-        if (any & (1u << s)) mbar_wait_bounded(bar(S::B_FULL + s), (lastpar >> s) & 1u, a.timeout_ns);
+        if (any & (1u << s)) mbar_wait_bounded(bar(b_full + s), (lastpar >> s) & 1u, a.timeout_ns);
   } else if (warp == 1) {
     // ---------------- tcgen05.mma issuer (one thread)
     if (lane == 0) {
@@ -737,12 +743,14 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       int i = 0, segord = 0;
       auto do_pv = [&](const Prev& pv, int j) -> bool {
         const int b = j % kSBufs;
-        if (!mbar_wait_bounded(bar(S::B_PFULL + b), (j / kSBufs) & 1, a.timeout_ns)) return false;
+        if (!mbar_wait_bounded(bar(S::B_PFULL + b), (j / kSBufs) & 1, a.timeout_ns) ||
+            !mbar_wait_bounded(bar(S::B_VFULL + pv.s), (j / NST) & 1, a.timeout_ns))
+          return false;
         // the first p.V of a segment overwrites O: the previous epilogue must have read it
         if (pv.first && pv.segord >= 1 && !mbar_wait_bounded(bar(S::B_OFREE), (pv.segord - 1) & 1, a.timeout_ns))
           return false;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + pv.s * S::STAGE + S::HALVES * S::KBLK);
+        const uint32_t v_base = smem_u32(smem + S::OFF_V + pv.s * S::KSTAGE);
         for (int c = 0; c < pv.np; ++c) {
           // 16-key chunk c (page c of the stage) belongs to key half c / 2.  P
           // chunk c: P_hi in columns [16c, 16c + 8), P_lo in [16c + 8, 16c + 16)
@@ -754,7 +762,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           umma_bf16_ts(d_o, a_p + 8, bd, idesc_o, 1u);
         }
         umma_commit(bar(S::B_PV + b));
-        umma_commit(bar(S::B_EMPTY + pv.s));
+        umma_commit(bar(S::B_VEMPTY + pv.s));
         return true;
       };
       for (int si = s_begin; si < s_end && ok; ++si) {
@@ -769,7 +777,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             break;
           }
           tc_fence_after();
-          const uint32_t k_base = smem_u32(smem + s * S::STAGE);
+          const uint32_t k_base = smem_u32(smem + S::OFF_K + s * S::KSTAGE);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             // Q and K: K-major 128-byte swizzle, 64-dim blocks, 8-row groups at +1 KB
@@ -778,6 +786,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             umma_bf16(tmem + S::T_S + b * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar(S::B_SFULL + b));
+          umma_commit(bar(S::B_EMPTY + s));  // the K slot is free once S is done
           if (have_prev && !do_pv(prev, i - 1)) {
             ok = false;
             break;
@@ -898,8 +907,10 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         tmem_st32(t_s, pw);
         if (kvalid < np * 16) {
           // V rows past the last valid key may hold NaN; p = 0 there but 0 * NaN
-          // would still poison the product, so those rows are zeroed
-          uint8_t* vst = smem + s * S::STAGE + S::HALVES * S::KBLK;
+          // would still poison the product, so those rows are zeroed (once the
+          // V tile has landed)
+          if (!warp_wait(bar(S::B_VFULL + s), (i / NST) & 1, a.timeout_ns)) { ok = false; break; }
+          uint8_t* vst = smem + S::OFF_V + s * S::KSTAGE;
           const int nz = np * 16 - kvalid;
           for (int idx = tid; idx < nz * S::HALVES * 8; idx += kSmaxThreads) {
             const int row = kvalid + idx / (S::HALVES * 8);
