@@ -57,6 +57,7 @@ struct Planner {
   const int32_t* bt;
   int max_pages, P, G, Hq, Hkv, D;
   uint32_t flags;
+  int num_pages_in_pool;
   std::vector<int>& order;
   std::vector<int>& npg;
   // outputs of the tree walk
@@ -74,6 +75,13 @@ struct Planner {
     const int off = (int)pages.size();
     const int32_t* r = row(rep);
     pages.insert(pages.end(), r + page_lo, r + page_hi);
+    // page ids are validated here: every (request, page) entry of the batch is
+    // copied into exactly one item (entries of a shared run are equal across
+    // its requests), so this checks each id once per item instead of once per
+    // request
+    uint32_t bad = 0;
+    for (int j = off; j < (int)pages.size(); ++j) bad |= (uint32_t)pages[j] >= (uint32_t)num_pages_in_pool ? 1u : 0u;
+    if (bad) invalid = true;
     if (simt) {
       items.push_back({off, (int)tokens, 1, (int)queries.size(), true});
       queries.push_back(qs[0]);
@@ -249,7 +257,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     sc.items.clear();
     sc.pages.clear();
     sc.queries.clear();
-    Planner pl{kv_lens, block_table, max_pages, P, G, Hq, Hkv, D, flags, sc.order, sc.npg,
+    Planner pl{kv_lens, block_table, max_pages, P, G, Hq, Hkv, D, flags, num_pages_in_pool, sc.order, sc.npg,
                sc.items, sc.pages, sc.queries, sc.qbuf};
     pl.kv_lens = kv_lens;
     pl.bt = block_table;
@@ -260,6 +268,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     pl.Hkv = Hkv;
     pl.D = D;
     pl.flags = flags;
+    pl.num_pages_in_pool = num_pages_in_pool;
     pl.npg.resize(batch);
     int64_t total_pages = 0;
     for (int b = 0; b < batch; ++b) {
@@ -267,10 +276,6 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       if (n < 1 || n > (int64_t)max_pages * P) { delete plan; return PA_ERR_INVALID; }
       pl.npg[b] = (int)ceil_div(n, P);
       total_pages += pl.npg[b];
-      const uint32_t* r = reinterpret_cast<const uint32_t*>(block_table + (size_t)b * max_pages);
-      uint32_t bad = 0;
-      for (int j = 0; j < pl.npg[b]; ++j) bad |= r[j] >= (uint32_t)num_pages_in_pool ? 1u : 0u;
-      if (bad) { delete plan; return PA_ERR_INVALID; }
     }
 
     // ---- tree-structured block table + profit model + emission

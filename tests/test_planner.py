@@ -126,6 +126,28 @@ def test_validation_errors():
         assert e.value.status == code, kw
 
 
+@pytest.mark.parametrize("flags", [0, pad.PA_PLAN_ALWAYS_SHARE, pad.PA_PLAN_NO_SHARING])
+def test_out_of_range_page_ids_anywhere_are_rejected(flags):
+    # pages 0-1 are shared by all three requests, page 2 by the first two,
+    # page 3 is each request's own (4 full pages each, pool of 10 pages)
+    bt = np.array([[5, 6, 7, 2], [5, 6, 7, 3], [5, 6, 8, 9]], dtype=np.int32)
+    kv = np.array([64, 64, 64], dtype=np.int32)
+    pad.Plan(kv, bt, 10, 4, 1, 64, flags=flags)
+    bad_cases = []
+    b = bt.copy(); b[:, 1] = 10; bad_cases.append(b)      # in a run shared by three
+    b = bt.copy(); b[:2, 2] = 11; bad_cases.append(b)     # in a run shared by two
+    b = bt.copy(); b[2, 3] = 12; bad_cases.append(b)      # in one request's own page
+    b = bt.copy(); b[1, 2] = -1; bad_cases.append(b)      # negative
+    for i, b in enumerate(bad_cases):
+        with pytest.raises(pad.PaError) as e:
+            pad.Plan(kv, b, 10, 4, 1, 64, flags=flags)
+        assert e.value.status == pad.PA_ERR_INVALID, i
+    # an entry past a request's last page is never read
+    ignored = bt.copy()
+    ignored[0, 3] = 99
+    pad.Plan(np.array([48, 64, 64], dtype=np.int32), ignored, 10, 4, 1, 64, flags=flags)
+
+
 def test_plan_is_deterministic():
     w = wl.make_config(3, with_values=False, scale=0.25)
     a = make_plan(w).host_image()
