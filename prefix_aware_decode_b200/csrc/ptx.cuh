@@ -70,7 +70,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
-// 2-D tiled tensor copy global -> shared (no multicast).  c0 is the innermost
+// 2-D tiled tensor copy global -> shared of this CTA only.  c0 is the innermost
 // coordinate in elements and must be a multiple of 16 bytes / element size.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
   asm volatile(
