@@ -596,7 +596,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
 // is unchanged.
 
 constexpr int kMmaKT = 64;           // keys per stage (4 pages)
-constexpr int kMmaWarps = 11;        // K producer, MMA issuer, 8 softmax warps, V producer
+constexpr int kMmaWarps = 12;        // K producer, S issuer, 8 softmax warps, p.V issuer, V producer
 constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kSmaxThreads = 256;    // softmax threads (two per tile row)
 constexpr int kSBufs = 3;            // S/P buffers in TMEM
@@ -665,7 +665,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     }
     mbar_init(bar(S::B_QFULL), kSmaxThreads);
     mbar_init(bar(S::B_OFREE), kSmaxThreads);
-    mbar_init(bar(S::B_DONE), 1);
+    mbar_init(bar(S::B_DONE), 2);
     for (int q = 0; q < 4; ++q) mbar_init(bar(S::B_XCH + q), 64);
     fence_mbar_init();
   }
@@ -732,73 +732,71 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     if (lane == 0)
       for (int s = 0; s < NST; ++s)
         if (any & (1u << s)) mbar_wait_bounded(bar(b_full + s), (lastpar >> s) & 1u, a.timeout_ns);
-  } else if (warp == 1) {
-    // ---------------- tcgen05.mma issuer (one thread)
+  } else if (warp == 1 || warp == kMmaWarps - 2) {
+    // ---------------- tcgen05.mma issuers: lane 0 of warp 1 issues the S
+    // products, lane 0 of the second-to-last warp the p.V products, each on its
+    // own waits, so neither issue path waits behind the other; a commit tracks
+    // the MMAs of the thread that issues it.
     if (lane == 0) {
+      const bool is_s = warp == 1;
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, kMmaKT, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, false, true);
-      struct Prev { int s, np, segord; bool first; };
-      Prev prev{0, 0, 0, false};
-      bool have_prev = false, ok = true;
+      bool ok = true;
       int i = 0, segord = 0;
-      auto do_pv = [&](const Prev& pv, int j) -> bool {
-        const int b = j % kSBufs;
-        if (!mbar_wait_bounded(bar(S::B_PFULL + b), (j / kSBufs) & 1, a.timeout_ns) ||
-            !mbar_wait_bounded(bar(S::B_VFULL + pv.s), (j / NST) & 1, a.timeout_ns))
-          return false;
-        // the first p.V of a segment overwrites O: the previous epilogue must have read it
-        if (pv.first && pv.segord >= 1 && !mbar_wait_bounded(bar(S::B_OFREE), (pv.segord - 1) & 1, a.timeout_ns))
-          return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + S::OFF_V + pv.s * S::KSTAGE);
-        for (int c = 0; c < pv.np; ++c) {
-          // 16-key chunk c (page c of the stage) belongs to key half c / 2.  P
-          // chunk c: P_hi in columns [16c, 16c + 8), P_lo in [16c + 8, 16c + 16)
-          // of the buffer; V: MN-major (64-dim atoms at +KBLK, 8-key groups at +1 KB)
-          const uint32_t d_o = tmem + S::T_O + (c >> 1) * D;
-          const uint32_t a_p = tmem + S::T_S + b * kMmaKT + 16 * c;
-          const uint64_t bd = umma_sdesc_sw128(v_base + c * 2048, S::KBLK >> 4, 64);
-          umma_bf16_ts(d_o, a_p, bd, idesc_o, (pv.first && (c & 1) == 0) ? 0u : 1u);
-          umma_bf16_ts(d_o, a_p + 8, bd, idesc_o, 1u);
-        }
-        umma_commit(bar(S::B_PV + b));
-        umma_commit(bar(S::B_VEMPTY + pv.s));
-        return true;
-      };
       for (int si = s_begin; si < s_end && ok; ++si) {
         const int npages = (a.segs[si].n_tokens + 15) >> 4;
         for (int st = 0; st < npages; st += 4, ++i) {
           const int s = i % NST, b = i % kSBufs;
           const bool first = st == 0;
-          if (!mbar_wait_bounded(bar(S::B_FULL + s), (i / NST) & 1, a.timeout_ns) ||
-              (first && !mbar_wait_bounded(bar(S::B_QFULL), segord & 1, a.timeout_ns)) ||
-              (i >= kSBufs && !mbar_wait_bounded(bar(S::B_PV + b), ((i / kSBufs) - 1) & 1, a.timeout_ns))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(smem + S::OFF_K + s * S::KSTAGE);
+          if (is_s) {
+            // K landed; Q of the segment loaded; the buffer's last p.V (stage i - 3) done
+            if (!mbar_wait_bounded(bar(S::B_FULL + s), (i / NST) & 1, a.timeout_ns) ||
+                (first && !mbar_wait_bounded(bar(S::B_QFULL), segord & 1, a.timeout_ns)) ||
+                (i >= kSBufs && !mbar_wait_bounded(bar(S::B_PV + b), ((i / kSBufs) - 1) & 1, a.timeout_ns))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(smem + S::OFF_K + s * S::KSTAGE);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // Q and K: K-major 128-byte swizzle, 64-dim blocks, 8-row groups at +1 KB
-            const uint64_t ad = umma_sdesc_sw128(q_base + (kk >> 2) * S::QBLK + (kk & 3) * 32, 1, 64);
-            const uint64_t bd = umma_sdesc_sw128(k_base + (kk >> 2) * S::KBLK + (kk & 3) * 32, 1, 64);
-            umma_bf16(tmem + S::T_S + b * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              // Q and K: K-major 128-byte swizzle, 64-dim blocks, 8-row groups at +1 KB
+              const uint64_t ad = umma_sdesc_sw128(q_base + (kk >> 2) * S::QBLK + (kk & 3) * 32, 1, 64);
+              const uint64_t bd = umma_sdesc_sw128(k_base + (kk >> 2) * S::KBLK + (kk & 3) * 32, 1, 64);
+              umma_bf16(tmem + S::T_S + b * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(S::B_SFULL + b));
+            umma_commit(bar(S::B_EMPTY + s));  // the K slot is free once S is done
+          } else {
+            // P written; V landed; the first p.V of a segment overwrites O, so the
+            // previous epilogue must have read it
+            if (!mbar_wait_bounded(bar(S::B_PFULL + b), (i / kSBufs) & 1, a.timeout_ns) ||
+                !mbar_wait_bounded(bar(S::B_VFULL + s), (i / NST) & 1, a.timeout_ns) ||
+                (first && segord >= 1 && !mbar_wait_bounded(bar(S::B_OFREE), (segord - 1) & 1, a.timeout_ns))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(smem + S::OFF_V + s * S::KSTAGE);
+            const int np = min(4, npages - st);
+            for (int c = 0; c < np; ++c) {
+              // 16-key chunk c (page c of the stage) belongs to key half c / 2.  P
+              // chunk c: P_hi in columns [16c, 16c + 8), P_lo in [16c + 8, 16c + 16)
+              // of the buffer; V: MN-major (64-dim atoms at +KBLK, 8-key groups at +1 KB)
+              const uint32_t d_o = tmem + S::T_O + (c >> 1) * D;
+              const uint32_t a_p = tmem + S::T_S + b * kMmaKT + 16 * c;
+              const uint64_t bd = umma_sdesc_sw128(v_base + c * 2048, S::KBLK >> 4, 64);
+              umma_bf16_ts(d_o, a_p, bd, idesc_o, (first && (c & 1) == 0) ? 0u : 1u);
+              umma_bf16_ts(d_o, a_p + 8, bd, idesc_o, 1u);
+            }
+            umma_commit(bar(S::B_PV + b));
+            umma_commit(bar(S::B_VEMPTY + s));
           }
-          umma_commit(bar(S::B_SFULL + b));
-          umma_commit(bar(S::B_EMPTY + s));  // the K slot is free once S is done
-          if (have_prev && !do_pv(prev, i - 1)) {
-            ok = false;
-            break;
-          }
-          prev = Prev{s, min(4, npages - st), segord, first};
-          have_prev = true;
         }
         ++segord;
       }
-      if (ok && have_prev) ok = do_pv(prev, i - 1);
-      if (!ok) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -3);
-      // every MMA issued by this thread has completed before TMEM is released
+      if (!ok) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, is_s ? -3 : -5);
+      // every MMA issued by either thread has completed before TMEM is released
       umma_commit(bar(S::B_DONE));
       mbar_wait_bounded(bar(S::B_DONE), 0, a.timeout_ns);
     }
