@@ -74,6 +74,7 @@ struct PinnedSlot {
   void* ptr = nullptr;
   size_t bytes = 0;
   cudaEvent_t done = nullptr;
+  bool lent = false;  // holds a plan image being built, its copy not yet enqueued
 };
 struct PinnedRing {
   PinnedSlot slot[kPinSlots];
@@ -87,6 +88,7 @@ PinnedSlot* pin_acquire(size_t n, int device) {
   if (device < 0 || device >= 64) return nullptr;
   PinnedRing& r = g_pin[device];
   PinnedSlot& s = r.slot[r.next];
+  if (s.lent) return nullptr;
   r.next = (r.next + 1) % kPinSlots;
   if (s.done && cudaEventSynchronize(s.done) != cudaSuccess) return nullptr;
   if (s.bytes < n) {
@@ -269,7 +271,29 @@ StepRing* step_ring(int& device) {
 
 // Uploads the plan image into the next slot and makes `stream` wait for it;
 // the plan's kernels then read their tables there.
-pa_status step_upload(pa_plan* plan, cudaStream_t stream, int* slot_out) {
+// pa_decode_step has the planner write the image straight into a pinned
+// staging buffer (no second copy); the buffer stays lent until its copy is
+// enqueued.
+struct ImageInPinned {
+  int device = 0;
+  PinnedSlot* slot = nullptr;
+};
+uint8_t* pinned_image_sink(size_t n, void* ctx) {
+  ImageInPinned* c = static_cast<ImageInPinned*>(ctx);
+  std::lock_guard<std::mutex> lock(g_pin_mu);
+  PinnedSlot* s = pin_acquire(n, c->device);
+  if (!s) return nullptr;
+  s->lent = true;
+  c->slot = s;
+  return static_cast<uint8_t*>(s->ptr);
+}
+void pinned_image_return(ImageInPinned& c) {
+  std::lock_guard<std::mutex> lock(g_pin_mu);
+  if (c.slot) c.slot->lent = false;
+  c.slot = nullptr;
+}
+
+pa_status step_upload(pa_plan* plan, cudaStream_t stream, int* slot_out, ImageInPinned* pinned) {
   std::lock_guard<std::mutex> lock(g_step_mu);
   int device = 0;
   StepRing* r = step_ring(device);
@@ -290,8 +314,16 @@ pa_status step_upload(pa_plan* plan, cudaStream_t stream, int* slot_out) {
   if (r->consumed_set[j] && cudaStreamWaitEvent(r->upload, r->consumed[j], 0) != cudaSuccess) return PA_ERR_CUDA;
   {
     std::lock_guard<std::mutex> pin_lock(g_pin_mu);
-    PinnedSlot* s = pin_acquire(n, device);
-    if (s) {
+    PinnedSlot* lent = pinned && pinned->slot && pinned->slot->ptr == plan->image.data() ? pinned->slot : nullptr;
+    PinnedSlot* s = lent ? nullptr : pin_acquire(n, device);
+    if (lent) {
+      // the image was built in this pinned buffer
+      const cudaError_t e1 = cudaMemcpyAsync(r->slot[j], lent->ptr, n, cudaMemcpyHostToDevice, r->upload);
+      const cudaError_t e2 = e1 == cudaSuccess ? cudaEventRecord(lent->done, r->upload) : e1;
+      lent->lent = false;
+      pinned->slot = nullptr;
+      if (e2 != cudaSuccess) return PA_ERR_CUDA;
+    } else if (s) {
       std::memcpy(s->ptr, plan->image.data(), n);
       if (cudaMemcpyAsync(r->slot[j], s->ptr, n, cudaMemcpyHostToDevice, r->upload) != cudaSuccess ||
           cudaEventRecord(s->done, r->upload) != cudaSuccess)
@@ -330,16 +362,36 @@ extern "C" pa_status pa_decode_step(const pa_config* cfg, int32_t batch, const i
                                     void* stream, pa_plan** plan_out) {
   if (plan_out) *plan_out = nullptr;
   pa_plan* plan = nullptr;
+  ImageInPinned pinned;
+  if (cudaGetDevice(&pinned.device) != cudaSuccess) return PA_ERR_CUDA;
+  pa_set_image_sink(pinned_image_sink, &pinned);
   pa_status st = pa_plan_create(cfg, batch, kv_lens, block_table, max_pages, num_pages_in_pool, &plan);
-  if (st != PA_OK) return st;
+  pa_set_image_sink(nullptr, nullptr);
+  if (st != PA_OK) {
+    pinned_image_return(pinned);
+    return st;
+  }
   if (profile_events) pa_plan_set_profile_events(plan, profile_events, 4);
   if (workspace_bytes < plan->hdr.workspace_bytes) st = PA_ERR_NOMEM;
   int slot = -1;
-  if (st == PA_OK) st = step_upload(plan, static_cast<cudaStream_t>(stream), &slot);
+  if (st == PA_OK) st = step_upload(plan, static_cast<cudaStream_t>(stream), &slot, &pinned);
+  pinned_image_return(pinned);  // no-op once the copy was enqueued
   if (st == PA_OK) st = pa_attend(plan, q, k_pool, v_pool, d_workspace, out, lse, stream);
   if (slot >= 0) {
     const pa_status rs = step_release(slot, static_cast<cudaStream_t>(stream));
     if (st == PA_OK) st = rs;
+  }
+  if (st == PA_OK && plan_out && !plan->image.owned) {
+    // the caller keeps the plan: give it its own copy of the image (the pinned
+    // buffer goes back to the staging ring)
+    try {
+      HostBuf own = hostbuf_acquire(plan->image.size);
+      std::memcpy(own.data(), plan->image.data(), plan->image.size);
+      plan->image = own;
+    } catch (...) {
+      pa_plan_destroy(plan);
+      return PA_ERR_NOMEM;
+    }
   }
   if (st == PA_OK && plan_out) *plan_out = plan;
   else pa_plan_destroy(plan);

@@ -207,8 +207,22 @@ HostBuf hostbuf_acquire(size_t n) {
   return b;
 }
 
+namespace {
+thread_local ImageSink t_sink = nullptr;
+thread_local void* t_sink_ctx = nullptr;
+}  // namespace
+
+void pa_set_image_sink(ImageSink sink, void* ctx) {
+  t_sink = sink;
+  t_sink_ctx = ctx;
+}
+
 void hostbuf_release(HostBuf& b) {
   if (!b.ptr) return;
+  if (!b.owned) {
+    b = HostBuf{};
+    return;
+  }
   constexpr size_t kMaxFreeBufs = 16;
   std::lock_guard<std::mutex> lock(g_buf_mu);
   if (g_buf_free.size() < kMaxFreeBufs) g_buf_free.push_back(b);
@@ -483,7 +497,14 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
     h.workspace_bytes = off;
 
-    plan->image = hostbuf_acquire(h.image_bytes);
+    uint8_t* lent = t_sink ? t_sink(h.image_bytes, t_sink_ctx) : nullptr;
+    if (lent) {
+      plan->image.ptr = lent;
+      plan->image.size = plan->image.cap = h.image_bytes;
+      plan->image.owned = false;
+    } else {
+      plan->image = hostbuf_acquire(h.image_bytes);
+    }
     uint8_t* img = plan->image.data();
     std::memcpy(img, &h, sizeof(h));
     std::memset(img + h.off_counters, 0, (size_t)batch * Hkv * 4);

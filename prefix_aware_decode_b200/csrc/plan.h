@@ -24,10 +24,18 @@ constexpr int kSimtMaxDeferred = 16;
 struct HostBuf {
   uint8_t* ptr = nullptr;
   size_t size = 0, cap = 0;
+  bool owned = true;  // false: memory lent by an image sink, not returned to the pool
   uint8_t* data() const { return ptr; }
 };
 HostBuf hostbuf_acquire(size_t n);
 void hostbuf_release(HostBuf& b);
+
+// Where pa_plan_create writes the plan image on this thread: by default a
+// pooled host buffer; a sink set here lends the memory instead (pa_decode_step
+// lends a pinned upload buffer, so the image needs no second copy).  The sink
+// returns a buffer of at least n bytes, or nullptr to fall back to the pool.
+using ImageSink = uint8_t* (*)(size_t n, void* ctx);
+void pa_set_image_sink(ImageSink sink, void* ctx);
 
 struct pa_plan {
   pa_config cfg;
