@@ -154,6 +154,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--layers", type=int, default=32,
+                    help="layers of the multi-layer step measured beside config 2 (0: skip)")
+    ap.add_argument("--amortise", type=int, default=1024,
+                    help="config-1 problems batched together for the amortised config-1 figure (0: skip)")
     args = ap.parse_args()
     rank, world, local = dist_env()
     if args.warmup < 3:
@@ -300,6 +304,72 @@ def main():
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clk,
     }
+
+    # config 1 is a few hundred KB, far below what one launch can stream: also
+    # time n independent config-1 problems planned together (device time of the
+    # forward + merge launches; plan time beside it, outside the timing)
+    if args.config == 1 and args.amortise > 0:
+        wa = wl.config1_stream(args.amortise, seed=w.seed)
+        qa, ka, va = dev(wa.q), dev(wa.k_pool), dev(wa.v_pool)
+        oa = torch.empty((wa.B, wa.Hq, wa.D), dtype=torch.bfloat16, device="cuda")
+        la = torch.empty((wa.B, wa.Hq), dtype=torch.float32, device="cuda")
+        pa_ = pad.Plan(wa.kv_lens, wa.block_table, wa.num_pages, wa.Hq, wa.Hkv, wa.D)
+        wsa = pa_.alloc_workspace()
+        pa_.upload(wsa, stream)
+        for _ in range(3):
+            pa_.attend(qa, ka, va, wsa, oa, la, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            pa_.attend(qa, ka, va, wsa, oa, la, stream)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        t_us = a0.elapsed_time(a1) / args.steps * 1e3
+        assert pa_.device_status(wsa, stream) == pad.PA_OK
+        line["amortised"] = {
+            "problems": args.amortise, "batch": wa.B, "unique_kv_bytes": wa.unique_kv_bytes,
+            "forward_merge_us": t_us, "queries_per_s": wa.B / (t_us * 1e-6),
+            "unique_kv_frac_of_hbm": wa.unique_kv_bytes / (t_us * 1e-6) / 1e9 / hbm_peak,
+            "plan_us": pa_.stats()["plan_us"],
+            "note": "one plan and upload, then forward + merge launches timed back to back on the device "
+                    "(the KV of all problems stays resident; 218 MB, above L2)"}
+        pa_.close()
+        del qa, ka, va, oa, la, wsa
+
+    # one decode step of a model: the plan is made and uploaded once and read by
+    # every layer's attention (each layer has its own KV pools)
+    if args.config == 2 and args.layers > 0:
+        lay = [(k0.clone(), v0.clone()) for _ in range(args.layers)]
+        wsl = workspaces[0]
+
+        def layer_step():
+            p_ = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+            p_.upload(wsl, stream)
+            for kl_, vl_ in lay:
+                p_.attend(q, kl_, vl_, wsl, out, lse, stream)
+            p_.close()
+
+        for _ in range(3):
+            layer_step()
+        torch.cuda.synchronize()
+        nst = max(3, args.steps // 10)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        th = time.perf_counter()
+        b0.record(stream)
+        for _ in range(nst):
+            layer_step()
+        b1.record(stream)
+        th = (time.perf_counter() - th) / nst * 1e6
+        torch.cuda.synchronize()
+        t_us = b0.elapsed_time(b1) / nst * 1e3
+        line["multi_layer"] = {
+            "layers": args.layers, "us_per_step": t_us, "us_per_layer": t_us / args.layers,
+            "queries_per_s_per_layer": w.B * args.layers / (t_us * 1e-6),
+            "unique_kv_frac_of_hbm": unique_bytes * args.layers / (t_us * 1e-6) / 1e9 / hbm_peak,
+            "host_us_per_step": th,
+            "note": "per step: pack + upload once, then one forward + merge per layer, each layer with its "
+                    f"own KV pools ({args.layers} x {pool_bytes / 2**20:.0f} MiB)"}
+        del lay
 
     # end to end through the public API with host buffers
     if not args.no_e2e:

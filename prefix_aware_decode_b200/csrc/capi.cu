@@ -120,7 +120,7 @@ struct TmapEntry {
   alignas(64) uint8_t map[128];
 };
 std::mutex g_tmap_mu;
-TmapEntry g_tmap[32];
+TmapEntry g_tmap[128];  // enough for both pools of every layer of a large model
 int g_tmap_next = 0;
 
 bool tmap_get(const pa_plan& p, const void* pool, void* out) {
@@ -136,7 +136,7 @@ bool tmap_get(const pa_plan& p, const void* pool, void* out) {
   e.ptr = pool;
   e.rows = rows;
   e.D = p.D;
-  g_tmap_next = (g_tmap_next + 1) % 32;
+  g_tmap_next = (g_tmap_next + 1) % (int)(sizeof(g_tmap) / sizeof(g_tmap[0]));
   std::memcpy(out, e.map, 128);
   return true;
 }

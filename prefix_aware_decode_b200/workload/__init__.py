@@ -345,6 +345,16 @@ CONFIG_NAMES = {
 }
 
 
+def config1_stream(n: int, seed: int = 1001, with_values: bool = True) -> "Workload":
+    """n independent problems shaped like config 1 (each: one shared 256-token
+    prefix and 4 suffixes uniform 16-64 tokens, 8/2 heads, D 64) in one batch of
+    4n requests: the amortised form of config 1, whose single instance is too
+    small to leave the launch latency."""
+    u = Uniform(seed, TAG_LEN)
+    roots = [Node(256, [Node(u.randint(16, 64)) for _ in range(4)]) for _ in range(n)]
+    return build_workload(f"config 1 x {n}", roots, 8, 2, 64, seed, with_values=with_values)
+
+
 def config_tree(config: int, seed: int, scale: float = 1.0):
     """Return (roots, Hq, Hkv, D) for one of the five configs.
 
