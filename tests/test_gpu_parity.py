@@ -191,3 +191,50 @@ def test_decode_step_matches_plan_path():
         step(w.kv_lens, w.block_table)
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), a.view(torch.int16)) and torch.equal(lse, la)
+
+
+def test_decode_steps_alternating_batches_and_one_plan_over_several_pools():
+    # pa_decode_step uploads each step's plan into one of two device slots on a
+    # copy stream of its own; alternating two different batches through the
+    # same stepper must give each batch its own result every time
+    wa = wl.make_config(1)
+    wb = wl.make_config(2, scale=0.25)
+    da, db = DevWorkload(wa), DevWorkload(wb)
+    refs = {}
+    for name, w in (("a", wa), ("b", wb)):
+        refs[name] = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    outs = {}
+    for name, w, d in (("a", wa, da), ("b", wb, db)):
+        p = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+        ws = p.alloc_workspace()
+        p.close()
+        o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        l = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        outs[name] = (pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, d.q, d.k, d.v, ws, o, l), o, l, w)
+    for step in range(6):
+        name = "ab"[step % 2]
+        stepper, o, l, w = outs[name]
+        stepper(w.kv_lens, w.block_table)
+        if step >= 4:
+            torch.cuda.synchronize()
+            assert_close(compare(o, l, *refs[name]), f"alternating step {step} ({name})")
+    # one uploaded plan read with three different pool pairs (as the layers of
+    # a model would): each result matches the oracle over that pool pair
+    w, d = wb, db
+    p = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    ws = p.alloc_workspace()
+    p.upload(ws)
+    # other contents with the NaN poison in the same places: K and V swapped,
+    # K with its signs flipped
+    flip = lambda a: (a.view(np.uint16) ^ np.uint16(0x8000)).view(a.dtype)
+    for layer, (k_np, v_np) in enumerate([(w.k_pool, w.v_pool), (w.v_pool, w.k_pool), (flip(w.k_pool), w.v_pool)]):
+        k_d = torch.from_numpy(np.ascontiguousarray(k_np).view(np.int16)).cuda().view(torch.bfloat16)
+        v_d = torch.from_numpy(np.ascontiguousarray(v_np).view(np.int16)).cuda().view(torch.bfloat16)
+        o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        l = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        p.attend(d.q, k_d, v_d, ws, o, l)
+        torch.cuda.synchronize()
+        ref = oracle.attend_paged(w.q, k_np, v_np, w.block_table, w.kv_lens)
+        assert_close(compare(o, l, *ref), f"pool pair {layer}")
+    assert p.device_status(ws) == pad.PA_OK
+    p.close()
