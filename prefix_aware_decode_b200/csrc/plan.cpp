@@ -320,7 +320,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
     const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 2.5e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
+    const double kMmaFlopsPerSmUs = 3.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
     int64_t simt_pages = 0, mma_pages = 0;
