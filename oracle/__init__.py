@@ -35,7 +35,7 @@ def build(force: bool = False) -> str:
     """Compile oracle.c into liboracle.so (gcc -O2; no fast-math, no FMA contraction)."""
     src = os.path.join(_HERE, "oracle.c")
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(src):
-        tmp = _LIB + ".tmp"
+        tmp = "%s.%d.tmp" % (_LIB, os.getpid())  # ranks started together may both build
         subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fPIC", "-shared",
                                "-pthread", src, "-o", tmp, "-lm"])
         os.replace(tmp, _LIB)
