@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "plan.h"
 #include "ptx.cuh"
@@ -828,6 +829,15 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       fence_proxy_async_smem();
       mbar_arrive(bar(S::B_QFULL));
     };
+    // S(i) is read from tensor memory into sv; inside a segment the load of
+    // S(i + 1) is issued while P(i) is being stored, when S(i + 1) is already
+    // there (else at the top of the next stage)
+    float sv[32];
+    auto load_s = [&](int i_) {
+      tc_fence_after();
+      tmem_ld32(tmem + S::T_S + (i_ % kSBufs) * kMmaKT + 32 * h + lane_off, sv);
+    };
+    bool have_s = false;
     if (s_begin < s_end) load_q(s_begin);
     for (int si = s_begin; si < s_end && ok; ++si) {
       const pa_seg seg = a.segs[si];
@@ -840,14 +850,16 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         const int np = min(4, npages - st);
         const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
         const int kv_h = max(0, min(32, kvalid - 32 * h));  // valid keys of this half
-        if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
-        tc_fence_after();
+        const bool last = st + 4 >= npages;
+        if (!have_s) {
+          if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
+          load_s(i);
+        }
+        have_s = false;
+        tmem_wait_ld_into(sv);
         const uint32_t t_s = tmem + S::T_S + b * kMmaKT + 32 * h + lane_off;
-        float sv[32];
-        tmem_ld32(t_s, sv);
-        tmem_wait_ld();
         // all S products of this segment are done: Q may be replaced by the next segment's
-        if (st + 4 >= npages && si + 1 < s_end) load_q(si + 1);
+        if (last && si + 1 < s_end) load_q(si + 1);
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (kv_h == 32) {
 #pragma unroll
@@ -887,22 +899,45 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         }
         const float ms = m_used == -INFINITY ? 0.f : m_used;
         // p, and its split P_hi + P_lo: P_hi keeps the top 16 bits of p (a
-        // truncated bf16), P_lo the top 16 bits of the exact remainder p - P_hi
+        // truncated bf16), P_lo the top 16 bits of the exact remainder p - P_hi.
+        // Each page of 16 keys is stored as soon as it is done (P_hi words, then
+        // P_lo words), so its store overlaps the next page's exponentials.
         float pw[32];
         float l4[4] = {0.f, 0.f, 0.f, 0.f};
+        auto page = [&](auto pg_tag, auto full_tag) {
+          constexpr int PG = decltype(pg_tag)::value;
+          constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = (2 * j < kv_h) ? ex2(fmaf(sv[2 * j], a.qscale, -ms)) : 0.f;
-          const float p1 = (2 * j + 1 < kv_h) ? ex2(fmaf(sv[2 * j + 1], a.qscale, -ms)) : 0.f;
-          l4[j & 3] += p0 + p1;
-          const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-          const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
-          const int w = (j >> 3) * 16 + (j & 7);
-          pw[w] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
-          pw[w + 8] = __uint_as_float(__byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632));
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = PG * 8 + jj;
+            float p0 = ex2(fmaf(sv[2 * j], a.qscale, -ms));
+            float p1 = ex2(fmaf(sv[2 * j + 1], a.qscale, -ms));
+            if (!FULL) {
+              p0 = 2 * j < kv_h ? p0 : 0.f;
+              p1 = 2 * j + 1 < kv_h ? p1 : 0.f;
+            }
+            l4[jj & 3] += p0 + p1;
+            const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+            const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
+            pw[PG * 16 + jj] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
+            pw[PG * 16 + jj + 8] = __uint_as_float(__byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632));
+          }
+          tmem_st16<PG * 16>(t_s + PG * 16, pw);
+        };
+        using I0 = std::integral_constant<int, 0>;
+        using I1 = std::integral_constant<int, 1>;
+        if (kv_h == 32) {
+          page(I0{}, std::true_type{});
+          page(I1{}, std::true_type{});
+        } else {
+          page(I0{}, std::false_type{});
+          page(I1{}, std::false_type{});
         }
         l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-        tmem_st32(t_s, pw);
+        if (!last && __all_sync(0xffffffffu, mbar_test_wait(bar(S::B_SFULL + (i + 1) % kSBufs), ((i + 1) / kSBufs) & 1))) {
+          load_s(i + 1);
+          have_s = true;
+        }
         if (kvalid < np * 16) {
           // V rows past the last valid key may hold NaN; p = 0 there but 0 * NaN
           // would still poison the product, so those rows are zeroed (once the
@@ -977,6 +1012,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       // these rows' pairs are merged by their last SIMT writer or the tail merge launch
       ++segord;
     }
+    tmem_wait_ld();  // a load of S issued ahead before a failed wait
     if (!ok && lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, warp);
   }
   tc_fence_before();

@@ -51,6 +51,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking: has the phase of parity `parity` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of parity `parity` to complete, giving up after
 // `timeout_ns` of global time.  Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -213,6 +224,33 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+// Whole warp: 16 columns of this warp's 32 TMEM lanes, v[off .. off + 16).
+template <int off>
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[off + 0])), "r"(__float_as_uint(v[off + 1])), "r"(__float_as_uint(v[off + 2])),
+      "r"(__float_as_uint(v[off + 3])), "r"(__float_as_uint(v[off + 4])), "r"(__float_as_uint(v[off + 5])),
+      "r"(__float_as_uint(v[off + 6])), "r"(__float_as_uint(v[off + 7])), "r"(__float_as_uint(v[off + 8])),
+      "r"(__float_as_uint(v[off + 9])), "r"(__float_as_uint(v[off + 10])), "r"(__float_as_uint(v[off + 11])),
+      "r"(__float_as_uint(v[off + 12])), "r"(__float_as_uint(v[off + 13])), "r"(__float_as_uint(v[off + 14])),
+      "r"(__float_as_uint(v[off + 15]))
+      : "memory");
+}
+// Waits for this thread's tensor-memory loads, with v tied to the wait: v was
+// the destination of a load issued earlier, and its values are read only after
+// this point.
+__device__ __forceinline__ void tmem_wait_ld_into(float (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]),
+                 "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]),
+                 "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]),
+                 "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+               :
+               : "memory");
 }
 // Whole warp: 2 columns of this warp's 32 TMEM lanes.
 __device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&v)[2]) {
