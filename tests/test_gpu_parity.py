@@ -193,6 +193,39 @@ def test_decode_step_matches_plan_path():
         assert torch.equal(out.view(torch.int16), a.view(torch.int16)) and torch.equal(lse, la)
 
 
+def test_arrival_counters_return_to_zero_with_mixed_pairs():
+    # mixed pairs (tensor-core and SIMT rows) are merged by the last SIMT arriver
+    # after the tensor-core launch; the merging warp puts the pair's arrival
+    # counter back to zero, so the uploaded plan gives the same bits launch after launch
+    import ctypes
+
+    dw = dev_config(2, scale=0.25)
+    w = dw.w
+    plan = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    st = plan.stats()
+    assert st["mma_ctas"] > 0 and st["simt_warps"] > 0 and st["num_tail_pairs"] == 0
+    h = pad.PaImageHeader.from_buffer_copy(plan.host_image()[: ctypes.sizeof(pad.PaImageHeader)].tobytes())
+    n_words = w.B * w.Hkv
+    ws = plan.alloc_workspace()
+    plan.upload(ws)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    first = None
+    for _ in range(4):
+        out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        plan.attend(dw.q, dw.k, dw.v, ws, out, lse)
+        torch.cuda.synchronize()
+        words = ws[h.off_counters: h.off_counters + 4 * n_words].cpu().numpy().view(np.int32)
+        assert not words.any(), np.nonzero(words)
+        if first is None:
+            first = (out.clone(), lse.clone())
+            assert_close(compare(out, lse, ref_o, ref_l), "attend() with mixed pairs")
+        else:
+            assert torch.equal(out.view(torch.int16), first[0].view(torch.int16)) and torch.equal(lse, first[1])
+    assert plan.device_status(ws) == pad.PA_OK
+    plan.close()
+
+
 def test_decode_steps_alternating_batches_and_one_plan_over_several_pools():
     # pa_decode_step uploads each step's plan into one of two device slots on a
     # copy stream of its own; alternating two different batches through the
