@@ -320,10 +320,11 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
     const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 3.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
+    const double kMmaFlopsPerSmUs = 5.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
+    const int kMmaSegPages = 38;               // fixed cost of a tensor-core segment (q load, epilogue), in pages
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
-    int64_t simt_pages = 0, mma_pages = 0;
+    int64_t simt_pages = 0, mma_pages = 0, mma_runs = 0;
     double mma_cost = 0;  // SM-us
     for (const auto& it : items) {
       const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
@@ -333,10 +334,11 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
         simt_pages += np + kSimtSegPages * Hkv;
       } else {
         mma_pages += np;
+        mma_runs += Hkv;
         // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
         const double rows = kMmaRowsPerCta;
         const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
-        mma_cost += np * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
+        mma_cost += (np + (int64_t)kMmaSegPages * Hkv) * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
       }
     }
     const int S = plan->num_sms;
@@ -393,7 +395,8 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       if (used > 0) warp_segs.push_back((int32_t)simt_segs.size());
     }
     if (mma_pages > 0) {
-      int64_t span = ceil_div(mma_pages, n_mma);
+      // each (item, kv head) run is a segment, and so is each cut at a CTA boundary
+      int64_t span = ceil_div(mma_pages + (int64_t)kMmaSegPages * (mma_runs + n_mma), n_mma);
       if (span < 16) span = 16;
       if (max_chunk_pages) span = std::min(span, max_chunk_pages);
       int64_t used = 0;
@@ -404,12 +407,22 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
         for (int g = 0; g < Hkv; ++g) {
           int pb = 0;
           while (pb < npages) {
-            const int take = (int)std::min<int64_t>(npages - pb, span - used);
+            // never more than n_mma CTAs: the last one takes whatever is left
+            bool last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
+            if (!last_cta && used > 0 && span - used - kMmaSegPages < 4) {
+              // no room for a stage after the segment's fixed cost: next CTA
+              mma_cta_segs.push_back((int32_t)mma_segs.size());
+              used = 0;
+              last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
+            }
+            used += kMmaSegPages;  // the segment's fixed cost
+            const int take = last_cta ? npages - pb
+                                      : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
             const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
             mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
             pb += take;
             used += take;
-            if (used == span) {
+            if (!last_cta && used >= span) {
               mma_cta_segs.push_back((int32_t)mma_segs.size());
               used = 0;
             }
