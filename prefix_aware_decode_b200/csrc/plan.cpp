@@ -321,10 +321,16 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
     const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
     const double kMmaFlopsPerSmUs = 5.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
-    const int kMmaSegPages = 38;               // fixed cost of a tensor-core segment (q load, epilogue), in pages
+    const int kMmaSegPages = 38;               // fixed cost of a 128-row tensor-core segment (q load, epilogue), in pages
+    // the epilogue's stores scale with the tile's rows: a tile of r rows pays
+    // kMmaSegPages * max(32, r) / 128
+    auto mma_seg_pages = [&](const ItemRec& it) -> int64_t {
+      const int rows = std::min(kMmaRowsPerCta, it.n_queries * G);
+      return (int64_t)kMmaSegPages * std::max(32, rows) / kMmaRowsPerCta;
+    };
     const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
     const double tile_bytes = 2.0 * 16 * D * 2;
-    int64_t simt_pages = 0, mma_pages = 0, mma_runs = 0;
+    int64_t simt_pages = 0, mma_pages = 0, mma_runs = 0, mma_seg_total = 0;
     double mma_cost = 0;  // SM-us
     for (const auto& it : items) {
       const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
@@ -335,10 +341,11 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       } else {
         mma_pages += np;
         mma_runs += Hkv;
+        mma_seg_total += mma_seg_pages(it) * Hkv;
         // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
         const double rows = kMmaRowsPerCta;
         const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
-        mma_cost += (np + (int64_t)kMmaSegPages * Hkv) * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
+        mma_cost += (np + mma_seg_pages(it) * Hkv) * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
       }
     }
     const int S = plan->num_sms;
@@ -347,11 +354,13 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
       n_mma = S;
     } else if (mma_pages > 0) {
       // T_simt = A / (S - k) and T_mma = C / k are equal at k = S C / (A + C);
-      // take the better of the two integers around it
+      // take the better of the two integers around it; no more CTAs than
+      // 16-page spans of tensor-core work
       const double A = simt_pages * tile_bytes / kSimtBytesPerSmUs, C = mma_cost;
-      const int k0 = std::max(1, std::min(S - 1, (int)(S * C / (A + C))));
+      const int k_cap = (int)std::min<int64_t>(S - 1, std::max<int64_t>(1, ceil_div(mma_pages, 16)));
+      const int k0 = std::max(1, std::min(k_cap, (int)(S * C / (A + C))));
       double best = 1e300;
-      for (int kk = k0; kk <= std::min(S - 1, k0 + 1); ++kk) {
+      for (int kk = k0; kk <= std::min(k_cap, k0 + 1); ++kk) {
         const double t = std::max(A / (S - kk), C / kk);
         if (t < best) { best = t; n_mma = kk; }
       }
@@ -396,7 +405,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     }
     if (mma_pages > 0) {
       // each (item, kv head) run is a segment, and so is each cut at a CTA boundary
-      int64_t span = ceil_div(mma_pages + (int64_t)kMmaSegPages * (mma_runs + n_mma), n_mma);
+      int64_t span = ceil_div(mma_pages + mma_seg_total + mma_seg_total / std::max<int64_t>(1, mma_runs) * n_mma, n_mma);
       if (span < 16) span = 16;
       if (max_chunk_pages) span = std::min(span, max_chunk_pages);
       int64_t used = 0;
@@ -408,14 +417,15 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
           int pb = 0;
           while (pb < npages) {
             // never more than n_mma CTAs: the last one takes whatever is left
+            const int64_t seg_cost = mma_seg_pages(it);
             bool last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
-            if (!last_cta && used > 0 && span - used - kMmaSegPages < 4) {
+            if (!last_cta && used > 0 && span - used - seg_cost < 4) {
               // no room for a stage after the segment's fixed cost: next CTA
               mma_cta_segs.push_back((int32_t)mma_segs.size());
               used = 0;
               last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
             }
-            used += kMmaSegPages;  // the segment's fixed cost
+            used += seg_cost;  // the segment's fixed cost
             const int take = last_cta ? npages - pb
                                       : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
             const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
