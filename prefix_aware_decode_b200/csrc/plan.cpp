@@ -556,6 +556,19 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     put(h.off_warp_segs, warp_segs);
     put(h.off_prow_off, prow_off);
     put(h.off_tail_pairs, tail_pairs);
+    // the alignment gaps after the regions are zeroed: the image depends on the inputs only
+    const uint64_t region_end[] = {sizeof(h),
+                                   h.off_nodes + items.size() * sizeof(pa_item),
+                                   h.off_segs + (uint64_t)h.num_segments * sizeof(pa_seg),
+                                   h.off_pages + pages.size() * 4,
+                                   h.off_queries + queries.size() * 4,
+                                   h.off_seg_prows + seg_prows.size() * 4,
+                                   h.off_mma_segs + mma_cta_segs.size() * 4,
+                                   h.off_counters + (uint64_t)batch * Hkv * 4,
+                                   h.off_warp_segs + warp_segs.size() * 4,
+                                   h.off_prow_off + prow_off.size() * 4,
+                                   h.off_tail_pairs + tail_pairs.size() * 4};
+    for (const uint64_t e : region_end) std::memset(img + e, 0, align256(e) - e);
 
     pa_plan_stats& st = plan->stats;
     st.batch = batch;

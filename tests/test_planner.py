@@ -151,5 +151,52 @@ def test_out_of_range_page_ids_anywhere_are_rejected(flags):
 def test_plan_is_deterministic():
     w = wl.make_config(3, with_values=False, scale=0.25)
     a = make_plan(w).host_image()
+    # a plan of other inputs in between leaves other bytes in the pooled host
+    # buffers; the alignment gaps of the image are zeroed, so the bytes match
+    other = make_plan(wl.make_config(2, with_values=False, scale=0.5))
+    other.close()
     b = make_plan(w).host_image()
     assert np.array_equal(a, b)
+
+
+def tensor_core_stats(w):
+    p = make_plan(w)
+    img = Image(p.host_image())
+    h = img.h
+    ns = h.num_segments_simt
+    mma_pages = sum((int(img.segs[i][3]) + 15) // 16 for i in range(ns, h.num_segments))
+    per_cta = [int(img.mma_segs[c + 1] - img.mma_segs[c]) for c in range(h.mma_ctas)]
+    return h, mma_pages, per_cta
+
+
+@pytest.mark.parametrize("config", [1, 2, 3, 5])
+def test_tensor_core_ctas_have_at_least_16_pages_each(config):
+    # at most one tensor-core CTA per 16 pages of tensor-core work: a small
+    # shared prefix (config 1: 16 pages x 2 kv heads) is not spread over many
+    # CTAs that each pay the segment's fixed cost
+    w = wl.make_config(config, with_values=False)
+    h, mma_pages, per_cta = tensor_core_stats(w)
+    assert h.mma_ctas >= 1 and h.mma_ctas <= -(-mma_pages // 16)
+    assert all(n >= 1 for n in per_cta)
+    if config == 1:
+        assert h.mma_ctas <= 2
+
+
+def test_tensor_core_spans_charge_a_cost_per_segment():
+    # config 3: the root's 128-row query tiles (one long run per kv head) and
+    # the 32-row leaf tiles (many short runs); a CTA that holds many short
+    # segments is given fewer pages than one holding a single long run
+    w = wl.make_config(3, with_values=False)
+    p = make_plan(w)
+    img = Image(p.host_image())
+    h = img.h
+    ns = h.num_segments_simt
+    pages, segs = [], []
+    for c in range(h.mma_ctas):
+        ss = range(ns + int(img.mma_segs[c]), ns + int(img.mma_segs[c + 1]))
+        pages.append(sum((int(img.segs[i][3]) + 15) // 16 for i in ss))
+        segs.append(len(ss))
+    pages, segs = np.array(pages), np.array(segs)
+    many, few = segs >= np.percentile(segs, 75), segs <= np.percentile(segs, 25)
+    assert many.any() and few.any() and segs[many].min() > segs[few].max()
+    assert pages[many].mean() < pages[few].mean()
