@@ -58,6 +58,7 @@ typedef enum {
 #define PA_PLAN_NO_SHARING (1u << 0)   /* query-centric: inline every shared node (baseline mode) */
 #define PA_PLAN_ALWAYS_SHARE (1u << 1) /* keep every shared node shared, whatever the profit model says */
 #define PA_PLAN_DEBUG_CHECKS (1u << 2) /* device-side index checks; failures set PA_ERR_DEVICE */
+#define PA_PLAN_KEEP_PACK (1u << 3)    /* keep the pack result in the plan, for pa_plan_advance */
 #define PA_PLAN_FAULT_DROP_LOAD (1u << 8) /* tests only: forward skips one KV load, so its bounded
                                              wait must expire and record PA_ERR_TIMEOUT */
 
@@ -96,7 +97,7 @@ typedef struct {
   int64_t read_kv_bytes;    /* read_tokens * 2 * Hkv * D * 2 */
   uint64_t workspace_bytes; /* device workspace the caller must provide */
   uint64_t image_bytes;     /* bytes pa_plan_upload copies to the device */
-  double plan_us;           /* host time spent in pa_plan_create */
+  double plan_us;           /* host time spent in pa_plan_create or pa_plan_advance */
 } pa_plan_stats;
 
 /*
@@ -117,6 +118,31 @@ typedef struct {
 pa_status pa_plan_create(const pa_config *cfg, int32_t batch, const int32_t *kv_lens,
                          const int32_t *block_table, int32_t max_pages, int32_t num_pages_in_pool,
                          pa_plan **out);
+
+/*
+ * Pack for the next decode step of the same batch, from the previous step's
+ * plan instead of a new walk of the block table (PAT, "Implementation": the
+ * pack scheduler runs every decode step; here its tree is carried over).
+ *   prev              a plan made with PA_PLAN_KEEP_PACK (by pa_plan_create or
+ *                     by this call); not modified
+ *   kv_lens, block_table, max_pages, num_pages_in_pool
+ *                     as for pa_plan_create, for the same batch
+ *   out               receives the new plan (NULL on error); it keeps its pack
+ *                     result, so it can be advanced in turn
+ * The caller asserts that the first ceil(prev_kv_len / page_size) entries of
+ * every row are the ones the previous plan was made from: the tree of shared
+ * nodes is reused as it was, and only each request's own tail grows (its one-
+ * request item takes the new tokens and pages; a request that ended exactly at
+ * the end of a shared node gets a new one-request item).  New page ids are
+ * range-checked.  A request whose kv_len shrank, or a smaller pool, makes the
+ * call plan from scratch (same result as pa_plan_create with prev's config).
+ * New pages that several requests share are read once per request (no new
+ * sharing is found; the next full pa_plan_create finds it).
+ * Errors: PA_ERR_INVALID for a prev without a kept pack result, a different
+ * batch size, or inputs pa_plan_create would reject.
+ */
+pa_status pa_plan_advance(const pa_plan *prev, const int32_t *kv_lens, const int32_t *block_table,
+                          int32_t max_pages, int32_t num_pages_in_pool, pa_plan **out);
 
 /* Device workspace size in bytes for this plan (256-byte aligned buffer required). */
 pa_status pa_plan_workspace_size(const pa_plan *plan, size_t *bytes);

@@ -19,6 +19,7 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_NOMEM, PA_ERR_CUDA, PA_ERR_TIM
 PA_PLAN_NO_SHARING = 1 << 0
 PA_PLAN_ALWAYS_SHARE = 1 << 1
 PA_PLAN_DEBUG_CHECKS = 1 << 2
+PA_PLAN_KEEP_PACK = 1 << 3
 PA_PLAN_FAULT_DROP_LOAD = 1 << 8
 
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_NOMEM", 4: "PA_ERR_CUDA",
@@ -62,7 +63,7 @@ class PaImageHeader(ctypes.Structure):
 
 
 # exported names, in the order pa.h declares them
-EXPORTS = ["pa_plan_create", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
+EXPORTS = ["pa_plan_create", "pa_plan_advance", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
            "pa_get_device_status", "pa_plan_get_stats", "pa_plan_host_image", "pa_plan_set_profile_events",
            "pa_decode_step", "pa_attend_noalloc", "pa_plan_destroy", "pa_status_string"]
 
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
     st = ctypes.c_int
     L.pa_plan_create.argtypes = [ctypes.POINTER(PaConfig), i32, vp, vp, i32, i32, ctypes.POINTER(vp)]
     L.pa_plan_create.restype = st
+    L.pa_plan_advance.argtypes = [vp, vp, vp, i32, i32, ctypes.POINTER(vp)]
+    L.pa_plan_advance.restype = st
     L.pa_plan_workspace_size.argtypes = [vp, ctypes.POINTER(sz)]
     L.pa_plan_workspace_size.restype = st
     L.pa_plan_upload.argtypes = [vp, vp, sz, vp]
@@ -156,6 +159,22 @@ class Plan:
                                         bt.shape[1], int(num_pages), ctypes.byref(h)), "pa_plan_create")
         self._h = h
         self.B, self.Hq, self.Hkv, self.D = int(kv.shape[0]), num_q_heads, num_kv_heads, head_dim
+
+    def advance(self, kv_lens, block_table, num_pages: int) -> "Plan":
+        """The next decode step's plan of the same batch (pa_plan_advance): this
+        plan must have been made with PA_PLAN_KEEP_PACK; the first
+        ceil(old kv_len / page_size) entries of every row must be unchanged."""
+        kv = np.ascontiguousarray(kv_lens, dtype=np.int32)
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        if bt.ndim != 2 or kv.ndim != 1 or bt.shape[0] != kv.shape[0] or kv.shape[0] != self.B:
+            raise ValueError("block_table must be [B][max_pages] and kv_lens [B], B as before")
+        h = ctypes.c_void_p()
+        _check(self._lib.pa_plan_advance(self._h, kv.ctypes.data, bt.ctypes.data, bt.shape[1], int(num_pages),
+                                         ctypes.byref(h)), "pa_plan_advance")
+        nxt = Plan.__new__(Plan)
+        nxt._lib, nxt._h = self._lib, h
+        nxt.B, nxt.Hq, nxt.Hkv, nxt.D = self.B, self.Hq, self.Hkv, self.D
+        return nxt
 
     def close(self):
         if self._h is not None and self._h.value:

@@ -21,6 +21,7 @@
 #include <mutex>
 #include <new>
 #include <numeric>
+#include <stdexcept>
 #include <vector>
 
 #include "plan.h"
@@ -182,6 +183,11 @@ struct Scratch {
   std::vector<int32_t> n_mma_rows;
 };
 
+Scratch& scratch() {
+  static thread_local Scratch sc;
+  return sc;
+}
+
 }  // namespace
 
 HostBuf hostbuf_acquire(size_t n) {
@@ -230,6 +236,339 @@ void hostbuf_release(HostBuf& b) {
   b = HostBuf{};
 }
 
+// What the split and the image need from the pack stage.
+struct PackCounts {
+  int64_t unique_tokens = 0, read_tokens = 0;
+  int num_nodes = 0, num_shared = 0, num_kept = 0;
+};
+
+// Split, partial rows and image of a plan whose pack result (items, their
+// pages and requests) is given; fills plan->hdr, plan->image and plan->stats.
+static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& items, const std::vector<int32_t>& pages,
+                 const std::vector<int32_t>& queries, const PackCounts& pc, const int32_t* kv_lens,
+                 std::chrono::steady_clock::time_point t0) {
+  const int batch = plan->B, Hq = plan->Hq, Hkv = plan->Hkv, G = plan->G, D = plan->D, P = plan->P;
+  const pa_config* cfg = &plan->cfg;
+
+  // ---- split and tile selection
+  // Tile class by rows (requests x G): one request -> SIMT class (CUDA
+  // cores); two or more -> MMA class (tensor cores, query tiles of <= 128 rows).
+  // The two classes run as two concurrent launches of one CTA per SM each; k
+  // SMs take the MMA class, the rest the SIMT class.  k balances the two
+  // classes' estimated times:
+  //   T_simt(k) = SIMT tile bytes / ((num_sms - k) * kSimtBytesPerSmUs)
+  //   T_mma(k)  = sum over MMA tiles of max(bytes / kMmaBytesPerSmUs,
+  //               flops / kMmaFlopsPerSmUs) / k
+  // Both classes split their work stream-K: the (item, kv head) page runs are
+  // concatenated and cut into equal spans, one span per SIMT warp or per MMA
+  // CTA; a span may end inside an item, so partial rows appear only at span
+  // boundaries (long-KV splitting without a fixed chunk size).
+  const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
+  const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
+  const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
+  const double kMmaFlopsPerSmUs = 5.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
+  const int kMmaSegPages = 38;               // fixed cost of a 128-row tensor-core segment (q load, epilogue), in pages
+  // the epilogue's stores scale with the tile's rows: a tile of r rows pays
+  // kMmaSegPages * max(32, r) / 128
+  auto mma_seg_pages = [&](const ItemRec& it) -> int64_t {
+    const int rows = std::min(kMmaRowsPerCta, it.n_queries * G);
+    return (int64_t)kMmaSegPages * std::max(32, rows) / kMmaRowsPerCta;
+  };
+  const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
+  const double tile_bytes = 2.0 * 16 * D * 2;
+  int64_t simt_pages = 0, mma_pages = 0, mma_runs = 0, mma_seg_total = 0;
+  double mma_cost = 0;  // SM-us
+  for (const auto& it : items) {
+    const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
+    if (it.simt) {
+      // a SIMT work unit also pays a fixed latency (q rows, partial row,
+      // arrival): counted as kSimtSegPages more pages
+      simt_pages += np + kSimtSegPages * Hkv;
+    } else {
+      mma_pages += np;
+      mma_runs += Hkv;
+      mma_seg_total += mma_seg_pages(it) * Hkv;
+      // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
+      const double rows = kMmaRowsPerCta;
+      const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
+      mma_cost += (np + mma_seg_pages(it) * Hkv) * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
+    }
+  }
+  const int S = plan->num_sms;
+  int n_mma = 0;  // SMs given to the MMA class
+  if (mma_pages > 0 && simt_pages == 0) {
+    n_mma = S;
+  } else if (mma_pages > 0) {
+    // T_simt = A / (S - k) and T_mma = C / k are equal at k = S C / (A + C);
+    // take the better of the two integers around it; no more CTAs than
+    // 16-page spans of tensor-core work
+    const double A = simt_pages * tile_bytes / kSimtBytesPerSmUs, C = mma_cost;
+    const int k_cap = (int)std::min<int64_t>(S - 1, std::max<int64_t>(1, ceil_div(mma_pages, 16)));
+    const int k0 = std::max(1, std::min(k_cap, (int)(S * C / (A + C))));
+    double best = 1e300;
+    for (int kk = k0; kk <= std::min(k_cap, k0 + 1); ++kk) {
+      const double t = std::max(A / (S - kk), C / kk);
+      if (t < best) { best = t; n_mma = kk; }
+    }
+  }
+  std::vector<SegRec>& simt_segs = sc.simt_segs;
+  std::vector<SegRec>& mma_segs = sc.mma_segs;
+  std::vector<int32_t>& warp_segs = sc.warp_segs;
+  std::vector<int32_t>& mma_cta_segs = sc.mma_cta_segs;
+  simt_segs.clear();
+  mma_segs.clear();
+  warp_segs.assign(1, 0);
+  mma_cta_segs.assign(1, 0);
+  if (simt_pages > 0) {
+    const int64_t W = (int64_t)(S - n_mma) * kSimtWarpsPerCta;
+    int64_t span = ceil_div(simt_pages, W);
+    if (span < 4) span = 4;
+    if (max_chunk_pages) span = std::min(span, max_chunk_pages);
+    simt_segs.reserve(items.size() * Hkv + simt_pages / span + 8);
+    int64_t used = 0;  // pages in the current warp's span
+    for (size_t i = 0; i < items.size(); ++i) {
+      const ItemRec& it = items[i];
+      if (!it.simt) continue;
+      const int npages = (int)ceil_div(it.n_tokens, P);
+      const int b = queries[it.query_off];
+      for (int g = 0; g < Hkv; ++g) {
+        int pb = 0;
+        used += kSimtSegPages;  // the unit's fixed cost
+        while (pb < npages) {
+          const int take = (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
+          const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
+          simt_segs.push_back({(int)i, g, pb, tok, -1, b});
+          pb += take;
+          used += take;
+          if (used >= span && (int64_t)warp_segs.size() < W) {  // never more than W warps
+            warp_segs.push_back((int32_t)simt_segs.size());
+            used = 0;
+          }
+        }
+      }
+    }
+    if (used > 0) warp_segs.push_back((int32_t)simt_segs.size());
+  }
+  if (mma_pages > 0) {
+    // each (item, kv head) run is a segment, and so is each cut at a CTA boundary
+    int64_t span = ceil_div(mma_pages + mma_seg_total + mma_seg_total / std::max<int64_t>(1, mma_runs) * n_mma, n_mma);
+    if (span < 16) span = 16;
+    if (max_chunk_pages) span = std::min(span, max_chunk_pages);
+    int64_t used = 0;
+    for (size_t i = 0; i < items.size(); ++i) {
+      const ItemRec& it = items[i];
+      if (it.simt) continue;
+      const int npages = (int)ceil_div(it.n_tokens, P);
+      for (int g = 0; g < Hkv; ++g) {
+        int pb = 0;
+        while (pb < npages) {
+          // never more than n_mma CTAs: the last one takes whatever is left
+          const int64_t seg_cost = mma_seg_pages(it);
+          bool last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
+          if (!last_cta && used > 0 && span - used - seg_cost < 4) {
+            // no room for a stage after the segment's fixed cost: next CTA
+            mma_cta_segs.push_back((int32_t)mma_segs.size());
+            used = 0;
+            last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
+          }
+          used += seg_cost;  // the segment's fixed cost
+          const int take = last_cta ? npages - pb
+                                    : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
+          const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
+          mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
+          pb += take;
+          used += take;
+          if (!last_cta && used >= span) {
+            mma_cta_segs.push_back((int32_t)mma_segs.size());
+            used = 0;
+          }
+        }
+      }
+    }
+    if (used > 0) mma_cta_segs.push_back((int32_t)mma_segs.size());
+  }
+
+  // ---- partial rows: contiguous per (request, kv head), in a fixed order
+  std::vector<int32_t>& prow_off = sc.prow_off;
+  prow_off.assign((size_t)batch * Hkv + 1, 0);
+  for (const auto& s : mma_segs) {
+    const ItemRec& it = items[s.item];
+    for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
+  }
+  // fused merge: the last SIMT partial row of a pair to be written merges the
+  // pair (after the tensor-core launch has finished if the pair also has
+  // tensor-core rows); pairs with tensor-core rows only are merged by the
+  // tail merge launch
+  std::vector<int32_t>& n_mma_rows = sc.n_mma_rows;
+  n_mma_rows.assign(prow_off.begin() + 1, prow_off.end());
+  for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
+  // a SIMT warp defers the merges of its mixed pairs to the end of its work;
+  // if some warp would defer more than kSimtMaxDeferred, every mixed pair
+  // goes to the tail merge launch instead
+  bool mixed_to_tail = false;
+  if (!mma_segs.empty()) {
+    for (size_t w = 0; w + 1 < warp_segs.size() && !mixed_to_tail; ++w) {
+      int n = 0;
+      for (int si = warp_segs[w]; si < warp_segs[w + 1]; ++si)
+        n += n_mma_rows[(size_t)simt_segs[si].query * Hkv + simt_segs[si].kv_head] > 0;
+      mixed_to_tail = n > kSimtMaxDeferred;
+    }
+  }
+  std::vector<int32_t>& tail_pairs = sc.tail_pairs;
+  tail_pairs.clear();
+  for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
+    if (n_mma_rows[bg] > 0 && (mixed_to_tail || prow_off[bg + 1] == n_mma_rows[bg]))
+      tail_pairs.push_back((int32_t)bg);
+  for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
+  std::vector<int32_t>& cursor = sc.cursor;
+  cursor.assign(prow_off.begin(), prow_off.end() - 1);
+  std::vector<int32_t>& seg_prows = sc.seg_prows;
+  seg_prows.clear();
+  for (auto& s : mma_segs) {
+    const ItemRec& it = items[s.item];
+    s.prow = (int)seg_prows.size();
+    for (int j = 0; j < it.n_queries; ++j)
+      seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
+  }
+  for (auto& s : simt_segs) s.prow = cursor[(size_t)s.query * Hkv + s.kv_head]++;
+  const int num_prows = prow_off.back();
+
+  // ---- image
+  pa_image_header& h = plan->hdr;
+  std::memset(&h, 0, sizeof(h));
+  h.magic = 0x50414231u;
+  h.batch = batch;
+  h.num_q_heads = Hq;
+  h.num_kv_heads = Hkv;
+  h.head_dim = D;
+  h.page_size = P;
+  h.num_items = (int32_t)items.size();
+  h.num_segments_simt = (int32_t)simt_segs.size();
+  h.num_segments_mma = (int32_t)mma_segs.size();
+  h.num_segments = h.num_segments_simt + h.num_segments_mma;
+  h.simt_warps = (int32_t)warp_segs.size() - 1;
+  h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
+  h.num_partial_rows = num_prows;
+  h.num_tail_pairs = (int32_t)tail_pairs.size();
+  uint64_t off = align256(sizeof(pa_image_header));
+  h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
+  h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
+  h.off_pages = off; off = align256(off + pages.size() * 4);
+  h.off_queries = off; off = align256(off + queries.size() * 4);
+  h.off_seg_prows = off; off = align256(off + seg_prows.size() * 4);
+  h.off_mma_segs = off; off = align256(off + mma_cta_segs.size() * 4);
+  h.off_counters = off; off = align256(off + (size_t)batch * Hkv * 4);
+  h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
+  h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
+  h.off_tail_pairs = off; off = align256(off + tail_pairs.size() * 4);
+  h.image_bytes = off;
+  h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
+  h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
+  h.workspace_bytes = off;
+
+  uint8_t* lent = t_sink ? t_sink(h.image_bytes, t_sink_ctx) : nullptr;
+  if (lent) {
+    plan->image.ptr = lent;
+    plan->image.size = plan->image.cap = h.image_bytes;
+    plan->image.owned = false;
+  } else {
+    plan->image = hostbuf_acquire(h.image_bytes);
+  }
+  uint8_t* img = plan->image.data();
+  std::memcpy(img, &h, sizeof(h));
+  std::memset(img + h.off_counters, 0, (size_t)batch * Hkv * 4);
+  pa_item* di = reinterpret_cast<pa_item*>(img + h.off_nodes);
+  for (size_t i = 0; i < items.size(); ++i)
+    di[i] = {items[i].page_off, items[i].n_tokens, items[i].n_queries, items[i].query_off};
+  pa_seg* ds = reinterpret_cast<pa_seg*>(img + h.off_segs);
+  size_t k = 0;
+  for (const auto& s : simt_segs) {
+    const size_t bg = (size_t)s.query * Hkv + s.kv_head;
+    const int n_rows = prow_off[bg + 1] - prow_off[bg], n_simt = n_rows - n_mma_rows[bg];
+    const int mode = n_mma_rows[bg] > 0 ? (mixed_to_tail ? 3 : 2) : n_rows == 1 ? 1 : 0;
+    const int sole = mode | (n_simt << 2);
+    ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
+               items[s.item].page_off + s.page_begin};
+  }
+  for (const auto& s : mma_segs)
+    ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, items[s.item].page_off + s.page_begin};
+  auto put = [&](uint64_t o, const std::vector<int32_t>& v) {
+    if (!v.empty()) std::memcpy(img + o, v.data(), v.size() * 4);
+  };
+  put(h.off_pages, pages);
+  put(h.off_queries, queries);
+  put(h.off_seg_prows, seg_prows);
+  put(h.off_mma_segs, mma_cta_segs);
+  put(h.off_warp_segs, warp_segs);
+  put(h.off_prow_off, prow_off);
+  put(h.off_tail_pairs, tail_pairs);
+  // the alignment gaps after the regions are zeroed: the image depends on the inputs only
+  const uint64_t region_end[] = {sizeof(h),
+                                 h.off_nodes + items.size() * sizeof(pa_item),
+                                 h.off_segs + (uint64_t)h.num_segments * sizeof(pa_seg),
+                                 h.off_pages + pages.size() * 4,
+                                 h.off_queries + queries.size() * 4,
+                                 h.off_seg_prows + seg_prows.size() * 4,
+                                 h.off_mma_segs + mma_cta_segs.size() * 4,
+                                 h.off_counters + (uint64_t)batch * Hkv * 4,
+                                 h.off_warp_segs + warp_segs.size() * 4,
+                                 h.off_prow_off + prow_off.size() * 4,
+                                 h.off_tail_pairs + tail_pairs.size() * 4};
+  for (const uint64_t e : region_end) std::memset(img + e, 0, align256(e) - e);
+
+  pa_plan_stats& st = plan->stats;
+  st.batch = batch;
+  st.num_nodes = pc.num_nodes;
+  st.num_shared_nodes = pc.num_shared;
+  st.num_kept_shared = pc.num_kept;
+  st.num_items = (int32_t)items.size();
+  st.num_segments = h.num_segments;
+  st.num_segments_simt = h.num_segments_simt;
+  st.num_segments_mma = h.num_segments_mma;
+  st.num_partial_rows = num_prows;
+  st.simt_warps = h.simt_warps;
+  st.mma_ctas = h.mma_ctas;
+  st.num_tail_pairs = h.num_tail_pairs;
+  st.unique_tokens = pc.unique_tokens;
+  int64_t naive = 0;
+  for (int b = 0; b < batch; ++b) naive += kv_lens[b];
+  st.naive_tokens = naive;
+  st.read_tokens = pc.read_tokens;
+  st.unique_kv_bytes = pc.unique_tokens * (int64_t)(2 * Hkv * D * 2);
+  st.read_kv_bytes = pc.read_tokens * (int64_t)(2 * Hkv * D * 2);
+  st.workspace_bytes = h.workspace_bytes;
+  st.image_bytes = h.image_bytes;
+  st.plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+}
+
+// Stores the pack result in the plan (PA_PLAN_KEEP_PACK) for pa_plan_advance.
+static void keep_pack(pa_plan* plan, const std::vector<ItemRec>& items, const std::vector<int32_t>& pages,
+                      const std::vector<int32_t>& queries, const PackCounts& pc, const int32_t* kv_lens) {
+  plan->pk_items.resize(items.size() * 5);
+  for (size_t i = 0; i < items.size(); ++i) {
+    int32_t* r = &plan->pk_items[i * 5];
+    r[0] = items[i].page_off;
+    r[1] = items[i].n_tokens;
+    r[2] = items[i].n_queries;
+    r[3] = items[i].query_off;
+    r[4] = items[i].simt ? 1 : 0;
+  }
+  plan->pk_pages = pages;
+  plan->pk_queries = queries;
+  plan->pk_kv_lens.assign(kv_lens, kv_lens + plan->B);
+  // a request's one-request item (there is at most one: it ends at the
+  // request's last page)
+  plan->pk_suffix.assign(plan->B, -1);
+  for (size_t i = 0; i < items.size(); ++i)
+    if (items[i].simt) plan->pk_suffix[queries[items[i].query_off]] = (int32_t)i;
+  plan->pk_unique_tokens = pc.unique_tokens;
+  plan->pk_read_tokens = pc.read_tokens;
+  plan->pk_num_nodes = pc.num_nodes;
+  plan->pk_num_shared = pc.num_shared;
+  plan->pk_num_kept = pc.num_kept;
+  plan->has_pack = true;
+}
+
 extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const int32_t* kv_lens,
                                     const int32_t* block_table, int32_t max_pages, int32_t num_pages_in_pool,
                                     pa_plan** out) {
@@ -267,7 +606,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     plan->wait_timeout_us = cfg->wait_timeout_us > 0 ? cfg->wait_timeout_us : 2000000;
 
     // ---- validation
-    static thread_local Scratch sc;
+    Scratch& sc = scratch();
     sc.items.clear();
     sc.pages.clear();
     sc.queries.clear();
@@ -303,296 +642,136 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     const std::vector<ItemRec>& items = pl.items;
     const std::vector<int32_t>& pages = pl.pages;
     const std::vector<int32_t>& queries = pl.queries;
+    PackCounts pc;
+    pc.unique_tokens = pl.unique_tokens;
+    pc.read_tokens = pl.read_tokens;
+    pc.num_nodes = pl.num_nodes;
+    pc.num_shared = pl.num_shared;
+    pc.num_kept = pl.num_kept;
+    finish_plan(plan, sc, items, pages, queries, pc, kv_lens, t0);
+    if (flags & PA_PLAN_KEEP_PACK) keep_pack(plan, items, pages, queries, pc, kv_lens);
+    *out = plan;
+    return PA_OK;
+  } catch (const std::bad_alloc&) {
+    delete plan;
+    return PA_ERR_NOMEM;
+  } catch (...) {
+    delete plan;
+    return PA_ERR_INVALID;
+  }
+}
 
-    // ---- split and tile selection
-    // Tile class by rows (requests x G): one request -> SIMT class (CUDA
-    // cores); two or more -> MMA class (tensor cores, query tiles of <= 128 rows).
-    // The two classes run as two concurrent launches of one CTA per SM each; k
-    // SMs take the MMA class, the rest the SIMT class.  k balances the two
-    // classes' estimated times:
-    //   T_simt(k) = SIMT tile bytes / ((num_sms - k) * kSimtBytesPerSmUs)
-    //   T_mma(k)  = sum over MMA tiles of max(bytes / kMmaBytesPerSmUs,
-    //               flops / kMmaFlopsPerSmUs) / k
-    // Both classes split their work stream-K: the (item, kv head) page runs are
-    // concatenated and cut into equal spans, one span per SIMT warp or per MMA
-    // CTA; a span may end inside an item, so partial rows appear only at span
-    // boundaries (long-KV splitting without a fixed chunk size).
-    const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
-    const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
-    const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
-    const double kMmaFlopsPerSmUs = 5.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
-    const int kMmaSegPages = 38;               // fixed cost of a 128-row tensor-core segment (q load, epilogue), in pages
-    // the epilogue's stores scale with the tile's rows: a tile of r rows pays
-    // kMmaSegPages * max(32, r) / 128
-    auto mma_seg_pages = [&](const ItemRec& it) -> int64_t {
-      const int rows = std::min(kMmaRowsPerCta, it.n_queries * G);
-      return (int64_t)kMmaSegPages * std::max(32, rows) / kMmaRowsPerCta;
+extern "C" pa_status pa_plan_advance(const pa_plan* prev, const int32_t* kv_lens, const int32_t* block_table,
+                                     int32_t max_pages, int32_t num_pages_in_pool, pa_plan** out) {
+  if (out) *out = nullptr;
+  if (!prev || !prev->has_pack || !kv_lens || !block_table || !out) return PA_ERR_INVALID;
+  auto t0 = std::chrono::steady_clock::now();
+  const int batch = prev->B, P = prev->P, Hkv = prev->Hkv;
+  if (max_pages < 1 || num_pages_in_pool < 1) return PA_ERR_INVALID;
+  if ((int64_t)num_pages_in_pool * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  bool rebuild = num_pages_in_pool < prev->num_pages_in_pool;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t n = kv_lens[b];
+    if (n < 1 || n > (int64_t)max_pages * P) return PA_ERR_INVALID;
+    if (n < prev->pk_kv_lens[b]) rebuild = true;
+  }
+  if (rebuild) {
+    const pa_status st = pa_plan_create(&prev->cfg, batch, kv_lens, block_table, max_pages, num_pages_in_pool, out);
+    if (st == PA_OK) (*out)->stats.plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+    return st;
+  }
+
+  pa_plan* plan = new (std::nothrow) pa_plan();
+  if (!plan) return PA_ERR_NOMEM;
+  try {
+    plan->cfg = prev->cfg;
+    plan->B = batch;
+    plan->Hq = prev->Hq;
+    plan->Hkv = Hkv;
+    plan->G = prev->G;
+    plan->D = prev->D;
+    plan->P = P;
+    plan->num_pages_in_pool = num_pages_in_pool;
+    plan->scale = prev->scale;
+    plan->num_sms = prev->num_sms;
+    plan->flags = prev->flags;
+    plan->wait_timeout_us = prev->wait_timeout_us;
+
+    Scratch& sc = scratch();
+    std::vector<ItemRec>& items = sc.items;
+    std::vector<int32_t>& pages = sc.pages;
+    std::vector<int32_t>& queries = sc.queries;
+    const size_t n_items_prev = prev->pk_items.size() / 5;
+    items.clear();
+    pages.clear();
+    queries.assign(prev->pk_queries.begin(), prev->pk_queries.end());
+    pages.reserve(prev->pk_pages.size() + 2 * (size_t)batch);
+    items.reserve(n_items_prev + batch);
+    PackCounts pc;
+    pc.unique_tokens = prev->pk_unique_tokens;
+    pc.read_tokens = prev->pk_read_tokens;
+    pc.num_nodes = prev->pk_num_nodes;
+    pc.num_shared = prev->pk_num_shared;
+    pc.num_kept = prev->pk_num_kept;
+    uint32_t bad = 0;
+    auto row = [&](int b) { return block_table + (size_t)b * max_pages; };
+    auto append_pages = [&](int b, int from, int to) {
+      const int32_t* r = row(b);
+      for (int j = from; j < to; ++j) {
+        bad |= (uint32_t)r[j] >= (uint32_t)num_pages_in_pool ? 1u : 0u;
+        pages.push_back(r[j]);
+      }
     };
-    const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
-    const double tile_bytes = 2.0 * 16 * D * 2;
-    int64_t simt_pages = 0, mma_pages = 0, mma_runs = 0, mma_seg_total = 0;
-    double mma_cost = 0;  // SM-us
-    for (const auto& it : items) {
-      const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
-      if (it.simt) {
-        // a SIMT work unit also pays a fixed latency (q rows, partial row,
-        // arrival): counted as kSimtSegPages more pages
-        simt_pages += np + kSimtSegPages * Hkv;
+    // the items in their old order; tiles of one node keep sharing their pages
+    int last_old_off = -1, last_new_off = -1;
+    for (size_t i = 0; i < n_items_prev; ++i) {
+      const int32_t* r = &prev->pk_items[i * 5];
+      ItemRec it{r[0], r[1], r[2], r[3], r[4] != 0};
+      const int np_old = (int)ceil_div(it.n_tokens, P);
+      if (!it.simt && it.page_off == last_old_off) {
+        it.page_off = last_new_off;  // another query tile of the same node
       } else {
-        mma_pages += np;
-        mma_runs += Hkv;
-        mma_seg_total += mma_seg_pages(it) * Hkv;
-        // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
-        const double rows = kMmaRowsPerCta;
-        const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
-        mma_cost += (np + mma_seg_pages(it) * Hkv) * std::max(tile_bytes / kMmaBytesPerSmUs, flops / kMmaFlopsPerSmUs);
-      }
-    }
-    const int S = plan->num_sms;
-    int n_mma = 0;  // SMs given to the MMA class
-    if (mma_pages > 0 && simt_pages == 0) {
-      n_mma = S;
-    } else if (mma_pages > 0) {
-      // T_simt = A / (S - k) and T_mma = C / k are equal at k = S C / (A + C);
-      // take the better of the two integers around it; no more CTAs than
-      // 16-page spans of tensor-core work
-      const double A = simt_pages * tile_bytes / kSimtBytesPerSmUs, C = mma_cost;
-      const int k_cap = (int)std::min<int64_t>(S - 1, std::max<int64_t>(1, ceil_div(mma_pages, 16)));
-      const int k0 = std::max(1, std::min(k_cap, (int)(S * C / (A + C))));
-      double best = 1e300;
-      for (int kk = k0; kk <= std::min(k_cap, k0 + 1); ++kk) {
-        const double t = std::max(A / (S - kk), C / kk);
-        if (t < best) { best = t; n_mma = kk; }
-      }
-    }
-    std::vector<SegRec>& simt_segs = sc.simt_segs;
-    std::vector<SegRec>& mma_segs = sc.mma_segs;
-    std::vector<int32_t>& warp_segs = sc.warp_segs;
-    std::vector<int32_t>& mma_cta_segs = sc.mma_cta_segs;
-    simt_segs.clear();
-    mma_segs.clear();
-    warp_segs.assign(1, 0);
-    mma_cta_segs.assign(1, 0);
-    if (simt_pages > 0) {
-      const int64_t W = (int64_t)(S - n_mma) * kSimtWarpsPerCta;
-      int64_t span = ceil_div(simt_pages, W);
-      if (span < 4) span = 4;
-      if (max_chunk_pages) span = std::min(span, max_chunk_pages);
-      simt_segs.reserve(items.size() * Hkv + simt_pages / span + 8);
-      int64_t used = 0;  // pages in the current warp's span
-      for (size_t i = 0; i < items.size(); ++i) {
-        const ItemRec& it = items[i];
-        if (!it.simt) continue;
-        const int npages = (int)ceil_div(it.n_tokens, P);
-        const int b = queries[it.query_off];
-        for (int g = 0; g < Hkv; ++g) {
-          int pb = 0;
-          used += kSimtSegPages;  // the unit's fixed cost
-          while (pb < npages) {
-            const int take = (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
-            const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
-            simt_segs.push_back({(int)i, g, pb, tok, -1, b});
-            pb += take;
-            used += take;
-            if (used >= span && (int64_t)warp_segs.size() < W) {  // never more than W warps
-              warp_segs.push_back((int32_t)simt_segs.size());
-              used = 0;
-            }
+        const int new_off = (int)pages.size();
+        pages.insert(pages.end(), prev->pk_pages.begin() + it.page_off, prev->pk_pages.begin() + it.page_off + np_old);
+        last_old_off = it.page_off;
+        last_new_off = new_off;
+        it.page_off = new_off;
+        if (it.simt) {
+          // the request's own tail: it takes the new tokens and pages
+          const int b = queries[it.query_off];
+          const int64_t grow = (int64_t)kv_lens[b] - prev->pk_kv_lens[b];
+          if (grow > 0) {
+            const int npg_old = (int)ceil_div(prev->pk_kv_lens[b], P), npg_new = (int)ceil_div(kv_lens[b], P);
+            append_pages(b, npg_old, npg_new);
+            it.n_tokens += (int)grow;
+            pc.unique_tokens += grow;
+            pc.read_tokens += grow;
           }
         }
       }
-      if (used > 0) warp_segs.push_back((int32_t)simt_segs.size());
+      items.push_back(it);
     }
-    if (mma_pages > 0) {
-      // each (item, kv head) run is a segment, and so is each cut at a CTA boundary
-      int64_t span = ceil_div(mma_pages + mma_seg_total + mma_seg_total / std::max<int64_t>(1, mma_runs) * n_mma, n_mma);
-      if (span < 16) span = 16;
-      if (max_chunk_pages) span = std::min(span, max_chunk_pages);
-      int64_t used = 0;
-      for (size_t i = 0; i < items.size(); ++i) {
-        const ItemRec& it = items[i];
-        if (it.simt) continue;
-        const int npages = (int)ceil_div(it.n_tokens, P);
-        for (int g = 0; g < Hkv; ++g) {
-          int pb = 0;
-          while (pb < npages) {
-            // never more than n_mma CTAs: the last one takes whatever is left
-            const int64_t seg_cost = mma_seg_pages(it);
-            bool last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
-            if (!last_cta && used > 0 && span - used - seg_cost < 4) {
-              // no room for a stage after the segment's fixed cost: next CTA
-              mma_cta_segs.push_back((int32_t)mma_segs.size());
-              used = 0;
-              last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
-            }
-            used += seg_cost;  // the segment's fixed cost
-            const int take = last_cta ? npages - pb
-                                      : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
-            const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
-            mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
-            pb += take;
-            used += take;
-            if (!last_cta && used >= span) {
-              mma_cta_segs.push_back((int32_t)mma_segs.size());
-              used = 0;
-            }
-          }
-        }
-      }
-      if (used > 0) mma_cta_segs.push_back((int32_t)mma_segs.size());
+    // requests that ended at the end of a shared node: a new tail item
+    for (int b = 0; b < batch; ++b) {
+      const int64_t grow = (int64_t)kv_lens[b] - prev->pk_kv_lens[b];
+      if (prev->pk_suffix[b] >= 0 || grow <= 0) continue;
+      const int npg_old = (int)ceil_div(prev->pk_kv_lens[b], P), npg_new = (int)ceil_div(kv_lens[b], P);
+      if ((int64_t)npg_old * P != prev->pk_kv_lens[b]) throw std::logic_error("request ends inside a shared page");
+      const int off = (int)pages.size();
+      append_pages(b, npg_old, npg_new);
+      items.push_back({off, (int)grow, 1, (int)queries.size(), true});
+      queries.push_back(b);
+      ++pc.num_nodes;
+      pc.unique_tokens += grow;
+      pc.read_tokens += grow;
     }
-
-    // ---- partial rows: contiguous per (request, kv head), in a fixed order
-    std::vector<int32_t>& prow_off = sc.prow_off;
-    prow_off.assign((size_t)batch * Hkv + 1, 0);
-    for (const auto& s : mma_segs) {
-      const ItemRec& it = items[s.item];
-      for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
+    if (bad) {
+      delete plan;
+      return PA_ERR_INVALID;
     }
-    // fused merge: the last SIMT partial row of a pair to be written merges the
-    // pair (after the tensor-core launch has finished if the pair also has
-    // tensor-core rows); pairs with tensor-core rows only are merged by the
-    // tail merge launch
-    std::vector<int32_t>& n_mma_rows = sc.n_mma_rows;
-    n_mma_rows.assign(prow_off.begin() + 1, prow_off.end());
-    for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
-    // a SIMT warp defers the merges of its mixed pairs to the end of its work;
-    // if some warp would defer more than kSimtMaxDeferred, every mixed pair
-    // goes to the tail merge launch instead
-    bool mixed_to_tail = false;
-    if (!mma_segs.empty()) {
-      for (size_t w = 0; w + 1 < warp_segs.size() && !mixed_to_tail; ++w) {
-        int n = 0;
-        for (int si = warp_segs[w]; si < warp_segs[w + 1]; ++si)
-          n += n_mma_rows[(size_t)simt_segs[si].query * Hkv + simt_segs[si].kv_head] > 0;
-        mixed_to_tail = n > kSimtMaxDeferred;
-      }
-    }
-    std::vector<int32_t>& tail_pairs = sc.tail_pairs;
-    tail_pairs.clear();
-    for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
-      if (n_mma_rows[bg] > 0 && (mixed_to_tail || prow_off[bg + 1] == n_mma_rows[bg]))
-        tail_pairs.push_back((int32_t)bg);
-    for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
-    std::vector<int32_t>& cursor = sc.cursor;
-    cursor.assign(prow_off.begin(), prow_off.end() - 1);
-    std::vector<int32_t>& seg_prows = sc.seg_prows;
-    seg_prows.clear();
-    for (auto& s : mma_segs) {
-      const ItemRec& it = items[s.item];
-      s.prow = (int)seg_prows.size();
-      for (int j = 0; j < it.n_queries; ++j)
-        seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
-    }
-    for (auto& s : simt_segs) s.prow = cursor[(size_t)s.query * Hkv + s.kv_head]++;
-    const int num_prows = prow_off.back();
-
-    // ---- image
-    pa_image_header& h = plan->hdr;
-    std::memset(&h, 0, sizeof(h));
-    h.magic = 0x50414231u;
-    h.batch = batch;
-    h.num_q_heads = Hq;
-    h.num_kv_heads = Hkv;
-    h.head_dim = D;
-    h.page_size = P;
-    h.num_items = (int32_t)items.size();
-    h.num_segments_simt = (int32_t)simt_segs.size();
-    h.num_segments_mma = (int32_t)mma_segs.size();
-    h.num_segments = h.num_segments_simt + h.num_segments_mma;
-    h.simt_warps = (int32_t)warp_segs.size() - 1;
-    h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
-    h.num_partial_rows = num_prows;
-    h.num_tail_pairs = (int32_t)tail_pairs.size();
-    uint64_t off = align256(sizeof(pa_image_header));
-    h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
-    h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
-    h.off_pages = off; off = align256(off + pages.size() * 4);
-    h.off_queries = off; off = align256(off + queries.size() * 4);
-    h.off_seg_prows = off; off = align256(off + seg_prows.size() * 4);
-    h.off_mma_segs = off; off = align256(off + mma_cta_segs.size() * 4);
-    h.off_counters = off; off = align256(off + (size_t)batch * Hkv * 4);
-    h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
-    h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
-    h.off_tail_pairs = off; off = align256(off + tail_pairs.size() * 4);
-    h.image_bytes = off;
-    h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
-    h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
-    h.workspace_bytes = off;
-
-    uint8_t* lent = t_sink ? t_sink(h.image_bytes, t_sink_ctx) : nullptr;
-    if (lent) {
-      plan->image.ptr = lent;
-      plan->image.size = plan->image.cap = h.image_bytes;
-      plan->image.owned = false;
-    } else {
-      plan->image = hostbuf_acquire(h.image_bytes);
-    }
-    uint8_t* img = plan->image.data();
-    std::memcpy(img, &h, sizeof(h));
-    std::memset(img + h.off_counters, 0, (size_t)batch * Hkv * 4);
-    pa_item* di = reinterpret_cast<pa_item*>(img + h.off_nodes);
-    for (size_t i = 0; i < items.size(); ++i)
-      di[i] = {items[i].page_off, items[i].n_tokens, items[i].n_queries, items[i].query_off};
-    pa_seg* ds = reinterpret_cast<pa_seg*>(img + h.off_segs);
-    size_t k = 0;
-    for (const auto& s : simt_segs) {
-      const size_t bg = (size_t)s.query * Hkv + s.kv_head;
-      const int n_rows = prow_off[bg + 1] - prow_off[bg], n_simt = n_rows - n_mma_rows[bg];
-      const int mode = n_mma_rows[bg] > 0 ? (mixed_to_tail ? 3 : 2) : n_rows == 1 ? 1 : 0;
-      const int sole = mode | (n_simt << 2);
-      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
-                 items[s.item].page_off + s.page_begin};
-    }
-    for (const auto& s : mma_segs)
-      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, items[s.item].page_off + s.page_begin};
-    auto put = [&](uint64_t o, const std::vector<int32_t>& v) {
-      if (!v.empty()) std::memcpy(img + o, v.data(), v.size() * 4);
-    };
-    put(h.off_pages, pages);
-    put(h.off_queries, queries);
-    put(h.off_seg_prows, seg_prows);
-    put(h.off_mma_segs, mma_cta_segs);
-    put(h.off_warp_segs, warp_segs);
-    put(h.off_prow_off, prow_off);
-    put(h.off_tail_pairs, tail_pairs);
-    // the alignment gaps after the regions are zeroed: the image depends on the inputs only
-    const uint64_t region_end[] = {sizeof(h),
-                                   h.off_nodes + items.size() * sizeof(pa_item),
-                                   h.off_segs + (uint64_t)h.num_segments * sizeof(pa_seg),
-                                   h.off_pages + pages.size() * 4,
-                                   h.off_queries + queries.size() * 4,
-                                   h.off_seg_prows + seg_prows.size() * 4,
-                                   h.off_mma_segs + mma_cta_segs.size() * 4,
-                                   h.off_counters + (uint64_t)batch * Hkv * 4,
-                                   h.off_warp_segs + warp_segs.size() * 4,
-                                   h.off_prow_off + prow_off.size() * 4,
-                                   h.off_tail_pairs + tail_pairs.size() * 4};
-    for (const uint64_t e : region_end) std::memset(img + e, 0, align256(e) - e);
-
-    pa_plan_stats& st = plan->stats;
-    st.batch = batch;
-    st.num_nodes = pl.num_nodes;
-    st.num_shared_nodes = pl.num_shared;
-    st.num_kept_shared = pl.num_kept;
-    st.num_items = (int32_t)items.size();
-    st.num_segments = h.num_segments;
-    st.num_segments_simt = h.num_segments_simt;
-    st.num_segments_mma = h.num_segments_mma;
-    st.num_partial_rows = num_prows;
-    st.simt_warps = h.simt_warps;
-    st.mma_ctas = h.mma_ctas;
-    st.num_tail_pairs = h.num_tail_pairs;
-    st.unique_tokens = pl.unique_tokens;
-    int64_t naive = 0;
-    for (int b = 0; b < batch; ++b) naive += kv_lens[b];
-    st.naive_tokens = naive;
-    st.read_tokens = pl.read_tokens;
-    st.unique_kv_bytes = pl.unique_tokens * (int64_t)(2 * Hkv * D * 2);
-    st.read_kv_bytes = pl.read_tokens * (int64_t)(2 * Hkv * D * 2);
-    st.workspace_bytes = h.workspace_bytes;
-    st.image_bytes = h.image_bytes;
-    st.plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+    finish_plan(plan, sc, items, pages, queries, pc, kv_lens, t0);
+    keep_pack(plan, items, pages, queries, pc, kv_lens);
+    plan->stats.plan_us = std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
     *out = plan;
     return PA_OK;
   } catch (const std::bad_alloc&) {

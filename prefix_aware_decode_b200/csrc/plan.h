@@ -60,6 +60,14 @@ struct pa_plan {
   // device copy of the image when it lives outside the caller's workspace
   // (pa_decode_step's image ring); nullptr: at the workspace base
   void* dev_image = nullptr;
+  // the pack result (PA_PLAN_KEEP_PACK), from which pa_plan_advance plans the
+  // next decode step: items (page_off, n_tokens, n_queries, query_off, simt),
+  // their pages and requests, each request's kv_len and one-request item (-1:
+  // none), and the pack counters
+  bool has_pack = false;
+  std::vector<int32_t> pk_items, pk_pages, pk_queries, pk_kv_lens, pk_suffix;
+  int64_t pk_unique_tokens = 0, pk_read_tokens = 0;
+  int pk_num_nodes = 0, pk_num_shared = 0, pk_num_kept = 0;
 };
 
 // Kernel launchers (kernels.cu).  Return 0 or a cudaError_t value.

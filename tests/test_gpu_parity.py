@@ -226,6 +226,49 @@ def test_arrival_counters_return_to_zero_with_mixed_pairs():
     plan.close()
 
 
+def test_advanced_plan_on_the_device_matches_the_oracle():
+    # pa_plan_advance over a few decode steps of a config-2-shaped batch: the
+    # carried-over plan runs through the same kernels and matches the oracle
+    w = wl.make_config(2, scale=0.25)
+    P = w.P
+    rng = np.random.default_rng(11)
+    kv = w.kv_lens.astype(np.int32).copy()
+    bt = np.full((w.B, w.block_table.shape[1] + 2), -1, np.int32)
+    bt[:, :w.block_table.shape[1]] = w.block_table
+    spare = 2 * w.B
+    k = np.concatenate([w.k_pool, np.full((spare,) + w.k_pool.shape[1:], wl.BF16_NAN, np.uint16)])
+    v = np.concatenate([w.v_pool, np.full((spare,) + w.v_pool.shape[1:], wl.BF16_NAN, np.uint16)])
+    n_pages, free = w.num_pages + spare, w.num_pages
+    plan = pad.Plan(kv, bt, n_pages, w.Hq, w.Hkv, w.D, flags=pad.PA_PLAN_KEEP_PACK)
+    q = torch.from_numpy(w.q.view(np.int16)).cuda().view(torch.bfloat16)
+    for step in range(3):
+        for b in range(w.B):
+            for _ in range(int(rng.integers(1, 4))):
+                pos = int(kv[b])
+                if pos % P == 0:
+                    bt[b, pos // P] = free
+                    free += 1
+                page = bt[b, pos // P]
+                k[page, :, pos % P, :] = rng.normal(size=(w.Hkv, w.D)).astype(np.float32).view(np.uint32) >> 16
+                v[page, :, pos % P, :] = rng.normal(size=(w.Hkv, w.D)).astype(np.float32).view(np.uint32) >> 16
+                kv[b] += 1
+        nxt = plan.advance(kv, bt, n_pages)
+        plan.close()
+        plan = nxt
+        kd = torch.from_numpy(k.view(np.int16)).cuda().view(torch.bfloat16)
+        vd = torch.from_numpy(v.view(np.int16)).cuda().view(torch.bfloat16)
+        ws = plan.alloc_workspace()
+        plan.upload(ws)
+        out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        plan.attend(q, kd, vd, ws, out, lse)
+        torch.cuda.synchronize()
+        assert plan.device_status(ws) == pad.PA_OK
+        ref_o, ref_l = oracle.attend_paged(w.q, k, v, bt, kv)
+        assert_close(compare(out, lse, ref_o, ref_l), f"advanced plan, step {step}")
+    plan.close()
+
+
 def test_decode_steps_alternating_batches_and_one_plan_over_several_pools():
     # pa_decode_step uploads each step's plan into one of two device slots on a
     # copy stream of its own; alternating two different batches through the

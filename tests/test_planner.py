@@ -200,3 +200,116 @@ def test_tensor_core_spans_charge_a_cost_per_segment():
     many, few = segs >= np.percentile(segs, 75), segs <= np.percentile(segs, 25)
     assert many.any() and few.any() and segs[many].min() > segs[few].max()
     assert pages[many].mean() < pages[few].mean()
+
+
+# ------------------------------------------------------------- decode steps
+
+def decode_steps(w, steps, seed):
+    """Yields (kv_lens, block_table, k_pool, v_pool, num_pages) after each of
+    `steps` decode steps: every request appends 0-2 tokens (random bf16 K/V),
+    taking a fresh page of its own whenever its last page is full."""
+    rng = np.random.default_rng(seed)
+    P = w.P
+    kv = w.kv_lens.astype(np.int32).copy()
+    spare = w.B * (2 * steps // P + 2)
+    k = np.concatenate([w.k_pool, np.full((spare,) + w.k_pool.shape[1:], wl.BF16_NAN, np.uint16)])
+    v = np.concatenate([w.v_pool, np.full((spare,) + w.v_pool.shape[1:], wl.BF16_NAN, np.uint16)])
+    cols = w.block_table.shape[1] + 2 * steps // P + 2
+    bt = np.full((w.B, cols), -1, np.int32)
+    bt[:, :w.block_table.shape[1]] = w.block_table
+    free = w.num_pages
+    for _ in range(steps):
+        for b in range(w.B):
+            for _ in range(int(rng.integers(0, 3))):
+                pos = int(kv[b])
+                pg, slot = pos // P, pos % P
+                if slot == 0:
+                    bt[b, pg] = free
+                    free += 1
+                page = bt[b, pg]
+                k[page, :, slot, :] = rng.normal(size=(w.Hkv, w.D)).astype(np.float32).view(np.uint32) >> 16
+                v[page, :, slot, :] = rng.normal(size=(w.Hkv, w.D)).astype(np.float32).view(np.uint32) >> 16
+                kv[b] += 1
+        yield kv.copy(), bt.copy(), k, v, free
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_advanced_plans_execute_to_oracle(seed):
+    # pa_plan_advance: the tree of the first step is carried over; each
+    # request's own tail takes the new tokens.  Every step's plan must cover
+    # each token once and execute to the oracle, and count the same tokens as
+    # a plan made from scratch
+    G = [1, 2, 4, 8][seed % 4]
+    D = [64, 128][seed % 2]
+    roots = wl.random_tree(seed=300 + seed, n_queries=9, depth=3, shared_pages=(1, 4), leaf_tokens=(1, 40))
+    w = wl.build_workload("rand", roots, Hq=2 * G, Hkv=2, D=D, seed=700 + seed)
+    p = make_plan(w, flags=pad.PA_PLAN_KEEP_PACK, max_chunk_tokens=32 * (seed % 2))
+    for kv, bt, k, v, n_pages in decode_steps(w, steps=20, seed=seed):
+        p = p.advance(kv, bt, n_pages)
+        img = Image(p.host_image())
+        check_structure(img, kv, bt)
+        out, lse = execute(img, w.q, k, v)
+        ref_o, ref_l = oracle.attend_paged(w.q, k, v, bt, kv)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+        st = p.stats()
+        full = pad.Plan(kv, bt, n_pages, w.Hq, w.Hkv, w.D, max_chunk_tokens=32 * (seed % 2)).stats()
+        for key in ("unique_tokens", "naive_tokens", "read_tokens", "num_shared_nodes", "num_kept_shared"):
+            assert st[key] == full[key], key
+
+
+def test_advance_falls_back_and_checks_its_inputs():
+    roots = wl.random_tree(seed=41, n_queries=6, depth=2, shared_pages=(1, 3), leaf_tokens=(1, 40))
+    w = wl.build_workload("rand", roots, Hq=8, Hkv=2, D=64, seed=42)
+    kept = make_plan(w, flags=pad.PA_PLAN_KEEP_PACK)
+    # a plan made without PA_PLAN_KEEP_PACK cannot be advanced
+    with pytest.raises(pad.PaError) as e:
+        make_plan(w).advance(w.kv_lens, w.block_table, w.num_pages)
+    assert e.value.status == pad.PA_ERR_INVALID
+    # a request that shrank: planned from scratch, same structure as pa_plan_create
+    kv = w.kv_lens.copy()
+    b = int(np.argmax(kv))
+    kv[b] -= 1
+    p = kept.advance(kv, w.block_table, w.num_pages)
+    check_structure(Image(p.host_image()), kv, w.block_table)
+    assert p.stats()["unique_tokens"] == make_plan(w).stats()["unique_tokens"] - 1
+    # a new page id outside the pool is rejected
+    steps = decode_steps(w, steps=16, seed=3)
+    kv2, bt2, _, _, n_pages = next(steps)
+    grown = np.nonzero(kv2 > w.kv_lens)[0]
+    assert len(grown)
+    bad = bt2.copy()
+    for r in grown:
+        bad[r, (kv2[r] - 1) // 16] = n_pages + 5 if (kv2[r] - 1) // 16 >= (w.kv_lens[r] + 15) // 16 else bad[r, (kv2[r] - 1) // 16]
+    if np.array_equal(bad, bt2):
+        pytest.skip("no request took a new page in the first step")
+    with pytest.raises(pad.PaError) as e:
+        kept.advance(kv2, bad, n_pages)
+    assert e.value.status == pad.PA_ERR_INVALID
+
+
+def test_advance_gives_a_request_that_ended_at_a_shared_node_its_own_tail():
+    # request 0's KV is exactly the shared node [5, 6] of requests 0-2 (kept
+    # shared), so it has no item of its own; its next token goes to a new page
+    P, Hkv, D, Hq = 16, 1, 64, 4
+    rng = np.random.default_rng(5)
+    n_pages = 12
+    bf = lambda *s: (rng.normal(size=s).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    k, v = bf(n_pages, Hkv, P, D), bf(n_pages, Hkv, P, D)
+    q = bf(3, Hq, D)
+    bt = np.array([[5, 6, -1, -1], [5, 6, 7, -1], [5, 6, 8, 9]], dtype=np.int32)
+    kv = np.array([32, 40, 50], dtype=np.int32)
+    p = pad.Plan(kv, bt, n_pages, Hq, Hkv, D, flags=pad.PA_PLAN_ALWAYS_SHARE | pad.PA_PLAN_KEEP_PACK)
+    before = Image(p.host_image())
+    assert sum(1 for it in before.items if it[2] == 1 and int(before.queries[it[3]]) == 0) == 0
+    bt2 = bt.copy()
+    bt2[0, 2] = 10
+    for kv2 in (np.array([33, 41, 50], dtype=np.int32), np.array([40, 47, 51], dtype=np.int32)):
+        p2 = p.advance(kv2, bt2, n_pages)
+        img = Image(p2.host_image())
+        check_structure(img, kv2, bt2, P)
+        out, lse = execute(img, q, k, v)
+        ref_o, ref_l = oracle.attend_paged(q, k, v, bt2, kv2)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+        assert p2.stats()["num_kept_shared"] == 1
