@@ -121,8 +121,9 @@ pa_status pa_plan_create(const pa_config *cfg, int32_t batch, const int32_t *kv_
 
 /*
  * Pack for the next decode step of the same batch, from the previous step's
- * plan instead of a new walk of the block table (PAT, "Implementation": the
- * pack scheduler runs every decode step; here its tree is carried over).
+ * plan instead of a new walk of the block table (PAT review, section 六,
+ * overhead analysis, Figure 16: the pack scheduler runs at every decode step;
+ * here its tree is carried over from one step to the next).
  *   prev              a plan made with PA_PLAN_KEEP_PACK (by pa_plan_create or
  *                     by this call); not modified
  *   kv_lens, block_table, max_pages, num_pages_in_pool
