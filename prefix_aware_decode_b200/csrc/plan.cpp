@@ -324,7 +324,17 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     int64_t span = ceil_div(simt_pages, W);
     if (span < 4) span = 4;
     if (max_chunk_pages) span = std::min(span, max_chunk_pages);
-    simt_segs.reserve(items.size() * Hkv + simt_pages / span + 8);
+    // one segment per (item, kv head) run plus one per warp boundary (the last
+    // warp takes whole runs), so this is enough unless max_chunk_tokens cuts
+    // finer; the writer grows the buffer if it is not
+    size_t n_units = 0;
+    for (const auto& it : items) n_units += it.simt;
+    simt_segs.resize(n_units * Hkv + (size_t)W + 8);
+    warp_segs.resize((size_t)W + 2);
+    SegRec* sp = simt_segs.data();
+    int32_t* wp = warp_segs.data() + 1;
+    int32_t n_seg = 0;
+    int64_t n_warp = 1;
     int64_t used = 0;  // pages in the current warp's span
     for (size_t i = 0; i < items.size(); ++i) {
       const ItemRec& it = items[i];
@@ -335,19 +345,31 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
         int pb = 0;
         used += kSimtSegPages;  // the unit's fixed cost
         while (pb < npages) {
-          const int take = (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
+          const bool last_warp = n_warp >= W;
+          const int take = last_warp ? npages - pb
+                                     : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
           const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
-          simt_segs.push_back({(int)i, g, pb, tok, -1, b});
+          if ((size_t)n_seg == simt_segs.size()) {
+            simt_segs.resize(2 * simt_segs.size());
+            sp = simt_segs.data();
+          }
+          sp[n_seg++] = {(int)i, g, pb, tok, -1, b};
           pb += take;
           used += take;
-          if (used >= span && (int64_t)warp_segs.size() < W) {  // never more than W warps
-            warp_segs.push_back((int32_t)simt_segs.size());
+          if (used >= span && n_warp < W) {  // never more than W warps
+            *wp++ = n_seg;
+            ++n_warp;
             used = 0;
           }
         }
       }
     }
-    if (used > 0) warp_segs.push_back((int32_t)simt_segs.size());
+    if (used > 0) {
+      *wp++ = n_seg;
+      ++n_warp;
+    }
+    simt_segs.resize(n_seg);
+    warp_segs.resize(n_warp);
   }
   if (mma_pages > 0) {
     // each (item, kv head) run is a segment, and so is each cut at a CTA boundary
