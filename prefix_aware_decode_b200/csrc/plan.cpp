@@ -324,9 +324,10 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     int64_t span = ceil_div(simt_pages, W);
     if (span < 4) span = 4;
     if (max_chunk_pages) span = std::min(span, max_chunk_pages);
-    // one segment per (item, kv head) run plus one per warp boundary (the last
-    // warp takes whole runs), so this is enough unless max_chunk_tokens cuts
-    // finer; the writer grows the buffer if it is not
+    // one segment per (item, kv head) run plus one per warp boundary; more
+    // when max_chunk_tokens caps the spans below the work per warp (the last
+    // warp then cuts its runs into one-page segments), so the writer grows the
+    // buffer if needed
     size_t n_units = 0;
     for (const auto& it : items) n_units += it.simt;
     simt_segs.resize(n_units * Hkv + (size_t)W + 8);
@@ -345,9 +346,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
         int pb = 0;
         used += kSimtSegPages;  // the unit's fixed cost
         while (pb < npages) {
-          const bool last_warp = n_warp >= W;
-          const int take = last_warp ? npages - pb
-                                     : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
+          const int take = (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
           const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
           if ((size_t)n_seg == simt_segs.size()) {
             simt_segs.resize(2 * simt_segs.size());
