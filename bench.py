@@ -156,6 +156,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--layers", type=int, default=32,
                     help="layers of the multi-layer step measured beside config 2 (0: skip)")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="config 2: also time this many growing decode steps of --layers layers whose plans "
+                         "come from pa_plan_advance (0: skip)")
     ap.add_argument("--amortise", type=int, default=1024,
                     help="config-1 problems batched together for the amortised config-1 figure (0: skip)")
     args = ap.parse_args()
@@ -370,6 +373,74 @@ def main():
             "note": "per step: pack + upload once, then one forward + merge per layer, each layer with its "
                     f"own KV pools ({args.layers} x {pool_bytes / 2**20:.0f} MiB)"}
         del lay
+
+    # decode steps of a model: every request gains one token per step (a page
+    # of its own when its last one is full); the plan of each step comes from
+    # the previous one by pa_plan_advance and serves every layer.  The host
+    # time of a plan made from scratch for the same inputs is taken beside it.
+    if args.config == 2 and args.decode_steps > 0 and args.layers > 0:
+        n = args.decode_steps
+        n_pages = w.num_pages + w.B * (n // w.P + 2)
+        kv = w.kv_lens.astype(np.int32).copy()
+        bt = np.full((w.B, w.block_table.shape[1] + n // w.P + 2), -1, np.int32)
+        bt[:, :w.block_table.shape[1]] = w.block_table
+
+        def grown(t):  # the pool with zeroed spare pages after the workload's
+            g = torch.zeros((n_pages,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+            g[:w.num_pages].copy_(t)
+            return g
+
+        lay2 = [(grown(k0), grown(v0)) for _ in range(args.layers)]
+        free = [w.num_pages]
+
+        def grow():
+            for b in range(w.B):
+                if kv[b] % w.P == 0:
+                    bt[b, kv[b] // w.P] = free[0]
+                    free[0] += 1
+                kv[b] += 1
+
+        plan = pad.Plan(kv, bt, n_pages, w.Hq, w.Hkv, w.D, flags=pad.PA_PLAN_KEEP_PACK)
+        wsd = torch.empty((2 * plan.workspace_bytes + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        adv_us, full_us = [], []
+
+        def decode_step(timed: bool):
+            nonlocal plan
+            grow()
+            t = time.perf_counter()
+            nxt = plan.advance(kv, bt, n_pages)
+            t = (time.perf_counter() - t) * 1e6
+            plan.close()
+            plan = nxt
+            if plan.workspace_bytes > wsd.numel():
+                raise RuntimeError("decode-steps workspace too small")
+            plan.upload(wsd, stream)
+            for kl_, vl_ in lay2:
+                plan.attend(q, kl_, vl_, wsd, out, lse, stream)
+            if timed:
+                adv_us.append(t)
+                fp = pad.Plan(kv, bt, n_pages, w.Hq, w.Hkv, w.D)
+                full_us.append(fp.stats()["plan_us"])
+                fp.close()
+
+        for _ in range(3):
+            decode_step(False)
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(n):
+            decode_step(True)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        assert plan.device_status(wsd, stream) == pad.PA_OK
+        t_us = c0.elapsed_time(c1) / n * 1e3
+        line["decode_steps"] = {
+            "steps": n, "layers": args.layers, "us_per_step": t_us, "us_per_layer": t_us / args.layers,
+            "advance_us_median": statistics.median(adv_us), "create_us_median": statistics.median(full_us),
+            "note": "each step: every request appends a token, pa_plan_advance, upload, then one forward + merge "
+                    "per layer; create_us is pa_plan_create on the same inputs (host only, for comparison)"}
+        plan.close()
+        del lay2, wsd
 
     # end to end through the public API with host buffers
     if not args.no_e2e:
