@@ -39,3 +39,54 @@ def local_batch(block_table: np.ndarray, kv_lens: np.ndarray, q: np.ndarray, own
     """The rank's slice of the batch (block table rows, kv lens, q rows)."""
     return (np.ascontiguousarray(block_table[owned]), np.ascontiguousarray(kv_lens[owned]),
             np.ascontiguousarray(q[owned]))
+
+
+# ------------------------------------------------------------- context parallel
+
+def context_slices(block_table: np.ndarray, kv_lens: np.ndarray, world: int):
+    """Context-parallel split of one batch: the pages of every request are cut
+    into `world` contiguous, page-aligned slices, slice r going to rank r, so a
+    long session's KV is spread over the GPUs.  Returns, per rank,
+    (requests, block_table, kv_lens): the requests holding at least one token
+    in the rank's slice, their slice's page ids (from column 0) and token
+    counts.  Requests that share a prefix share it inside each slice too (the
+    slices are cut at the same page positions), so each rank's plan still packs
+    the shared pages.  Slice boundaries sit at page multiples, so only a
+    request's last slice may end inside a page."""
+    P = 16
+    B = len(kv_lens)
+    npg = (kv_lens.astype(np.int64) + P - 1) // P
+    out = []
+    for r in range(world):
+        lo = npg * r // world
+        hi = npg * (r + 1) // world
+        reqs = np.nonzero(hi > lo)[0]
+        width = int((hi - lo)[reqs].max()) if len(reqs) else 1
+        bt = np.full((len(reqs), max(1, width)), -1, dtype=np.int32)
+        kl = np.zeros(len(reqs), dtype=np.int32)
+        for i, b in enumerate(reqs):
+            bt[i, :hi[b] - lo[b]] = block_table[b, lo[b]:hi[b]]
+            kl[i] = min(int(kv_lens[b]), int(hi[b]) * P) - int(lo[b]) * P
+        out.append((reqs.astype(np.int64), bt, kl))
+    return out
+
+
+def merge_context_partials(B: int, parts):
+    """Combines per-rank results of context_slices: parts[r] = (requests,
+    out [n][Hq][D], lse [n][Hq]) with out the rank's attention over its slice
+    (normalised) and lse its log-sum-exp.  The result over the whole KV is the
+    same log-sum-exp combine as the merge stage: lse = ln Σ_r e^{lse_r},
+    out = Σ_r e^{lse_r − lse} out_r.  Host fp64 reference of the exchange step;
+    on GPUs the parts arrive by an all-gather."""
+    shape_o = parts[0][1].shape[1:]
+    shape_l = parts[0][2].shape[1:]
+    m = np.full((B,) + shape_l, -np.inf)
+    for reqs, _, l in parts:
+        m[reqs] = np.maximum(m[reqs], l)
+    z = np.zeros((B,) + shape_l)
+    acc = np.zeros((B,) + shape_o)
+    for reqs, o, l in parts:
+        wgt = np.exp(l - m[reqs])
+        z[reqs] += wgt
+        acc[reqs] += wgt[..., None] * o
+    return acc / z[..., None], m + np.log(z)

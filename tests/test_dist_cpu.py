@@ -59,6 +59,73 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
+def _cp_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+    import prefix_aware_decode_b200 as pad
+    from plan_exec import Image, check_structure, execute
+    from prefix_aware_decode_b200 import workload as wl
+    from prefix_aware_decode_b200.shard import context_slices, merge_context_partials
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # long sessions (config-5 shaped, scaled down): every rank holds a
+        # page-aligned slice of every session's KV and plans it on its own
+        w = wl.make_config(5, scale=1 / 64)
+        reqs, bt, kl = context_slices(w.block_table, w.kv_lens, world)[rank]
+        plan = pad.Plan(kl, bt, w.num_pages, w.Hq, w.Hkv, w.D)
+        img = Image(plan.host_image())
+        check_structure(img, kl, bt)
+        o, l = execute(img, w.q[reqs], w.k_pool, w.v_pool)
+        parts = [None] * world
+        dist.all_gather_object(parts, (reqs, o, l))
+        if rank == 0:
+            import oracle
+            out, lse = merge_context_partials(w.B, parts)
+            ro, rl = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+            q.put((float(np.abs(out - ro).max()), float(np.abs(lse - rl).max()),
+                   [int(p_[2].shape[0]) for p_ in parts], plan.stats()["num_kept_shared"]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_context_parallel_sessions_match_oracle():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=240)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    err_o, err_l, rows, kept = q.get(timeout=5)
+    assert err_o < 1e-12 and err_l < 1e-12
+    assert all(r > 0 for r in rows)  # both ranks hold part of every session
+    assert kept > 0                  # the slice of a shared context is still packed as shared
+
+
+def test_context_slices_cover_each_token_once():
+    from prefix_aware_decode_b200 import workload as wl
+    from prefix_aware_decode_b200.shard import context_slices
+    w = wl.make_config(3, with_values=False, scale=0.25)
+    for world in (2, 3, 5):
+        seen = {b: [] for b in range(w.B)}
+        for reqs, bt, kl in context_slices(w.block_table, w.kv_lens, world):
+            assert (kl > 0).all()
+            for i, b in enumerate(reqs):
+                n = (int(kl[i]) + 15) // 16
+                seen[int(b)].extend(bt[i, :n].tolist())
+                assert int(kl[i]) % 16 == 0 or seen[int(b)][-1] == w.block_table[b, (w.kv_lens[b] - 1) // 16]
+        for b in range(w.B):
+            n = (int(w.kv_lens[b]) + 15) // 16
+            assert seen[b] == w.block_table[b, :n].tolist()
+
+
 def test_two_rank_sharded_batch_matches_oracle():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
