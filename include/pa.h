@@ -223,7 +223,9 @@ pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t
  * while the kernels of step k do, and `stream` waits for it (an event) before
  * its launches.  A slot is refilled only after the launches that read it have
  * completed.  The device status word of the step is in its slot: read it with
- * pa_get_device_status on the plan returned through plan_out.
+ * pa_get_device_status on the plan returned through plan_out, before two more
+ * pa_decode_step calls on the device refill that slot.  pa_plan_upload (or
+ * pa_attend_noalloc) of that plan makes it refer to the new copy instead.
  * profile_events: NULL, or four cudaEvent_t as for pa_plan_set_profile_events.
  * plan_out: NULL (the plan is released before returning; its upload has
  * already been staged) or receives the plan, which the caller then releases.

@@ -150,6 +150,9 @@ extern "C" pa_status pa_plan_upload(const pa_plan* plan, void* d_workspace, size
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return PA_ERR_CUDA;
+  // from here on the plan's image is the copy at the workspace base (a plan
+  // that pa_decode_step returned stops referring to the library's slot)
+  plan->dev_image = nullptr;
   std::lock_guard<std::mutex> lock(g_pin_mu);
   PinnedSlot* s = pin_acquire(plan->image.size, device);
   if (!s) {

@@ -52,5 +52,6 @@ extern "C" pa_status pa_attend_noalloc(const pa_plan* plan, const void* q, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(ws, plan->image.data(), plan->image.size, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return PA_ERR_CUDA;
+  plan->dev_image = nullptr;  // the launches read this copy
   return pa_attend_ws(plan, q, k_pool, v_pool, ws, out, lse, stream);
 }

@@ -58,8 +58,9 @@ struct pa_plan {
   // [0,1] forward launch (pa_forward / pa_attend), [2,3] merge launch
   void* prof[4] = {};
   // device copy of the image when it lives outside the caller's workspace
-  // (pa_decode_step's image ring); nullptr: at the workspace base
-  void* dev_image = nullptr;
+  // (pa_decode_step's image ring); nullptr: at the workspace base.  A later
+  // pa_plan_upload or pa_attend_noalloc copies the image again and resets it.
+  mutable void* dev_image = nullptr;
   // the pack result (PA_PLAN_KEEP_PACK), from which pa_plan_advance plans the
   // next decode step: items (page_off, n_tokens, n_queries, query_off, simt),
   // their pages and requests, each request's kv_len and one-request item (-1:
