@@ -17,6 +17,11 @@ review's Merge stage).  Parity status of each function, and what pins it:
                         closed form of two one-key parts.
   oracle_attend_paged   pinned: dense gather done independently in numpy, then
                         torch fp64 SDPA; GQA head mapping by explicit repeat.
+  attend_rows           (a later workload: a chunk of new tokens appended to a
+                        session's persistent KV, each attending causally)
+                        pinned: torch fp64 SDPA with an explicit causal mask
+                        over the gathered context + chunk, the decode special
+                        case, invariance to the order of context tokens.
 """
 from __future__ import annotations
 
@@ -119,3 +124,32 @@ def attend_paged(q, k_pool, v_pool, block_table, kv_lens, scale=None, queries=No
     if rc != 0:
         raise ValueError("oracle_attend_paged: invalid arguments")
     return out, lse
+
+
+def attend_rows(q_rows, row_req, row_pos, k_pool, v_pool, block_table, scale=None, nthreads=None):
+    """Attention of query rows over a prefix of their request's paged KV, fp64.
+
+    Row r belongs to request row_req[r] and sits at token position row_pos[r]
+    of it; it attends over that request's tokens 0 .. row_pos[r] (its own
+    included), all already in the paged cache.  A chunk of C new tokens
+    appended to a session of L tokens is C rows at positions L .. L + C - 1
+    (causal inside the chunk; the persistent context before it); a decode
+    token is the row at position kv_len - 1.  This is the stateful-session
+    workload of "Attention Once Is All You Need" (new data advances the
+    session's KV; a query consumes it), with the PAT review's formula per row.
+
+    q_rows uint16[N][Hq][D]; row_req, row_pos int[N]; pools and block_table as
+    for attend_paged.  Returns (out float64[N][Hq][D], lse float64[N][Hq]).
+    Each row is the paged decode attention of a one-row batch whose block
+    table row is its request's and whose length is row_pos + 1.
+    """
+    bt = _c(block_table, np.int32)
+    req = np.asarray(row_req, dtype=np.int64)
+    pos = np.asarray(row_pos, dtype=np.int64)
+    if len(req) != len(pos) or len(req) != len(q_rows):
+        raise ValueError("attend_rows: q_rows, row_req and row_pos differ in length")
+    if (pos < 0).any() or (pos >= bt.shape[1] * k_pool.shape[2]).any():
+        raise ValueError("attend_rows: row position outside the block table")
+    rows_bt = np.ascontiguousarray(bt[req])
+    rows_len = (pos + 1).astype(np.int32)
+    return attend_paged(q_rows, k_pool, v_pool, rows_bt, rows_len, scale=scale, nthreads=nthreads)

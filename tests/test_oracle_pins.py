@@ -246,3 +246,59 @@ def test_paged_rejects_bad_inputs():
     kl[1] = 0
     with pytest.raises(ValueError):
         oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, kl)
+
+
+# ------------------------------------------------------------- session chunk append (attend_rows)
+
+def _session_chunk_case(seed, G, D, ctx, chunk):
+    """One session request whose last `chunk` tokens are new rows (causal), and
+    two other requests sharing its first pages; rows at positions ctx..ctx+chunk-1."""
+    roots = [wl.Node(32, [wl.Node(ctx + chunk - 32), wl.Node(21)]), wl.Node(40)]
+    w = wl.build_workload("chunk", roots, Hq=2 * G, Hkv=2, D=D, seed=seed)
+    (match,) = np.nonzero(w.kv_lens == ctx + chunk)
+    assert len(match) == 1
+    b = int(match[0])
+    rng = np.random.default_rng(seed)
+    qr = to_bf16_bits(rng.normal(size=(chunk, w.Hq, w.D)))
+    return w, b, qr
+
+
+@pytest.mark.parametrize("G,D,ctx,chunk", [(1, 64, 37, 5), (4, 128, 64, 16), (8, 64, 100, 19), (2, 128, 32, 1)])
+def test_attend_rows_matches_causal_sdpa(G, D, ctx, chunk):
+    w, b, qr = _session_chunk_case(7 + G + D, G, D, ctx, chunk)
+    pos = np.arange(ctx, ctx + chunk)
+    out, lse = oracle.attend_rows(qr, np.full(chunk, b), pos, w.k_pool, w.v_pool, w.block_table)
+    k, v = dense_gather(w, b)  # [Hkv][ctx+chunk][D]
+    K = torch.from_numpy(k).repeat_interleave(G, dim=0)  # [Hq][n][D]
+    V = torch.from_numpy(v).repeat_interleave(G, dim=0)
+    q = torch.from_numpy(wl.bf16_bits_to_f32(qr).astype(np.float64)).permute(1, 0, 2)  # [Hq][C][D]
+    n = ctx + chunk
+    allowed = torch.arange(n)[None, :] <= torch.from_numpy(pos)[:, None]  # [C][n]: key t <= row position
+    ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, attn_mask=allowed)  # [Hq][C][D]
+    logits = torch.einsum("hcd,hnd->hcn", q, K) / math.sqrt(D)
+    ref_lse = torch.logsumexp(logits.masked_fill(~allowed, float("-inf")), dim=-1)  # [Hq][C]
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse.permute(1, 0).numpy(), rtol=0, atol=1e-12)
+
+
+def test_attend_rows_last_row_is_decode_and_context_order_does_not_matter():
+    G, D, ctx, chunk = 4, 64, 96, 6
+    w, b, qr = _session_chunk_case(99, G, D, ctx, chunk)
+    pos = np.arange(ctx, ctx + chunk)
+    out, lse = oracle.attend_rows(qr, np.full(chunk, b), pos, w.k_pool, w.v_pool, w.block_table)
+    # the last row attends over the whole request: the decode attention of a
+    # batch whose query for request b is that row
+    qd = w.q.copy()
+    qd[b] = qr[-1]
+    do, dl = oracle.attend_paged(qd, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=[b])
+    np.testing.assert_allclose(out[-1], do[0], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[-1], dl[0], rtol=0, atol=1e-13)
+    # swapping two full context pages of the request changes no row (every row
+    # sees the whole context; attention does not depend on the order of keys)
+    bt2 = w.block_table.copy()
+    bt2[b, [1, 3]] = bt2[b, [3, 1]]
+    o2, l2 = oracle.attend_rows(qr, np.full(chunk, b), pos, w.k_pool, w.v_pool, bt2)
+    np.testing.assert_allclose(o2, out, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l2, lse, rtol=0, atol=1e-13)
+    # while a row earlier in the chunk sees fewer keys than the one after it
+    assert np.abs(out[0] - out[1]).max() > 1e-6
