@@ -313,3 +313,22 @@ def test_advance_gives_a_request_that_ended_at_a_shared_node_its_own_tail():
         np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
         assert p2.stats()["num_kept_shared"] == 1
+
+
+@pytest.mark.parametrize("config,scale", [(5, 1 / 64), (3, 1 / 16)])
+def test_advanced_plans_of_session_and_tree_batches(config, scale):
+    # shapes with tensor-core items of many rows (config 5: sessions of 16
+    # requests over one context; config 3: a three-level tree), a few decode
+    # steps through pa_plan_advance, executed against the oracle
+    w = wl.make_config(config, scale=scale)
+    p = make_plan(w, flags=pad.PA_PLAN_KEEP_PACK)
+    assert p.stats()["num_segments_mma"] > 0
+    for kv, bt, k, v, n_pages in decode_steps(w, steps=3, seed=config):
+        p = p.advance(kv, bt, n_pages)
+        img = Image(p.host_image())
+        check_structure(img, kv, bt)
+        out, lse = execute(img, w.q, k, v)
+        ref_o, ref_l = oracle.attend_paged(w.q, k, v, bt, kv)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+        assert p.stats()["num_segments_mma"] > 0
