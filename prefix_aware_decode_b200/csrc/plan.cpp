@@ -310,6 +310,9 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
       const double t = std::max(A / (S - kk), C / kk);
       if (t < best) { best = t; n_mma = kk; }
     }
+    // one SM: each class still gets one CTA (the two launches then run one
+    // after the other instead of side by side)
+    if (n_mma < 1) n_mma = 1;
   }
   std::vector<SegRec>& simt_segs = sc.simt_segs;
   std::vector<SegRec>& mma_segs = sc.mma_segs;
@@ -320,7 +323,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   warp_segs.assign(1, 0);
   mma_cta_segs.assign(1, 0);
   if (simt_pages > 0) {
-    const int64_t W = (int64_t)(S - n_mma) * kSimtWarpsPerCta;
+    const int64_t W = (int64_t)std::max(1, S - n_mma) * kSimtWarpsPerCta;
     int64_t span = ceil_div(simt_pages, W);
     if (span < 4) span = 4;
     if (max_chunk_pages) span = std::min(span, max_chunk_pages);

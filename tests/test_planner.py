@@ -332,3 +332,20 @@ def test_advanced_plans_of_session_and_tree_batches(config, scale):
         np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
         assert p.stats()["num_segments_mma"] > 0
+
+
+@pytest.mark.parametrize("num_sms", [1, 2, 3])
+def test_plans_for_very_few_sms(num_sms):
+    # both tile classes with one to three SMs: each class still gets at least
+    # one CTA (with one SM the two launches run one after the other)
+    w = wl.make_config(2, scale=0.125)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    p = make_plan(w, num_sms=num_sms)
+    st = p.stats()
+    assert st["mma_ctas"] >= 1 and st["simt_warps"] >= 1
+    assert st["mma_ctas"] + -(-st["simt_warps"] // 8) <= max(2, num_sms)
+    img = Image(p.host_image())
+    check_structure(img, w.kv_lens, w.block_table)
+    out, lse = execute(img, w.q, w.k_pool, w.v_pool)
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
