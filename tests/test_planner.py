@@ -349,3 +349,34 @@ def test_plans_for_very_few_sms(num_sms):
     out, lse = execute(img, w.q, w.k_pool, w.v_pool)
     np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+
+
+def test_random_plans_and_advances_against_the_oracle():
+    # a fixed-seed sweep over tree shapes, GQA groups, head dims, SM counts,
+    # planner flags and chunk caps: a plan, then decode steps through
+    # pa_plan_advance (some requests shrink, which plans from scratch), every
+    # plan checked for coverage and the last one executed against the oracle
+    rng = np.random.default_rng(2024)
+    done = 0
+    while done < 60:
+        seed = int(rng.integers(1 << 30))
+        G, D, Hkv = int(rng.choice([1, 2, 4, 8])), int(rng.choice([64, 128])), int(rng.choice([1, 2]))
+        roots = wl.random_tree(seed=seed, n_queries=int(rng.integers(2, 20)), depth=int(rng.integers(1, 4)),
+                               shared_pages=(1, int(rng.integers(1, 6))), leaf_tokens=(1, int(rng.integers(2, 80))))
+        w = wl.build_workload("sweep", roots, Hq=G * Hkv, Hkv=Hkv, D=D, seed=seed % 1000)
+        flags = int(rng.choice([0, pad.PA_PLAN_ALWAYS_SHARE, pad.PA_PLAN_NO_SHARING]))
+        p = make_plan(w, flags=flags | pad.PA_PLAN_KEEP_PACK, num_sms=int(rng.choice([1, 2, 7, 148])),
+                      max_chunk_tokens=int(rng.choice([0, 16, 64])))
+        for kv, bt, k, v, n_pages in decode_steps(w, steps=int(rng.integers(1, 8)), seed=seed % 97):
+            kv = kv.copy()
+            b = int(rng.integers(0, w.B))
+            if rng.random() < 0.2 and kv[b] > w.kv_lens[b]:
+                kv[b] -= 1
+            p = p.advance(kv, bt, n_pages)
+            img = Image(p.host_image())
+            check_structure(img, kv, bt)
+        out, lse = execute(img, w.q, k, v)
+        ref_o, ref_l = oracle.attend_paged(w.q, k, v, bt, kv)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+        done += 1
