@@ -46,7 +46,7 @@ extern "C" {
 
 typedef enum {
   PA_OK = 0,
-  PA_ERR_INVALID = 1,     /* bad argument: page id, kv_len, shape, partial shared page */
+  PA_ERR_INVALID = 1,     /* bad argument: page id, kv_len, shape */
   PA_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim, GQA ratio, page size */
   PA_ERR_NOMEM = 3,       /* host allocation failed, or workspace too small */
   PA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
@@ -111,8 +111,12 @@ typedef struct {
  *   num_pages_in_pool size of the pools' first dimension
  *   out               receives the new plan (NULL on error)
  * Two requests share a page when their rows hold the same page id at the same
- * position after an identical prefix (prefix caching).  A shared page must be
- * full for every request that shares it, else PA_ERR_INVALID.  Inputs are read
+ * position after an identical prefix (prefix caching).  A shared page is
+ * packed as shared (read once for all its requests) where it is full for all
+ * of them; a page that is the last, partial page of some of the requests that
+ * hold it (the queries of one session sharing its partial last page, or a
+ * request continuing in a page another one ends in) is read by each of those
+ * requests in its own item.  Inputs are read
  * during the call only.
  */
 pa_status pa_plan_create(const pa_config *cfg, int32_t batch, const int32_t *kv_lens,

@@ -134,11 +134,37 @@ struct Planner {
     for (int i = lo + 1; i < hi && l > depth; ++i) l = first_diff(r0, row(order[i]), depth, l);
     bool keep = false;
     int next_eff = eff_lo;
+    if (l > depth) {
+      // a page is packed as shared only where it is full for every request
+      // that holds it: the shared node stops before the first page that is
+      // partial for one of them
+      int lf = l;
+      for (int i = lo; i < hi; ++i) lf = std::min(lf, kv_lens[order[i]] / P);
+      if (lf <= depth) {
+        // page `depth` is the last, partial page of some requests (the same
+        // page id for all of them): those read their own tail; the requests
+        // for which it is full are walked again without them
+        auto mid = std::partition(order.begin() + lo, order.begin() + hi,
+                                  [&](int b) { return kv_lens[b] / P <= depth; });
+        const int e = (int)(mid - order.begin());
+        int64_t tail = 0;
+        for (int i = lo; i < e; ++i) {
+          const int b = order[i];
+          tail = std::max<int64_t>(tail, kv_lens[b] - (int64_t)depth * P);
+          add_item(b, eff_lo, npg[b], kv_lens[b] - (int64_t)eff_lo * P, &b, 1, true);
+        }
+        if (e < hi) {
+          walk(e, hi, depth, eff_lo);  // they hold page `depth` whole: it counts there
+        } else {
+          ++num_nodes;
+          unique_tokens += tail;
+        }
+        return;
+      }
+      l = lf;
+    }
     const int nq = hi - lo;
     if (l > depth) {
-      // a shared page must be full for every request that shares it
-      for (int i = lo; i < hi; ++i)
-        if (kv_lens[order[i]] / P < l) { invalid = true; return; }
       ++num_nodes;
       ++num_shared;
       unique_tokens += (int64_t)(l - depth) * P;

@@ -112,7 +112,6 @@ def test_validation_errors():
         (dict(kv_lens=np.array([0, 30], dtype=np.int32)), pad.PA_ERR_INVALID),      # empty request
         (dict(kv_lens=np.array([20, 33], dtype=np.int32)), pad.PA_ERR_INVALID),     # beyond max_pages * P
         (dict(num_pages=3), pad.PA_ERR_INVALID),                                     # page id 3 out of range
-        (dict(kv_lens=np.array([10, 30], dtype=np.int32)), pad.PA_ERR_INVALID),     # shared page 1 partial
         (dict(num_q_heads=12, num_kv_heads=4), pad.PA_ERR_UNSUPPORTED),              # G = 3
         (dict(num_q_heads=8, num_kv_heads=3), pad.PA_ERR_INVALID),                   # not a multiple
         (dict(head_dim=96), pad.PA_ERR_UNSUPPORTED),
@@ -124,6 +123,42 @@ def test_validation_errors():
         with pytest.raises(pad.PaError) as e:
             pad.Plan(**args)
         assert e.value.status == code, kw
+
+
+@pytest.mark.parametrize("flags", [0, pad.PA_PLAN_ALWAYS_SHARE, pad.PA_PLAN_NO_SHARING])
+def test_partially_filled_shared_pages(flags):
+    # a page several requests hold is packed as shared only where it is full
+    # for all of them; a page that is the last, partial page of some of them is
+    # read by each of those in its own item (sessions whose queries share the
+    # session's partial last page; a request that continues in a page another
+    # one ends in)
+    P, Hkv, D, Hq = 16, 2, 64, 8
+    rng = np.random.default_rng(3)
+    bf = lambda *sh: (rng.normal(size=sh).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    n_pages = 12
+    k, v = bf(n_pages, Hkv, P, D), bf(n_pages, Hkv, P, D)
+    cases = [
+        # three queries of one session: pages 4, 5 full, page 6 holds 7 tokens
+        (np.array([[4, 5, 6]] * 3, dtype=np.int32), np.array([39, 39, 39], dtype=np.int32)),
+        # request 0 ends 10 tokens into page 1, request 1 fills it and goes on
+        (np.array([[1, 2], [1, 3]], dtype=np.int32), np.array([10, 30], dtype=np.int32)),
+        # the same page partial for two requests of different lengths, full for a third
+        (np.array([[7, 8, 9], [7, 8, 10], [7, 8, 11]], dtype=np.int32), np.array([20, 28, 40], dtype=np.int32)),
+        # a shared run of full pages, then one page partial for all four at different lengths
+        (np.array([[0, 1, 2]] * 4, dtype=np.int32), np.array([33, 35, 40, 47], dtype=np.int32)),
+    ]
+    for bt, kv in cases:
+        q = bf(len(kv), Hq, D)
+        p = pad.Plan(kv, bt, n_pages, Hq, Hkv, D, flags=flags)
+        img = Image(p.host_image())
+        check_structure(img, kv, bt, P)
+        out, lse = execute(img, q, k, v)
+        ref_o, ref_l = oracle.attend_paged(q, k, v, bt, kv)
+        np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+    # the session's full pages stay one shared node
+    p = pad.Plan(cases[0][1], cases[0][0], n_pages, Hq, Hkv, D, flags=pad.PA_PLAN_ALWAYS_SHARE)
+    assert p.stats()["num_kept_shared"] == 1 and p.stats()["num_segments_mma"] > 0
 
 
 @pytest.mark.parametrize("flags", [0, pad.PA_PLAN_ALWAYS_SHARE, pad.PA_PLAN_NO_SHARING])
