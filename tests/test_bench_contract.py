@@ -1,5 +1,5 @@
 """bench.py's reference arm runs on the host (the fp64 oracle): its JSON line
-keeps the contract the driver reads.  The GPU arm is covered on a B200."""
+keeps the benchmark line's contract.  The GPU arm is covered on a B200."""
 import json
 import os
 import subprocess
