@@ -415,3 +415,35 @@ def test_random_plans_and_advances_against_the_oracle():
         np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
         done += 1
+
+
+def test_random_partially_shared_pages_against_the_oracle():
+    # block tables whose rows share random prefixes of a few page chains and
+    # end anywhere (so shared pages are often partial for some holders), then
+    # grown in place; plan, advance and execute against the oracle
+    rng = np.random.default_rng(77)
+    P = 16
+    for _ in range(40):
+        B, maxp = int(rng.integers(1, 10)), int(rng.integers(1, 7))
+        Hkv, G, D = int(rng.choice([1, 2])), int(rng.choice([1, 2, 4, 8])), int(rng.choice([64, 128]))
+        chains = [rng.permutation(100)[:maxp] for _ in range(int(rng.integers(1, 4)))]
+        bt = np.full((B, maxp), -1, np.int32)
+        nxt = 100
+        for b in range(B):
+            share = int(rng.integers(0, maxp + 1))
+            bt[b, :share] = chains[int(rng.integers(0, len(chains)))][:share]
+            bt[b, share:] = np.arange(nxt, nxt + maxp - share)
+            nxt += maxp - share
+        kv = rng.integers(1, maxp * P + 1, size=B).astype(np.int32)
+        bf = lambda *sh: (rng.normal(size=sh).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        k, v, q = bf(nxt, Hkv, P, D), bf(nxt, Hkv, P, D), bf(B, G * Hkv, D)
+        flags = int(rng.choice([0, pad.PA_PLAN_ALWAYS_SHARE, pad.PA_PLAN_NO_SHARING]))
+        p = pad.Plan(kv, bt, nxt, G * Hkv, Hkv, D, flags=flags | pad.PA_PLAN_KEEP_PACK)
+        kv2 = np.minimum(kv + rng.integers(0, 20, size=B), maxp * P).astype(np.int32)
+        for plan, lens in ((p, kv), (p.advance(kv2, bt, nxt), kv2)):
+            img = Image(plan.host_image())
+            check_structure(img, lens, bt)
+            out, lse = execute(img, q, k, v)
+            ref_o, ref_l = oracle.attend_paged(q, k, v, bt, lens)
+            np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
