@@ -3,20 +3,26 @@
 
 One step = the whole hot path over one decode batch: pack on the host
 (pa_plan_create: tree block table, profit model, split, tile selection), the
-async upload of the plan, forward and merge on the GPU.  The default workload is
-the Llama-3-8B-shaped decode layer (batch 64, 32/8 heads, head_dim 128, one
-shared 2048-token prefix plus suffixes uniform 128-1024, page 16).
+async upload of the plan, forward and merge on the GPU (pa_decode_step).  The
+headline workload is the largest one of the five (stateful sessions: 32
+sessions of 32768-131072 context tokens, 16 single-token queries each, batch
+512, 32/8 heads, head_dim 128); the four others are measured in the same run
+and reported under "per_config".
 
 Metric: decode-attention queries/s (B / time per step), with the unique-KV bytes
-per second reported beside it as a fraction of the measured HBM bandwidth.
+per second beside it as a fraction of the measured HBM bandwidth.  The roofline
+object credits the algorithmic bytes of the forward + merge launches: unique
+KV (each shared page once), q, out, lse, the fp32 partial rows that are
+written and read back, and the plan image.
 
 Timing: W warm-up steps, then K steps bracketed by a barrier and a device sync
 on both sides, timed with CUDA events on the launching stream; max over ranks.
-Between steps the KV pools rotate over several device copies whose total size
-exceeds L2, so no step finds its KV in L2.
+KV pools larger than L2 are used as they are; smaller ones rotate over device
+copies whose total exceeds L2, so no step finds its KV in L2.
 
-Under torchrun each rank runs its own batch (seed + rank): weak scaling, no
-collective on the data path.
+--gpus N: N ranks, one per GPU, each with its own batch (seed + rank): weak
+scaling, no collective on the data path.  Under torchrun the ranks come from
+the environment; without it bench.py starts them itself.
 """
 from __future__ import annotations
 
@@ -48,7 +54,7 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled during a timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -95,16 +101,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
+def kernels_hash() -> str:
+    import hashlib
+    src = open(os.path.join(_ROOT, "prefix_aware_decode_b200", "csrc", "kernels.cu"), "rb").read()
+    return hashlib.sha256(src).hexdigest()[:16]
+
+
 def measured_traffic(config: int):
     """DRAM bytes per step of the forward launches from the committed ncu capture,
     or None when the kernels have changed since it was taken."""
-    import hashlib
     try:
         t = json.load(open(os.path.join(_ROOT, "profiles", "traffic.json")))
-        src = open(os.path.join(_ROOT, "prefix_aware_decode_b200", "csrc", "kernels.cu"), "rb").read()
+        if kernels_hash() != t.get("kernels_cu_sha256_16"):
+            return None
     except OSError:
-        return None
-    if hashlib.sha256(src).hexdigest()[:16] != t.get("kernels_cu_sha256_16"):
         return None
     w = t.get("workloads", {}).get(str(config))
     return sum(w.values()) if w else None
@@ -112,6 +122,20 @@ def measured_traffic(config: int):
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def spawn_ranks(n: int) -> int:
+    """Runs this script as n ranks (one per GPU) under torch.distributed.run."""
+    import socket
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = ["timeout", "-k", "60", "1800", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def reference_arm(args, rank, world):
@@ -142,178 +166,190 @@ def reference_arm(args, rank, world):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
-    ap.add_argument("--config", type=int, default=2)
-    ap.add_argument("--copies", type=int, default=0, help="KV pool copies rotated between steps (0: enough to exceed L2)")
-    ap.add_argument("--ref-queries", type=int, default=64)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--layers", type=int, default=32,
-                    help="layers of the multi-layer step measured beside config 2 (0: skip)")
-    ap.add_argument("--decode-steps", type=int, default=0,
-                    help="config 2: also time this many growing decode steps of --layers layers whose plans "
-                         "come from pa_plan_advance (0: skip)")
-    ap.add_argument("--amortise", type=int, default=1024,
-                    help="config-1 problems batched together for the amortised config-1 figure (0: skip)")
-    args = ap.parse_args()
-    rank, world, local = dist_env()
-    if args.warmup < 3:
-        args.warmup = 3
-
-    if args.impl == "reference":
-        reference_arm(args, rank, world)
-        return
-
-    import torch
+def merged_rows(plan) -> int:
+    """Partial rows that go through the fp32 partial buffers (pairs with two or
+    more partial rows; a pair with one row is written straight to the output)."""
+    import ctypes
 
     import prefix_aware_decode_b200 as pad
-    from prefix_aware_decode_b200 import workload as wl
+    img = plan.host_image()
+    h = pad.PaImageHeader.from_buffer_copy(img[:ctypes.sizeof(pad.PaImageHeader)].tobytes())
+    n = h.batch * h.num_kv_heads
+    off = np.frombuffer(img[h.off_prow_off:h.off_prow_off + 4 * (n + 1)].tobytes(), dtype=np.int32)
+    cnt = np.diff(off)
+    return int(cnt[cnt > 1].sum())
 
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
 
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    hbm_peak, bf16_peak, peak_kind = peaks()
-    w = wl.make_config(args.config, seed=1000 + args.config + 7919 * rank)
-    unique_bytes = w.unique_kv_bytes
-    pool_bytes = w.k_pool.nbytes + w.v_pool.nbytes
-    copies = args.copies or max(2, int(np.ceil(3 * L2_BYTES / pool_bytes)) + 1)
-
-    def dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
-
-    q = dev(w.q)
-    k0, v0 = dev(w.k_pool), dev(w.v_pool)
-    pools = [(k0, v0)] + [(k0.clone(), v0.clone()) for _ in range(copies - 1)]
-    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
-    stream = torch.cuda.current_stream()
-    kv_lens, block_table = w.kv_lens, w.block_table
-
-    probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
-    pst = probe.stats()
-    ws_bytes = probe.workspace_bytes
-    probe.close()
-    workspaces = [torch.empty((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device="cuda") for _ in range(2)]
-
-    # per-step profiling events around each launch (recorded once so they exist)
-    def mk_events(n):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        for e in evs:
-            e.record(stream)
-        return evs
-
-    nsteps = args.warmup + args.steps
-    prof_every = 4  # profiling events on every 4th step of the timed region
-    step_events = [mk_events(4) if i % prof_every == 0 else None for i in range(nsteps)]
-    host_us = []
-    stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, q, k0, v0, workspaces[0], out, lse, stream=stream)
-
-    def step(i):
-        t = time.perf_counter()
-        stepper.set_pools(*pools[i % copies])
-        stepper(kv_lens, block_table, events=step_events[i])
-        host_us.append((time.perf_counter() - t) * 1e6)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
-    probe.upload(workspaces[0], stream)
-    status = probe.device_status(workspaces[0], stream)
-    probe.close()
-    assert status == pad.PA_OK, status
-
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
-    time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    host_us.clear()
-    ev0.record(stream)
-    for i in range(args.warmup, nsteps):
-        step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    ms_step = ms / args.steps
-
-    # forward (both classes) + merge time inside the timed region, per step
-    def ev_ms(a_, b_):
-        return statistics.mean(step_events[i][a_].elapsed_time(step_events[i][b_])
-                               for i in range(args.warmup, nsteps) if step_events[i] is not None)
-
-    fwd_ms = ev_ms(0, 1)
-    # the tensor-core and CUDA-core forward launches (concurrent), the tail merge launch
-    launches_per_step = (pst["mma_ctas"] > 0) + (pst["simt_warps"] > 0) + (pst["num_tail_pairs"] > 0)
-
-    # algorithmic bytes of one forward: the KV of its (page, kv head) tiles (each
-    # node read once per query tile), the q rows, the fp32 partial rows written
-    # and read back, and the bf16 output and fp32 lse
+def algorithmic_bytes(w, st: dict, n_merged: int) -> dict:
+    """Bytes the forward + merge launches must move for one batch: the unique
+    KV, q, out and lse, the partial rows written and read back (G rows of D + 1
+    floats each), and the plan image."""
     G = w.Hq // w.Hkv
-    tile_bytes = 2 * 16 * w.D * 2
-    fwd_bytes = (pst["read_kv_bytes"] + w.q.nbytes + 2 * pst["num_partial_rows"] * G * (w.D + 1) * 4
-                 + w.B * w.Hq * (w.D * 2 + 4))
-    achieved = fwd_bytes / (fwd_ms * 1e-3) / 1e9
+    parts = {"unique_kv": int(w.unique_kv_bytes), "q": int(w.q.nbytes), "out": w.B * w.Hq * w.D * 2,
+             "lse": w.B * w.Hq * 4, "partials": 2 * n_merged * G * (w.D + 1) * 4, "image": int(st["image_bytes"])}
+    parts["total"] = sum(parts.values())
+    return parts
 
-    queries_per_s = w.B * world / (ms_step * 1e-3)
-    line = {
-        "metric": METRIC, "value": queries_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.CONFIG_NAMES[args.config], "batch": w.B, "heads": f"{w.Hq}/{w.Hkv}",
-                   "head_dim": w.D, "page": w.P, "seed": w.seed, "unique_kv_bytes": unique_bytes,
-                   "prefix_ratio": round(w.prefix_ratio, 4), "l2": f"KV pools rotated over {copies} device copies "
-                   f"({copies * pool_bytes / 2**20:.0f} MiB > L2 {L2_BYTES // 2**20} MiB)",
-                   "step": "pack (host) + upload + forward + merge", "parallelism": f"replicas x{world}"},
-        "unique_kv_gbs": unique_bytes / (ms_step * 1e-3) / 1e9,
-        "unique_kv_frac_of_hbm": unique_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak,
-        "device_ms": {"forward_merge": fwd_ms, "profiled_steps": sum(e is not None for e in step_events[args.warmup:])},
-        "forward_queries_per_s": w.B / (fwd_ms * 1e-3),
-        "forward_unique_kv_frac": unique_bytes / (fwd_ms * 1e-3) / 1e9 / hbm_peak,
-        "plan_us": pst["plan_us"],
-        "host_us_per_step_median": statistics.median(host_us),
-        "plan": {k: pst[k] for k in ("num_segments_simt", "num_segments_mma", "simt_warps", "mma_ctas",
-                                     "num_tail_pairs", "num_partial_rows", "read_kv_bytes", "workspace_bytes",
-                                     "image_bytes")},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": measured_traffic(args.config),
-                     "traffic_unit": "bytes per step (DRAM read + write of the forward launches, ncu)",
-                     "kernel": "mma_fwd_kernel + simt_fwd_kernel (concurrent launches, merge fused into the "
-                               "SIMT launch) + merge_kernel over tensor-core-only pairs if any, timed together",
-                     "launches_per_step": launches_per_step,
-                     "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)"},
-        "gpu_launches": args.steps * launches_per_step,
-        "clocks": clk,
-    }
 
-    # config 1 is a few hundred KB, far below what one launch can stream: also
-    # time n independent config-1 problems planned together (device time of the
-    # forward + merge launches; plan time beside it, outside the timing)
-    if args.config == 1 and args.amortise > 0:
+class Bench:
+    def __init__(self, args, rank, world, local):
+        import torch
+
+        self.torch = torch
+        self.args, self.rank, self.world = args, rank, world
+        torch.cuda.set_device(local)
+        self.dist = None
+        if world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+            self.dist = dist
+        self.hbm_peak, self.bf16_peak, self.peak_kind = peaks()
+        self.stream = torch.cuda.current_stream()
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.dist is None:
+            return x
+        t = self.torch.tensor([x], device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def dev(self, a):
+        return self.torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(self.torch.bfloat16)
+
+    def measure(self, config: int, headline: bool) -> dict:
+        """Times K steps of pa_decode_step on one workload; returns its fields."""
+        torch, args, stream = self.torch, self.args, self.stream
+        import prefix_aware_decode_b200 as pad
+        from prefix_aware_decode_b200 import workload as wl
+
+        w = wl.make_config(config, seed=1000 + config + 7919 * self.rank)
+        pool_bytes = w.k_pool.nbytes + w.v_pool.nbytes
+        copies = args.copies or (1 if pool_bytes > 3 * L2_BYTES else int(np.ceil(3 * L2_BYTES / pool_bytes)) + 1)
+        q = self.dev(w.q)
+        k0, v0 = self.dev(w.k_pool), self.dev(w.v_pool)
+        pools = [(k0, v0)] + [(k0.clone(), v0.clone()) for _ in range(copies - 1)]
+        out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        kv_lens, block_table = w.kv_lens, w.block_table
+
+        probe = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+        pst = probe.stats()
+        n_merged = merged_rows(probe)
+        ws_bytes = probe.workspace_bytes
+        probe.close()
+        algo = algorithmic_bytes(w, pst, n_merged)
+        ws = torch.empty((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+
+        def mk_events(n):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+            for e in evs:
+                e.record(stream)
+            return evs
+
+        nsteps = args.warmup + args.steps
+        prof_every = 4  # profiling events on every 4th step of the timed region
+        step_events = [mk_events(4) if i % prof_every == 0 else None for i in range(nsteps)]
+        host_us = []
+        stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, q, k0, v0, ws, out, lse, stream=stream)
+
+        def step(i):
+            t = time.perf_counter()
+            stepper.set_pools(*pools[i % copies])
+            stepper(kv_lens, block_table, events=step_events[i])
+            host_us.append((time.perf_counter() - t) * 1e6)
+
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        chk = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+        chk.upload(ws, stream)
+        chk.attend(q, k0, v0, ws, out, lse, stream)
+        status = chk.device_status(ws, stream)
+        chk.close()
+        assert status == pad.PA_OK, status
+
+        clocks = ClockSampler(torch.cuda.current_device())
+        clocks.start()
+        time.sleep(0.3)
+        self.barrier()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        host_us.clear()
+        ev0.record(stream)
+        for i in range(args.warmup, nsteps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        self.barrier()
+        clk = clocks.stop()
+        ms_step = self.max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
+        fwd_ms = statistics.mean(step_events[i][0].elapsed_time(step_events[i][1])
+                                 for i in range(args.warmup, nsteps) if step_events[i] is not None)
+        launches = (pst["mma_ctas"] > 0) + (pst["simt_warps"] > 0) + (pst["num_tail_pairs"] > 0)
+        achieved = algo["total"] / (fwd_ms * 1e-3) / 1e9
+        hbm = self.hbm_peak
+        res = {
+            "workload": wl.CONFIG_NAMES[config], "batch": w.B, "seed": w.seed,
+            "unique_kv_bytes": int(w.unique_kv_bytes), "prefix_ratio": round(w.prefix_ratio, 4),
+            "l2": (f"KV pools ({pool_bytes / 2**20:.0f} MiB) larger than L2" if copies == 1 else
+                   f"KV pools rotated over {copies} device copies ({copies * pool_bytes / 2**20:.0f} MiB > L2)"),
+            "ms_per_step": ms_step, "queries_per_s": w.B * self.world / (ms_step * 1e-3),
+            "unique_kv_frac_of_hbm": w.unique_kv_bytes / (ms_step * 1e-3) / 1e9 / hbm,
+            "forward_merge_us": fwd_ms * 1e3,
+            "forward_queries_per_s": w.B / (fwd_ms * 1e-3),
+            "forward_unique_kv_frac_of_hbm": w.unique_kv_bytes / (fwd_ms * 1e-3) / 1e9 / hbm,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": measured_traffic(config),
+                         "algorithmic_bytes": algo,
+                         "kernel": "forward launches of both tile classes with the merge fused, plus the tail "
+                                   "merge launch when the plan has one, timed together with CUDA events",
+                         "launches_per_step": launches,
+                         "peak_kind": f"{self.peak_kind} hbm_gbs (copy, burst)"},
+            "plan_us": pst["plan_us"], "host_us_per_step_median": statistics.median(host_us),
+            "plan": {k: pst[k] for k in ("num_segments_simt", "num_segments_mma", "simt_warps", "mma_ctas",
+                                         "num_tail_pairs", "num_partial_rows", "read_kv_bytes",
+                                         "workspace_bytes", "image_bytes")},
+            "clocks": clk, "gpu_launches": args.steps * launches,
+        }
+
+        if config == 1 and args.amortise > 0:
+            res["amortised"] = self.amortised(w)
+        if config == 2 and args.layers > 0:
+            res["multi_layer"] = self.multi_layer(w, q, k0, v0, ws, out, lse, pool_bytes)
+        if config == 2 and args.decode_steps > 0 and args.layers > 0:
+            res["decode_steps"] = self.decode_steps(w, q, k0, v0, out, lse)
+        if headline and not args.no_e2e:
+            res.update(self.e2e(w, q, k0, v0, out, lse, ws_bytes))
+        if headline and self.rank == 0 and not args.no_cpu_baseline:
+            import oracle
+            cores = os.cpu_count() or 1
+            n = min(w.B, args.ref_queries)
+            qs = np.arange(n, dtype=np.int32)
+            t0 = time.perf_counter()
+            oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs, nthreads=cores)
+            dt = time.perf_counter() - t0
+            res["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                   "sample": f"first {n} of {w.B} queries of the same workload, one pass"}
+        del pools, q, k0, v0, out, lse, ws, stepper
+        torch.cuda.empty_cache()
+        return res
+
+    def amortised(self, w) -> dict:
+        # config 1 is a few hundred KB, far below what one launch can stream:
+        # n independent config-1 problems planned together, forward + merge
+        # launches timed on the device (plan time beside it, outside the timing)
+        torch, args, stream = self.torch, self.args, self.stream
+        import prefix_aware_decode_b200 as pad
+        from prefix_aware_decode_b200 import workload as wl
+
         wa = wl.config1_stream(args.amortise, seed=w.seed)
-        qa, ka, va = dev(wa.q), dev(wa.k_pool), dev(wa.v_pool)
+        qa, ka, va = self.dev(wa.q), self.dev(wa.k_pool), self.dev(wa.v_pool)
         oa = torch.empty((wa.B, wa.Hq, wa.D), dtype=torch.bfloat16, device="cuda")
         la = torch.empty((wa.B, wa.Hq), dtype=torch.float32, device="cuda")
         pa_ = pad.Plan(wa.kv_lens, wa.block_table, wa.num_pages, wa.Hq, wa.Hkv, wa.D)
@@ -329,27 +365,30 @@ def main():
         torch.cuda.synchronize()
         t_us = a0.elapsed_time(a1) / args.steps * 1e3
         assert pa_.device_status(wsa, stream) == pad.PA_OK
-        line["amortised"] = {
-            "problems": args.amortise, "batch": wa.B, "unique_kv_bytes": wa.unique_kv_bytes,
-            "forward_merge_us": t_us, "queries_per_s": wa.B / (t_us * 1e-6),
-            "unique_kv_frac_of_hbm": wa.unique_kv_bytes / (t_us * 1e-6) / 1e9 / hbm_peak,
-            "plan_us": pa_.stats()["plan_us"],
-            "note": "one plan and upload, then forward + merge launches timed back to back on the device "
-                    "(the KV of all problems stays resident; 218 MB, above L2)"}
+        algo = algorithmic_bytes(wa, pa_.stats(), merged_rows(pa_))
+        r = {"problems": args.amortise, "batch": wa.B, "unique_kv_bytes": int(wa.unique_kv_bytes),
+             "forward_merge_us": t_us, "queries_per_s": wa.B / (t_us * 1e-6),
+             "unique_kv_frac_of_hbm": wa.unique_kv_bytes / (t_us * 1e-6) / 1e9 / self.hbm_peak,
+             "roofline_frac": algo["total"] / (t_us * 1e-6) / 1e9 / self.hbm_peak,
+             "plan_us": pa_.stats()["plan_us"],
+             "note": "one plan and upload, then forward + merge launches timed back to back on the device "
+                     f"(the KV of all problems stays resident; {wa.unique_kv_bytes / 1e6:.0f} MB, above L2)"}
         pa_.close()
-        del qa, ka, va, oa, la, wsa
+        return r
 
-    # one decode step of a model: the plan is made and uploaded once and read by
-    # every layer's attention (each layer has its own KV pools)
-    if args.config == 2 and args.layers > 0:
+    def multi_layer(self, w, q, k0, v0, ws, out, lse, pool_bytes) -> dict:
+        # one decode step of a model: the plan is made and uploaded once and
+        # read by every layer's attention (each layer has its own KV pools)
+        torch, args, stream = self.torch, self.args, self.stream
+        import prefix_aware_decode_b200 as pad
+
         lay = [(k0.clone(), v0.clone()) for _ in range(args.layers)]
-        wsl = workspaces[0]
 
         def layer_step():
-            p_ = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
-            p_.upload(wsl, stream)
+            p_ = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+            p_.upload(ws, stream)
             for kl_, vl_ in lay:
-                p_.attend(q, kl_, vl_, wsl, out, lse, stream)
+                p_.attend(q, kl_, vl_, ws, out, lse, stream)
             p_.close()
 
         for _ in range(3):
@@ -365,20 +404,23 @@ def main():
         th = (time.perf_counter() - th) / nst * 1e6
         torch.cuda.synchronize()
         t_us = b0.elapsed_time(b1) / nst * 1e3
-        line["multi_layer"] = {
-            "layers": args.layers, "us_per_step": t_us, "us_per_layer": t_us / args.layers,
-            "queries_per_s_per_layer": w.B * args.layers / (t_us * 1e-6),
-            "unique_kv_frac_of_hbm": unique_bytes * args.layers / (t_us * 1e-6) / 1e9 / hbm_peak,
-            "host_us_per_step": th,
-            "note": "per step: pack + upload once, then one forward + merge per layer, each layer with its "
-                    f"own KV pools ({args.layers} x {pool_bytes / 2**20:.0f} MiB)"}
         del lay
+        return {"layers": args.layers, "us_per_step": t_us, "us_per_layer": t_us / args.layers,
+                "queries_per_s_per_layer": w.B * args.layers / (t_us * 1e-6),
+                "unique_kv_frac_of_hbm": w.unique_kv_bytes * args.layers / (t_us * 1e-6) / 1e9 / self.hbm_peak,
+                "host_us_per_step": th,
+                "note": "per step: pack + upload once, then one forward + merge per layer, each layer with its "
+                        f"own KV pools ({args.layers} x {pool_bytes / 2**20:.0f} MiB)"}
 
-    # decode steps of a model: every request gains one token per step (a page
-    # of its own when its last one is full); the plan of each step comes from
-    # the previous one by pa_plan_advance and serves every layer.  The host
-    # time of a plan made from scratch for the same inputs is taken beside it.
-    if args.config == 2 and args.decode_steps > 0 and args.layers > 0:
+    def decode_steps(self, w, q, k0, v0, out, lse) -> dict:
+        # decode steps of a model: every request gains one token per step (a
+        # page of its own when its last one is full); the plan of each step
+        # comes from the previous one by pa_plan_advance and serves every
+        # layer.  The host time of a plan made from scratch for the same
+        # inputs is taken beside it.
+        torch, args, stream = self.torch, self.args, self.stream
+        import prefix_aware_decode_b200 as pad
+
         n = args.decode_steps
         n_pages = w.num_pages + w.B * (n // w.P + 2)
         kv = w.kv_lens.astype(np.int32).copy()
@@ -434,33 +476,35 @@ def main():
         torch.cuda.synchronize()
         assert plan.device_status(wsd, stream) == pad.PA_OK
         t_us = c0.elapsed_time(c1) / n * 1e3
-        line["decode_steps"] = {
-            "steps": n, "layers": args.layers, "us_per_step": t_us, "us_per_layer": t_us / args.layers,
-            "advance_us_median": statistics.median(adv_us), "create_us_median": statistics.median(full_us),
-            "note": "each step: every request appends a token, pa_plan_advance, upload, then one forward + merge "
-                    "per layer; create_us is pa_plan_create on the same inputs (host only, for comparison)"}
         plan.close()
         del lay2, wsd
+        return {"steps": n, "layers": args.layers, "us_per_step": t_us, "us_per_layer": t_us / args.layers,
+                "advance_us_median": statistics.median(adv_us), "create_us_median": statistics.median(full_us),
+                "note": "each step: every request appends a token, pa_plan_advance, upload, then one forward + "
+                        "merge per layer; create_us is pa_plan_create on the same inputs (host only)"}
 
-    # end to end through the public API with host buffers
-    if not args.no_e2e:
+    def e2e(self, w, q, k0, v0, out, lse, ws_bytes) -> dict:
+        # end to end through the public API with host buffers: every input
+        # copied from pinned host memory each step, the result read back
+        torch, args, stream = self.torch, self.args, self.stream
+        import prefix_aware_decode_b200 as pad
+
         hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).pin_memory()
         hk = torch.from_numpy(np.ascontiguousarray(w.k_pool).view(np.int16)).pin_memory()
         hv = torch.from_numpy(np.ascontiguousarray(w.v_pool).view(np.int16)).pin_memory()
         ho = torch.empty((w.B, w.Hq, w.D), dtype=torch.int16).pin_memory()
         hl = torch.empty((w.B, w.Hq), dtype=torch.float32).pin_memory()
         dq = torch.empty_like(q)
-        dk, dv = torch.empty_like(k0), torch.empty_like(v0)
-
-        e2e_stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, dq, dk, dv, workspaces[1], out, lse,
-                                     stream=stream)
+        dk, dv = k0, v0  # the device pools are overwritten by the copies
+        ws = torch.empty((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, dq, dk, dv, ws, out, lse, stream=stream)
 
         def e2e_step(copy_kv: bool):
             dq.view(torch.int16).copy_(hq, non_blocking=True)
             if copy_kv:
                 dk.view(torch.int16).copy_(hk, non_blocking=True)
                 dv.view(torch.int16).copy_(hv, non_blocking=True)
-            e2e_stepper(kv_lens, block_table)
+            stepper(w.kv_lens, w.block_table)
             ho.copy_(out.view(torch.int16), non_blocking=True)
             hl.copy_(lse, non_blocking=True)
 
@@ -475,31 +519,88 @@ def main():
                 e2e_step(copy_kv)
             b.record(stream)
             torch.cuda.synchronize()
-            res[copy_kv] = a.elapsed_time(b) / args.e2e_steps
+            res[copy_kv] = self.max_over_ranks(a.elapsed_time(b)) / args.e2e_steps
         h2d = w.q.nbytes + w.k_pool.nbytes + w.v_pool.nbytes
         d2h = out.numel() * 2 + lse.numel() * 4
-        line["e2e"] = {"value": w.B * world / (res[True] * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h,
-                       "note": "every input (q and both KV pools) copied from pinned host memory each step"}
-        line["e2e_kv_resident"] = {"value": w.B * world / (res[False] * 1e-3), "unit": UNIT,
-                                   "h2d_bytes_per_step": w.q.nbytes, "d2h_bytes_per_step": d2h,
-                                   "note": "q from pinned host memory, KV cache resident on the device"}
+        del hq, hk, hv, ho, hl
+        return {"e2e": {"value": w.B * self.world / (res[True] * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h,
+                        "note": "every input (q and both KV pools) copied from pinned host memory each step; "
+                                "bound by the host link, not by the kernels"},
+                "e2e_kv_resident": {"value": w.B * self.world / (res[False] * 1e-3), "unit": UNIT,
+                                    "h2d_bytes_per_step": w.q.nbytes, "d2h_bytes_per_step": d2h,
+                                    "note": "the serving case: q from pinned host memory, the KV cache resident "
+                                            "on the device, out and lse read back each step"}}
 
-    if rank == 0 and not args.no_cpu_baseline:
-        import oracle
-        cores = os.cpu_count() or 1
-        n = min(w.B, args.ref_queries)
-        qs = np.arange(n, dtype=np.int32)
-        t0 = time.perf_counter()
-        oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs, nthreads=cores)
-        dt = time.perf_counter() - t0
-        line["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"first {n} of {w.B} queries of the same workload, one pass"}
 
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
+    ap.add_argument("--config", type=int, default=5, help="headline workload (1-5)")
+    ap.add_argument("--per-config", default="1,2,3,4",
+                    help="other workloads measured in the same run (comma list; empty: none)")
+    ap.add_argument("--copies", type=int, default=0, help="KV pool copies rotated between steps (0: enough to exceed L2)")
+    ap.add_argument("--ref-queries", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--layers", type=int, default=32,
+                    help="layers of the multi-layer step measured beside config 2 (0: skip)")
+    ap.add_argument("--decode-steps", type=int, default=16,
+                    help="config 2: also time this many growing decode steps of --layers layers whose plans "
+                         "come from pa_plan_advance (0: skip)")
+    ap.add_argument("--amortise", type=int, default=1024,
+                    help="config-1 problems batched together for the amortised config-1 figure (0: skip)")
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    if args.warmup < 3:
+        args.warmup = 3
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(spawn_ranks(args.gpus))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        sys.exit(2)
+
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+
+    bench = Bench(args, rank, world, local)
+    head = bench.measure(args.config, headline=True)
+    per = {}
+    for c in [int(x) for x in args.per_config.split(",") if x.strip()]:
+        if c != args.config:
+            per[str(c)] = bench.measure(c, headline=False)
+
+    line = {
+        "metric": METRIC, "value": head["queries_per_s"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": head["workload"], "batch": head["batch"], "heads": "32/8" if args.config > 1 else "8/2",
+                   "head_dim": 128 if args.config > 1 else 64, "page": 16, "seed": head["seed"],
+                   "unique_kv_bytes": head["unique_kv_bytes"], "prefix_ratio": head["prefix_ratio"],
+                   "l2": head["l2"], "step": "pack (host) + upload + forward + merge",
+                   "parallelism": f"replicas x{world}"},
+        "unique_kv_gbs": head["unique_kv_bytes"] / (head["ms_per_step"] * 1e-3) / 1e9,
+        "unique_kv_frac_of_hbm": head["unique_kv_frac_of_hbm"],
+        "device_ms": {"forward_merge": head["forward_merge_us"] * 1e-3},
+        "forward_queries_per_s": head["forward_queries_per_s"],
+        "forward_unique_kv_frac": head["forward_unique_kv_frac_of_hbm"],
+        "plan_us": head["plan_us"], "host_us_per_step_median": head["host_us_per_step_median"],
+        "plan": head["plan"], "roofline": head["roofline"], "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+    }
+    for k in ("e2e", "e2e_kv_resident", "cpu_baseline"):
+        if k in head:
+            line[k] = head[k]
+    line["per_config"] = per
     if rank == 0:
         print(json.dumps(line))
-    if dist is not None:
-        dist.destroy_process_group()
+    if bench.dist is not None:
+        bench.dist.destroy_process_group()
 
 
 if __name__ == "__main__":

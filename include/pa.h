@@ -102,6 +102,12 @@ typedef struct {
 
 /*
  * Pack: build a plan for one decode batch (host only; no device call).
+ * Source: the PAT review, section 三, Pack-Forward-merge 范式 item 1 (group the
+ * queries of a batch into CTA work by shared prefix, with a profit-model
+ * heuristic) and Pack Scheduler 工作流, Figure 7 (the tree-structured block
+ * table; packing scheme 1 keeps a parent node apart from its leaves, scheme 2
+ * folds it into them); item 2 of the same list for the tile selector and the
+ * split of long KV that the plan also fixes.
  *   cfg               head configuration and planner options (copied)
  *   batch             B >= 1
  *   kv_lens           host int32[B], each in [1, max_pages * page_size]
@@ -149,12 +155,16 @@ pa_status pa_plan_create(const pa_config *cfg, int32_t batch, const int32_t *kv_
 pa_status pa_plan_advance(const pa_plan *prev, const int32_t *kv_lens, const int32_t *block_table,
                           int32_t max_pages, int32_t num_pages_in_pool, pa_plan **out);
 
-/* Device workspace size in bytes for this plan (256-byte aligned buffer required). */
+/* Device workspace size in bytes for this plan (256-byte aligned buffer required).
+ * The workspace holds the plan image and the forward stage's fp32 partial
+ * results (the intermediate results the PAT review's Merge stage combines). */
 pa_status pa_plan_workspace_size(const pa_plan *plan, size_t *bytes);
 
 /*
  * Copy the plan (item, segment and page tables, and a zeroed status word) into
  * the caller's device workspace, asynchronously on `stream` (cudaStream_t).
+ * This is the hand-over from the host pack stage to the device forward stage
+ * of the PAT review's Pack-Forward-merge 范式 (section 三).
  * The image is first copied into a library-owned pinned staging buffer (a
  * small pool reused once each copy has completed), so the call does not wait
  * for earlier work on the stream and the plan may be destroyed right after it
@@ -165,7 +175,10 @@ pa_status pa_plan_upload(const pa_plan *plan, void *d_workspace, size_t bytes, v
 
 /*
  * Forward: partial attention of every planned work unit into the workspace's
- * fp32 partial buffers.  q, k_pool, v_pool are device pointers in the layouts
+ * fp32 partial buffers.  Source: the PAT review, section 三, Forward 阶段
+ * (multi-tile kernels, a runtime tile selector per CTA, multi-stream execution
+ * and long-KV splitting) and Figure 3 (decode attention as two GEMVs, q.K^T
+ * and p.V, fed by a tiling pipeline from global memory).  q, k_pool, v_pool are device pointers in the layouts
  * above; k_pool and v_pool must be 16-byte aligned.  Needs a prior
  * pa_plan_upload to the same workspace (ordered before on the stream).
  * Asynchronous on `stream`; launch failures return PA_ERR_CUDA.
@@ -176,14 +189,16 @@ pa_status pa_forward(const pa_plan *plan, const void *q, const void *k_pool, con
 /*
  * Merge: log-sum-exp combine of the partials of every (request, head) into
  * out (bf16 [B][Hq][D], round-to-nearest-even) and lse (fp32 [B][Hq]; may be
- * NULL).  Asynchronous on `stream`, ordered after pa_forward.
+ * NULL).  Asynchronous on `stream`, ordered after pa_forward.  Source: the PAT
+ * review, section 三, Merge 阶段 (a light online-softmax kernel that combines
+ * each query's intermediate results across CTAs).
  */
 pa_status pa_merge(const pa_plan *plan, void *d_workspace, void *out, float *lse, void *stream);
 
 /*
  * Forward with the merge fused into it (one launch): the warp that writes the
  * last partial row of a (request, kv head) pair merges that pair into out and
- * lse.  Same results as pa_forward + pa_merge, bit for bit.  The arrival
+ * lse (the PAT review's Forward and Merge stages, section 三, in one pass).  Same results as pa_forward + pa_merge, bit for bit.  The arrival
  * counters it uses are left at zero, so the uploaded plan can be run again.
  */
 pa_status pa_attend(const pa_plan *plan, const void *q, const void *k_pool, const void *v_pool,
@@ -192,7 +207,10 @@ pa_status pa_attend(const pa_plan *plan, const void *q, const void *k_pool, cons
 /*
  * Read the device status word of the workspace (synchronises `stream`).
  * *out = PA_OK, PA_ERR_TIMEOUT or PA_ERR_DEVICE.  The word is cleared by the
- * next pa_plan_upload.
+ * next pa_plan_upload.  d_workspace == NULL reads the word of the static
+ * workspace of pa_attend_noalloc instead (the status of the last call made
+ * there, by any plan).  The pages have no counterpart of this call: it
+ * reports the device-side bounded waits and checks of this library.
  */
 pa_status pa_get_device_status(const pa_plan *plan, const void *d_workspace, void *stream, pa_status *out);
 
@@ -218,26 +236,35 @@ pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t
 
 /*
  * One decode step in one call: pa_plan_create, the upload of the plan image and
- * pa_attend (forward with the merge fused) on `stream`.  workspace_bytes must
- * cover the plan's workspace (pa_plan_workspace_size of a plan of the same
- * batch); the workspace holds the partial rows.  The image itself goes to one
- * of two device slots that the library owns per device (allocated on first use
- * and grown when a larger image comes, the only device allocation of this
- * call), copied on a stream of the library's own: the copy for step k+1 runs
- * while the kernels of step k do, and `stream` waits for it (an event) before
- * its launches.  A slot is refilled only after the launches that read it have
- * completed.  The device status word of the step is in its slot: read it with
- * pa_get_device_status on the plan returned through plan_out, before two more
- * pa_decode_step calls on the device refill that slot.  pa_plan_upload (or
- * pa_attend_noalloc) of that plan makes it refer to the new copy instead.
+ * pa_attend (forward with the merge fused) on `stream`.  Source: the PAT review,
+ * section 六, 开销分析 and Figure 16 (the pack scheduler runs at every decode
+ * step of the serving system, beside the attention kernels).
+ *   d_workspace, workspace_bytes
+ *                     caller-owned device buffer for the partial rows; must
+ *                     cover pa_plan_workspace_size of a plan of the same batch
+ *   d_images, images_bytes
+ *                     caller-owned device buffer (256-byte aligned) for the
+ *                     plan images; its two halves are used alternately, so a
+ *                     plan whose image exceeds images_bytes / 2 (rounded down
+ *                     to 256 bytes) is refused with PA_ERR_NOMEM
+ * The image is copied into the next half on a stream of the library's own (the
+ * library keeps one copy stream and four events per device, and no device
+ * memory): the copy for step k+1 runs while the kernels of step k do, and
+ * `stream` waits for it (an event) before its launches.  A half is refilled
+ * only after the launches that read it have completed.  The device status word
+ * of the step is in its half: read it with pa_get_device_status on the plan
+ * returned through plan_out, before two more pa_decode_step calls refill that
+ * half.  pa_plan_upload (or pa_attend_noalloc) of that plan makes it refer to
+ * the new copy instead.
  * profile_events: NULL, or four cudaEvent_t as for pa_plan_set_profile_events.
  * plan_out: NULL (the plan is released before returning; its upload has
  * already been staged) or receives the plan, which the caller then releases.
  */
 pa_status pa_decode_step(const pa_config *cfg, int32_t batch, const int32_t *kv_lens, const int32_t *block_table,
                          int32_t max_pages, int32_t num_pages_in_pool, const void *q, const void *k_pool,
-                         const void *v_pool, void *d_workspace, size_t workspace_bytes, void *out, float *lse,
-                         void *const *profile_events, void *stream, pa_plan **plan_out);
+                         const void *v_pool, void *d_workspace, size_t workspace_bytes, void *d_images,
+                         size_t images_bytes, void *out, float *lse, void *const *profile_events, void *stream,
+                         pa_plan **plan_out);
 
 /*
  * pa_attend without a caller workspace, for callers that cannot allocate
@@ -258,8 +285,9 @@ pa_status pa_decode_step(const pa_config *cfg, int32_t batch, const int32_t *kv_
  *   must be ordered by the caller.
  *   The first call on a device looks up the array's device address (with that
  *   device current); make that first call before any stream capture.
- * Returns as pa_attend; the device status word is in the shared array and is
- * not readable through pa_get_device_status.
+ * Returns as pa_attend.  The device status word of the call is in the shared
+ * array: pa_get_device_status(plan, NULL, stream, &st) reads it (until the
+ * next call overwrites it).
  */
 pa_status pa_attend_noalloc(const pa_plan *plan, const void *q, const void *k_pool, const void *v_pool, void *out,
                             float *lse, void *stream);

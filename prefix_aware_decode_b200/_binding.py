@@ -102,8 +102,8 @@ def lib() -> ctypes.CDLL:
     L.pa_plan_host_image.restype = st
     L.pa_plan_set_profile_events.argtypes = [vp, ctypes.POINTER(vp), i32]
     L.pa_plan_set_profile_events.restype = st
-    L.pa_decode_step.argtypes = [ctypes.POINTER(PaConfig), i32, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp,
-                                 ctypes.POINTER(vp), vp, ctypes.POINTER(vp)]
+    L.pa_decode_step.argtypes = [ctypes.POINTER(PaConfig), i32, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, sz, vp,
+                                 vp, ctypes.POINTER(vp), vp, ctypes.POINTER(vp)]
     L.pa_decode_step.restype = st
     L.pa_attend_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     L.pa_attend_noalloc.restype = st
@@ -248,9 +248,11 @@ class Plan:
                                            _stream_ptr(stream)), "pa_attend_noalloc")
 
     def device_status(self, ws, stream=None) -> int:
+        """The device status word of the workspace `ws`; ws=None reads the
+        static workspace of attend_noalloc."""
         out = ctypes.c_int()
-        _check(self._lib.pa_get_device_status(self._h, _dptr(ws, "workspace", 256), _stream_ptr(stream),
-                                              ctypes.byref(out)), "pa_get_device_status")
+        _check(self._lib.pa_get_device_status(self._h, _dptr(ws, "workspace", 256) if ws is not None else None,
+                                              _stream_ptr(stream), ctypes.byref(out)), "pa_get_device_status")
         return out.value
 
 
@@ -282,18 +284,27 @@ def attend(q, k_pool, v_pool, block_table, kv_lens, softmax_scale: float = 0.0, 
 class DecodeStep:
     """Repeated decode steps through pa_decode_step (one C call per step).
 
-    The fixed arguments (shapes, pools, workspace, outputs) are marshalled
-    once; each call passes the step's kv_lens / block_table (host arrays).
+    The fixed arguments (shapes, pools, workspace, image buffer, outputs) are
+    marshalled once; each call passes the step's kv_lens / block_table (host
+    arrays).  `images` is the device buffer whose two halves hold the plan
+    images of consecutive steps (allocated here, image_bytes per half, when
+    not given).
     """
 
     def __init__(self, num_pages, num_q_heads, num_kv_heads, head_dim, q, k_pool, v_pool, workspace, out, lse=None,
-                 page_size=16, softmax_scale=0.0, flags=0, max_chunk_tokens=0, stream=None):
+                 page_size=16, softmax_scale=0.0, flags=0, max_chunk_tokens=0, stream=None, images=None,
+                 image_bytes=8 << 20):
+        import torch
         self._lib = lib()
         self.cfg = PaConfig(num_q_heads, num_kv_heads, head_dim, page_size, softmax_scale, 0, max_chunk_tokens,
                             flags, 0)
         self.num_pages = int(num_pages)
+        if images is None:
+            images = torch.empty(2 * ((image_bytes + 255) // 256 * 256), dtype=torch.uint8, device=q.device)
+        self.images = images
         self.args = (_dptr(q, "q"), _dptr(k_pool, "k_pool"), _dptr(v_pool, "v_pool"),
                      _dptr(workspace, "workspace", 256), workspace.numel() * workspace.element_size(),
+                     _dptr(images, "images", 256), images.numel() * images.element_size(),
                      _dptr(out, "out"), _dptr(lse, "lse", 4) if lse is not None else None)
         self.stream = _stream_ptr(stream)
         self._events = None
@@ -308,7 +319,7 @@ class DecodeStep:
         if events is not None:
             self._events = (ctypes.c_void_p * 4)(*[e.cuda_event if e is not None else None for e in events])
             ev = self._events
-        q, k, v, ws, wsb, out, lse = self.args
+        q, k, v, ws, wsb, im, imb, out, lse = self.args
         _check(self._lib.pa_decode_step(ctypes.byref(self.cfg), kv_lens.shape[0], kv_lens.ctypes.data,
                                         block_table.ctypes.data, block_table.shape[1], self.num_pages, q, k, v,
-                                        ws, wsb, out, lse, ev, self.stream, None), "pa_decode_step")
+                                        ws, wsb, im, imb, out, lse, ev, self.stream, None), "pa_decode_step")

@@ -230,10 +230,13 @@ pa_status pa_attend_ws(const pa_plan* plan, const void* q, const void* k_pool, c
 
 extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_workspace, void* stream,
                                           pa_status* out) {
-  if (!plan || !d_workspace || !out) return PA_ERR_INVALID;
+  if (!plan || !out) return PA_ERR_INVALID;
   int32_t word = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const uint8_t* base = static_cast<const uint8_t*>(plan->dev_image ? plan->dev_image : d_workspace);
+  // NULL workspace: the static array of pa_attend_noalloc
+  const void* ws = d_workspace ? d_workspace : pa_noalloc_scratch();
+  if (!ws) return PA_ERR_CUDA;
+  const uint8_t* base = static_cast<const uint8_t*>(d_workspace && plan->dev_image ? plan->dev_image : ws);
   const uint8_t* src = base + offsetof(pa_image_header, status);
   if (cudaMemcpyAsync(&word, src, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
@@ -243,15 +246,15 @@ extern "C" pa_status pa_get_device_status(const pa_plan* plan, const void* d_wor
 
 namespace {
 
-// Per-step plan images of pa_decode_step: two device slots per device used
-// alternately, uploaded on a stream of the library's own so that the upload of
-// step k+1 runs while the kernels of step k do.  The compute stream waits for
-// the upload (an event) before its launches, and records when it has finished
-// reading the slot; the upload that next fills the slot waits for that.
+// Per-step plan images of pa_decode_step: the two halves of the caller's image
+// buffer, used alternately and uploaded on a stream of the library's own so
+// that the upload of step k+1 runs while the kernels of step k do.  The compute
+// stream waits for the upload (an event) before its launches, and records when
+// it has finished reading the slot; the upload that next fills the slot waits
+// for that.  The library holds only the copy stream and the events (per
+// device); the device memory is the caller's.
 struct StepRing {
   cudaStream_t upload = nullptr;
-  void* slot[2] = {nullptr, nullptr};
-  size_t cap[2] = {0, 0};
   cudaEvent_t uploaded[2] = {nullptr, nullptr}, consumed[2] = {nullptr, nullptr};
   bool consumed_set[2] = {false, false};
   int next = 0;
@@ -272,8 +275,8 @@ StepRing* step_ring(int& device) {
   return &r;
 }
 
-// Uploads the plan image into the next slot and makes `stream` wait for it;
-// the plan's kernels then read their tables there.
+// Uploads the plan image into the next half of the caller's image buffer and
+// makes `stream` wait for it; the plan's kernels then read their tables there.
 // pa_decode_step has the planner write the image straight into a pinned
 // staging buffer (no second copy); the buffer stays lent until its copy is
 // enqueued.
@@ -296,24 +299,16 @@ void pinned_image_return(ImageInPinned& c) {
   c.slot = nullptr;
 }
 
-pa_status step_upload(pa_plan* plan, cudaStream_t stream, int* slot_out, ImageInPinned* pinned) {
+pa_status step_upload(pa_plan* plan, cudaStream_t stream, uint8_t* images, size_t half, int* slot_out,
+                      ImageInPinned* pinned) {
   std::lock_guard<std::mutex> lock(g_step_mu);
   int device = 0;
   StepRing* r = step_ring(device);
   if (!r) return PA_ERR_CUDA;
   const int j = r->next;
   const size_t n = plan->image.size;
-  if (r->cap[j] < n) {
-    // grow (rare): the slot's previous readers must be done before it is freed
-    if (r->consumed_set[j] && cudaEventSynchronize(r->consumed[j]) != cudaSuccess) return PA_ERR_CUDA;
-    if (r->slot[j]) cudaFree(r->slot[j]);
-    r->slot[j] = nullptr;
-    r->cap[j] = 0;
-    size_t cap = 1 << 20;
-    while (cap < n) cap <<= 1;
-    if (cudaMalloc(&r->slot[j], cap) != cudaSuccess) return PA_ERR_NOMEM;
-    r->cap[j] = cap;
-  }
+  if (n > half) return PA_ERR_NOMEM;
+  void* dst = images + (size_t)j * half;
   if (r->consumed_set[j] && cudaStreamWaitEvent(r->upload, r->consumed[j], 0) != cudaSuccess) return PA_ERR_CUDA;
   {
     std::lock_guard<std::mutex> pin_lock(g_pin_mu);
@@ -321,25 +316,24 @@ pa_status step_upload(pa_plan* plan, cudaStream_t stream, int* slot_out, ImageIn
     PinnedSlot* s = lent ? nullptr : pin_acquire(n, device);
     if (lent) {
       // the image was built in this pinned buffer
-      const cudaError_t e1 = cudaMemcpyAsync(r->slot[j], lent->ptr, n, cudaMemcpyHostToDevice, r->upload);
+      const cudaError_t e1 = cudaMemcpyAsync(dst, lent->ptr, n, cudaMemcpyHostToDevice, r->upload);
       const cudaError_t e2 = e1 == cudaSuccess ? cudaEventRecord(lent->done, r->upload) : e1;
       lent->lent = false;
       pinned->slot = nullptr;
       if (e2 != cudaSuccess) return PA_ERR_CUDA;
     } else if (s) {
       std::memcpy(s->ptr, plan->image.data(), n);
-      if (cudaMemcpyAsync(r->slot[j], s->ptr, n, cudaMemcpyHostToDevice, r->upload) != cudaSuccess ||
+      if (cudaMemcpyAsync(dst, s->ptr, n, cudaMemcpyHostToDevice, r->upload) != cudaSuccess ||
           cudaEventRecord(s->done, r->upload) != cudaSuccess)
         return PA_ERR_CUDA;
-    } else if (cudaMemcpyAsync(r->slot[j], plan->image.data(), n, cudaMemcpyHostToDevice, r->upload) !=
-               cudaSuccess) {
+    } else if (cudaMemcpyAsync(dst, plan->image.data(), n, cudaMemcpyHostToDevice, r->upload) != cudaSuccess) {
       return PA_ERR_CUDA;
     }
   }
   if (cudaEventRecord(r->uploaded[j], r->upload) != cudaSuccess ||
       cudaStreamWaitEvent(stream, r->uploaded[j], 0) != cudaSuccess)
     return PA_ERR_CUDA;
-  plan->dev_image = r->slot[j];
+  plan->dev_image = dst;
   r->next = j ^ 1;
   *slot_out = j;
   return PA_OK;
@@ -361,9 +355,12 @@ pa_status step_release(int j, cudaStream_t stream) {
 extern "C" pa_status pa_decode_step(const pa_config* cfg, int32_t batch, const int32_t* kv_lens,
                                     const int32_t* block_table, int32_t max_pages, int32_t num_pages_in_pool,
                                     const void* q, const void* k_pool, const void* v_pool, void* d_workspace,
-                                    size_t workspace_bytes, void* out, float* lse, void* const* profile_events,
-                                    void* stream, pa_plan** plan_out) {
+                                    size_t workspace_bytes, void* d_images, size_t images_bytes, void* out,
+                                    float* lse, void* const* profile_events, void* stream, pa_plan** plan_out) {
   if (plan_out) *plan_out = nullptr;
+  if (!d_images || (reinterpret_cast<uintptr_t>(d_images) & 255)) return PA_ERR_INVALID;
+  const size_t half = (images_bytes / 2) & ~size_t(255);
+  if (half == 0) return PA_ERR_NOMEM;
   pa_plan* plan = nullptr;
   ImageInPinned pinned;
   if (cudaGetDevice(&pinned.device) != cudaSuccess) return PA_ERR_CUDA;
@@ -377,7 +374,8 @@ extern "C" pa_status pa_decode_step(const pa_config* cfg, int32_t batch, const i
   if (profile_events) pa_plan_set_profile_events(plan, profile_events, 4);
   if (workspace_bytes < plan->hdr.workspace_bytes) st = PA_ERR_NOMEM;
   int slot = -1;
-  if (st == PA_OK) st = step_upload(plan, static_cast<cudaStream_t>(stream), &slot, &pinned);
+  if (st == PA_OK)
+    st = step_upload(plan, static_cast<cudaStream_t>(stream), static_cast<uint8_t*>(d_images), half, &slot, &pinned);
   pinned_image_return(pinned);  // no-op once the copy was enqueued
   if (st == PA_OK) st = pa_attend(plan, q, k_pool, v_pool, d_workspace, out, lse, stream);
   if (slot >= 0) {

@@ -587,8 +587,9 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
 // 64-key stage i (S/P buffer i % 3 in TMEM):
 //   S(i) = Q K^T                  -> TMEM, 64 columns
 //   p = exp2(s - m)               -> P = P_hi + P_lo, two bf16 matrices written
-//                                    over S(i) in TMEM (P_lo = p - P_hi, both
-//                                    truncated, so P keeps about 15 bits)
+//                                    over S(i) in TMEM (P_hi truncated, P_lo =
+//                                    p - P_hi rounded to nearest: P keeps about
+//                                    16 bits of p)
 //   O_h += P_hi,h V_h + P_lo,h V_h  (A operand read from TMEM)
 // S(i+1) is issued before p.V(i), so the tensor core overlaps the softmax; a
 // buffer is reused for S(i+3) only after p.V(i) has completed.  A half's
@@ -899,7 +900,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         }
         const float ms = m_used == -INFINITY ? 0.f : m_used;
         // p, and its split P_hi + P_lo: P_hi keeps the top 16 bits of p (a
-        // truncated bf16), P_lo the top 16 bits of the exact remainder p - P_hi.
+        // truncated bf16, so the remainder p - P_hi is exact in fp32), P_lo is
+        // that remainder rounded to the nearest bf16 (P_hi + P_lo is within
+        // 2^-16 p of p, with no one-sided bias).
         // Each page of 16 keys is stored as soon as it is done (P_hi words, then
         // P_lo words), so its store overlaps the next page's exponentials.
         float pw[32];
@@ -920,7 +923,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
             const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
             pw[PG * 16 + jj] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
-            pw[PG * 16 + jj + 8] = __uint_as_float(__byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632));
+            pw[PG * 16 + jj + 8] = __uint_as_float(pack_bf16x2(r0, r1));
           }
           tmem_st16<PG * 16>(t_s + PG * 16, pw);
         };

@@ -40,6 +40,8 @@ void* scratch_address() {
 
 }  // namespace
 
+void* pa_noalloc_scratch() { return scratch_address(); }
+
 extern "C" pa_status pa_attend_noalloc(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
                                        void* out, float* lse, void* stream) {
   if (!plan || !q || !k_pool || !v_pool || !out) return PA_ERR_INVALID;

@@ -57,8 +57,8 @@ struct pa_plan {
   // optional cudaEvent_t handles recorded around the launches (profiling):
   // [0,1] forward launch (pa_forward / pa_attend), [2,3] merge launch
   void* prof[4] = {};
-  // device copy of the image when it lives outside the caller's workspace
-  // (pa_decode_step's image ring); nullptr: at the workspace base.  A later
+  // device copy of the image when it lives outside the workspace (a half of
+  // pa_decode_step's image buffer); nullptr: at the workspace base.  A later
   // pa_plan_upload or pa_attend_noalloc copies the image again and resets it.
   mutable void* dev_image = nullptr;
   // the pack result (PA_PLAN_KEEP_PACK), from which pa_plan_advance plans the
@@ -97,6 +97,10 @@ int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
 int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 // Merge of the pairs in the plan's tail list (after a fused forward launch).
 int pa_launch_tail_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
+
+// Device address of the static workspace of pa_attend_noalloc on the current
+// device (looked up on first use), or nullptr on error.
+void* pa_noalloc_scratch();
 
 // pa_attend on a workspace whose plan image is already (being) uploaded.
 pa_status pa_attend_ws(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool, void* ws,

@@ -1,8 +1,11 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle.
 
 Inputs are the seeded synthetic workloads (NaN-poisoned spare pages and
-tails); tolerances: max abs 2e-3 and max relative 1e-2 (floored by the row rms)
-on bf16 outputs, 1e-4 on fp32 lse.
+tails).  Tolerances (gpu_util): max abs 2e-3 wherever |o| < 1, and half a bf16
+ulp plus 2^-15 |o| above (where rounding the output to bf16 alone exceeds
+2e-3); max relative 1e-2 floored by the row rms; 1e-4 on fp32 lse.  Configs
+1-4 are compared on every request, config 5 on three queries of each of its
+32 sessions (the first and the last among them).
 """
 import numpy as np
 import pytest
@@ -28,14 +31,6 @@ def dev_config(c, scale=1.0):
     return _cache[key]
 
 
-def sample(B, n, seed=0):
-    if B <= n:
-        return np.arange(B, dtype=np.int32)
-    r = np.random.default_rng(seed)
-    s = np.sort(r.choice(B, size=n - 2, replace=False))
-    return np.unique(np.concatenate([[0, B - 1], s])).astype(np.int32)
-
-
 @pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("config", [1, 2])
 def test_small_configs_full_parity(config, fused):
@@ -47,27 +42,32 @@ def test_small_configs_full_parity(config, fused):
     assert_close(m, f"config {config}")
 
 
-@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("config", [3, 4])
-def test_large_configs_sampled_parity(config, fused):
+def test_large_configs_full_parity(config):
+    # every request of the workload, both the two-launch path (pa_forward +
+    # pa_merge) and the fused one (pa_attend)
     dw = dev_config(config)
     w = dw.w
-    out, lse, st, _ = run(dw, fused=fused)
-    qs = sample(w.B, 40, seed=config)
-    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs)
-    assert_close(compare(out, lse, ref_o, ref_l, queries=qs), f"config {config}")
-    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    for fused in (False, True):
+        out, lse, st, _ = run(dw, fused=fused)
+        assert_close(compare(out, lse, ref_o, ref_l), f"config {config} fused={fused}")
 
 
-def test_config5_sampled_parity():
+def test_config5_every_session_parity():
+    # 32 sessions x 16 registered queries (request 16 s + j is query j of
+    # session s): the first and the last query of every session, plus one
+    # from the middle of each, against the oracle
     dw = dev_config(5)
     w = dw.w
-    out, lse, st, _ = run(dw)
-    assert st["num_segments_mma"] > 0
-    qs = np.array([0, 1, 15, 16, 255, 256, 500, 511], dtype=np.int32)
+    S = w.B // 16
+    qs = np.array(sorted({16 * s + j for s in range(S) for j in (0, 15, (5 * s) % 14 + 1)}), dtype=np.int32)
     ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens, queries=qs)
-    assert_close(compare(out, lse, ref_o, ref_l, queries=qs), "config 5")
-    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    for fused in (False, True):
+        out, lse, st, _ = run(dw, fused=fused)
+        assert st["num_segments_mma"] > 0
+        assert_close(compare(out, lse, ref_o, ref_l, queries=qs), f"config 5 fused={fused} ({len(qs)} queries)")
+        assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
 
 
 @pytest.mark.parametrize("flags,chunk", [(pad.PA_PLAN_NO_SHARING, 0), (pad.PA_PLAN_ALWAYS_SHARE, 64),
