@@ -155,6 +155,32 @@ pa_status pa_plan_create(const pa_config *cfg, int32_t batch, const int32_t *kv_
 pa_status pa_plan_advance(const pa_plan *prev, const int32_t *kv_lens, const int32_t *block_table,
                           int32_t max_pages, int32_t num_pages_in_pool, pa_plan **out);
 
+/*
+ * Pack for chunks of new tokens appended to sessions (prefix-aware grouped
+ * prefill of stateful sessions).  Source: the stateful-streaming summary
+ * ("Attention Once Is All You Need", 方法拆解: a session's KV cache persists
+ * and is advanced as new data arrives; the scheduler groups the prefill of the
+ * sessions prefix-aware) and the short-term-memory page (技术原理: a token's K
+ * and V are appended before it attends, so each new token sees the context and
+ * the chunk up to itself).
+ *   n_sessions        S >= 1
+ *   ctx_lens          host int32[S]: tokens of session s before its chunk (>= 0)
+ *   chunk_lens        host int32[S]: new tokens of session s (>= 1)
+ *   block_table       host int32[S][max_pages]: session s's pages, covering its
+ *                     ctx_lens[s] + chunk_lens[s] tokens (K and V of the chunk
+ *                     already written there)
+ * The plan has one row per new token, sessions in order and each chunk in
+ * token order: row i of session s attends over tokens 0 .. ctx_lens[s] + i of
+ * the session.  q, out and lse of pa_forward / pa_merge / pa_attend are then
+ * [sum(chunk_lens)][Hq][D] (lse [rows][Hq]).  The rows of a session share the
+ * context's full pages, so the pack stage reads those once for all of a
+ * session's rows (chunk x G rows on the tensor cores); the chunk's own pages
+ * are read per row up to its position.  Errors as pa_plan_create.
+ */
+pa_status pa_plan_create_append(const pa_config *cfg, int32_t n_sessions, const int32_t *ctx_lens,
+                                const int32_t *chunk_lens, const int32_t *block_table, int32_t max_pages,
+                                int32_t num_pages_in_pool, pa_plan **out);
+
 /* Device workspace size in bytes for this plan (256-byte aligned buffer required).
  * The workspace holds the plan image and the forward stage's fp32 partial
  * results (the intermediate results the PAT review's Merge stage combines). */

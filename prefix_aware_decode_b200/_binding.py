@@ -63,7 +63,7 @@ class PaImageHeader(ctypes.Structure):
 
 
 # exported names, in the order pa.h declares them
-EXPORTS = ["pa_plan_create", "pa_plan_advance", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
+EXPORTS = ["pa_plan_create", "pa_plan_advance", "pa_plan_create_append", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
            "pa_get_device_status", "pa_plan_get_stats", "pa_plan_host_image", "pa_plan_set_profile_events",
            "pa_decode_step", "pa_attend_noalloc", "pa_plan_destroy", "pa_status_string"]
 
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
     L.pa_plan_create.restype = st
     L.pa_plan_advance.argtypes = [vp, vp, vp, i32, i32, ctypes.POINTER(vp)]
     L.pa_plan_advance.restype = st
+    L.pa_plan_create_append.argtypes = [ctypes.POINTER(PaConfig), i32, vp, vp, vp, i32, i32, ctypes.POINTER(vp)]
+    L.pa_plan_create_append.restype = st
     L.pa_plan_workspace_size.argtypes = [vp, ctypes.POINTER(sz)]
     L.pa_plan_workspace_size.restype = st
     L.pa_plan_upload.argtypes = [vp, vp, sz, vp]
@@ -159,6 +161,30 @@ class Plan:
                                         bt.shape[1], int(num_pages), ctypes.byref(h)), "pa_plan_create")
         self._h = h
         self.B, self.Hq, self.Hkv, self.D = int(kv.shape[0]), num_q_heads, num_kv_heads, head_dim
+
+    @classmethod
+    def append(cls, ctx_lens, chunk_lens, block_table, num_pages: int, num_q_heads: int, num_kv_heads: int,
+               head_dim: int, page_size: int = 16, softmax_scale: float = 0.0, num_sms: int = 0,
+               max_chunk_tokens: int = 0, flags: int = 0, wait_timeout_us: int = 0) -> "Plan":
+        """Plan for chunks of new tokens appended to sessions
+        (pa_plan_create_append): one row per new token, sessions in order;
+        row i of session s attends over tokens 0 .. ctx_lens[s] + i."""
+        ctx = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+        ch = np.ascontiguousarray(chunk_lens, dtype=np.int32)
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        if bt.ndim != 2 or ctx.ndim != 1 or ch.shape != ctx.shape or bt.shape[0] != ctx.shape[0]:
+            raise ValueError("block_table must be [S][max_pages], ctx_lens and chunk_lens [S]")
+        self = cls.__new__(cls)
+        self._lib = lib()
+        cfg = PaConfig(num_q_heads, num_kv_heads, head_dim, page_size, softmax_scale, num_sms, max_chunk_tokens,
+                       flags, wait_timeout_us)
+        h = ctypes.c_void_p()
+        _check(self._lib.pa_plan_create_append(ctypes.byref(cfg), ctx.shape[0], ctx.ctypes.data, ch.ctypes.data,
+                                               bt.ctypes.data, bt.shape[1], int(num_pages), ctypes.byref(h)),
+               "pa_plan_create_append")
+        self._h = h
+        self.B, self.Hq, self.Hkv, self.D = int(ch.sum()), num_q_heads, num_kv_heads, head_dim
+        return self
 
     def advance(self, kv_lens, block_table, num_pages: int) -> "Plan":
         """The next decode step's plan of the same batch (pa_plan_advance): this

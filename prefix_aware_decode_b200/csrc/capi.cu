@@ -186,7 +186,7 @@ pa_status launch(const pa_plan* plan, const void* q, const void* k_pool, const v
   d.q = static_cast<const uint16_t*>(q);
   d.k_pool = static_cast<const uint16_t*>(k_pool);
   d.v_pool = static_cast<const uint16_t*>(v_pool);
-  if (plan->hdr.mma_ctas > 0 && (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool)) {
+  if (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool) {
     if (!tmap_get(*plan, k_pool, plan->tma_k) || !tmap_get(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
     plan->tma_k_ptr = k_pool;
     plan->tma_v_ptr = v_pool;

@@ -41,6 +41,7 @@ namespace pa {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kSmemMax = 232448;  // opt-in shared memory per CTA on sm_100
+constexpr float kRescaleLog2 = 8.f;  // a running maximum is raised only when it grows by more than this (log2 units)
 
 struct FwdArgs {
   const uint16_t* q;
@@ -64,6 +65,8 @@ struct FwdArgs {
   float qscale;  // softmax scale * log2(e): scores are kept in base-2 units
   uint64_t timeout_ns;
   int fault_drop;
+  int debug_checks;  // PA_PLAN_DEBUG_CHECKS: page and request ids are range-checked before any load
+  int num_pages, B;
 };
 
 // ---------------------------------------------------------------- merge of one (request, kv head)
@@ -153,25 +156,41 @@ __device__ __forceinline__ void merge_and_reset(const FwdArgs& a, int bg, int la
   if (lane == 0) a.counters[bg] = 0;  // ready for the next launch
 }
 
-// ---------------------------------------------------------------- SIMT class
+// ---------------------------------------------------------------- small-row class (one request, G rows)
+//
+// Each of 8 warps streams its own run of (page, kv head) tiles through a
+// private ring in shared memory: per tile, K and V arrive as D/64 boxes of 16
+// keys x 64 dims each (2-D TMA, 128-byte swizzle, completed on the stage's
+// mbarrier).  The G query rows of the request stay in registers as the B
+// operand of warp-level tensor-core products (mma.sync m16n8k16, bf16 in,
+// fp32 accumulate), with the keys as the M dimension so one request's rows
+// never leave the warp:
+//   S^T (16 keys x 8 rows) = K (16 x D) . Q^T            D/16 products
+//   online softmax per row over the keys (3 shuffles per row pair)
+//   P^T = P_hi + P_lo, each a bf16 B operand (transposed in registers)
+//   O^T (D x 8 rows) += V^T (D x 16 keys) . P^T          2 D/16 products
+// Rows past G are zero q rows whose results are dropped.  Per tile a warp
+// issues about a hundred instructions (against about 800 for the same work on
+// the CUDA cores with packed fp32 FMAs), so the class is bound by the bytes in
+// flight, not by issue.
 
 template <int D, int G>
 struct SimtShape {
-  static constexpr int DPL = (64 / G) < (D / 2) ? (64 / G) : (D / 2);  // head dims per lane
-  static constexpr int LPG = D / DPL;                                  // lanes per key group
-  static constexpr int NG = 32 / LPG;                                  // key groups per warp
-  static constexpr int KPG = 16 / NG;                                  // keys per group per page
-  static constexpr int CPL = DPL / 8;                                  // 16-byte chunks per lane per row
-  static constexpr int TILE = 16 * D * 2;                              // one (page, kv head) tile
-  static constexpr int QT = G * D * 2;                                 // the G query rows
+  static constexpr int TILE = 16 * D * 2;   // K (or V) of one (page, kv head) tile: D/64 swizzled 2 KB boxes
+  static constexpr int QT = G * D * 2;      // the G query rows
   static constexpr int STAGE = 2 * TILE;
   static constexpr int W = kSimtWarpsPerCta;
-  static constexpr int NST_FIT = (kSmemMax - W * (2 * QT + 8 * 8)) / (W * STAGE);
+  static constexpr int KT = D / 16;         // k steps of K.Q^T, d tiles of V^T.P^T
+  static constexpr int FIXED = W * 2 * QT + 1024 + W * 8 * 8;  // q slots, alignment slack, barriers
+  static constexpr int NST_FIT = (kSmemMax - FIXED) / (W * STAGE);
   static constexpr int NST = NST_FIT < (D == 128 ? 3 : 6) ? NST_FIT : (D == 128 ? 3 : 6);  // ring stages
-  static constexpr int WARP_BYTES = NST * STAGE + 2 * QT;
-  static constexpr int SMEM = W * WARP_BYTES + W * (NST + 2) * 8;
-  static_assert(NG * LPG == 32 && KPG * NG == 16 && DPL % 8 == 0, "bad SIMT shape");
-  static_assert(NST >= 2 && SMEM <= kSmemMax, "SIMT ring does not fit in shared memory");
+  static constexpr int RING = NST * STAGE;  // one warp's ring (a multiple of 1 KB: swizzle atoms stay aligned)
+  static constexpr int OFF_Q = W * RING;
+  static constexpr int OFF_BAR = OFF_Q + W * 2 * QT;
+  static constexpr int SMEM = OFF_BAR + W * (NST + 2) * 8 + 1024;
+  static_assert(NST >= 2 && SMEM <= kSmemMax, "ring does not fit in shared memory");
+  static_assert(RING % 1024 == 0 && TILE % 2048 == 0, "swizzle atoms must stay 1 KB aligned");
+  static_assert(G <= 8, "at most 8 rows per request");
 };
 
 struct SegInfo {
@@ -194,135 +213,129 @@ __device__ __forceinline__ SegInfo load_seg(const pa_seg* segs, int i, int end) 
   return r;
 }
 
-// One page of 16 keys for one warp: scores, online softmax, p.V.  PARTIAL: the
-// page holds fewer than 16 valid keys (its tail may hold NaN).
+// Shared-memory address of 16-byte chunk `ch` (8 dims) of key row `r` of a
+// tile stored as D/64 boxes of 16 rows x 128 bytes with the 128-byte swizzle
+// (chunk c of row r sits at chunk c ^ (r % 8) of the row).
+__device__ __forceinline__ uint32_t swz(uint32_t base, int r, int ch) {
+  return base + (ch >> 3) * 2048 + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+}
+
+// One tile of 16 keys for one warp: scores, online softmax (base-2 units,
+// maximum raised lazily), p.V.  Thread (g, t) = (lane / 4, lane % 4) holds the
+// scores of keys g and g + 8 for rows 2t and 2t + 1, and the accumulator
+// O^T[d][2t..2t+1] for d = 16 i + g and 16 i + g + 8.  PARTIAL: the tile holds
+// fewer than 16 valid keys (the rest may hold NaN).
 template <int D, int G, bool PARTIAL>
-__device__ __forceinline__ void simt_page(const uint8_t* kt, const uint8_t* vt, int nvalid, int grp, int li,
-                                          const float2 (&qf)[G][SimtShape<D, G>::CPL][4],
-                                          float2 (&o)[G][SimtShape<D, G>::CPL][4], float (&m)[G], float (&l)[G]) {
-  using S = SimtShape<D, G>;
-  constexpr int LPG = S::LPG, KPG = S::KPG, CPL = S::CPL;
-  float s[KPG][G];
+__device__ __forceinline__ void tile_step(uint32_t kt, uint32_t vt, int nvalid, int lane, float c,
+                                          const uint32_t (&qb)[D / 16][2], float (&o)[D / 16][4], float (&ms)[2],
+                                          float (&l)[2]) {
+  constexpr int KT = D / 16;
+  const int g = lane >> 2, t = lane & 3;
+  // S^T = K . Q^T, two accumulation chains
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int kk = 0; kk < KPG; ++kk) {
-    const int key = grp * KPG + kk;
-    const uint32_t msk = (!PARTIAL || key < nvalid) ? 0xffffffffu : 0u;
-    float2 acc[G];
-#pragma unroll
-    for (int r = 0; r < G; ++r) acc[r] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      uint4 w = *reinterpret_cast<const uint4*>(kt + key * D * 2 + (li + LPG * j) * 16);
-      if (PARTIAL) {
-        w.x &= msk;
-        w.y &= msk;
-        w.z &= msk;
-        w.w &= msk;
-      }
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 kf = bf16x2_to_f2(ws[e]);
-#pragma unroll
-        for (int r = 0; r < G; ++r) acc[r] = ffma2(qf[r][j][e], kf, acc[r]);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < G; ++r) s[kk][r] = acc[r].x + acc[r].y;
+  for (int kk = 0; kk < KT; ++kk) {
+    uint32_t af[4];
+    ldsm_x4(swz(kt, lane & 15, 2 * kk + (lane >> 4)), af);
+    if (kk & 1) mma_bf16_16816(sb, af, qb[kk][0], qb[kk][1]);
+    else mma_bf16_16816(sa, af, qb[kk][0], qb[kk][1]);
   }
+  float s[4];
 #pragma unroll
-  for (int off = 1; off < LPG; off <<= 1)
-#pragma unroll
-    for (int kk = 0; kk < KPG; ++kk)
-#pragma unroll
-      for (int r = 0; r < G; ++r) s[kk][r] += __shfl_xor_sync(0xffffffffu, s[kk][r], off);
+  for (int i = 0; i < 4; ++i) s[i] = sa[i] + sb[i];
+  // s[0]: key g row 2t, s[1]: key g row 2t+1, s[2]: key g+8 row 2t, s[3]: key g+8 row 2t+1
   if (PARTIAL) {
-#pragma unroll
-    for (int kk = 0; kk < KPG; ++kk)
-      if (grp * KPG + kk >= nvalid)
-#pragma unroll
-        for (int r = 0; r < G; ++r) s[kk][r] = -INFINITY;
+    if (g >= nvalid) s[0] = s[1] = -INFINITY;
+    if (g + 8 >= nvalid) s[2] = s[3] = -INFINITY;
   }
-  // online softmax (per group; every lane of a group holds the same values)
-  bool grow = false;
-  float mnew[G];
+  if (2 * t >= G) s[0] = s[2] = -INFINITY;
+  if (2 * t + 1 >= G) s[1] = s[3] = -INFINITY;
+  float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
 #pragma unroll
-  for (int r = 0; r < G; ++r) {
-    float pm = s[0][r];
-#pragma unroll
-    for (int kk = 1; kk < KPG; ++kk) pm = fmaxf(pm, s[kk][r]);
-    mnew[r] = fmaxf(m[r], pm);
-    grow |= mnew[r] > m[r];
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
   }
-  if (__any_sync(0xffffffffu, grow)) {
+  const float mn0 = mx0 * c, mn1 = mx1 * c;
+  const bool up0 = mn0 > ms[0] + kRescaleLog2, up1 = mn1 > ms[1] + kRescaleLog2;
+  if (up0 || up1) {
+    // the running maximum moves up only when it grows by more than 2^8: p stays
+    // below 256, and the accumulator is rescaled rarely
+    const float a0 = up0 ? ex2(ms[0] - mn0) : 1.f, a1 = up1 ? ex2(ms[1] - mn1) : 1.f;
 #pragma unroll
-    for (int r = 0; r < G; ++r) {
-      if (mnew[r] > m[r]) {
-        const float alpha = ex2(m[r] - mnew[r]);
-        l[r] *= alpha;
-        const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int j = 0; j < CPL; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) o[r][j][e] = fmul2(o[r][j][e], a2);
-        m[r] = mnew[r];
-      }
+    for (int i = 0; i < KT; ++i) {
+      o[i][0] *= a0;
+      o[i][1] *= a1;
+      o[i][2] *= a0;
+      o[i][3] *= a1;
     }
+    l[0] *= a0;
+    l[1] *= a1;
+    if (up0) ms[0] = mn0;
+    if (up1) ms[1] = mn1;
   }
-  float2 p[KPG][G];
-#pragma unroll
-  for (int r = 0; r < G; ++r) {
-    const float mr = m[r] == -INFINITY ? 0.f : m[r];
-#pragma unroll
-    for (int kk = 0; kk < KPG; ++kk) {
-      const float pv = ex2(s[kk][r] - mr);
-      p[kk][r] = make_float2(pv, pv);
-      l[r] += pv;
-    }
+  const float m0 = ms[0] == -INFINITY ? 0.f : ms[0], m1 = ms[1] == -INFINITY ? 0.f : ms[1];
+  const float p0 = ex2(fmaf(s[0], c, -m0)), p1 = ex2(fmaf(s[1], c, -m1));
+  const float p2 = ex2(fmaf(s[2], c, -m0)), p3 = ex2(fmaf(s[3], c, -m1));
+  l[0] += p0 + p2;
+  l[1] += p1 + p3;
+  // P = P_hi + P_lo: P_hi the truncated bf16 of p (so p - P_hi is exact),
+  // P_lo that remainder rounded to the nearest bf16; then each 8x8 block
+  // (keys x rows) is transposed into the B-operand layout (keys 2t, 2t+1 of row g)
+  const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+  const uint32_t u2 = __float_as_uint(p2), u3 = __float_as_uint(p3);
+  const uint32_t h01 = __byte_perm(u0, u1, 0x7632), h23 = __byte_perm(u2, u3, 0x7632);
+  const uint32_t l01 = pack_bf16x2(p0 - __uint_as_float(u0 & 0xFFFF0000u), p1 - __uint_as_float(u1 & 0xFFFF0000u));
+  const uint32_t l23 = pack_bf16x2(p2 - __uint_as_float(u2 & 0xFFFF0000u), p3 - __uint_as_float(u3 & 0xFFFF0000u));
+  const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+  const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+  // V rows past the last valid key may hold NaN: p = 0 there, but 0 * NaN would
+  // still poison the product, so those keys' V values are zeroed
+  uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+  if (PARTIAL) {
+    mlo = (2 * t < nvalid ? 0x0000ffffu : 0u) | (2 * t + 1 < nvalid ? 0xffff0000u : 0u);
+    mhi = (2 * t + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t + 9 < nvalid ? 0xffff0000u : 0u);
   }
+  // O^T += V^T . P^T: matrices (keys 0-7 | 8-15) x (dims 16i..16i+7 | 16i+8..16i+15)
+  const int vrow = (lane & 7) + ((lane >> 4) << 3), vch = (lane >> 3) & 1;
 #pragma unroll
-  for (int kk = 0; kk < KPG; ++kk) {
-    const int key = grp * KPG + kk;
-    const uint32_t msk = (!PARTIAL || key < nvalid) ? 0xffffffffu : 0u;
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      uint4 w = *reinterpret_cast<const uint4*>(vt + key * D * 2 + (li + LPG * j) * 16);
-      if (PARTIAL) {
-        w.x &= msk;
-        w.y &= msk;
-        w.z &= msk;
-        w.w &= msk;
-      }
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 vf = bf16x2_to_f2(ws[e]);
-#pragma unroll
-        for (int r = 0; r < G; ++r) o[r][j][e] = ffma2(p[kk][r], vf, o[r][j][e]);
-      }
+  for (int i = 0; i < KT; ++i) {
+    uint32_t af[4];
+    ldsm_x4_trans(swz(vt, vrow, 2 * i + vch), af);
+    if (PARTIAL) {
+      af[0] &= mlo;
+      af[1] &= mlo;
+      af[2] &= mhi;
+      af[3] &= mhi;
     }
+    mma_bf16_16816(o[i], af, bh0, bh1);
+    mma_bf16_16816(o[i], af, bl0, bl1);
   }
 }
 
 template <int D, int G>
-__device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
+__device__ __forceinline__ void simt_role(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
+                                          uint8_t* smem_raw) {
   using S = SimtShape<D, G>;
-  constexpr int NST = S::NST, LPG = S::LPG, CPL = S::CPL;
+  constexpr int NST = S::NST, KT = S::KT;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp >= kSimtWarpsPerCta) return;
   const int gw = blockIdx.x * kSimtWarpsPerCta + warp;
   if (gw >= a.n_simt_warps) return;  // no block-wide barrier in this role
-  uint8_t* wbase_smem = smem + warp * S::WARP_BYTES;
-  uint8_t* qslot = wbase_smem + NST * S::STAGE;  // two q-row slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSimtWarpsPerCta * S::WARP_BYTES) + warp * (NST + 2);
+  const uint32_t ring = smem_u32(smem + warp * S::RING);
+  uint8_t* qslot = smem + S::OFF_Q + warp * 2 * S::QT;  // two q-row slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR) + warp * (NST + 2);
   uint64_t* qbars = bars + NST;
   if (lane == 0) {
     for (int s = 0; s < NST + 2; ++s) mbar_init(smem_u32(&bars[s]), 1);
     fence_mbar_init();
+    prefetch_tmap(tk);
+    prefetch_tmap(tv);
   }
   __syncwarp();
 
-  const int grp = lane / LPG, li = lane % LPG;
+  const int g8 = lane >> 2, t4 = lane & 3;
   const int seg_begin = a.warp_segs[gw], seg_end = a.warp_segs[gw + 1];
   const bool drop_first = a.fault_drop && gw == 0;
 
@@ -332,7 +345,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   // prefix sums; a window of 32 tile ids (page * Hkv + kv head) is filled by a
   // per-lane binary search over the group plus one page-id load, and the next
   // window is fetched one window ahead.
-  int sg_base = seg_begin;          // first segment of the current group
+  int sg_base = seg_begin;  // first segment of the current group
   int sg_pstart = 0, sg_npg = 0, sg_g = 0, sg_off = 0, sg_tot = 0, sg_n = 0;
   auto load_group = [&]() {
     sg_n = min(32, seg_end - sg_base);
@@ -365,9 +378,15 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
     const int ps = __shfl_sync(0xffffffffu, sg_pstart, lo);
     const int o0 = __shfl_sync(0xffffffffu, sg_off, lo);
     const int g = __shfl_sync(0xffffffffu, sg_g, lo);
-    return x < sg_tot ? a.pages[ps + (x - o0)] * a.Hkv + g : 0;
+    if (x >= sg_tot) return 0;
+    int page = a.pages[ps + (x - o0)];
+    if (a.debug_checks && (uint32_t)page >= (uint32_t)a.num_pages) {
+      record_status(a.status, PA_ERR_DEVICE, gw, page);
+      page = 0;
+    }
+    return page * a.Hkv + g;
   };
-  int ld_x = 0, wbase = 0;          // next load (within the group), current window base
+  int ld_x = 0, wbase = 0;  // next load (within the group), current window base
   bool ld_more = seg_begin < seg_end;
   int win_cur = 0, win_nxt = 0;
   if (ld_more) {
@@ -402,12 +421,14 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
     const bool drop = drop_first && first_load;
     first_load = false;
     if (lane == 0 && !drop) {
-      uint8_t* st = wbase_smem + stage * S::STAGE;
+      const uint32_t st = ring + stage * S::STAGE;
       const uint32_t bar = smem_u32(&bars[stage]);
       mbar_arrive_expect_tx(bar, 2 * S::TILE);
-      const size_t off = (size_t)tile * (16 * D);
-      bulk_g2s(smem_u32(st), a.k_pool + off, S::TILE, bar);
-      bulk_g2s(smem_u32(st + S::TILE), a.v_pool + off, S::TILE, bar);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_2d(st + h * 2048, tk, 64 * h, tile * 16, bar);
+        tma_load_2d(st + S::TILE + h * 2048, tv, 64 * h, tile * 16, bar);
+      }
     }
     if (!drop) inflight |= 1u << stage;
     ++ld_x;
@@ -416,9 +437,14 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   // q rows (b, g*G .. g*G+G-1) are contiguous: q + (b*Hq + g*G)*D
   auto issue_q = [&](int slot, const SegInfo& si) {
     if (lane == 0) {
+      int b = si.query;
+      if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
+        record_status(a.status, PA_ERR_DEVICE, gw, -1 - b);
+        b = 0;
+      }
       const uint32_t bar = smem_u32(&qbars[slot]);
       mbar_arrive_expect_tx(bar, S::QT);
-      bulk_g2s(smem_u32(qslot + slot * S::QT), a.q + ((size_t)si.query * a.Hq + si.kv_head * G) * D, S::QT, bar);
+      bulk_g2s(smem_u32(qslot + slot * S::QT), a.q + ((size_t)b * a.Hq + si.kv_head * G) * D, S::QT, bar);
     }
     inflight |= 1u << (NST + slot);
   };
@@ -434,6 +460,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
   if (seg_begin < seg_end) issue_q(0, cur);
   for (int s = 0; s < NST; ++s) issue(s);
 
+  const float c = a.qscale;  // scale * log2(e), applied to the fp32 scores
   int stage = 0;
   bool failed = false;
   for (int si = seg_begin; si < seg_end; ++si) {
@@ -446,34 +473,26 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
     }
     inflight &= ~(1u << (NST + qs));
     parity ^= 1u << (NST + qs);
-    float2 qf[G][CPL][4];
+    // B operand of K.Q^T: b0 = q[row g][16 kk + 2t, +1], b1 = q[row g][16 kk + 2t + 8, +9]
+    uint32_t qb[KT][2];
+    {
+      const uint8_t* qrow = qslot + qs * S::QT + (g8 < G ? g8 : 0) * D * 2;
 #pragma unroll
-    for (int r = 0; r < G; ++r)
-#pragma unroll
-      for (int j = 0; j < CPL; ++j) {
-        const uint4 w = *reinterpret_cast<const uint4*>(qslot + qs * S::QT + r * D * 2 + (li + LPG * j) * 16);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = bf16x2_to_f2(ws[e]);
-          qf[r][j][e] = make_float2(f.x * a.qscale, f.y * a.qscale);
-        }
+      for (int kk = 0; kk < KT; ++kk) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(qrow + (16 * kk + 2 * t4) * 2);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(qrow + (16 * kk + 2 * t4 + 8) * 2);
+        qb[kk][0] = g8 < G ? w0 : 0u;
+        qb[kk][1] = g8 < G ? w1 : 0u;
       }
+    }
     __syncwarp();
     if (si + 1 < seg_end) issue_q(qs ^ 1, nx);
 
     const int npages = (cur.n_tokens + 15) >> 4;
-    float2 o[G][CPL][4];
-    float m[G], l[G];
+    float o[KT][4];
 #pragma unroll
-    for (int r = 0; r < G; ++r) {
-      m[r] = -INFINITY;
-      l[r] = 0.f;
-#pragma unroll
-      for (int j = 0; j < CPL; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[r][j][e] = make_float2(0.f, 0.f);
-    }
+    for (int i = 0; i < KT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float ms[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     for (int pg = 0; pg < npages; ++pg) {
       if (!mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u, a.timeout_ns)) {
         if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, gw, si);
@@ -482,69 +501,48 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, uint8_t* smem) {
       }
       inflight &= ~(1u << stage);
       parity ^= 1u << stage;
-      const uint8_t* kt = wbase_smem + stage * S::STAGE;
+      const uint32_t kt = ring + stage * S::STAGE;
       const int nvalid = cur.n_tokens - pg * 16;
-      if (nvalid >= 16) simt_page<D, G, false>(kt, kt + S::TILE, 16, grp, li, qf, o, m, l);
-      else simt_page<D, G, true>(kt, kt + S::TILE, nvalid, grp, li, qf, o, m, l);
+      if (nvalid >= 16) tile_step<D, G, false>(kt, kt + S::TILE, 16, lane, c, qb, o, ms, l);
+      else tile_step<D, G, true>(kt, kt + S::TILE, nvalid, lane, c, qb, o, ms, l);
       __syncwarp();
       issue(stage);
       stage = stage + 1 == NST ? 0 : stage + 1;
     }
     if (failed) break;
 
-    // combine the NG key groups (butterfly over the group bits of the lane id)
+    // the sum over the keys of each row: the 8 lanes that share t
 #pragma unroll
-    for (int msk = LPG; msk < 32; msk <<= 1) {
-#pragma unroll
-      for (int r = 0; r < G; ++r) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m[r], msk);
-        const float lo = __shfl_xor_sync(0xffffffffu, l[r], msk);
-        const float mn = fmaxf(m[r], mo);
-        const float ca = m[r] == -INFINITY ? 0.f : ex2(m[r] - mn);
-        const float cb = mo == -INFINITY ? 0.f : ex2(mo - mn);
-        l[r] = l[r] * ca + lo * cb;
-        m[r] = mn;
-        const float2 ca2 = make_float2(ca, ca), cb2 = make_float2(cb, cb);
-#pragma unroll
-        for (int j = 0; j < CPL; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 other;
-            other.x = __shfl_xor_sync(0xffffffffu, o[r][j][e].x, msk);
-            other.y = __shfl_xor_sync(0xffffffffu, o[r][j][e].y, msk);
-            o[r][j][e] = ffma2(o[r][j][e], ca2, fmul2(other, cb2));
-          }
-      }
+    for (int off = 4; off < 32; off <<= 1) {
+      l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
+      l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
     }
-    // write: group k writes rows r with r % NG == k; a (request, kv head) with a
-    // single partial row goes straight to the output when the merge is fused
+    // write: thread (g, t) holds dims 16 i + g and 16 i + g + 8 of rows 2t, 2t+1;
+    // a (request, kv head) with a single partial row goes straight to the
+    // output when the merge is fused
     const bool direct = a.out && cur.mode == 1;
 #pragma unroll
-    for (int r = 0; r < G; ++r) {
-      if (r % S::NG != grp) continue;
-      const float inv = 1.f / l[r];
-      const float lse_r = (m[r] + lg2(l[r])) * kLn2;
+    for (int j = 0; j < 2; ++j) {
+      const int r = 2 * t4 + j;
+      if (r >= G) continue;
+      const float inv = 1.f / l[j];
+      const float lse_r = (ms[j] + lg2(l[j])) * kLn2;
       if (direct) {
-        __nv_bfloat16* dst = a.out + ((size_t)cur.query * a.Hq + cur.kv_head * G + r) * D;
+        __nv_bfloat16* dst = a.out + ((size_t)cur.query * a.Hq + cur.kv_head * G + r) * D + g8;
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(o[r][j][0].x * inv, o[r][j][0].y * inv);
-          w.y = pack_bf16x2(o[r][j][1].x * inv, o[r][j][1].y * inv);
-          w.z = pack_bf16x2(o[r][j][2].x * inv, o[r][j][2].y * inv);
-          w.w = pack_bf16x2(o[r][j][3].x * inv, o[r][j][3].y * inv);
-          *reinterpret_cast<uint4*>(dst + (li + LPG * j) * 8) = w;
+        for (int i = 0; i < KT; ++i) {
+          dst[16 * i] = __float2bfloat16_rn(o[i][j] * inv);
+          dst[16 * i + 8] = __float2bfloat16_rn(o[i][2 + j] * inv);
         }
-        if (li == 0 && a.lse) a.lse[(size_t)cur.query * a.Hq + cur.kv_head * G + r] = lse_r;
+        if (g8 == 0 && a.lse) a.lse[(size_t)cur.query * a.Hq + cur.kv_head * G + r] = lse_r;
       } else {
-        float* dst = a.partial_o + ((size_t)cur.prow * G + r) * D;
+        float* dst = a.partial_o + ((size_t)cur.prow * G + r) * D + g8;
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-          float4* d4 = reinterpret_cast<float4*>(dst + (li + LPG * j) * 8);
-          d4[0] = make_float4(o[r][j][0].x * inv, o[r][j][0].y * inv, o[r][j][1].x * inv, o[r][j][1].y * inv);
-          d4[1] = make_float4(o[r][j][2].x * inv, o[r][j][2].y * inv, o[r][j][3].x * inv, o[r][j][3].y * inv);
+        for (int i = 0; i < KT; ++i) {
+          dst[16 * i] = o[i][j] * inv;
+          dst[16 * i + 8] = o[i][2 + j] * inv;
         }
-        if (li == 0) a.partial_lse[(size_t)cur.prow * G + r] = lse_r;
+        if (g8 == 0) a.partial_lse[(size_t)cur.prow * G + r] = lse_r;
       }
     }
     if (a.out && (cur.mode == 0 || cur.mode == 2)) {
@@ -603,7 +601,7 @@ constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kSmaxThreads = 256;    // softmax threads (two per tile row)
 constexpr int kSBufs = 3;            // S/P buffers in TMEM
 constexpr uint32_t kTmemCols = 512;  // the whole tensor memory of the SM (one CTA per SM)
-constexpr float kRescaleThreshold = 8.f;  // log2 units
+constexpr float kRescaleThreshold = kRescaleLog2;
 
 template <int D>
 struct MmaShape {
@@ -696,14 +694,23 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const pa_seg seg = a.segs[si];
       const int32_t* pg = a.pages + a.items[seg.item].page_off + seg.page_begin;
       const int npages = (seg.n_tokens + 15) >> 4;
+      auto page_at = [&](int x) -> int {
+        if (x >= npages) return 0;
+        int pid = pg[x];
+        if (a.debug_checks && (uint32_t)pid >= (uint32_t)a.num_pages) {
+          record_status(a.status, PA_ERR_DEVICE, blockIdx.x, pid);
+          pid = 0;
+        }
+        return pid;
+      };
       int wbase = 0;
-      int wcur = lane < npages ? pg[lane] : 0;
-      int wnxt = 32 + lane < npages ? pg[32 + lane] : 0;
+      int wcur = page_at(lane);
+      int wnxt = page_at(32 + lane);
       for (int st = 0; st < npages; st += 4, ++i) {
         if (st - wbase >= 32) {
           wbase += 32;
           wcur = wnxt;
-          wnxt = wbase + 32 + lane < npages ? pg[wbase + 32 + lane] : 0;
+          wnxt = page_at(wbase + 32 + lane);
         }
         const int s = i % NST;
         if (i >= NST && !warp_wait(bar(b_empty + s), ((i / NST) - 1) & 1, a.timeout_ns)) {
@@ -818,7 +825,11 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const int R = item.n_queries * G;
       const uint16_t* src = nullptr;
       if (r < R) {
-        const int b = a.queries[item.query_off + r / G];
+        int b = a.queries[item.query_off + r / G];
+        if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
+          record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
+          b = 0;
+        }
         src = a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
       }
 #pragma unroll
@@ -1038,9 +1049,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
 // a tensor-core launch it does not end before that launch has, so work later
 // in the stream sees both.
 template <int D, int G>
-__global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1) simt_fwd_kernel(const FwdArgs a) {
+__global__ void __launch_bounds__(kSimtWarpsPerCta * 32, 1)
+    simt_fwd_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  simt_role<D, G>(a, smem);
+  simt_role<D, G>(a, &tk, &tv, smem);
   griddep_wait();
 }
 
@@ -1092,6 +1104,9 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.qscale = p.scale * kLog2e;
   a.timeout_ns = (uint64_t)p.wait_timeout_us * 1000ull;
   a.fault_drop = (p.flags & PA_PLAN_FAULT_DROP_LOAD) ? 1 : 0;
+  a.debug_checks = (p.flags & PA_PLAN_DEBUG_CHECKS) ? 1 : 0;
+  a.num_pages = p.num_pages_in_pool;
+  a.B = p.B;
   return a;
 }
 
@@ -1115,11 +1130,11 @@ template <int D, int G>
 int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
   static bool attr_mma[64] = {}, attr_simt[64] = {};
   const int n_simt_ctas = (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
+  const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
+  const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
   if (a.n_mma_ctas > 0) {
     auto k = mma_fwd_kernel<D, G>;
     if (int e = set_smem_attr(k, attr_mma)) return e;
-    const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
-    const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
     k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D>::SMEM, st>>>(a, *tk, *tv);
     if (cudaError_t e = cudaGetLastError()) return (int)e;
   }
@@ -1136,7 +1151,7 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.n_mma_ctas > 0 ? 1 : 0;
-    if (cudaError_t e = cudaLaunchKernelEx(&cfg, k, a)) return (int)e;
+    if (cudaError_t e = cudaLaunchKernelEx(&cfg, k, a, *tk, *tv)) return (int)e;
   }
   return 0;
 }

@@ -637,7 +637,8 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
   if (cfg->max_chunk_tokens < 0 || cfg->wait_timeout_us < 0 || cfg->num_sms < 0) return PA_ERR_INVALID;
   const uint32_t flags = cfg->flags;
   if ((flags & PA_PLAN_NO_SHARING) && (flags & PA_PLAN_ALWAYS_SHARE)) return PA_ERR_INVALID;
-  if ((int64_t)num_pages_in_pool * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  // the kernels address a pool as rows of D values (page, kv head, slot): a TMA coordinate is int32
+  if ((int64_t)num_pages_in_pool * Hkv * P > INT32_MAX) return PA_ERR_UNSUPPORTED;
 
   pa_plan* plan = new (std::nothrow) pa_plan();
   if (!plan) return PA_ERR_NOMEM;
@@ -718,7 +719,7 @@ extern "C" pa_status pa_plan_advance(const pa_plan* prev, const int32_t* kv_lens
   auto t0 = std::chrono::steady_clock::now();
   const int batch = prev->B, P = prev->P, Hkv = prev->Hkv;
   if (max_pages < 1 || num_pages_in_pool < 1) return PA_ERR_INVALID;
-  if ((int64_t)num_pages_in_pool * Hkv > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if ((int64_t)num_pages_in_pool * Hkv * P > INT32_MAX) return PA_ERR_UNSUPPORTED;
   bool rebuild = num_pages_in_pool < prev->num_pages_in_pool;
   for (int b = 0; b < batch; ++b) {
     const int64_t n = kv_lens[b];
@@ -830,6 +831,40 @@ extern "C" pa_status pa_plan_advance(const pa_plan* prev, const int32_t* kv_lens
   } catch (...) {
     delete plan;
     return PA_ERR_INVALID;
+  }
+}
+
+extern "C" pa_status pa_plan_create_append(const pa_config* cfg, int32_t n_sessions, const int32_t* ctx_lens,
+                                           const int32_t* chunk_lens, const int32_t* block_table, int32_t max_pages,
+                                           int32_t num_pages_in_pool, pa_plan** out) {
+  if (out) *out = nullptr;
+  if (!cfg || !ctx_lens || !chunk_lens || !block_table || !out || n_sessions < 1 || max_pages < 1)
+    return PA_ERR_INVALID;
+  // one row per new token: row i of session s is a request over the session's
+  // block-table row whose length stops at its own token (ctx_lens[s] + i + 1),
+  // so it sees the whole context and the chunk tokens up to itself (causal
+  // inside the chunk); the rows of a session share the context's full pages,
+  // which the pack stage then reads once for all of them
+  int64_t rows = 0;
+  for (int s = 0; s < n_sessions; ++s) {
+    if (ctx_lens[s] < 0 || chunk_lens[s] < 1) return PA_ERR_INVALID;
+    if ((int64_t)ctx_lens[s] + chunk_lens[s] > (int64_t)max_pages * cfg->page_size) return PA_ERR_INVALID;
+    rows += chunk_lens[s];
+  }
+  if (rows > INT32_MAX / 2) return PA_ERR_UNSUPPORTED;
+  try {
+    std::vector<int32_t> kv((size_t)rows), bt((size_t)rows * max_pages);
+    size_t r = 0;
+    for (int s = 0; s < n_sessions; ++s) {
+      const int32_t* src = block_table + (size_t)s * max_pages;
+      for (int i = 0; i < chunk_lens[s]; ++i, ++r) {
+        kv[r] = ctx_lens[s] + i + 1;
+        std::memcpy(&bt[r * max_pages], src, sizeof(int32_t) * max_pages);
+      }
+    }
+    return pa_plan_create(cfg, (int32_t)rows, kv.data(), bt.data(), max_pages, num_pages_in_pool, out);
+  } catch (const std::bad_alloc&) {
+    return PA_ERR_NOMEM;
   }
 }
 

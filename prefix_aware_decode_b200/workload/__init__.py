@@ -355,6 +355,22 @@ def config1_stream(n: int, seed: int = 1001, with_values: bool = True) -> "Workl
     return build_workload(f"config 1 x {n}", roots, 8, 2, 64, seed, with_values=with_values)
 
 
+def session_chunks(ctx_lens, chunk_lens, Hq: int, Hkv: int, D: int, seed: int):
+    """Sessions that each append a chunk of new tokens (the prefix-aware
+    grouped prefill of stateful sessions): session s holds ctx_lens[s] context
+    tokens followed by its chunk_lens[s] new tokens, all already in the paged
+    pool (append, then attend).  Returns (workload, q_rows): the workload's
+    request s is session s over all its tokens; q_rows uint16 [sum chunk][Hq][D]
+    are the new tokens' queries, sessions in order, each chunk in token order."""
+    roots = [Node(int(c) + int(n)) for c, n in zip(ctx_lens, chunk_lens)]
+    w = build_workload("chunks", roots, Hq, Hkv, D, seed)
+    rows = int(np.sum(chunk_lens))
+    q = np.empty((rows, Hq, D), dtype=np.uint16)
+    for r in range(rows):
+        q[r] = normal_bf16(seed, TAG_Q, 1 << 20 | r, Hq * D).reshape(Hq, D)
+    return w, q
+
+
 def config_tree(config: int, seed: int, scale: float = 1.0):
     """Return (roots, Hq, Hkv, D) for one of the five configs.
 

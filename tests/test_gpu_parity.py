@@ -314,3 +314,39 @@ def test_decode_steps_alternating_batches_and_one_plan_over_several_pools():
         assert_close(compare(o, l, *ref), f"pool pair {layer}")
     assert p.device_status(ws) == pad.PA_OK
     p.close()
+
+
+@pytest.mark.parametrize("flags", [pad.PA_PLAN_NO_SHARING, pad.PA_PLAN_ALWAYS_SHARE])
+def test_debug_checks_catch_a_corrupted_page_id(flags):
+    """PA_PLAN_DEBUG_CHECKS range-checks every page id the kernels read from
+    the device image before any load is issued.  The pools here hold 8 NaN
+    pages more than the plan declares, and the uploaded image's first page id
+    is overwritten with one of them: still inside the allocation (an unchecked
+    read would stay in bounds) but past the declared pool, so the check must
+    record PA_ERR_DEVICE.  The first page id belongs to request 0's own item
+    (small-row class) without sharing, and to the shared prefix (tensor-core
+    class) with it.  A clean run on the same plan is correct again."""
+    import ctypes
+
+    w = wl.make_config(1)
+    extra = np.full((8,) + w.k_pool.shape[1:], wl.BF16_NAN, np.uint16)
+    k = torch.from_numpy(np.concatenate([w.k_pool, extra]).view(np.int16)).cuda().view(torch.bfloat16)
+    v = torch.from_numpy(np.concatenate([w.v_pool, extra]).view(np.int16)).cuda().view(torch.bfloat16)
+    q = torch.from_numpy(w.q.view(np.int16)).cuda().view(torch.bfloat16)
+    plan = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D,
+                    flags=flags | pad.PA_PLAN_DEBUG_CHECKS)
+    h = pad.PaImageHeader.from_buffer_copy(plan.host_image()[: ctypes.sizeof(pad.PaImageHeader)].tobytes())
+    ws = plan.alloc_workspace()
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    plan.upload(ws)
+    torch.cuda.synchronize()
+    ws[h.off_pages:h.off_pages + 4].view(torch.int32).fill_(w.num_pages + 3)
+    plan.attend(q, k, v, ws, out, lse)
+    assert plan.device_status(ws) == pad.PA_ERR_DEVICE
+    plan.upload(ws)
+    plan.attend(q, k, v, ws, out, lse)
+    assert plan.device_status(ws) == pad.PA_OK
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    assert_close(compare(out, lse, ref_o, ref_l), "debug checks, clean run")
+    plan.close()

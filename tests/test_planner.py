@@ -447,3 +447,34 @@ def test_random_partially_shared_pages_against_the_oracle():
             ref_o, ref_l = oracle.attend_paged(q, k, v, bt, lens)
             np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
             np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("G,D", [(1, 64), (4, 128), (8, 64)])
+def test_append_plan_executes_to_the_oracle_rows(G, D):
+    # chunks of 1, 5, 16 and 19 new tokens over contexts that end on and off
+    # page boundaries (0 tokens included): each row must see the context and
+    # the chunk up to itself, nothing after it
+    ctx = np.array([0, 37, 48, 200, 333], dtype=np.int32)
+    chunk = np.array([5, 19, 1, 16, 19], dtype=np.int32)
+    w, q = wl.session_chunks(ctx, chunk, Hq=2 * G, Hkv=2, D=D, seed=11 * G + D)
+    plan = pad.Plan.append(ctx, chunk, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    st = plan.stats()
+    assert st["batch"] == chunk.sum()
+    img = Image(plan.host_image())
+    row_req = np.repeat(np.arange(len(ctx)), chunk)
+    row_pos = np.concatenate([c + np.arange(n) for c, n in zip(ctx, chunk)])
+    check_structure(img, (row_pos + 1).astype(np.int32), w.block_table[row_req])
+    o, l = execute(img, q, w.k_pool, w.v_pool)
+    ro, rl = oracle.attend_rows(q, row_req, row_pos, w.k_pool, w.v_pool, w.block_table)
+    assert np.abs(o - ro).max() < 1e-12 and np.abs(l - rl).max() < 1e-12
+    # the rows of a session with a long context share its full pages
+    assert st["num_kept_shared"] >= 1
+    plan.close()
+
+
+def test_append_plan_rejects_bad_chunks():
+    bt = np.zeros((1, 4), np.int32)
+    with pytest.raises(pad.PaError):
+        pad.Plan.append([10], [0], bt, 4, 8, 2, 64)
+    with pytest.raises(pad.PaError):
+        pad.Plan.append([60], [5], bt, 4, 8, 2, 64)  # 65 tokens > 4 pages
