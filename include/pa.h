@@ -222,6 +222,40 @@ pa_status pa_forward(const pa_plan *plan, const void *q, const void *k_pool, con
 pa_status pa_merge(const pa_plan *plan, void *d_workspace, void *out, float *lse, void *stream);
 
 /*
+ * Merge into fp32 instead of bf16: out is fp32 [B][Hq][D] (not rounded), lse
+ * fp32 [B][Hq] (may be NULL).  This is the per-rank result of context
+ * parallelism, which pa_merge_rows combines after the ranks' rows have been
+ * gathered; otherwise as pa_merge (the PAT review's Merge 阶段, section 三).
+ */
+pa_status pa_merge_f32(const pa_plan *plan, void *d_workspace, float *out, float *lse, void *stream);
+
+/*
+ * Merge of attention rows gathered from several parts of the KV (context
+ * parallelism: each part is one rank's result over its slice of every
+ * request's pages).  The combine is the merge stage's log-sum-exp rule (the
+ * PAT review, section 三, Merge 阶段), taken over the parts in order:
+ *   lse[b][h] = log sum_p e^{lse_p}, out[b][h] = sum_p e^{lse_p - lse} o_p.
+ *   n_parts, rows_per_part
+ *                     parts of the gather, each padded to rows_per_part rows
+ *   batch, num_q_heads, head_dim
+ *                     B, Hq, D (64 or 128) of the whole batch
+ *   d_part_req        device int32 [n_parts][rows_per_part]: the request of
+ *                     each row, ascending within a part, -1 for padding rows
+ *                     (which must come last)
+ *   d_part_o          device fp32 [n_parts][rows_per_part][Hq][D] (pa_merge_f32
+ *                     of each part), 16-byte aligned
+ *   d_part_lse        device fp32 [n_parts][rows_per_part][Hq]
+ *   out               device bf16 [B][Hq][D] (round-to-nearest-even), lse fp32
+ *                     [B][Hq] (may be NULL); a request in no part gets zeros
+ *                     and lse = -inf
+ * Asynchronous on `stream`; errors PA_ERR_INVALID / PA_ERR_UNSUPPORTED before
+ * anything is enqueued, PA_ERR_CUDA on a launch failure.
+ */
+pa_status pa_merge_rows(int32_t n_parts, int32_t rows_per_part, int32_t batch, int32_t num_q_heads,
+                        int32_t head_dim, const int32_t *d_part_req, const float *d_part_o, const float *d_part_lse,
+                        void *out, float *lse, void *stream);
+
+/*
  * Forward with the merge fused into it (one launch): the warp that writes the
  * last partial row of a (request, kv head) pair merges that pair into out and
  * lse (the PAT review's Forward and Merge stages, section 三, in one pass).  Same results as pa_forward + pa_merge, bit for bit.  The arrival

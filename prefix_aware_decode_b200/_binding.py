@@ -63,7 +63,7 @@ class PaImageHeader(ctypes.Structure):
 
 
 # exported names, in the order pa.h declares them
-EXPORTS = ["pa_plan_create", "pa_plan_advance", "pa_plan_create_append", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_attend",
+EXPORTS = ["pa_plan_create", "pa_plan_advance", "pa_plan_create_append", "pa_plan_workspace_size", "pa_plan_upload", "pa_forward", "pa_merge", "pa_merge_f32", "pa_merge_rows", "pa_attend",
            "pa_get_device_status", "pa_plan_get_stats", "pa_plan_host_image", "pa_plan_set_profile_events",
            "pa_decode_step", "pa_attend_noalloc", "pa_plan_destroy", "pa_status_string"]
 
@@ -94,6 +94,10 @@ def lib() -> ctypes.CDLL:
     L.pa_forward.restype = st
     L.pa_merge.argtypes = [vp, vp, vp, vp, vp]
     L.pa_merge.restype = st
+    L.pa_merge_f32.argtypes = [vp, vp, vp, vp, vp]
+    L.pa_merge_f32.restype = st
+    L.pa_merge_rows.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.pa_merge_rows.restype = st
     L.pa_attend.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
     L.pa_attend.restype = st
     L.pa_get_device_status.argtypes = [vp, vp, vp, ctypes.POINTER(ctypes.c_int)]
@@ -252,6 +256,13 @@ class Plan:
                                   _dptr(lse, "lse", 4) if lse is not None else None, _stream_ptr(stream)),
                "pa_merge")
 
+    def merge_f32(self, ws, out, lse=None, stream=None):
+        """pa_merge_f32: out fp32 [B][Hq][D], not rounded (a rank's part of a
+        context-parallel batch)."""
+        _check(self._lib.pa_merge_f32(self._h, _dptr(ws, "workspace", 256), _dptr(out, "out"),
+                                      _dptr(lse, "lse", 4) if lse is not None else None, _stream_ptr(stream)),
+               "pa_merge_f32")
+
     def attend(self, q, k_pool, v_pool, ws, out, lse=None, stream=None):
         _check(self._lib.pa_attend(self._h, _dptr(q, "q"), _dptr(k_pool, "k_pool"), _dptr(v_pool, "v_pool"),
                                    _dptr(ws, "workspace", 256), _dptr(out, "out"),
@@ -280,6 +291,18 @@ class Plan:
         _check(self._lib.pa_get_device_status(self._h, _dptr(ws, "workspace", 256) if ws is not None else None,
                                               _stream_ptr(stream), ctypes.byref(out)), "pa_get_device_status")
         return out.value
+
+
+def merge_rows(part_req, part_o, part_lse, batch: int, out, lse=None, stream=None):
+    """pa_merge_rows: combine rows gathered from several parts of the KV.
+    part_req int32 [P][R] (ascending, -1 padding last), part_o fp32 [P][R][Hq][D],
+    part_lse fp32 [P][R][Hq] (CUDA tensors); out bf16 [batch][Hq][D]."""
+    P, R = part_req.shape
+    Hq, D = part_o.shape[2], part_o.shape[3]
+    _check(lib().pa_merge_rows(P, R, batch, Hq, D, _dptr(part_req, "part_req", 4), _dptr(part_o, "part_o"),
+                               _dptr(part_lse, "part_lse", 4), _dptr(out, "out"),
+                               _dptr(lse, "lse", 4) if lse is not None else None, _stream_ptr(stream)),
+           "pa_merge_rows")
 
 
 def attend(q, k_pool, v_pool, block_table, kv_lens, softmax_scale: float = 0.0, flags: int = 0,

@@ -217,6 +217,30 @@ extern "C" pa_status pa_merge(const pa_plan* plan, void* d_workspace, void* out,
   return e == 0 ? PA_OK : PA_ERR_CUDA;
 }
 
+extern "C" pa_status pa_merge_f32(const pa_plan* plan, void* d_workspace, float* out, float* lse, void* stream) {
+  if (!plan || !d_workspace || !out) return PA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(d_workspace) & 255))
+    return PA_ERR_INVALID;
+  PaDevPtrs d = dev_ptrs(*plan, d_workspace);
+  record_profile(*plan, 2, static_cast<cudaStream_t>(stream));
+  const int e = pa_launch_merge(*plan, d, out, lse, stream, true);
+  record_profile(*plan, 3, static_cast<cudaStream_t>(stream));
+  return e == 0 ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" pa_status pa_merge_rows(int32_t n_parts, int32_t rows_per_part, int32_t batch, int32_t num_q_heads,
+                                   int32_t head_dim, const int32_t* d_part_req, const float* d_part_o,
+                                   const float* d_part_lse, void* out, float* lse, void* stream) {
+  if (n_parts < 1 || rows_per_part < 1 || batch < 1 || num_q_heads < 1 || !d_part_req || !d_part_o || !d_part_lse ||
+      !out)
+    return PA_ERR_INVALID;
+  if (!(head_dim == 64 || head_dim == 128)) return PA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(d_part_o) | reinterpret_cast<uintptr_t>(out)) & 15) return PA_ERR_INVALID;
+  const int e = pa_launch_merge_rows(n_parts, rows_per_part, batch, num_q_heads, head_dim, d_part_req, d_part_o,
+                                     d_part_lse, out, lse, stream);
+  return e == 0 ? PA_OK : PA_ERR_CUDA;
+}
+
 extern "C" pa_status pa_attend(const pa_plan* plan, const void* q, const void* k_pool, const void* v_pool,
                                void* d_workspace, void* out, float* lse, void* stream) {
   if (!out) return PA_ERR_INVALID;

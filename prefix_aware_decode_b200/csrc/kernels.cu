@@ -77,8 +77,8 @@ struct FwdArgs {
 // whose loads are all issued before any is used, so a pair costs about one
 // memory round trip per NB partial rows.  Partial rows are read through L2
 // (they may have been written by other SMs in the same launch).
-template <int D, int G>
-__device__ __forceinline__ void merge_pair(const float* partial_lse, const float* partial_o, __nv_bfloat16* out,
+template <int D, int G, typename OutT = __nv_bfloat16>
+__device__ __forceinline__ void merge_pair(const float* partial_lse, const float* partial_o, OutT* out,
                                            float* lse, int Hq, int b, int g, int p0, int p1, int lane) {
   constexpr int LPR = 32 / G;   // lanes per row
   constexpr int VPL = D / LPR;  // head dims per lane
@@ -130,10 +130,15 @@ __device__ __forceinline__ void merge_pair(const float* partial_lse, const float
     m = mn;
   }
   const float inv = 1.f / z;
-  __nv_bfloat16* dst = out + ((size_t)b * Hq + g * G + r) * D + d0;
+  OutT* dst = out + ((size_t)b * Hq + g * G + r) * D + d0;
+  if constexpr (std::is_same<OutT, float>::value) {
 #pragma unroll
-  for (int i = 0; i < VPL; i += 2)
-    *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+    for (int i = 0; i < VPL; i += 2) *reinterpret_cast<float2*>(dst + i) = make_float2(acc[i] * inv, acc[i + 1] * inv);
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; i += 2)
+      *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+  }
   if (lse && lane % LPR == 0) lse[(size_t)b * Hq + g * G + r] = m + logf(z);
 }
 
@@ -1060,9 +1065,10 @@ struct MergeArgs {
   const int32_t* prow_off;
   const float* partial_lse;
   const float* partial_o;
-  __nv_bfloat16* out;
+  void* out;  // bf16 [B][Hq][D], or fp32 when out_f32
   float* lse;
   int B, Hq, Hkv, G;
+  int out_f32;
 };
 
 // One warp per (request, kv head) pair: every pair (list == nullptr), or the
@@ -1072,8 +1078,68 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a, const int
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (w >= n) return;
   const int bg = list ? list[w] : w;
-  merge_pair<D, G>(a.partial_lse, a.partial_o, a.out, a.lse, a.Hq, bg / a.Hkv, bg % a.Hkv, a.prow_off[bg],
-                   a.prow_off[bg + 1], lane);
+  if (a.out_f32)
+    merge_pair<D, G, float>(a.partial_lse, a.partial_o, static_cast<float*>(a.out), a.lse, a.Hq, bg / a.Hkv,
+                            bg % a.Hkv, a.prow_off[bg], a.prow_off[bg + 1], lane);
+  else
+    merge_pair<D, G>(a.partial_lse, a.partial_o, static_cast<__nv_bfloat16*>(a.out), a.lse, a.Hq, bg / a.Hkv,
+                     bg % a.Hkv, a.prow_off[bg], a.prow_off[bg + 1], lane);
+}
+
+// Merge of rows gathered from several parts (context parallelism: each part
+// is one rank's attention over its slice of the requests' KV, normalised, in
+// fp32, with its log-sum-exp).  Part p holds rows_per_part rows; row j of part
+// p is request req[p][j] (ascending within a part; -1 marks padding).  One
+// warp per (request, query head): for each part, a binary search finds the
+// request's row, and the rows found are combined with the merge stage's
+// log-sum-exp rule in part order.
+template <int D>
+__global__ void __launch_bounds__(256)
+    merge_rows_kernel(int n_parts, int rows_per_part, int B, int Hq, const int32_t* __restrict__ req,
+                      const float* __restrict__ part_o, const float* __restrict__ part_lse, __nv_bfloat16* out,
+                      float* lse) {
+  constexpr int VPL = D / 32;
+  const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (w >= B * Hq) return;
+  const int b = w / Hq, h = w % Hq;
+  float m = -INFINITY, z = 0.f, acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  for (int p = 0; p < n_parts; ++p) {
+    const int32_t* rq = req + (size_t)p * rows_per_part;
+    int lo = 0, hi = rows_per_part;  // first row whose request is >= b (padding counts as past the end)
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      const int v = rq[mid];
+      if (v >= 0 && v < b) lo = mid + 1;
+      else hi = mid;
+    }
+    if (lo >= rows_per_part || rq[lo] != b) continue;
+    const size_t row = (size_t)p * rows_per_part + lo;
+    const float lp = part_lse[row * Hq + h];
+    if (lp == -INFINITY) continue;
+    const float* src = part_o + (row * Hq + h) * D + lane * VPL;
+    float o[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; i += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src + i);
+      o[i] = v.x;
+      o[i + 1] = v.y;
+    }
+    const float mn = fmaxf(m, lp);
+    const float sa = m == -INFINITY ? 0.f : expf(m - mn);
+    const float wgt = expf(lp - mn);
+    z = z * sa + wgt;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] = fmaf(o[i], wgt, acc[i] * sa);
+    m = mn;
+  }
+  __nv_bfloat16* dst = out + ((size_t)b * Hq + h) * D + lane * VPL;
+  const float inv = z > 0.f ? 1.f / z : 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; i += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+  if (lse && lane == 0) lse[(size_t)b * Hq + h] = z > 0.f ? m + logf(z) : -INFINITY;
 }
 
 FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse) {
@@ -1186,13 +1252,14 @@ int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
 namespace {
 
 int launch_merge_list(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, const int32_t* list, int n,
-                      void* stream) {
+                      void* stream, bool out_f32 = false) {
   if (n <= 0) return 0;
   MergeArgs a;
   a.prow_off = d.prow_off;
   a.partial_lse = d.partial_lse;
   a.partial_o = d.partial_o;
-  a.out = static_cast<__nv_bfloat16*>(out);
+  a.out = out;
+  a.out_f32 = out_f32 ? 1 : 0;
   a.lse = lse;
   a.B = p.B;
   a.Hq = p.Hq;
@@ -1215,8 +1282,22 @@ int launch_merge_list(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
 
 }  // namespace
 
-int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {
-  return launch_merge_list(p, d, out, lse, nullptr, p.B * p.Hkv, stream);
+int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream, bool out_f32) {
+  return launch_merge_list(p, d, out, lse, nullptr, p.B * p.Hkv, stream, out_f32);
+}
+
+int pa_launch_merge_rows(int n_parts, int rows_per_part, int B, int Hq, int D, const int32_t* req,
+                         const float* part_o, const float* part_lse, void* out, float* lse, void* stream) {
+  const int n = B * Hq;
+  if (n <= 0) return 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  if (D == 128) merge_rows_kernel<128><<<(n + 7) / 8, 256, 0, st>>>(n_parts, rows_per_part, B, Hq, req, part_o,
+                                                                    part_lse, o, lse);
+  else if (D == 64) merge_rows_kernel<64><<<(n + 7) / 8, 256, 0, st>>>(n_parts, rows_per_part, B, Hq, req, part_o,
+                                                                       part_lse, o, lse);
+  else return (int)cudaErrorInvalidValue;
+  return (int)cudaGetLastError();
 }
 
 int pa_launch_tail_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream) {

@@ -94,7 +94,10 @@ struct PaDevPtrs {
 
 // out == nullptr: partial rows only; else the merge is fused into the launch.
 int pa_launch_forward(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
-int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
+int pa_launch_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream, bool out_f32 = false);
+// Merge of per-part rows gathered across ranks (pa_merge_rows).
+int pa_launch_merge_rows(int n_parts, int rows_per_part, int B, int Hq, int D, const int32_t* req,
+                         const float* part_o, const float* part_lse, void* out, float* lse, void* stream);
 // Merge of the pairs in the plan's tail list (after a fused forward launch).
 int pa_launch_tail_merge(const pa_plan& p, const PaDevPtrs& d, void* out, float* lse, void* stream);
 

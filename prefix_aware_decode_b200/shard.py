@@ -1,6 +1,6 @@
 """Data-parallel sharding of one decode batch across ranks (host logic).
 
-Requests are grouped by the page id of their first block: requests in
+Data parallelism: requests are grouped by the page id of their first block: requests in
 different groups share no prefix, so whole groups (root subtrees of the tree
 block table) are assigned to ranks and no shared node is split across GPUs.
 Groups go to the least-loaded rank in decreasing order of KV tokens (longest
@@ -71,22 +71,34 @@ def context_slices(block_table: np.ndarray, kv_lens: np.ndarray, world: int):
     return out
 
 
-def merge_context_partials(B: int, parts):
-    """Combines per-rank results of context_slices: parts[r] = (requests,
-    out [n][Hq][D], lse [n][Hq]) with out the rank's attention over its slice
-    (normalised) and lse its log-sum-exp.  The result over the whole KV is the
-    same log-sum-exp combine as the merge stage: lse = ln Σ_r e^{lse_r},
-    out = Σ_r e^{lse_r − lse} out_r.  Host fp64 reference of the exchange step;
-    on GPUs the parts arrive by an all-gather."""
-    shape_o = parts[0][1].shape[1:]
-    shape_l = parts[0][2].shape[1:]
-    m = np.full((B,) + shape_l, -np.inf)
-    for reqs, _, l in parts:
-        m[reqs] = np.maximum(m[reqs], l)
-    z = np.zeros((B,) + shape_l)
-    acc = np.zeros((B,) + shape_o)
-    for reqs, o, l in parts:
-        wgt = np.exp(l - m[reqs])
-        z[reqs] += wgt
-        acc[reqs] += wgt[..., None] * o
-    return acc / z[..., None], m + np.log(z)
+def exchange_context_parts(reqs, out_f32, lse_f32, batch: int, out, lse=None, group=None):
+    """The exchange step of context parallelism on GPUs: every rank's
+    (request ids, fp32 out [n][Hq][D], lse [n][Hq]) of its slice, padded to the
+    largest slice, is all-gathered over NCCL (torch.distributed, the process
+    group's backend), and the rows are merged on the device by pa_merge_rows
+    into out (bf16 [batch][Hq][D]) and lse.  Every rank ends with the whole
+    batch's result.  All tensors are CUDA tensors."""
+    import torch
+    import torch.distributed as dist
+
+    from ._binding import merge_rows
+
+    world = dist.get_world_size(group)
+    n = torch.tensor([len(reqs)], device=out_f32.device, dtype=torch.int64)
+    dist.all_reduce(n, op=dist.ReduceOp.MAX, group=group)
+    R = max(1, int(n.item()))
+    Hq, D = out_f32.shape[1], out_f32.shape[2]
+    req = torch.full((R,), -1, dtype=torch.int32, device=out_f32.device)
+    o = torch.zeros((R, Hq, D), dtype=torch.float32, device=out_f32.device)
+    ls = torch.full((R, Hq), float("-inf"), dtype=torch.float32, device=out_f32.device)
+    k = len(reqs)
+    req[:k] = torch.as_tensor(np.asarray(reqs), dtype=torch.int32, device=out_f32.device)
+    o[:k] = out_f32[:k]
+    ls[:k] = lse_f32[:k]
+    all_req = torch.empty((world, R), dtype=torch.int32, device=out_f32.device)
+    all_o = torch.empty((world, R, Hq, D), dtype=torch.float32, device=out_f32.device)
+    all_l = torch.empty((world, R, Hq), dtype=torch.float32, device=out_f32.device)
+    dist.all_gather_into_tensor(all_req, req, group=group)
+    dist.all_gather_into_tensor(all_o, o, group=group)
+    dist.all_gather_into_tensor(all_l, ls, group=group)
+    merge_rows(all_req, all_o, all_l, batch, out, lse)

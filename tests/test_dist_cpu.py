@@ -69,7 +69,7 @@ def _cp_worker(rank, world, port, q):
     import prefix_aware_decode_b200 as pad
     from plan_exec import Image, check_structure, execute
     from prefix_aware_decode_b200 import workload as wl
-    from prefix_aware_decode_b200.shard import context_slices, merge_context_partials
+    from prefix_aware_decode_b200.shard import context_slices
 
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -85,7 +85,14 @@ def _cp_worker(rank, world, port, q):
         dist.all_gather_object(parts, (reqs, o, l))
         if rank == 0:
             import oracle
-            out, lse = merge_context_partials(w.B, parts)
+            # the exchange step's combine, done here with the oracle's merge
+            # (on GPUs: pa_merge_rows after an NCCL all-gather)
+            out = np.zeros((w.B, w.Hq, w.D))
+            lse = np.zeros((w.B, w.Hq))
+            for b in range(w.B):
+                for h in range(w.Hq):
+                    rows = [(o_[list(r_).index(b), h], l_[list(r_).index(b), h]) for r_, o_, l_ in parts if b in r_]
+                    out[b, h], lse[b, h] = oracle.merge(np.stack([x[0] for x in rows]), np.array([x[1] for x in rows]))
             ro, rl = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
             q.put((float(np.abs(out - ro).max()), float(np.abs(lse - rl).max()),
                    [int(p_[2].shape[0]) for p_ in parts], plan.stats()["num_kept_shared"]))

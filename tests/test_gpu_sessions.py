@@ -126,3 +126,47 @@ def test_registered_queries_against_growing_sessions():
         assert_close(compare(out, lse, ref_o, ref_l), f"live sessions step {step}")
     assert plan.stats()["num_kept_shared"] >= 1
     plan.close()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_slices_merged_on_the_device(world):
+    # long sessions (config-5 shaped, 4 sessions x 16 queries): the batch's
+    # pages cut into `world` page-aligned slices (one per rank), each slice
+    # planned and run on its own with an fp32 result (pa_merge_f32), the rows
+    # stacked as an all-gather would deliver them, and merged by pa_merge_rows
+    from prefix_aware_decode_b200.shard import context_slices
+
+    w = wl.make_config(5, scale=0.125)
+    qd, kd, vd = bf16_dev(w.q), bf16_dev(w.k_pool), bf16_dev(w.v_pool)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    parts = context_slices(w.block_table, w.kv_lens, world)
+    R = max(len(reqs) for reqs, _, _ in parts)
+    all_req = torch.full((world, R), -1, dtype=torch.int32, device="cuda")
+    all_o = torch.zeros((world, R, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    all_l = torch.full((world, R, w.Hq), float("-inf"), dtype=torch.float32, device="cuda")
+    for r, (reqs, bt, kl) in enumerate(parts):
+        plan = pad.Plan(kl, bt, w.num_pages, w.Hq, w.Hkv, w.D)
+        assert plan.stats()["num_kept_shared"] >= 1  # each slice of a session is still packed as shared
+        ws = plan.alloc_workspace()
+        qr = qd[torch.as_tensor(reqs, device="cuda")].contiguous()
+        plan.upload(ws)
+        plan.forward(qr, kd, vd, ws)
+        o32 = torch.empty((len(reqs), w.Hq, w.D), dtype=torch.float32, device="cuda")
+        l32 = torch.empty((len(reqs), w.Hq), dtype=torch.float32, device="cuda")
+        plan.merge_f32(ws, o32, l32)
+        # the fp32 result rounds to exactly what the bf16 merge writes
+        o16 = torch.empty((len(reqs), w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        l16 = torch.empty_like(l32)
+        plan.merge(ws, o16, l16)
+        assert plan.device_status(ws) == pad.PA_OK
+        assert torch.equal(o32.to(torch.bfloat16).view(torch.int16), o16.view(torch.int16))
+        assert torch.equal(l32, l16)
+        all_req[r, :len(reqs)] = torch.as_tensor(reqs, dtype=torch.int32, device="cuda")
+        all_o[r, :len(reqs)] = o32
+        all_l[r, :len(reqs)] = l32
+        plan.close()
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    pad.merge_rows(all_req, all_o, all_l, w.B, out, lse)
+    torch.cuda.synchronize()
+    assert_close(compare(out, lse, ref_o, ref_l), f"context parallel, {world} slices")
