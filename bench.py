@@ -324,6 +324,11 @@ class Bench:
             res["multi_layer"] = self.multi_layer(w, q, k0, v0, ws, out, lse, pool_bytes)
         if config == 2 and args.decode_steps > 0 and args.layers > 0:
             res["decode_steps"] = self.decode_steps(w, q, k0, v0, out, lse)
+        if config == 5 and args.session_steps > 0:
+            del pools
+            pools = None
+            torch.cuda.empty_cache()
+            res["sessions"] = self.sessions(w)
         if headline and not args.no_e2e:
             res.update(self.e2e(w, q, k0, v0, out, lse, ws_bytes))
         if headline and self.rank == 0 and not args.no_cpu_baseline:
@@ -339,6 +344,66 @@ class Bench:
         del pools, q, k0, v0, out, lse, ws, stepper
         torch.cuda.empty_cache()
         return res
+
+    def sessions(self, w) -> dict:
+        # registered queries against live sessions (config-5 shape: 32
+        # sessions x 16 queries): each session's context grows by a quarter of
+        # its final length per step through the session page allocator, and
+        # every step's batch of registered queries is planned and run;
+        # reported: forward + merge time against the mean context length
+        torch, args, stream = self.torch, self.args, self.stream
+        import prefix_aware_decode_b200 as pad
+        from prefix_aware_decode_b200.session import SessionPool
+
+        n = args.session_steps
+        final = [int(w.kv_lens[16 * s]) for s in range(w.B // 16)]
+        n_pages = sum((L + 15) // 16 for L in final) + 64
+        pool = SessionPool(n_pages, 16)
+        # pool contents do not change the work: one bf16 N(0,1) fill on the device
+        kp = torch.randn((n_pages, w.Hkv, 16, w.D), device="cuda", dtype=torch.float32).to(torch.bfloat16)
+        vp = torch.randn_like(kp)
+        q = torch.randn((w.B, w.Hq, w.D), device="cuda", dtype=torch.float32).to(torch.bfloat16)
+        for sid in range(len(final)):
+            pool.open(sid)
+            for j in range(16):
+                pool.register(sid, 16 * sid + j)
+        out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        points = []
+        grown = [0] * len(final)
+        for step in range(n):
+            for sid, L in enumerate(final):
+                target = L * (step + 1) // n
+                pool.append(sid, target - grown[sid])
+                grown[sid] = target
+            qids, _, bt, kv = pool.batch()
+            plan = pad.Plan(kv, bt, n_pages, w.Hq, w.Hkv, w.D)
+            st = plan.stats()
+            ws = plan.alloc_workspace()
+            plan.upload(ws, stream)
+            for _ in range(3):
+                plan.attend(q, kp, vp, ws, out, lse, stream)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.steps):
+                plan.attend(q, kp, vp, ws, out, lse, stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            assert plan.device_status(ws, stream) == pad.PA_OK
+            us = a.elapsed_time(b) / args.steps * 1e3
+            points.append({"mean_context_tokens": float(np.mean(kv)), "forward_merge_us": us,
+                           "queries_per_s": len(qids) / (us * 1e-6),
+                           "unique_kv_frac_of_hbm": st["unique_kv_bytes"] / (us * 1e-6) / 1e9 / self.hbm_peak,
+                           "plan_us": st["plan_us"]})
+            plan.close()
+            del ws
+        del kp, vp
+        torch.cuda.empty_cache()
+        return {"steps": points,
+                "note": "32 sessions x 16 registered queries; contexts grow to the workload's lengths in equal "
+                        "steps through session.SessionPool; each step plans the registered queries' batch and "
+                        "times forward + merge on the device (KV resident); time per query grows with the "
+                        "context's bytes, the unique-KV fraction of HBM is the per-step efficiency"}
 
     def amortised(self, w) -> dict:
         # config 1 is a few hundred KB, far below what one launch can stream:
@@ -552,6 +617,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=16,
                     help="config 2: also time this many growing decode steps of --layers layers whose plans "
                          "come from pa_plan_advance (0: skip)")
+    ap.add_argument("--session-steps", type=int, default=4,
+                    help="config 5: growing-session steps of registered queries (0: skip)")
     ap.add_argument("--amortise", type=int, default=1024,
                     help="config-1 problems batched together for the amortised config-1 figure (0: skip)")
     args = ap.parse_args()

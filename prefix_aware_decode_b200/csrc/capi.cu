@@ -111,34 +111,55 @@ void record_profile(const pa_plan& p, int which, cudaStream_t st) {
   if (p.prof[which]) cudaEventRecord(static_cast<cudaEvent_t>(p.prof[which]), st);
 }
 
-// Encoded tensor maps, cached process-wide by (pool pointer, rows, head dim):
-// a pool keeps its map for every plan that reads it.
+// 3-D view of a pool for whole (page, kv head) tiles in one copy: dims (64
+// dims, row, half of D) with strides (D * 2 bytes per row, 128 bytes per half);
+// box 64 x 16 x 2 with 128-byte swizzle lands as two 16-row x 128-byte boxes,
+// the second 2 KB after the first (the layout of two 2-D copies).  Only for
+// D = 128; returns false when the driver refuses the view.
+bool encode_pool_tiles(const pa_plan& p, const void* pool, void* out) {
+  auto fn = encode_fn();
+  if (!fn || p.D != 128) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)p.num_pages_in_pool * p.Hkv * p.P, 2};
+  cuuint64_t strides[2] = {(cuuint64_t)p.D * 2, 128};
+  cuuint32_t box[3] = {64, 16, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(reinterpret_cast<CUtensorMap*>(out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Encoded tensor maps, cached process-wide by (pool pointer, rows, head dim,
+// view): a pool keeps its maps for every plan that reads it.
 struct TmapEntry {
   const void* ptr = nullptr;
   uint64_t rows = 0;
   int D = 0;
+  int view = 0;  // 0: 2-D rows x D; 1: 3-D whole tiles; -1 (in `ok`): refused
+  bool ok = false;
   alignas(64) uint8_t map[128];
 };
 std::mutex g_tmap_mu;
 TmapEntry g_tmap[128];  // enough for both pools of every layer of a large model
 int g_tmap_next = 0;
 
-bool tmap_get(const pa_plan& p, const void* pool, void* out) {
+bool tmap_get(const pa_plan& p, const void* pool, void* out, int view = 0) {
   const uint64_t rows = (uint64_t)p.num_pages_in_pool * p.Hkv * p.P;
   std::lock_guard<std::mutex> lock(g_tmap_mu);
   for (const TmapEntry& e : g_tmap)
-    if (e.ptr == pool && e.rows == rows && e.D == p.D) {
-      std::memcpy(out, e.map, 128);
-      return true;
+    if (e.ptr == pool && e.rows == rows && e.D == p.D && e.view == view) {
+      if (e.ok) std::memcpy(out, e.map, 128);
+      return e.ok;
     }
   TmapEntry& e = g_tmap[g_tmap_next];
-  if (!encode_pool(p, pool, e.map)) return false;
+  e.ok = view == 0 ? encode_pool(p, pool, e.map) : encode_pool_tiles(p, pool, e.map);
   e.ptr = pool;
   e.rows = rows;
   e.D = p.D;
+  e.view = view;
   g_tmap_next = (g_tmap_next + 1) % (int)(sizeof(g_tmap) / sizeof(g_tmap[0]));
-  std::memcpy(out, e.map, 128);
-  return true;
+  if (e.ok) std::memcpy(out, e.map, 128);
+  return e.ok;
 }
 
 }  // namespace
@@ -188,6 +209,8 @@ pa_status launch(const pa_plan* plan, const void* q, const void* k_pool, const v
   d.v_pool = static_cast<const uint16_t*>(v_pool);
   if (plan->tma_k_ptr != k_pool || plan->tma_v_ptr != v_pool) {
     if (!tmap_get(*plan, k_pool, plan->tma_k) || !tmap_get(*plan, v_pool, plan->tma_v)) return PA_ERR_CUDA;
+    // whole-tile maps for the small-row class when the driver takes them
+    plan->tma_tiles = tmap_get(*plan, k_pool, plan->tma_k3, 1) && tmap_get(*plan, v_pool, plan->tma_v3, 1);
     plan->tma_k_ptr = k_pool;
     plan->tma_v_ptr = v_pool;
   }

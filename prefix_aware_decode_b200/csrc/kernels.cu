@@ -66,6 +66,7 @@ struct FwdArgs {
   uint64_t timeout_ns;
   int fault_drop;
   int debug_checks;  // PA_PLAN_DEBUG_CHECKS: page and request ids are range-checked before any load
+  int tile_maps;     // the small-row class got whole-tile (3-D) maps: one copy per K or V tile
   int num_pages, B;
 };
 
@@ -429,10 +430,15 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, const CUtensorMap* t
       const uint32_t st = ring + stage * S::STAGE;
       const uint32_t bar = smem_u32(&bars[stage]);
       mbar_arrive_expect_tx(bar, 2 * S::TILE);
+      if (D == 128 && a.tile_maps) {
+        tma_load_3d(st, tk, 0, tile * 16, 0, bar);
+        tma_load_3d(st + S::TILE, tv, 0, tile * 16, 0, bar);
+      } else {
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        tma_load_2d(st + h * 2048, tk, 64 * h, tile * 16, bar);
-        tma_load_2d(st + S::TILE + h * 2048, tv, 64 * h, tile * 16, bar);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(st + h * 2048, tk, 64 * h, tile * 16, bar);
+          tma_load_2d(st + S::TILE + h * 2048, tv, 64 * h, tile * 16, bar);
+        }
       }
     }
     if (!drop) inflight |= 1u << stage;
@@ -615,19 +621,20 @@ struct MmaShape {
   static constexpr int KSTAGE = HALVES * KBLK;     // K (or V) of one stage
   static constexpr int STAGE = 2 * KSTAGE;         // K and V of one stage
   static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
-  static constexpr int FIXED = HALVES * QBLK + 512 + 1024;  // Q, barriers, alignment slack
+  static constexpr int QBUF = HALVES * QBLK;       // the Q rows of one segment
+  static constexpr int FIXED = 2 * QBUF + 512 + 1024;  // two Q buffers, barriers, alignment slack
   static constexpr int NST_FIT = (kSmemMax - FIXED) / STAGE;
   static constexpr int NST = NST_FIT < 8 ? NST_FIT : 8;  // slots of the K ring and of the V ring
   static constexpr int OFF_K = 0, OFF_V = NST * KSTAGE;
   static constexpr int OFF_Q = NST * STAGE;
-  static constexpr int OFF_BAR = OFF_Q + HALVES * QBLK;
+  static constexpr int OFF_BAR = OFF_Q + 2 * QBUF;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;
   // barriers: K full / empty and V full / empty per ring slot; S full, P full,
-  // p.V done per buffer; Q loaded; O read out; all MMAs retired; the two halves
-  // of each lane quarter have exchanged (m, l)
+  // p.V done per buffer; Q loaded per Q buffer; O read out; all MMAs retired;
+  // the two halves of each lane quarter have exchanged (m, l)
   static constexpr int B_FULL = 0, B_EMPTY = NST, B_VFULL = 2 * NST, B_VEMPTY = 3 * NST,
                        B_SFULL = 4 * NST, B_PFULL = B_SFULL + kSBufs,
-                       B_PV = B_PFULL + kSBufs, B_QFULL = B_PV + kSBufs, B_OFREE = B_QFULL + 1, B_DONE = B_OFREE + 1,
+                       B_PV = B_PFULL + kSBufs, B_QFULL = B_PV + kSBufs, B_OFREE = B_QFULL + 2, B_DONE = B_OFREE + 1,
                        B_XCH = B_DONE + 1, NBARS = B_XCH + 4;
   // tensor memory columns: S/P buffers, the two half accumulators, (m, l) exchange
   static constexpr uint32_t T_S = 0, T_O = kSBufs * kMmaKT, T_X = T_O + 2 * D;
@@ -669,6 +676,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       mbar_init(bar(S::B_PV + b), 1);
     }
     mbar_init(bar(S::B_QFULL), kSmaxThreads);
+    mbar_init(bar(S::B_QFULL + 1), kSmaxThreads);
     mbar_init(bar(S::B_OFREE), kSmaxThreads);
     mbar_init(bar(S::B_DONE), 2);
     for (int q = 0; q < 4; ++q) mbar_init(bar(S::B_XCH + q), 64);
@@ -765,17 +773,18 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           if (is_s) {
             // K landed; Q of the segment loaded; the buffer's last p.V (stage i - 3) done
             if (!mbar_wait_bounded(bar(S::B_FULL + s), (i / NST) & 1, a.timeout_ns) ||
-                (first && !mbar_wait_bounded(bar(S::B_QFULL), segord & 1, a.timeout_ns)) ||
+                (first && !mbar_wait_bounded(bar(S::B_QFULL + (segord & 1)), (segord >> 1) & 1, a.timeout_ns)) ||
                 (i >= kSBufs && !mbar_wait_bounded(bar(S::B_PV + b), ((i / kSBufs) - 1) & 1, a.timeout_ns))) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t k_base = smem_u32(smem + S::OFF_K + s * S::KSTAGE);
+            const uint32_t qb = q_base + (segord & 1) * S::QBUF;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               // Q and K: K-major 128-byte swizzle, 64-dim blocks, 8-row groups at +1 KB
-              const uint64_t ad = umma_sdesc_sw128(q_base + (kk >> 2) * S::QBLK + (kk & 3) * 32, 1, 64);
+              const uint64_t ad = umma_sdesc_sw128(qb + (kk >> 2) * S::QBLK + (kk & 3) * 32, 1, 64);
               const uint64_t bd = umma_sdesc_sw128(k_base + (kk >> 2) * S::KBLK + (kk & 3) * 32, 1, 64);
               umma_bf16(tmem + S::T_S + b * kMmaKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
             }
@@ -824,28 +833,47 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     constexpr int QCH = D / 16;  // 16-byte q chunks per row loaded by each half
     bool ok = true;
     int i = 0, segord = 0;
-    auto load_q = [&](int si) {
+    // The q row this thread copies for segment si (nullptr: a row past the tile's)
+    auto q_src = [&](int si) -> const uint16_t* {
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
-      const int R = item.n_queries * G;
-      const uint16_t* src = nullptr;
-      if (r < R) {
-        int b = a.queries[item.query_off + r / G];
-        if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
-          record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
-          b = 0;
-        }
-        src = a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
+      if (r >= item.n_queries * G) return nullptr;
+      int b = a.queries[item.query_off + r / G];
+      if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
+        record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
+        b = 0;
       }
+      return a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
+    };
+    // This thread's half of row r into Q buffer qbuf (K-major, 128-byte swizzle).
+    auto q_dst = [&](int qbuf, int c) -> uint8_t* {
+      return smem + S::OFF_Q + qbuf * S::QBUF + (c >> 3) * S::QBLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+    };
+    // the first segment: plain loads
+    auto load_q = [&](int si) {
+      const uint16_t* src = q_src(si);
 #pragma unroll
       for (int cc = 0; cc < QCH; ++cc) {
         const int c = h * QCH + cc;
         const uint4 v = src ? *reinterpret_cast<const uint4*>(src + 8 * c) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(smem + S::OFF_Q + (c >> 3) * S::QBLK + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(q_dst(0, c)) = v;
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(S::B_QFULL));
     };
+    // later segments: copied asynchronously while the previous segment runs
+    // (16-byte cp.async, zero-filled past the tile's rows), published on the
+    // buffer's barrier a stage later
+    auto prefetch_q = [&](int si, int qbuf) {
+      const uint16_t* src = q_src(si);
+#pragma unroll
+      for (int cc = 0; cc < QCH; ++cc) {
+        const int c = h * QCH + cc;
+        cp_async16(smem_u32(q_dst(qbuf, c)), src ? src + 8 * c : a.q, src ? 16u : 0u);
+      }
+      cp_async_commit();
+    };
+    bool q_pending = false;
     // S(i) is read from tensor memory into sv; inside a segment the load of
     // S(i + 1) is issued while P(i) is being stored, when S(i + 1) is already
     // there (else at the top of the next stage)
@@ -860,6 +888,10 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
       const int R = item.n_queries * G;
+      // a warp whose lane quarter lies past the tile's rows keeps every
+      // barrier of the protocol but skips the arithmetic (its P and O rows are
+      // never read out)
+      const bool act = quad * 32 < R;
       const int npages = (seg.n_tokens + 15) >> 4;
       float m_used = -INFINITY, l = 0.f;
       for (int st = 0; st < npages; st += 4, ++i) {
@@ -870,13 +902,25 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         const bool last = st + 4 >= npages;
         if (!have_s) {
           if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
-          load_s(i);
+          if (act) load_s(i);
         }
         have_s = false;
-        tmem_wait_ld_into(sv);
+        if (act) tmem_wait_ld_into(sv);
         const uint32_t t_s = tmem + S::T_S + b * kMmaKT + 32 * h + lane_off;
-        // all S products of this segment are done: Q may be replaced by the next segment's
-        if (last && si + 1 < s_end) load_q(si + 1);
+        // the Q buffer of the previous segment is free (all its S products have
+        // been read): the next segment's rows are copied into it, and published
+        // a stage later (or at this segment's last stage)
+        if (st == 0 && si + 1 < s_end) {
+          prefetch_q(si + 1, (segord + 1) & 1);
+          q_pending = true;
+        }
+        if (q_pending && (st > 0 || last)) {
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(bar(S::B_QFULL + ((segord + 1) & 1)));
+          q_pending = false;
+        }
+        if (act) {
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (kv_h == 32) {
 #pragma unroll
@@ -957,6 +1001,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           load_s(i + 1);
           have_s = true;
         }
+        }  // act
         if (kvalid < np * 16) {
           // V rows past the last valid key may hold NaN; p = 0 there but 0 * NaN
           // would still poison the product, so those rows are zeroed (once the
@@ -983,7 +1028,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
       }
       tc_fence_after();
-      {
+      if (act) {
         const uint32_t mine[2] = {__float_as_uint(m_used), __float_as_uint(l)};
         tmem_st2(tmem + S::T_X + 2 * h + lane_off, mine);
         tmem_wait_st();
@@ -992,6 +1037,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       mbar_arrive(bar(S::B_XCH + quad));
       if (!warp_wait(bar(S::B_XCH + quad), segord & 1, a.timeout_ns)) { ok = false; break; }
       tc_fence_after();
+      if (act) {
       uint32_t other[2];
       tmem_ld2(tmem + S::T_X + 2 * (1 - h) + lane_off, other);
       tmem_wait_ld();
@@ -1026,12 +1072,14 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           }
         }
       }
+      }  // act
       tc_fence_before();
       mbar_arrive(bar(S::B_OFREE));
       // these rows' pairs are merged by their last SIMT writer or the tail merge launch
       ++segord;
     }
     tmem_wait_ld();  // a load of S issued ahead before a failed wait
+    cp_async_wait_all();  // a Q prefetch still in flight after a failed wait
     if (!ok && lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, warp);
   }
   tc_fence_before();
@@ -1171,6 +1219,7 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.timeout_ns = (uint64_t)p.wait_timeout_us * 1000ull;
   a.fault_drop = (p.flags & PA_PLAN_FAULT_DROP_LOAD) ? 1 : 0;
   a.debug_checks = (p.flags & PA_PLAN_DEBUG_CHECKS) ? 1 : 0;
+  a.tile_maps = p.tma_tiles ? 1 : 0;
   a.num_pages = p.num_pages_in_pool;
   a.B = p.B;
   return a;
@@ -1205,6 +1254,8 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
     if (cudaError_t e = cudaGetLastError()) return (int)e;
   }
   if (n_simt_ctas > 0) {
+    const CUtensorMap* sk = p.tma_tiles ? reinterpret_cast<const CUtensorMap*>(p.tma_k3) : tk;
+    const CUtensorMap* sv = p.tma_tiles ? reinterpret_cast<const CUtensorMap*>(p.tma_v3) : tv;
     auto k = simt_fwd_kernel<D, G>;
     if (int e = set_smem_attr(k, attr_simt)) return e;
     cudaLaunchConfig_t cfg = {};
@@ -1217,7 +1268,7 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.n_mma_ctas > 0 ? 1 : 0;
-    if (cudaError_t e = cudaLaunchKernelEx(&cfg, k, a, *tk, *tv)) return (int)e;
+    if (cudaError_t e = cudaLaunchKernelEx(&cfg, k, a, *sk, *sv)) return (int)e;
   }
   return 0;
 }

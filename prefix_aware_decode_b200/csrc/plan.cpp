@@ -289,11 +289,11 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   // concatenated and cut into equal spans, one span per SIMT warp or per MMA
   // CTA; a span may end inside an item, so partial rows appear only at span
   // boundaries (long-KV splitting without a fixed chunk size).
-  const double kSimtBytesPerSmUs = 36.0e3;   // bytes per us per SM, CUDA-core class
+  const double kSimtBytesPerSmUs = 56.0e3;   // bytes per us per SM, small-row class
   const int kSimtSegPages = 2;               // fixed cost of a SIMT work unit, in pages
   const double kMmaBytesPerSmUs = 40.0e3;    // bytes per us per SM, tensor-core class
   const double kMmaFlopsPerSmUs = 5.0e6;     // flop per us per SM, tcgen05 class, running beside the SIMT class
-  const int kMmaSegPages = 38;               // fixed cost of a 128-row tensor-core segment (q load, epilogue), in pages
+  const int kMmaSegPages = 24;               // fixed cost of a 128-row tensor-core segment (epilogue), in pages
   // the epilogue's stores scale with the tile's rows: a tile of r rows pays
   // kMmaSegPages * max(32, r) / 128
   auto mma_seg_pages = [&](const ItemRec& it) -> int64_t {

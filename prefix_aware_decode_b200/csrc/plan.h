@@ -54,6 +54,11 @@ struct pa_plan {
   mutable const void* tma_v_ptr = nullptr;
   alignas(64) mutable uint8_t tma_k[128] = {};
   alignas(64) mutable uint8_t tma_v[128] = {};
+  // whole-tile (3-D) maps of the same pools, used by the small-row class when
+  // tma_tiles is set (else it copies each tile as D/64 boxes of the 2-D maps)
+  mutable bool tma_tiles = false;
+  alignas(64) mutable uint8_t tma_k3[128] = {};
+  alignas(64) mutable uint8_t tma_v3[128] = {};
   // optional cudaEvent_t handles recorded around the launches (profiling):
   // [0,1] forward launch (pa_forward / pa_attend), [2,3] merge launch
   void* prof[4] = {};
