@@ -12,7 +12,7 @@
  *   "Q is a single token in decode") and the short-term-memory page (技术原理:
  *   K_t, V_t are appended to the cache, then the token attends over K_1..K_t).
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings where the pages are silent (the plainest reading in each case):
  *   - GQA: query head h reads kv head h / G with G = Hq / Hkv (contiguous groups).
  *   - The 1/sqrt(d) scale multiplies the fp64 dot products (d = head_dim).
  *   - lse is the natural log of the sum of exp(scaled logits).

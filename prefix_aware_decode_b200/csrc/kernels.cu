@@ -237,14 +237,23 @@ __device__ __forceinline__ void tile_step(uint32_t kt, uint32_t vt, int nvalid, 
                                           float (&l)[2]) {
   constexpr int KT = D / 16;
   const int g = lane >> 2, t = lane & 3;
-  // S^T = K . Q^T, two accumulation chains
+  // S^T = K . Q^T, two accumulation chains; every K fragment is loaded before
+  // the first product, and every V fragment (matrices (keys 0-7 | 8-15) x
+  // (dims 16i..16i+7 | 16i+8..16i+15)) right after the last one, so the V loads
+  // overlap the softmax
+  uint32_t kf[KT][4], vf[KT][4];
+#pragma unroll
+  for (int kk = 0; kk < KT; ++kk) ldsm_x4(swz(kt, lane & 15, 2 * kk + (lane >> 4)), kf[kk]);
   float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int kk = 0; kk < KT; ++kk) {
-    uint32_t af[4];
-    ldsm_x4(swz(kt, lane & 15, 2 * kk + (lane >> 4)), af);
-    if (kk & 1) mma_bf16_16816(sb, af, qb[kk][0], qb[kk][1]);
-    else mma_bf16_16816(sa, af, qb[kk][0], qb[kk][1]);
+    if (kk & 1) mma_bf16_16816(sb, kf[kk], qb[kk][0], qb[kk][1]);
+    else mma_bf16_16816(sa, kf[kk], qb[kk][0], qb[kk][1]);
+  }
+  {
+    const int vrow = (lane & 7) + ((lane >> 4) << 3), vch = (lane >> 3) & 1;
+#pragma unroll
+    for (int i = 0; i < KT; ++i) ldsm_x4_trans(swz(vt, vrow, 2 * i + vch), vf[i]);
   }
   float s[4];
 #pragma unroll
@@ -302,12 +311,10 @@ __device__ __forceinline__ void tile_step(uint32_t kt, uint32_t vt, int nvalid, 
     mlo = (2 * t < nvalid ? 0x0000ffffu : 0u) | (2 * t + 1 < nvalid ? 0xffff0000u : 0u);
     mhi = (2 * t + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t + 9 < nvalid ? 0xffff0000u : 0u);
   }
-  // O^T += V^T . P^T: matrices (keys 0-7 | 8-15) x (dims 16i..16i+7 | 16i+8..16i+15)
-  const int vrow = (lane & 7) + ((lane >> 4) << 3), vch = (lane >> 3) & 1;
+  // O^T += V^T . P^T
 #pragma unroll
   for (int i = 0; i < KT; ++i) {
-    uint32_t af[4];
-    ldsm_x4_trans(swz(vt, vrow, 2 * i + vch), af);
+    uint32_t (&af)[4] = vf[i];
     if (PARTIAL) {
       af[0] &= mlo;
       af[1] &= mlo;

@@ -350,3 +350,44 @@ def test_debug_checks_catch_a_corrupted_page_id(flags):
     ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
     assert_close(compare(out, lse, ref_o, ref_l), "debug checks, clean run")
     plan.close()
+
+
+@pytest.mark.parametrize("config,scale", [(2, 0.25), (5, 0.125)])
+def test_canaries_around_outputs_and_workspace_survive(config, scale):
+    # every device buffer the library writes (workspace, out, lse) sits inside
+    # a larger allocation with a canary pattern of 4 KiB on both sides; the
+    # two-launch path, the fused path and the fp32 merge leave the canaries as
+    # they were
+    w = wl.make_config(config, scale=scale)
+    dw = DevWorkload(w)
+    pad_b = 4096
+    canary = 0x5A
+
+    def guarded(nbytes):
+        buf = torch.full((nbytes + 2 * pad_b,), canary, dtype=torch.uint8, device="cuda")
+        return buf, buf[pad_b:pad_b + nbytes]
+
+    def intact(buf, nbytes):
+        return bool((buf[:pad_b] == canary).all() and (buf[pad_b + nbytes:] == canary).all())
+
+    plan = pad.Plan(w.kv_lens, w.block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+    nws = (plan.workspace_bytes + 255) // 256 * 256
+    wsb, ws = guarded(nws)
+    nout, nlse, nf32 = w.B * w.Hq * w.D * 2, w.B * w.Hq * 4, w.B * w.Hq * w.D * 4
+    outb, out_raw = guarded(nout)
+    lseb, lse_raw = guarded(nlse)
+    f32b, f32_raw = guarded(nf32)
+    out = out_raw.view(torch.bfloat16).view(w.B, w.Hq, w.D)
+    lse = lse_raw.view(torch.float32).view(w.B, w.Hq)
+    o32 = f32_raw.view(torch.float32).view(w.B, w.Hq, w.D)
+    plan.upload(ws)
+    plan.forward(dw.q, dw.k, dw.v, ws)
+    plan.merge(ws, out, lse)
+    plan.merge_f32(ws, o32, lse)
+    plan.attend(dw.q, dw.k, dw.v, ws, out, lse)
+    assert plan.device_status(ws) == pad.PA_OK
+    torch.cuda.synchronize()
+    assert intact(wsb, nws) and intact(outb, nout) and intact(lseb, nlse) and intact(f32b, nf32)
+    ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    assert_close(compare(out, lse, ref_o, ref_l), f"canaries config {config}")
+    plan.close()
