@@ -660,7 +660,7 @@ def main():
         "plan": head["plan"], "roofline": head["roofline"], "gpu_launches": head["gpu_launches"],
         "clocks": head["clocks"],
     }
-    for k in ("e2e", "e2e_kv_resident", "cpu_baseline"):
+    for k in ("e2e", "e2e_kv_resident", "cpu_baseline", "sessions"):
         if k in head:
             line[k] = head[k]
     line["per_config"] = per
