@@ -228,7 +228,7 @@ class Bench:
         import prefix_aware_decode_b200 as pad
         from prefix_aware_decode_b200 import workload as wl
 
-        w = wl.make_config(config, seed=1000 + config + 7919 * self.rank)
+        w = wl.make_config(config, seed=1000 + config + 7919 * self.rank, scale=args.scale)
         pool_bytes = w.k_pool.nbytes + w.v_pool.nbytes
         copies = args.copies or (1 if pool_bytes > 3 * L2_BYTES else int(np.ceil(3 * L2_BYTES / pool_bytes)) + 1)
         q = self.dev(w.q)
@@ -617,6 +617,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=16,
                     help="config 2: also time this many growing decode steps of --layers layers whose plans "
                          "come from pa_plan_advance (0: skip)")
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="shrink the workloads (batch and lengths) for small profiler captures; 1 = the named sizes")
     ap.add_argument("--session-steps", type=int, default=4,
                     help="config 5: growing-session steps of registered queries (0: skip)")
     ap.add_argument("--amortise", type=int, default=1024,
