@@ -368,8 +368,9 @@ const char *pa_status_string(pa_status s);
  *   pages       int32[num_page_entries]       page ids, per item
  *   queries     int32[num_query_entries]      request ids, per item
  *   seg_prows   int32[num_query_entries_mma]  partial row of each (MMA seg, query)
- *   mma_segs    int32[mma_ctas + 1]           MMA CTA c runs MMA segs [mma_segs[c], mma_segs[c+1])
- *                                             (indices counted from the first MMA seg)
+ *   mma_segs    int32[2]                      {0, num_segments_mma}: the tensor-core work units,
+ *                                             longest first; the tensor-core CTAs take them one
+ *                                             at a time from the counter mma_next of the header
  *   counters    int32[B * Hkv]                arrival counters of the fused merge (zero)
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
  *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
@@ -414,7 +415,9 @@ typedef struct {
   int32_t num_items, num_segments, num_segments_simt, num_segments_mma, simt_warps;
   int32_t num_partial_rows, mma_ctas;
   int32_t num_tail_pairs; /* pairs merged by the tail launch of pa_attend / pa_decode_step */
-  int32_t reserved;
+  int32_t mma_next;       /* tensor-core work units taken so far in the running launch: 0 after
+                             upload, and back at 0 after every launch that completes (after a
+                             device-side error, upload the plan again) */
   uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_mma_segs, off_counters, off_warp_segs,
       off_prow_off, off_tail_pairs;
   uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;

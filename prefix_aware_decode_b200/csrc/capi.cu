@@ -32,6 +32,7 @@ PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   d.partial_lse = reinterpret_cast<float*>(w + h.off_partial_lse);
   d.partial_o = reinterpret_cast<float*>(w + h.off_partial_o);
   d.status = reinterpret_cast<int32_t*>(b + offsetof(pa_image_header, status));
+  d.mma_next = reinterpret_cast<int32_t*>(b + offsetof(pa_image_header, mma_next));
   return d;
 }
 

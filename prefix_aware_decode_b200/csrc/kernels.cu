@@ -53,7 +53,6 @@ struct FwdArgs {
   const int32_t* queries;
   const int32_t* seg_prows;
   const int32_t* warp_segs;
-  const int32_t* mma_cta_segs;
   const int32_t* prow_off;
   int32_t* counters;
   float* partial_lse;
@@ -68,6 +67,8 @@ struct FwdArgs {
   int debug_checks;  // PA_PLAN_DEBUG_CHECKS: page and request ids are range-checked before any load
   int tile_maps;     // the small-row class got whole-tile (3-D) maps: one copy per K or V tile
   int num_pages, B;
+  int n_segs_mma;
+  int32_t* mma_next;  // the counter of tensor-core work units taken (image header)
 };
 
 // ---------------------------------------------------------------- merge of one (request, kv head)
@@ -618,6 +619,8 @@ constexpr int kMmaWarps = 12;        // K producer, S issuer, 8 softmax warps, p
 constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kSmaxThreads = 256;    // softmax threads (two per tile row)
 constexpr int kSBufs = 3;            // S/P buffers in TMEM
+constexpr int kSegQ = 8;             // entries of a CTA's queue of work units taken from the shared counter
+constexpr int kSegQConsumers = 11;   // V producer, S issuer, p.V issuer, 8 softmax warps
 constexpr uint32_t kTmemCols = 512;  // the whole tensor memory of the SM (one CTA per SM)
 constexpr float kRescaleThreshold = kRescaleLog2;
 
@@ -629,24 +632,24 @@ struct MmaShape {
   static constexpr int STAGE = 2 * KSTAGE;         // K and V of one stage
   static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
   static constexpr int QBUF = HALVES * QBLK;       // the Q rows of one segment
-  static constexpr int FIXED = 2 * QBUF + 512 + 1024;  // two Q buffers, barriers, alignment slack
+  static constexpr int FIXED = 2 * QBUF + 1024 + 1024;  // two Q buffers, barriers and queue, alignment slack
   static constexpr int NST_FIT = (kSmemMax - FIXED) / STAGE;
   static constexpr int NST = NST_FIT < 8 ? NST_FIT : 8;  // slots of the K ring and of the V ring
   static constexpr int OFF_K = 0, OFF_V = NST * KSTAGE;
   static constexpr int OFF_Q = NST * STAGE;
   static constexpr int OFF_BAR = OFF_Q + 2 * QBUF;
-  static constexpr int SMEM = OFF_BAR + 512 + 1024;
+  static constexpr int SMEM = OFF_BAR + 1024 + 1024;
   // barriers: K full / empty and V full / empty per ring slot; S full, P full,
   // p.V done per buffer; Q loaded per Q buffer; O read out; all MMAs retired;
   // the two halves of each lane quarter have exchanged (m, l)
   static constexpr int B_FULL = 0, B_EMPTY = NST, B_VFULL = 2 * NST, B_VEMPTY = 3 * NST,
                        B_SFULL = 4 * NST, B_PFULL = B_SFULL + kSBufs,
                        B_PV = B_PFULL + kSBufs, B_QFULL = B_PV + kSBufs, B_OFREE = B_QFULL + 2, B_DONE = B_OFREE + 1,
-                       B_XCH = B_DONE + 1, NBARS = B_XCH + 4;
+                       B_XCH = B_DONE + 1, B_QF = B_XCH + 4, B_QE = B_QF + kSegQ, NBARS = B_QE + kSegQ;
   // tensor memory columns: S/P buffers, the two half accumulators, (m, l) exchange
   static constexpr uint32_t T_S = 0, T_O = kSBufs * kMmaKT, T_X = T_O + 2 * D;
   static_assert(NST >= 3 && SMEM <= kSmemMax, "MMA ring does not fit");
-  static_assert(NBARS * 8 + 8 <= 512, "barrier area");
+  static_assert(NBARS * 8 + 8 + kSegQ * 4 <= 1024, "barrier area");
   static_assert(T_X + 4 <= kTmemCols, "tensor memory plan does not fit");
 };
 
@@ -664,11 +667,32 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::NBARS);
+  volatile int32_t* segq = reinterpret_cast<int32_t*>(bars + S::NBARS + 1);  // work units taken, in order
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s_begin = a.n_segs_simt + a.mma_cta_segs[blockIdx.x];
-  const int s_end = a.n_segs_simt + a.mma_cta_segs[blockIdx.x + 1];
   const uint32_t q_base = smem_u32(smem + S::OFF_Q);
+  // The work units (segments) are taken one at a time from the counter in the
+  // image: the K producer takes the next one as soon as it has issued the
+  // loads of the current one and puts it into this CTA's queue (kSegQ
+  // entries, full / empty barriers); the other roles read the queue in order.
+  // -1 ends the CTA's work.  Queue entry n is slot n % kSegQ, phase n / kSegQ.
+  // Returns the global segment index, -1 at the end, -2 if a wait gave up.
+  auto seg_take = [&](int& n, bool arrive) -> int {
+    const int j = n % kSegQ;
+    if (!mbar_wait_bounded(bar(S::B_QF + j), (n / kSegQ) & 1, a.timeout_ns)) return -2;
+    const int v = segq[j];
+    if (arrive) mbar_arrive(bar(S::B_QE + j));
+    ++n;
+    return v < 0 ? -1 : a.n_segs_simt + v;
+  };
+  // The entry after n, if the K producer has already put it there (no wait).
+  auto seg_peek = [&](int n, int& si) -> bool {
+    const int j = n % kSegQ;
+    if (!mbar_test_wait(bar(S::B_QF + j), (n / kSegQ) & 1)) return false;
+    const int v = segq[j];
+    si = v < 0 ? -1 : a.n_segs_simt + v;
+    return true;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -687,6 +711,10 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     mbar_init(bar(S::B_OFREE), kSmaxThreads);
     mbar_init(bar(S::B_DONE), 2);
     for (int q = 0; q < 4; ++q) mbar_init(bar(S::B_XCH + q), 64);
+    for (int q = 0; q < kSegQ; ++q) {
+      mbar_init(bar(S::B_QF + q), 1);
+      mbar_init(bar(S::B_QE + q), kSegQConsumers);
+    }
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -708,9 +736,43 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     uint8_t* ring = smem + (is_v ? S::OFF_V : S::OFF_K);
     if (lane == 0) prefetch_tmap(tm);
     uint32_t lastpar = 0, any = 0;
-    int i = 0;
+    int i = 0, qn = 0;
     bool ok = true;
-    for (int si = s_begin; si < s_end && ok; ++si) {
+    for (;;) {
+      int si;
+      if (!is_v) {
+        // take the next work unit from the shared counter and queue it
+        const int j = qn % kSegQ;
+        if (qn >= kSegQ && !warp_wait(bar(S::B_QE + j), ((qn / kSegQ) - 1) & 1, a.timeout_ns)) {
+          if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -6);
+          ok = false;
+          break;
+        }
+        int v = -1;
+        if (lane == 0) {
+          const int idx = atomicAdd(a.mma_next, 1);
+          if (idx < a.n_segs_mma) v = idx;
+          else if (idx == a.n_segs_mma + (int)gridDim.x - 1) *a.mma_next = 0;  // the launch's last take
+          segq[j] = v;
+          mbar_arrive(bar(S::B_QF + j));
+        }
+        v = __shfl_sync(0xffffffffu, v, 0);
+        ++qn;
+        if (v < 0) break;
+        si = a.n_segs_simt + v;
+      } else {
+        int v = 0;
+        if (lane == 0) v = seg_take(qn, true);
+        v = __shfl_sync(0xffffffffu, v, 0);
+        if (lane != 0) ++qn;
+        if (v == -2) {
+          if (lane == 0) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, -7);
+          ok = false;
+          break;
+        }
+        if (v < 0) break;
+        si = v;
+      }
       const pa_seg seg = a.segs[si];
       const int32_t* pg = a.pages + a.items[seg.item].page_off + seg.page_begin;
       const int npages = (seg.n_tokens + 15) >> 4;
@@ -757,6 +819,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         lastpar = (lastpar & ~(1u << s)) | ((uint32_t)((i / NST) & 1) << s);
         any |= 1u << s;
       }
+      if (!ok) break;
     }
     if (lane == 0)
       for (int s = 0; s < NST; ++s)
@@ -771,8 +834,11 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, kMmaKT, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, false, true);
       bool ok = true;
-      int i = 0, segord = 0;
-      for (int si = s_begin; si < s_end && ok; ++si) {
+      int i = 0, segord = 0, qn = 0;
+      for (;;) {
+        const int si = seg_take(qn, true);
+        if (si == -2) ok = false;
+        if (si < 0) break;
         const int npages = (a.segs[si].n_tokens + 15) >> 4;
         for (int st = 0; st < npages; st += 4, ++i) {
           const int s = i % NST, b = i % kSBufs;
@@ -823,6 +889,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             umma_commit(bar(S::B_VEMPTY + s));
           }
         }
+        if (!ok) break;
         ++segord;
       }
       if (!ok) record_status(a.status, PA_ERR_TIMEOUT, blockIdx.x, is_s ? -3 : -5);
@@ -890,8 +957,21 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       tmem_ld32(tmem + S::T_S + (i_ % kSBufs) * kMmaKT + 32 * h + lane_off, sv);
     };
     bool have_s = false;
-    if (s_begin < s_end) load_q(s_begin);
-    for (int si = s_begin; si < s_end && ok; ++si) {
+    int qn = 0;
+    // the next queue entry, by the whole warp (lane 0 frees the entry)
+    auto take = [&]() -> int {
+      const int j = qn % kSegQ;
+      const bool got = warp_wait(bar(S::B_QF + j), (qn / kSegQ) & 1, a.timeout_ns);
+      const int v = segq[j];
+      __syncwarp();
+      if (lane == 0 && got) mbar_arrive(bar(S::B_QE + j));
+      ++qn;
+      return !got ? -2 : v < 0 ? -1 : a.n_segs_simt + v;
+    };
+    int si = take();
+    if (si == -2) ok = false;
+    if (si >= 0) load_q(si);
+    while (si >= 0 && ok) {
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
       const int R = item.n_queries * G;
@@ -901,6 +981,8 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const bool act = quad * 32 < R;
       const int npages = (seg.n_tokens + 15) >> 4;
       float m_used = -INFINITY, l = 0.f;
+      bool q_known = false;  // the next work unit has been seen in the queue
+      int q_at = 0;          // the stage at which its Q rows were requested
       for (int st = 0; st < npages; st += 4, ++i) {
         const int s = i % NST, b = i % kSBufs;
         const int np = min(4, npages - st);
@@ -915,13 +997,28 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         if (act) tmem_wait_ld_into(sv);
         const uint32_t t_s = tmem + S::T_S + b * kMmaKT + 32 * h + lane_off;
         // the Q buffer of the previous segment is free (all its S products have
-        // been read): the next segment's rows are copied into it, and published
-        // a stage later (or at this segment's last stage)
-        if (st == 0 && si + 1 < s_end) {
-          prefetch_q(si + 1, (segord + 1) & 1);
-          q_pending = true;
+        // been read): the next work unit's rows are copied into it as soon as
+        // the unit is in the queue, and published a stage later (or at this
+        // segment's last stage).  At the last stage the wait for the queue entry
+        // is a real one: the K producer has issued this segment's loads by then
+        // and takes the next unit at once.
+        if (!q_known) {
+          int nsi = -1;
+          bool seen = seg_peek(qn, nsi);
+          if (!seen && last) {
+            if (!mbar_wait_bounded(bar(S::B_QF + qn % kSegQ), (qn / kSegQ) & 1, a.timeout_ns)) { ok = false; break; }
+            seen = seg_peek(qn, nsi);
+          }
+          if (seen) {
+            q_known = true;
+            q_at = st;
+            if (nsi >= 0) {
+              prefetch_q(nsi, (segord + 1) & 1);
+              q_pending = true;
+            }
+          }
         }
-        if (q_pending && (st > 0 || last)) {
+        if (q_pending && (st > q_at || last)) {
           cp_async_wait_all();
           fence_proxy_async_smem();
           mbar_arrive(bar(S::B_QFULL + ((segord + 1) & 1)));
@@ -1084,6 +1181,8 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       mbar_arrive(bar(S::B_OFREE));
       // these rows' pairs are merged by their last SIMT writer or the tail merge launch
       ++segord;
+      si = take();
+      if (si == -2) ok = false;
     }
     tmem_wait_ld();  // a load of S issued ahead before a failed wait
     cp_async_wait_all();  // a Q prefetch still in flight after a failed wait
@@ -1208,7 +1307,6 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.queries = d.queries;
   a.seg_prows = d.seg_prows;
   a.warp_segs = d.warp_segs;
-  a.mma_cta_segs = d.mma_cta_segs;
   a.prow_off = d.prow_off;
   a.counters = d.counters;
   a.partial_lse = d.partial_lse;
@@ -1227,6 +1325,8 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.fault_drop = (p.flags & PA_PLAN_FAULT_DROP_LOAD) ? 1 : 0;
   a.debug_checks = (p.flags & PA_PLAN_DEBUG_CHECKS) ? 1 : 0;
   a.tile_maps = p.tma_tiles ? 1 : 0;
+  a.n_segs_mma = p.hdr.num_segments_mma;
+  a.mma_next = d.mma_next;
   a.num_pages = p.num_pages_in_pool;
   a.B = p.B;
   return a;

@@ -302,7 +302,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   };
   const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
   const double tile_bytes = 2.0 * 16 * D * 2;
-  int64_t simt_pages = 0, mma_pages = 0, mma_runs = 0, mma_seg_total = 0;
+  int64_t simt_pages = 0, mma_pages = 0, mma_seg_total = 0;
   double mma_cost = 0;  // SM-us
   for (const auto& it : items) {
     const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
@@ -312,7 +312,6 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
       simt_pages += np + kSimtSegPages * Hkv;
     } else {
       mma_pages += np;
-      mma_runs += Hkv;
       mma_seg_total += mma_seg_pages(it) * Hkv;
       // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
       const double rows = kMmaRowsPerCta;
@@ -400,42 +399,35 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     warp_segs.resize(n_warp);
   }
   if (mma_pages > 0) {
-    // each (item, kv head) run is a segment, and so is each cut at a CTA boundary
-    int64_t span = ceil_div(mma_pages + mma_seg_total + mma_seg_total / std::max<int64_t>(1, mma_runs) * n_mma, n_mma);
-    if (span < 16) span = 16;
-    if (max_chunk_pages) span = std::min(span, max_chunk_pages);
-    int64_t used = 0;
+    // Tensor-core work units: every (item, kv head) run cut into equal chunks
+    // of at most `chunk` pages, about kMmaChunksPerCta per CTA.  The CTAs take
+    // the chunks one after another from a counter in the image (the K producer
+    // of each CTA fetches the next one), longest first, so an SM that runs
+    // faster takes more of them: the same stage of the same work was measured
+    // to take from 1.3k to 2.4k cycles on different SMs of one launch.
+    const int kMmaChunksPerCta = 2;
+    int64_t chunk = ceil_div(mma_pages + mma_seg_total, (int64_t)n_mma * kMmaChunksPerCta);
+    if (chunk < 16) chunk = 16;
+    if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
     for (size_t i = 0; i < items.size(); ++i) {
       const ItemRec& it = items[i];
       if (it.simt) continue;
       const int npages = (int)ceil_div(it.n_tokens, P);
+      const int n = (int)ceil_div(npages, chunk);
       for (int g = 0; g < Hkv; ++g) {
         int pb = 0;
-        while (pb < npages) {
-          // never more than n_mma CTAs: the last one takes whatever is left
-          const int64_t seg_cost = mma_seg_pages(it);
-          bool last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
-          if (!last_cta && used > 0 && span - used - seg_cost < 4) {
-            // no room for a stage after the segment's fixed cost: next CTA
-            mma_cta_segs.push_back((int32_t)mma_segs.size());
-            used = 0;
-            last_cta = (int64_t)mma_cta_segs.size() >= n_mma;
-          }
-          used += seg_cost;  // the segment's fixed cost
-          const int take = last_cta ? npages - pb
-                                    : (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
+        for (int c = 0; c < n; ++c) {
+          const int take = npages / n + (c < npages % n ? 1 : 0);
           const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
           mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
           pb += take;
-          used += take;
-          if (!last_cta && used >= span) {
-            mma_cta_segs.push_back((int32_t)mma_segs.size());
-            used = 0;
-          }
         }
       }
     }
-    if (used > 0) mma_cta_segs.push_back((int32_t)mma_segs.size());
+    std::stable_sort(mma_segs.begin(), mma_segs.end(),
+                     [](const SegRec& x, const SegRec& y) { return x.n_tokens > y.n_tokens; });
+    n_mma = (int)std::min<int64_t>(n_mma, (int64_t)mma_segs.size());
+    mma_cta_segs.push_back((int32_t)mma_segs.size());
   }
 
   // ---- partial rows: contiguous per (request, kv head), in a fixed order
@@ -497,7 +489,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   h.num_segments_mma = (int32_t)mma_segs.size();
   h.num_segments = h.num_segments_simt + h.num_segments_mma;
   h.simt_warps = (int32_t)warp_segs.size() - 1;
-  h.mma_ctas = (int32_t)mma_cta_segs.size() - 1;
+  h.mma_ctas = mma_segs.empty() ? 0 : n_mma;
   h.num_partial_rows = num_prows;
   h.num_tail_pairs = (int32_t)tail_pairs.size();
   uint64_t off = align256(sizeof(pa_image_header));

@@ -95,6 +95,7 @@ struct PaDevPtrs {
   float* partial_lse;
   float* partial_o;
   int32_t* status;
+  int32_t* mma_next;
 };
 
 // out == nullptr: partial rows only; else the merge is fused into the launch.

@@ -35,7 +35,7 @@ class Image:
         self.pages = arr(h.off_pages, n_pages)
         self.queries = arr(h.off_queries, (h.off_seg_prows - h.off_queries) // 4)
         self.seg_prows = arr(h.off_seg_prows, (h.off_mma_segs - h.off_seg_prows) // 4)
-        self.mma_segs = arr(h.off_mma_segs, h.mma_ctas + 1)
+        self.mma_segs = arr(h.off_mma_segs, 2 if h.num_segments_mma else 1)
         self.counters = arr(h.off_counters, h.batch * h.num_kv_heads)
         self.warp_segs = arr(h.off_warp_segs, h.simt_warps + 1)
         self.prow_off = arr(h.off_prow_off, h.batch * h.num_kv_heads + 1)
@@ -46,12 +46,17 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
     h = img.h
     B, Hkv, G = h.batch, h.num_kv_heads, h.num_q_heads // h.num_kv_heads
     nseg_simt = h.num_segments_simt
-    # MMA CTA lists partition the MMA segments; arrival counters start at zero
+    # the tensor-core work units form one list, longest first, taken by the
+    # CTAs from the header's counter (zero after upload); arrival counters
+    # start at zero
     if h.num_segments_mma:
-        assert img.mma_segs[0] == 0 and img.mma_segs[-1] == h.num_segments_mma
-        assert np.all(np.diff(img.mma_segs) > 0)
+        assert list(img.mma_segs) == [0, h.num_segments_mma]
+        assert 1 <= h.mma_ctas <= h.num_segments_mma
+        toks = img.segs[nseg_simt:, 3]
+        assert np.all(np.diff(toks) <= 0)
     else:
         assert h.mma_ctas == 0
+    assert h.mma_next == 0
     assert np.all(img.counters == 0)
     # pairs with tensor-core rows; the tail list holds those without SIMT rows, ascending
     mma_pairs, simt_rows = set(), {}

@@ -194,47 +194,49 @@ def test_plan_is_deterministic():
     assert np.array_equal(a, b)
 
 
-def tensor_core_stats(w):
+def tensor_core_units(w):
     p = make_plan(w)
     img = Image(p.host_image())
     h = img.h
     ns = h.num_segments_simt
-    mma_pages = sum((int(img.segs[i][3]) + 15) // 16 for i in range(ns, h.num_segments))
-    per_cta = [int(img.mma_segs[c + 1] - img.mma_segs[c]) for c in range(h.mma_ctas)]
-    return h, mma_pages, per_cta
+    pages = [(int(img.segs[i][3]) + 15) // 16 for i in range(ns, h.num_segments)]
+    runs = {}
+    for i in range(ns, h.num_segments):
+        item, g = int(img.segs[i][0]), int(img.segs[i][1])
+        runs.setdefault((item, g), []).append(i)
+    return h, img, pages, runs
 
 
 @pytest.mark.parametrize("config", [1, 2, 3, 5])
-def test_tensor_core_ctas_have_at_least_16_pages_each(config):
-    # at most one tensor-core CTA per 16 pages of tensor-core work: a small
-    # shared prefix (config 1: 16 pages x 2 kv heads) is not spread over many
-    # CTAs that each pay the segment's fixed cost
+def test_tensor_core_work_units_are_chunks_of_at_least_16_pages(config):
+    # at most one tensor-core CTA per 16 pages of tensor-core work (a small
+    # shared prefix, config 1: 16 pages x 2 kv heads, is not spread over many
+    # CTAs that each pay the segment's fixed cost); every (item, kv head) run
+    # is cut into equal chunks of at least 16 pages (or the whole run), and
+    # there are at least as many chunks as CTAs
     w = wl.make_config(config, with_values=False)
-    h, mma_pages, per_cta = tensor_core_stats(w)
-    assert h.mma_ctas >= 1 and h.mma_ctas <= -(-mma_pages // 16)
-    assert all(n >= 1 for n in per_cta)
+    h, img, pages, runs = tensor_core_units(w)
+    mma_pages = sum(pages)
+    assert 1 <= h.mma_ctas <= -(-mma_pages // 16) and h.mma_ctas <= len(pages)
     if config == 1:
         assert h.mma_ctas <= 2
-
-
-def test_tensor_core_spans_charge_a_cost_per_segment():
-    # config 3: the root's 128-row query tiles (one long run per kv head) and
-    # the 32-row leaf tiles (many short runs); a CTA that holds many short
-    # segments is given fewer pages than one holding a single long run
-    w = wl.make_config(3, with_values=False)
-    p = make_plan(w)
-    img = Image(p.host_image())
-    h = img.h
     ns = h.num_segments_simt
-    pages, segs = [], []
-    for c in range(h.mma_ctas):
-        ss = range(ns + int(img.mma_segs[c]), ns + int(img.mma_segs[c + 1]))
-        pages.append(sum((int(img.segs[i][3]) + 15) // 16 for i in ss))
-        segs.append(len(ss))
-    pages, segs = np.array(pages), np.array(segs)
-    many, few = segs >= np.percentile(segs, 75), segs <= np.percentile(segs, 25)
-    assert many.any() and few.any() and segs[many].min() > segs[few].max()
-    assert pages[many].mean() < pages[few].mean()
+    for ids in runs.values():
+        sizes = [pages[i - ns] for i in ids]
+        total = sum(sizes)
+        assert max(sizes) - min(sizes) <= 1
+        assert len(sizes) == 1 or min(sizes) >= min(16, total)
+
+
+def test_tensor_core_work_units_longest_first_about_two_per_cta():
+    # config 3: root runs (256 pages per kv head and 128-row tile) and branch
+    # runs (64 pages): the CTAs take the units longest first from a shared
+    # counter, so a CTA that runs faster takes more of them; about two units
+    # per CTA (each unit pays an epilogue, so not many more)
+    w = wl.make_config(3, with_values=False)
+    h, img, pages, runs = tensor_core_units(w)
+    assert pages == sorted(pages, reverse=True)
+    assert h.mma_ctas <= len(pages) <= 4 * h.mma_ctas + len(runs)
 
 
 # ------------------------------------------------------------- decode steps
