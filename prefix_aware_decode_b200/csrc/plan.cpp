@@ -347,6 +347,44 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   mma_segs.clear();
   warp_segs.assign(1, 0);
   mma_cta_segs.assign(1, 0);
+  if (mma_pages > 0) {
+    // Tensor-core work units: every (item, kv head) run cut into equal chunks
+    // of at most `chunk` pages, about kMmaChunksPerCta per CTA.  The CTAs take
+    // the chunks one after another from a counter in the image (the K producer
+    // of each CTA fetches the next one), longest first, so an SM that runs
+    // faster takes more of them: the same stage of the same work was measured
+    // to take from 1.3k to 2.4k cycles on different SMs of one launch.
+    // A chunk is at least kMmaMinChunkPages long: each one pays an epilogue
+    // (≈3 us, during which its CTA's tensor pipe waits), so short chunks cost
+    // more than the balance they buy.  When that leaves about one chunk per
+    // CTA, each chunk gets a CTA of its own.
+    const int kMmaChunksPerCta = 2, kMmaMinChunkPages = 64;
+    int64_t chunk = ceil_div(mma_pages + mma_seg_total, (int64_t)n_mma * kMmaChunksPerCta);
+    if (chunk < kMmaMinChunkPages) chunk = kMmaMinChunkPages;
+    if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
+    for (size_t i = 0; i < items.size(); ++i) {
+      const ItemRec& it = items[i];
+      if (it.simt) continue;
+      const int npages = (int)ceil_div(it.n_tokens, P);
+      const int n = (int)ceil_div(npages, chunk);
+      for (int g = 0; g < Hkv; ++g) {
+        int pb = 0;
+        for (int c = 0; c < n; ++c) {
+          const int take = npages / n + (c < npages % n ? 1 : 0);
+          const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
+          mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
+          pb += take;
+        }
+      }
+    }
+    std::stable_sort(mma_segs.begin(), mma_segs.end(),
+                     [](const SegRec& x, const SegRec& y) { return x.n_tokens > y.n_tokens; });
+    const int64_t n_chunks = (int64_t)mma_segs.size();
+    if (2 * n_chunks <= 3 * (int64_t)n_mma) n_mma = (int)std::min<int64_t>(n_chunks, std::max(1, S - 1));
+    n_mma = (int)std::min<int64_t>(n_mma, n_chunks);
+    mma_cta_segs.push_back((int32_t)mma_segs.size());
+  }
+
   if (simt_pages > 0) {
     const int64_t W = (int64_t)std::max(1, S - n_mma) * kSimtWarpsPerCta;
     int64_t span = ceil_div(simt_pages, W);
@@ -398,38 +436,6 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     simt_segs.resize(n_seg);
     warp_segs.resize(n_warp);
   }
-  if (mma_pages > 0) {
-    // Tensor-core work units: every (item, kv head) run cut into equal chunks
-    // of at most `chunk` pages, about kMmaChunksPerCta per CTA.  The CTAs take
-    // the chunks one after another from a counter in the image (the K producer
-    // of each CTA fetches the next one), longest first, so an SM that runs
-    // faster takes more of them: the same stage of the same work was measured
-    // to take from 1.3k to 2.4k cycles on different SMs of one launch.
-    const int kMmaChunksPerCta = 2;
-    int64_t chunk = ceil_div(mma_pages + mma_seg_total, (int64_t)n_mma * kMmaChunksPerCta);
-    if (chunk < 16) chunk = 16;
-    if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
-    for (size_t i = 0; i < items.size(); ++i) {
-      const ItemRec& it = items[i];
-      if (it.simt) continue;
-      const int npages = (int)ceil_div(it.n_tokens, P);
-      const int n = (int)ceil_div(npages, chunk);
-      for (int g = 0; g < Hkv; ++g) {
-        int pb = 0;
-        for (int c = 0; c < n; ++c) {
-          const int take = npages / n + (c < npages % n ? 1 : 0);
-          const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
-          mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
-          pb += take;
-        }
-      }
-    }
-    std::stable_sort(mma_segs.begin(), mma_segs.end(),
-                     [](const SegRec& x, const SegRec& y) { return x.n_tokens > y.n_tokens; });
-    n_mma = (int)std::min<int64_t>(n_mma, (int64_t)mma_segs.size());
-    mma_cta_segs.push_back((int32_t)mma_segs.size());
-  }
-
   // ---- partial rows: contiguous per (request, kv head), in a fixed order
   std::vector<int32_t>& prow_off = sc.prow_off;
   prow_off.assign((size_t)batch * Hkv + 1, 0);
