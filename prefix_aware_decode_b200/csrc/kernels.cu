@@ -957,8 +957,6 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       tmem_ld32(tmem + S::T_S + (i_ % kSBufs) * kMmaKT + 32 * h + lane_off, sv);
     };
     bool have_s = false;
-    bool p_pending = false;  // this thread's P of stage p_buf is stored but not yet handed over
-    int p_buf = 0;
     int qn = 0;
     // the next queue entry, by the whole warp (lane 0 frees the entry)
     auto take = [&]() -> int {
@@ -997,14 +995,6 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         }
         have_s = false;
         if (act) tmem_wait_ld_into(sv);
-        // the previous stage's P is handed over only now: its stores complete
-        // while this stage's S is loaded, instead of being waited for at once
-        if (p_pending) {
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(S::B_PFULL + p_buf));
-          p_pending = false;
-        }
         const uint32_t t_s = tmem + S::T_S + b * kMmaKT + 32 * h + lane_off;
         // the Q buffer of the previous segment is free (all its S products have
         // been read): the next work unit's rows are copied into it as soon as
@@ -1130,14 +1120,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           }
           fence_proxy_async_smem();
         }
-        p_pending = true;
-        p_buf = b;
-      }
-      if (p_pending) {
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(S::B_PFULL + p_buf));
-        p_pending = false;
+        mbar_arrive(bar(S::B_PFULL + b));
       }
       if (!ok) break;
       // ---- epilogue: combine the two key halves of each row; this thread
