@@ -194,9 +194,11 @@ def test_decode_step_matches_plan_path():
 
 
 def test_arrival_counters_return_to_zero_with_mixed_pairs():
-    # mixed pairs (tensor-core and SIMT rows) are merged by the last SIMT arriver
-    # after the tensor-core launch; the merging warp puts the pair's arrival
-    # counter back to zero, so the uploaded plan gives the same bits launch after launch
+    # mixed pairs (tensor-core and small-row rows) are merged by the last
+    # small-row arriver after the tensor-core launch; the merging warp puts the
+    # pair's arrival counter back to zero, and the launch's last take of a
+    # tensor-core work unit puts the unit counter back to zero, so the uploaded
+    # plan gives the same bits launch after launch
     import ctypes
 
     dw = dev_config(2, scale=0.25)
@@ -217,6 +219,9 @@ def test_arrival_counters_return_to_zero_with_mixed_pairs():
         torch.cuda.synchronize()
         words = ws[h.off_counters: h.off_counters + 4 * n_words].cpu().numpy().view(np.int32)
         assert not words.any(), np.nonzero(words)
+        # the counter of tensor-core work units taken is back at zero too
+        off_next = pad.PaImageHeader.mma_next.offset
+        assert int(ws[off_next:off_next + 4].cpu().numpy().view(np.int32)[0]) == 0
         if first is None:
             first = (out.clone(), lse.clone())
             assert_close(compare(out, lse, ref_o, ref_l), "attend() with mixed pairs")
