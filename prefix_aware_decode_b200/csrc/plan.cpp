@@ -436,12 +436,17 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     simt_segs.resize(n_seg);
     warp_segs.resize(n_warp);
   }
-  // ---- partial rows: contiguous per (request, kv head), in a fixed order
+  // ---- partial rows: contiguous per (request, kv head), in a fixed order.
+  // A tensor-core segment of at most 64 rows runs its rows twice (lanes 0-63
+  // and 64-127 of the tile, each copy on half of every stage's keys), so it
+  // writes two partial rows per request (mma_copies)
   std::vector<int32_t>& prow_off = sc.prow_off;
   prow_off.assign((size_t)batch * Hkv + 1, 0);
+  auto mma_copies = [&](const ItemRec& it) { return it.n_queries * G <= kMmaRowsPerCta / 2 ? 2 : 1; };
   for (const auto& s : mma_segs) {
     const ItemRec& it = items[s.item];
-    for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
+    for (int j = 0; j < it.n_queries; ++j)
+      prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1] += mma_copies(it);
   }
   // fused merge: the last SIMT partial row of a pair to be written merges the
   // pair (after the tensor-core launch has finished if the pair also has
@@ -475,8 +480,10 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   for (auto& s : mma_segs) {
     const ItemRec& it = items[s.item];
     s.prow = (int)seg_prows.size();
-    for (int j = 0; j < it.n_queries; ++j)
-      seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
+    // copy c of the rows: entries [c * n_queries, (c + 1) * n_queries)
+    for (int c = 0; c < mma_copies(it); ++c)
+      for (int j = 0; j < it.n_queries; ++j)
+        seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
   }
   for (auto& s : simt_segs) s.prow = cursor[(size_t)s.query * Hkv + s.kv_head]++;
   const int num_prows = prow_off.back();
