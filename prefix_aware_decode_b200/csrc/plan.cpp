@@ -349,7 +349,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   mma_cta_segs.assign(1, 0);
   if (mma_pages > 0) {
     // Tensor-core work units: every (item, kv head) run cut into equal chunks
-    // of at most `chunk` pages, about kMmaChunksPerCta per CTA.  The CTAs take
+    // of at most `chunk` pages, two to eight per CTA.  The CTAs take
     // the chunks one after another from a counter in the image (the K producer
     // of each CTA fetches the next one), longest first, so an SM that runs
     // faster takes more of them: the same stage of the same work was measured
@@ -358,8 +358,14 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     // (≈3 us, during which its CTA's tensor pipe waits), so short chunks cost
     // more than the balance they buy.  When that leaves about one chunk per
     // CTA, each chunk gets a CTA of its own.
-    const int kMmaChunksPerCta = 2, kMmaMinChunkPages = 64;
-    int64_t chunk = ceil_div(mma_pages + mma_seg_total, (int64_t)n_mma * kMmaChunksPerCta);
+    // Long work is cut finer, up to 8 chunks per CTA while a chunk stays at
+    // least 20 times its epilogue's cost (≈480 pages): a CTA then ends at most
+    // one short chunk after the others.
+    const int kMmaMinChunkPages = 64;
+    const int64_t work = mma_pages + mma_seg_total;
+    const int64_t per_cta = ceil_div(work, n_mma);
+    const int64_t chunks_per_cta = std::max<int64_t>(2, std::min<int64_t>(8, per_cta / (20 * kMmaSegPages)));
+    int64_t chunk = ceil_div(work, (int64_t)n_mma * chunks_per_cta);
     if (chunk < kMmaMinChunkPages) chunk = kMmaMinChunkPages;
     if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
     for (size_t i = 0; i < items.size(); ++i) {
