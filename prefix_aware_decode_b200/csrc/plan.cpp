@@ -348,38 +348,42 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   warp_segs.assign(1, 0);
   mma_cta_segs.assign(1, 0);
   if (mma_pages > 0) {
-    // Tensor-core work units: every (item, kv head) run cut into equal chunks
-    // of at most `chunk` pages, two to eight per CTA.  The CTAs take
-    // the chunks one after another from a counter in the image (the K producer
-    // of each CTA fetches the next one), longest first, so an SM that runs
-    // faster takes more of them: the same stage of the same work was measured
-    // to take from 1.3k to 2.4k cycles on different SMs of one launch.
-    // A chunk is at least kMmaMinChunkPages long: each one pays an epilogue
-    // (≈3 us, during which its CTA's tensor pipe waits), so short chunks cost
-    // more than the balance they buy.  When that leaves about one chunk per
-    // CTA, each chunk gets a CTA of its own.
-    // Long work is cut finer, up to 8 chunks per CTA while a chunk stays at
-    // least 20 times its epilogue's cost (≈480 pages): a CTA then ends at most
-    // one short chunk after the others.
-    const int kMmaMinChunkPages = 64;
+    // Tensor-core work units: the CTAs take them one after another from a
+    // counter in the image (the K producer of each CTA fetches the next one),
+    // longest first, so an SM that runs faster takes more of them: the same
+    // stage of the same work was measured to take from 1.3k to 2.4k cycles on
+    // different SMs of one launch.  Every unit pays an epilogue and adds a
+    // partial row per request to write and merge, so units stay few:
+    //   - long work (per CTA, at least 80 segment costs): each (item, kv head)
+    //     run cut into kMmaPieces pieces of decreasing length (weights
+    //     kMmaPieces : ... : 1), so the last units taken are the short ones and
+    //     the CTAs end together;
+    //   - otherwise: each run cut into equal chunks, about two per CTA, at
+    //     least kMmaMinChunkPages long; when that leaves about one chunk per
+    //     CTA, each chunk gets a CTA of its own.
+    const int kMmaMinChunkPages = 64, kMmaPieces = 2;
     const int64_t work = mma_pages + mma_seg_total;
-    const int64_t per_cta = ceil_div(work, n_mma);
-    const int64_t chunks_per_cta = std::max<int64_t>(2, std::min<int64_t>(8, per_cta / (20 * kMmaSegPages)));
-    int64_t chunk = ceil_div(work, (int64_t)n_mma * chunks_per_cta);
+    const bool long_work = ceil_div(work, n_mma) >= 80 * kMmaSegPages;
+    int64_t chunk = ceil_div(work, (int64_t)n_mma * 2);
     if (chunk < kMmaMinChunkPages) chunk = kMmaMinChunkPages;
     if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
     for (size_t i = 0; i < items.size(); ++i) {
       const ItemRec& it = items[i];
       if (it.simt) continue;
       const int npages = (int)ceil_div(it.n_tokens, P);
-      const int n = (int)ceil_div(npages, chunk);
       for (int g = 0; g < Hkv; ++g) {
         int pb = 0;
-        for (int c = 0; c < n; ++c) {
-          const int take = npages / n + (c < npages % n ? 1 : 0);
+        auto emit = [&](int take) {
           const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
           mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
           pb += take;
+        };
+        if (long_work && !max_chunk_pages && npages >= kMmaPieces * 20 * kMmaSegPages) {
+          const int wsum = kMmaPieces * (kMmaPieces + 1) / 2;
+          for (int c = kMmaPieces; c >= 1; --c) emit(c == 1 ? npages - pb : (int)((int64_t)npages * c / wsum));
+        } else {
+          const int n = (int)ceil_div(npages, chunk);
+          for (int c = 0; c < n; ++c) emit(npages / n + (c < npages % n ? 1 : 0));
         }
       }
     }
