@@ -367,11 +367,7 @@ const char *pa_status_string(pa_status s);
  *   segs        pa_seg[num_segments]          SIMT segments first, then MMA
  *   pages       int32[num_page_entries]       page ids, per item
  *   queries     int32[num_query_entries]      request ids, per item
- *   seg_prows   int32[...]                    partial row of each (MMA seg, query); a segment of
- *                                             at most 64 rows has two per query (entries of copy 0,
- *                                             then of copy 1: the rows run twice, copy c on keys
- *                                             [16c, 16c + 16) and [32 + 16c, 48 + 16c) of every
- *                                             64-key stage)
+ *   seg_prows   int32[num_query_entries_mma]  partial row of each (MMA seg, query)
  *   mma_segs    int32[2]                      {0, num_segments_mma}: the tensor-core work units,
  *                                             longest first; the tensor-core CTAs take them one
  *                                             at a time from the counter mma_next of the header

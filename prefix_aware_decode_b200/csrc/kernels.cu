@@ -911,15 +911,13 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     auto q_src = [&](int si) -> const uint16_t* {
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
-      const int R_ = item.n_queries * G;
-      const int rr = R_ <= 64 ? (r & 63) : r;  // tiles of <= 64 rows: lanes 64-127 repeat rows 0-63
-      if (rr >= R_) return nullptr;
-      int b = a.queries[item.query_off + rr / G];
+      if (r >= item.n_queries * G) return nullptr;
+      int b = a.queries[item.query_off + r / G];
       if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
         record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
         b = 0;
       }
-      return a.q + ((size_t)b * a.Hq + seg.kv_head * G + (rr % G)) * D;
+      return a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
     };
     // This thread's half of row r into Q buffer qbuf (K-major, 128-byte swizzle).
     auto q_dst = [&](int qbuf, int c) -> uint8_t* {
@@ -954,13 +952,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     // S(i + 1) is issued while P(i) is being stored, when S(i + 1) is already
     // there (else at the top of the next stage)
     float sv[32];
-    int cbase = 32 * h;  // first S/P column of this thread in a stage (set per segment)
-    bool dup = false;    // the segment's rows run twice (tiles of <= 64 rows)
     auto load_s = [&](int i_) {
       tc_fence_after();
-      const uint32_t ta = tmem + S::T_S + (i_ % kSBufs) * kMmaKT + cbase + lane_off;
-      if (dup) tmem_ld16(ta, sv);
-      else tmem_ld32(ta, sv);
+      tmem_ld32(tmem + S::T_S + (i_ % kSBufs) * kMmaKT + 32 * h + lane_off, sv);
     };
     bool have_s = false;
     int qn = 0;
@@ -981,19 +975,10 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
       const int R = item.n_queries * G;
-      // A tile of at most 64 rows runs its rows twice, in lanes 0-63 and
-      // 64-127 (copy 0 and 1): of the 16-key chunks of a stage, copy c takes
-      // chunk 2h + c of its key half and writes zeros as P of the other chunk,
-      // so each accumulator row sums its own copy's keys only; the two copies
-      // leave two partial rows per request, combined by the merge.  Otherwise a
-      // warp whose lane quarter lies past the tile's rows keeps every barrier of
-      // the protocol but skips the arithmetic (its P and O rows are never read).
-      dup = R <= 64;
-      const int copy = dup ? quad >> 1 : 0;
-      const int lrow = dup ? (r & 63) : r;  // the tile row this lane holds
-      cbase = dup ? 16 * (2 * h + copy) : 32 * h;
-      const int nk = dup ? 16 : 32;         // keys of a stage this thread handles
-      const bool act = dup || quad * 32 < R;
+      // a warp whose lane quarter lies past the tile's rows keeps every
+      // barrier of the protocol but skips the arithmetic (its P and O rows are
+      // never read out)
+      const bool act = quad * 32 < R;
       const int npages = (seg.n_tokens + 15) >> 4;
       float m_used = -INFINITY, l = 0.f;
       bool q_known = false;  // the next work unit has been seen in the queue
@@ -1002,7 +987,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         const int s = i % NST, b = i % kSBufs;
         const int np = min(4, npages - st);
         const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
-        const int kv_h = max(0, min(nk, kvalid - cbase));  // valid keys of this thread
+        const int kv_h = max(0, min(32, kvalid - 32 * h));  // valid keys of this half
         const bool last = st + 4 >= npages;
         if (!have_s) {
           if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
@@ -1010,7 +995,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         }
         have_s = false;
         if (act) tmem_wait_ld_into(sv);
-        const uint32_t t_s = tmem + S::T_S + b * kMmaKT + cbase + lane_off;
+        const uint32_t t_s = tmem + S::T_S + b * kMmaKT + 32 * h + lane_off;
         // the Q buffer of the previous segment is free (all its S products have
         // been read): the next work unit's rows are copied into it as soon as
         // the unit is in the queue, and published a stage later (or at this
@@ -1044,9 +1029,6 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         if (kv_h == 32) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
-        } else if (kv_h == 16 && dup) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -1111,13 +1093,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         };
         using I0 = std::integral_constant<int, 0>;
         using I1 = std::integral_constant<int, 1>;
-        if (dup) {
-          if (kv_h == 16) page(I0{}, std::true_type{});
-          else page(I0{}, std::false_type{});
-          // zeros as P (hi and lo) of the other copy's chunk, in this lane
-          const float zr[32] = {};
-          tmem_st16<0>(tmem + S::T_S + b * kMmaKT + (cbase ^ 16) + lane_off, zr);
-        } else if (kv_h == 32) {
+        if (kv_h == 32) {
           page(I0{}, std::true_type{});
           page(I1{}, std::true_type{});
         } else {
@@ -1174,14 +1150,12 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       const float mm = fmaxf(m0, m1);
       const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
       const float L = w0 * l0 + w1 * l1;
-      // a copy that saw no key (a segment of at most 16 tokens) writes o = 0,
-      // lse = -inf: a weight of zero in the merge
-      const float c0 = L > 0.f ? w0 / L : 0.f, c1 = L > 0.f ? w1 / L : 0.f;
+      const float c0 = w0 / L, c1 = w1 / L;
       float* dst = nullptr;
-      if (lrow < R) {
-        const int prow = a.seg_prows[seg.prow + copy * item.n_queries + lrow / G];
-        dst = a.partial_o + ((size_t)prow * G + (lrow % G)) * D + h * (D / 2);
-        if (h == 0) a.partial_lse[(size_t)prow * G + (lrow % G)] = L > 0.f ? (mm + lg2(L)) * kLn2 : -INFINITY;
+      if (r < R) {
+        const int prow = a.seg_prows[seg.prow + r / G];
+        dst = a.partial_o + ((size_t)prow * G + (r % G)) * D + h * (D / 2);
+        if (h == 0) a.partial_lse[(size_t)prow * G + (r % G)] = (mm + lg2(L)) * kLn2;
       }
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {

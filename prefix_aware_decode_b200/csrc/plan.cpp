@@ -348,42 +348,32 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   warp_segs.assign(1, 0);
   mma_cta_segs.assign(1, 0);
   if (mma_pages > 0) {
-    // Tensor-core work units: the CTAs take them one after another from a
-    // counter in the image (the K producer of each CTA fetches the next one),
-    // longest first, so an SM that runs faster takes more of them: the same
-    // stage of the same work was measured to take from 1.3k to 2.4k cycles on
-    // different SMs of one launch.  Every unit pays an epilogue and adds a
-    // partial row per request to write and merge, so units stay few:
-    //   - long work (per CTA, at least 80 segment costs): each (item, kv head)
-    //     run cut into kMmaPieces pieces of decreasing length (weights
-    //     kMmaPieces : ... : 1), so the last units taken are the short ones and
-    //     the CTAs end together;
-    //   - otherwise: each run cut into equal chunks, about two per CTA, at
-    //     least kMmaMinChunkPages long; when that leaves about one chunk per
-    //     CTA, each chunk gets a CTA of its own.
-    const int kMmaMinChunkPages = 64, kMmaPieces = 2;
-    const int64_t work = mma_pages + mma_seg_total;
-    const bool long_work = ceil_div(work, n_mma) >= 80 * kMmaSegPages;
-    int64_t chunk = ceil_div(work, (int64_t)n_mma * 2);
+    // Tensor-core work units: every (item, kv head) run cut into equal chunks
+    // of at most `chunk` pages, about kMmaChunksPerCta per CTA.  The CTAs take
+    // the chunks one after another from a counter in the image (the K producer
+    // of each CTA fetches the next one), longest first, so an SM that runs
+    // faster takes more of them: the same stage of the same work was measured
+    // to take from 1.3k to 2.4k cycles on different SMs of one launch.
+    // A chunk is at least kMmaMinChunkPages long: each one pays an epilogue
+    // (≈3 us, during which its CTA's tensor pipe waits), so short chunks cost
+    // more than the balance they buy.  When that leaves about one chunk per
+    // CTA, each chunk gets a CTA of its own.
+    const int kMmaChunksPerCta = 2, kMmaMinChunkPages = 64;
+    int64_t chunk = ceil_div(mma_pages + mma_seg_total, (int64_t)n_mma * kMmaChunksPerCta);
     if (chunk < kMmaMinChunkPages) chunk = kMmaMinChunkPages;
     if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
     for (size_t i = 0; i < items.size(); ++i) {
       const ItemRec& it = items[i];
       if (it.simt) continue;
       const int npages = (int)ceil_div(it.n_tokens, P);
+      const int n = (int)ceil_div(npages, chunk);
       for (int g = 0; g < Hkv; ++g) {
         int pb = 0;
-        auto emit = [&](int take) {
+        for (int c = 0; c < n; ++c) {
+          const int take = npages / n + (c < npages % n ? 1 : 0);
           const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
           mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
           pb += take;
-        };
-        if (long_work && !max_chunk_pages && npages >= kMmaPieces * 20 * kMmaSegPages) {
-          const int wsum = kMmaPieces * (kMmaPieces + 1) / 2;
-          for (int c = kMmaPieces; c >= 1; --c) emit(c == 1 ? npages - pb : (int)((int64_t)npages * c / wsum));
-        } else {
-          const int n = (int)ceil_div(npages, chunk);
-          for (int c = 0; c < n; ++c) emit(npages / n + (c < npages % n ? 1 : 0));
         }
       }
     }
@@ -446,17 +436,12 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     simt_segs.resize(n_seg);
     warp_segs.resize(n_warp);
   }
-  // ---- partial rows: contiguous per (request, kv head), in a fixed order.
-  // A tensor-core segment of at most 64 rows runs its rows twice (lanes 0-63
-  // and 64-127 of the tile, each copy on half of every stage's keys), so it
-  // writes two partial rows per request (mma_copies)
+  // ---- partial rows: contiguous per (request, kv head), in a fixed order
   std::vector<int32_t>& prow_off = sc.prow_off;
   prow_off.assign((size_t)batch * Hkv + 1, 0);
-  auto mma_copies = [&](const ItemRec& it) { return it.n_queries * G <= kMmaRowsPerCta / 2 ? 2 : 1; };
   for (const auto& s : mma_segs) {
     const ItemRec& it = items[s.item];
-    for (int j = 0; j < it.n_queries; ++j)
-      prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1] += mma_copies(it);
+    for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
   }
   // fused merge: the last SIMT partial row of a pair to be written merges the
   // pair (after the tensor-core launch has finished if the pair also has
@@ -490,10 +475,8 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   for (auto& s : mma_segs) {
     const ItemRec& it = items[s.item];
     s.prow = (int)seg_prows.size();
-    // copy c of the rows: entries [c * n_queries, (c + 1) * n_queries)
-    for (int c = 0; c < mma_copies(it); ++c)
-      for (int j = 0; j < it.n_queries; ++j)
-        seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
+    for (int j = 0; j < it.n_queries; ++j)
+      seg_prows.push_back(cursor[(size_t)queries[it.query_off + j] * Hkv + s.kv_head]++);
   }
   for (auto& s : simt_segs) s.prow = cursor[(size_t)s.query * Hkv + s.kv_head]++;
   const int num_prows = prow_off.back();

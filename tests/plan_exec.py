@@ -98,11 +98,16 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
         item, g, pb, nt, prow, q0 = img.segs[si]
         po, itok, nq, qo = img.items[item]
         assert 1 <= nt and pb * P + nt <= itok
-        for b, pr, toks in segment_rows(img, si, P):
+        qs = img.queries[qo: qo + nq]
+        if si < nseg_simt:
+            prs = [prow]
+        else:
+            prs = img.seg_prows[prow: prow + nq]
+        for b, pr in zip(qs, prs):
             assert img.prow_off[b * Hkv + g] <= pr < img.prow_off[b * Hkv + g + 1]
             prows_written[pr] += 1
-            for tok in toks:
-                key = (int(b), int(g), int(img.pages[po + tok // P]), int(tok) % P)
+            for tok in range(pb * P, pb * P + nt):
+                key = (int(b), int(g), int(img.pages[po + tok // P]), tok % P)
                 seen[key] = seen.get(key, 0) + 1
     assert np.all(prows_written == 1)
     assert all(v == 1 for v in seen.values())
@@ -112,30 +117,6 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
             for tok in range(n):
                 assert seen.get((b, g, int(block_table[b, tok // P]), tok % P)) == 1, (b, g, tok)
     assert len(seen) == int(np.sum(kv_lens)) * Hkv
-
-
-def segment_rows(img: Image, si: int, P=16):
-    """(request, partial row, token indices within the item) of every partial
-    row segment si writes.  A tensor-core segment of at most 64 rows runs its
-    rows twice; copy c reads keys [16c, 16c + 16) and [32 + 16c, 48 + 16c) of
-    every 64-key stage of the segment."""
-    h = img.h
-    G = h.num_q_heads // h.num_kv_heads
-    item, g, pb, nt, prow, q0 = img.segs[si]
-    po, itok, nq, qo = img.items[item]
-    qs = img.queries[qo: qo + nq]
-    toks = np.arange(pb * P, pb * P + nt)
-    if si < h.num_segments_simt:
-        return [(int(qs[0]), int(prow), toks)]
-    if nq * G > 64:
-        return [(int(b), int(pr), toks) for b, pr in zip(qs, img.seg_prows[prow: prow + nq])]
-    rel = (toks - pb * P) % 64 // 16
-    out = []
-    for c in range(2):
-        sel = toks[(rel == c) | (rel == c + 2)]
-        prs = img.seg_prows[prow + c * nq: prow + (c + 1) * nq]
-        out.extend((int(b), int(pr), sel) for b, pr in zip(qs, prs))
-    return out
 
 
 def execute(img: Image, q, k_pool, v_pool, scale=None, P=16):
@@ -151,10 +132,13 @@ def execute(img: Image, q, k_pool, v_pool, scale=None, P=16):
     for si in range(h.num_segments):
         item, g, pb, nt, prow, q0 = img.segs[si]
         po, itok, nq, qo = img.items[item]
-        for b, pr, toks in segment_rows(img, si, P):
-            pg = img.pages[po + toks // P]
-            K = kf[pg, g, toks % P]
-            V = vf[pg, g, toks % P]
+        toks = np.arange(pb * P, pb * P + nt)
+        pg = img.pages[po + toks // P]
+        K = kf[pg, g, toks % P]
+        V = vf[pg, g, toks % P]
+        qs = img.queries[qo: qo + nq]
+        prs = [prow] if si < h.num_segments_simt else img.seg_prows[prow: prow + nq]
+        for b, pr in zip(qs, prs):
             for r in range(G):
                 o, l = oracle.attend_dense(qf[b, g * G + r], K, V, scale)
                 po_[pr, r] = o
