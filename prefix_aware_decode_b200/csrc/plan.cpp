@@ -106,10 +106,14 @@ struct Planner {
   // (n - 1) extra reads of the node; what it costs is one more fp32 partial row
   // per request and head (written by forward, read by merge) and a fixed
   // per-item overhead C_item.  Otherwise the node is folded into its children.
+  // C_item is a tensor-core work unit's fixed cost (an epilogue of ≈3.7 us,
+  // the Q rows, the pipeline ramp) in bytes of re-reading instead: a 16-page
+  // prefix shared by 4 requests (config 1, 393 KB saved) ran slower shared
+  // than inlined (1024 such problems: 129 us against 107 us on one B200).
   bool keep_shared(int n, int64_t L) const {
     if (flags & PA_PLAN_NO_SHARING) return false;
     if (flags & PA_PLAN_ALWAYS_SHARE) return true;
-    const double Bt = 2.0 * Hkv * D * 2, C_item = 64.0 * 1024;
+    const double Bt = 2.0 * Hkv * D * 2, C_item = 512.0 * 1024;
     return (n - 1) * (double)L * Bt > n * (double)Hq * (4.0 * D + 4.0) * 2.0 + C_item;
   }
 

@@ -38,7 +38,10 @@ def run_batch(pool, kv_pool, q_of, plan=None):
     qids, _, bt, kv = pool.batch()
     q = np.stack([q_of[i] for i in qids])
     if plan is None:
-        plan = pad.Plan(kv, bt, pool.num_pages, G * HKV, HKV, D, flags=pad.PA_PLAN_KEEP_PACK)
+        # these sessions are small (tens of tokens): the profit model would
+        # inline them, so sharing is forced to exercise the shared path
+        plan = pad.Plan(kv, bt, pool.num_pages, G * HKV, HKV, D,
+                        flags=pad.PA_PLAN_KEEP_PACK | pad.PA_PLAN_ALWAYS_SHARE)
     else:
         plan = plan.advance(kv, bt, pool.num_pages)
     img = Image(plan.host_image())
