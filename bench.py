@@ -27,6 +27,7 @@ the environment; without it bench.py starts them itself.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -54,30 +55,50 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled during a timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled during a timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Samples carry nvidia-smi's own timestamps; only those inside the timed
+    region (marked by mark_start / mark_end, plus 100 ms for the lag of the
+    driver's counters) are summarised, so idle samples taken before and after
+    it do not enter the median."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int):
         self.idx = device_index
         self.samples = []
         self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def _read(self):
         for line in self.proc.stdout:
             self.samples.append([x.strip() for x in line.split(",")])
+
+    @staticmethod
+    def _when(field: str):
+        try:
+            return datetime.datetime.strptime(field, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self) -> dict:
         if self.proc is None:
@@ -88,17 +109,24 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm = [float(s[1]) for s in self.samples if len(s) >= 9 and s[1].replace(".", "").isdigit()]
-        smax = [float(s[2]) for s in self.samples if len(s) >= 9 and s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = [s for s in self.samples if len(s) >= 10 and s[2].replace(".", "").isdigit()]
+        t0, t1 = self.t0, (self.t1 or time.time()) + 0.1
+        inside = [s for s in rows if t0 is None or (self._when(s[0]) or 0.0) >= t0 and (self._when(s[0]) or 0.0) <= t1]
+        if not inside and t0 is not None:  # a region shorter than the sampling period: the next sample
+            later = [s for s in rows if (self._when(s[0]) or 0.0) >= t0]
+            inside = later[:1]
+        sm = [float(s[2]) for s in inside]
+        smax = [float(s[3]) for s in rows if s[3].replace(".", "").isdigit()]
+        power = [float(s[4]) for s in inside if s[4].replace(".", "").isdigit()]
         reasons = set()
-        for s in self.samples:
-            if len(s) >= 9:
-                for n, v in zip(names, s[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(self.samples)}
+        for s in inside:
+            for n, v in zip(self.REASONS, s[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_min_mhz": min(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "note": "samples inside the timed region only (nvidia-smi timestamps, 20 ms period)"}
 
 
 def kernels_hash() -> str:
@@ -281,11 +309,13 @@ class Bench:
         torch.cuda.synchronize()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         host_us.clear()
+        clocks.mark_start()
         ev0.record(stream)
         for i in range(args.warmup, nsteps):
             step(i)
         ev1.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_end()
         self.barrier()
         clk = clocks.stop()
         ms_step = self.max_over_ranks(ev0.elapsed_time(ev1)) / args.steps

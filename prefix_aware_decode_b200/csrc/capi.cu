@@ -84,7 +84,27 @@ struct PinnedRing {
 std::mutex g_pin_mu;
 PinnedRing g_pin[64];
 
+// Replaces the buffer of an idle slot by one of >= n bytes (a power of two, at
+// least 64 KiB).
+bool pin_grow(PinnedSlot& s, size_t n) {
+  if (s.ptr) cudaFreeHost(s.ptr);
+  s.ptr = nullptr;
+  s.bytes = 0;
+  size_t cap = 1 << 16;
+  while (cap < n) cap <<= 1;
+  if (cudaMallocHost(&s.ptr, cap) != cudaSuccess) {
+    s.ptr = nullptr;
+    return false;
+  }
+  s.bytes = cap;
+  return true;
+}
+
 // Returns a free pinned slot of >= n bytes for the current device, or nullptr.
+// A slot that must grow takes every idle slot with it: a pinned allocation
+// costs a millisecond or more of host time, and paid one slot per step it
+// would stall the steps that follow the first (the host has no lead on the
+// device yet).
 PinnedSlot* pin_acquire(size_t n, int device) {
   if (device < 0 || device >= 64) return nullptr;
   PinnedRing& r = g_pin[device];
@@ -93,16 +113,9 @@ PinnedSlot* pin_acquire(size_t n, int device) {
   r.next = (r.next + 1) % kPinSlots;
   if (s.done && cudaEventSynchronize(s.done) != cudaSuccess) return nullptr;
   if (s.bytes < n) {
-    if (s.ptr) cudaFreeHost(s.ptr);
-    s.ptr = nullptr;
-    s.bytes = 0;
-    size_t cap = 1 << 16;
-    while (cap < n) cap <<= 1;
-    if (cudaMallocHost(&s.ptr, cap) != cudaSuccess) {
-      s.ptr = nullptr;
-      return nullptr;
-    }
-    s.bytes = cap;
+    if (!pin_grow(s, n)) return nullptr;
+    for (PinnedSlot& o : r.slot)
+      if (&o != &s && o.bytes < n && !o.lent && (!o.done || cudaEventQuery(o.done) == cudaSuccess)) pin_grow(o, n);
   }
   if (!s.done && cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess) return nullptr;
   return &s;

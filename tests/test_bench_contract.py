@@ -45,3 +45,36 @@ def test_world_size_that_differs_from_gpus_is_refused():
                         "--gpus", "2", "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
                        timeout=300, cwd=ROOT, env=env)
     assert r.returncode == 2 and "WORLD_SIZE" in r.stderr
+
+
+def test_clock_summary_keeps_only_samples_inside_the_timed_region():
+    # rows as nvidia-smi prints them: idle samples at the maximum clock before
+    # and after the region, power-capped samples inside it
+    import importlib.util
+    import datetime
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    base = datetime.datetime(2026, 1, 2, 3, 4, 5)
+
+    def row(dt_ms, mhz, cap):
+        ts = (base + datetime.timedelta(milliseconds=dt_ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return [ts, "0", str(mhz), "1965", "700.0", "0x4" if cap else "0x0", "Not Active", "Not Active",
+                "Not Active", "Active" if cap else "Not Active"]
+
+    s = bench.ClockSampler(0)
+    s.proc = _FakeProc()
+    s.samples = ([row(t, 1965, False) for t in range(-500, 0, 20)] + [row(t, 1520, True) for t in range(0, 300, 20)]
+                 + [row(t, 1965, False) for t in range(420, 900, 20)])
+    s.t0, s.t1 = base.timestamp(), base.timestamp() + 0.29
+    out = s.stop()
+    assert out["sm_mhz"] == 1520 and out["sm_min_mhz"] == 1520 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 15
+
+
+class _FakeProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
