@@ -597,11 +597,13 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, const CUtensorMap* t
 // Its own launch of one CTA per SM, each running a list of segments (item of
 // <= 128 rows, kv head g, key range).  Warp 0: TMA producer of 64-key K/V
 // stages.  Warp 1: TMEM owner and single-thread tcgen05.mma issuer.  Warps
-// 2-9: softmax, two threads per tile row (TMEM lane): warps 2-5 take keys
-// 0-31 of every stage, warps 6-9 keys 32-63, each half with its own running
-// maximum, sum and accumulator, so the halves never wait on each other inside
-// a segment; the two partial results are combined once per segment.  Per
-// 64-key stage i (S/P buffer i % 3 in TMEM):
+// 2-9: softmax: warps 2-5 take keys 0-31 of every stage, warps 6-9 keys 32-63,
+// each half with its own running maximum, sum and accumulator, so the halves
+// never wait on each other inside a segment; the two partial results are
+// combined once per segment.  Tiles of more than 64 rows are M = 128 products
+// (two threads per row); tiles of at most 64 rows are M = 64 products, whose
+// rows the TMEM layout spreads over all four lane quarters (four threads per
+// row, 16 keys each).  Per 64-key stage i (S/P buffer i % 3 in TMEM):
 //   S(i) = Q K^T                  -> TMEM, 64 columns
 //   p = exp2(s - m)               -> P = P_hi + P_lo, two bf16 matrices written
 //                                    over S(i) in TMEM (P_hi truncated, P_lo =
@@ -831,15 +833,22 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     // the MMAs of the thread that issues it.
     if (lane == 0) {
       const bool is_s = warp == 1;
-      constexpr uint32_t idesc_s = umma_idesc_bf16(128, kMmaKT, false, false);
-      constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, false, true);
+      // tiles of at most 64 rows: M = 64 products (rows in the first 16 lanes of
+      // each lane quarter, the layout the softmax reads them in)
+      constexpr uint32_t idesc_s128 = umma_idesc_bf16(128, kMmaKT, false, false);
+      constexpr uint32_t idesc_o128 = umma_idesc_bf16(128, D, false, true);
+      constexpr uint32_t idesc_s64 = umma_idesc_bf16(64, kMmaKT, false, false);
+      constexpr uint32_t idesc_o64 = umma_idesc_bf16(64, D, false, true);
       bool ok = true;
       int i = 0, segord = 0, qn = 0;
       for (;;) {
         const int si = seg_take(qn, true);
         if (si == -2) ok = false;
         if (si < 0) break;
-        const int npages = (a.segs[si].n_tokens + 15) >> 4;
+        const pa_seg seg = a.segs[si];
+        const bool m64 = a.items[seg.item].n_queries * G <= 64;
+        const uint32_t idesc_s = m64 ? idesc_s64 : idesc_s128, idesc_o = m64 ? idesc_o64 : idesc_o128;
+        const int npages = (seg.n_tokens + 15) >> 4;
         for (int st = 0; st < npages; st += 4, ++i) {
           const int s = i % NST, b = i % kSBufs;
           const bool first = st == 0;
@@ -898,10 +907,13 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       mbar_wait_bounded(bar(S::B_DONE), 0, a.timeout_ns);
     }
   } else {
-    // ---------------- softmax: thread = (tile row = TMEM lane, key half)
+    // ---------------- softmax: warps 2-5 take key half 0 of every stage, warps
+    // 6-9 key half 1; the rows a thread holds depend on the tile's shape
+    // (run_segment below)
     const int h = (warp - 2) >> 2;
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
+    const int hw = lane >> 4;
+    const int rq = quad * 32 + lane;  // the Q row this thread copies
     const int tid = (warp - 2) * 32 + lane;  // 0 .. 255
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     constexpr int QCH = D / 16;  // 16-byte q chunks per row loaded by each half
@@ -911,17 +923,17 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     auto q_src = [&](int si) -> const uint16_t* {
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
-      if (r >= item.n_queries * G) return nullptr;
-      int b = a.queries[item.query_off + r / G];
+      if (rq >= item.n_queries * G) return nullptr;
+      int b = a.queries[item.query_off + rq / G];
       if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
         record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
         b = 0;
       }
-      return a.q + ((size_t)b * a.Hq + seg.kv_head * G + (r % G)) * D;
+      return a.q + ((size_t)b * a.Hq + seg.kv_head * G + (rq % G)) * D;
     };
-    // This thread's half of row r into Q buffer qbuf (K-major, 128-byte swizzle).
+    // This thread's half of Q row rq into Q buffer qbuf (K-major, 128-byte swizzle).
     auto q_dst = [&](int qbuf, int c) -> uint8_t* {
-      return smem + S::OFF_Q + qbuf * S::QBUF + (c >> 3) * S::QBLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+      return smem + S::OFF_Q + qbuf * S::QBUF + (c >> 3) * S::QBLK + rq * 128 + (((c & 7) ^ (rq & 7)) << 4);
     };
     // the first segment: plain loads
     auto load_q = [&](int si) {
@@ -952,10 +964,6 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     // S(i + 1) is issued while P(i) is being stored, when S(i + 1) is already
     // there (else at the top of the next stage)
     float sv[32];
-    auto load_s = [&](int i_) {
-      tc_fence_after();
-      tmem_ld32(tmem + S::T_S + (i_ % kSBufs) * kMmaKT + 32 * h + lane_off, sv);
-    };
     bool have_s = false;
     int qn = 0;
     // the next queue entry, by the whole warp (lane 0 frees the entry)
@@ -971,14 +979,29 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     int si = take();
     if (si == -2) ok = false;
     if (si >= 0) load_q(si);
-    while (si >= 0 && ok) {
-      const pa_seg seg = a.segs[si];
-      const pa_item item = a.items[seg.item];
-      const int R = item.n_queries * G;
-      // a warp whose lane quarter lies past the tile's rows keeps every
-      // barrier of the protocol but skips the arithmetic (its P and O rows are
-      // never read out)
-      const bool act = quad * 32 < R;
+    // One work unit, in the TMEM layout of its tile shape.  Tiles of more than
+    // 64 rows use M = 128 products: row r in lane r, thread (r, h) holds keys
+    // [32h, 32h + 32) of every stage.  Tiles of at most 64 rows use M = 64
+    // products, whose rows sit in the first 16 lanes of each lane quarter (row
+    // 16q + j in lane 32q + j): thread (row, h, hw = lane / 16) holds keys
+    // [32h + 16hw, 32h + 16hw + 16), so all four quarters, and with them all four
+    // SM sub-partitions, share the exponentials of a 64-row tile; the two
+    // half-warps of a row combine their maxima with one shuffle per stage and
+    // their sums in the epilogue.  Returns false if a wait gave up.
+    auto run_segment = [&](auto m64_tag, const pa_seg& seg, const int R) -> bool {
+      constexpr bool M64 = decltype(m64_tag)::value;
+      constexpr int KT = M64 ? 16 : 32;  // keys of a stage held by this thread
+      const int r = M64 ? quad * 16 + (lane & 15) : rq;
+      const int kt0 = M64 ? 32 * h + 16 * hw : 32 * h;  // its first key in the stage
+      // a warp whose rows all lie past the tile's keeps every barrier of the
+      // protocol but skips the arithmetic (its P and O rows are never read out)
+      const bool act = (M64 ? quad * 16 : quad * 32) < R;
+      auto load_s_tile = [&](int i_) {
+        tc_fence_after();
+        const uint32_t ta = tmem + S::T_S + (i_ % kSBufs) * kMmaKT + 32 * h + lane_off;
+        if constexpr (M64) tmem_ld16x2_x16<16>(ta, sv);
+        else tmem_ld32(ta, sv);
+      };
       const int npages = (seg.n_tokens + 15) >> 4;
       float m_used = -INFINITY, l = 0.f;
       bool q_known = false;  // the next work unit has been seen in the queue
@@ -987,11 +1010,11 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         const int s = i % NST, b = i % kSBufs;
         const int np = min(4, npages - st);
         const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
-        const int kv_h = max(0, min(32, kvalid - 32 * h));  // valid keys of this half
+        const int kv_t = max(0, min(KT, kvalid - kt0));  // valid keys of this thread
         const bool last = st + 4 >= npages;
         if (!have_s) {
-          if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
-          if (act) load_s(i);
+          if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) return false;
+          if (act) load_s_tile(i);
         }
         have_s = false;
         if (act) tmem_wait_ld_into(sv);
@@ -1006,7 +1029,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           int nsi = -1;
           bool seen = seg_peek(qn, nsi);
           if (!seen && last) {
-            if (!mbar_wait_bounded(bar(S::B_QF + qn % kSegQ), (qn / kSegQ) & 1, a.timeout_ns)) { ok = false; break; }
+            if (!mbar_wait_bounded(bar(S::B_QF + qn % kSegQ), (qn / kSegQ) & 1, a.timeout_ns)) return false;
             seen = seg_peek(qn, nsi);
           }
           if (seen) {
@@ -1025,92 +1048,114 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           q_pending = false;
         }
         if (act) {
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (kv_h == 32) {
+          // the unmasked path only when every lane of the warp has all its keys
+          // (with M = 64 the two half-warps can differ): the tensor-memory
+          // stores below are .sync.aligned, so the branch must not diverge
+          const bool full = __all_sync(0xffffffffu, kv_t == KT);
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (full) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
-        } else {
+            for (int j = 0; j < KT; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
+          } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < kv_h) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
-        }
-        const float mraw = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        const float mnew = fmaxf(m_used, mraw == -INFINITY ? -INFINITY : mraw * a.qscale);
-        if (st == 0) {
-          m_used = mnew;
-        } else {
-          const bool need = mnew > m_used + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, need)) {
-            // O_h must hold every earlier p.V product before it is rescaled
-            const int j = i - 1;
-            if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
-            tc_fence_after();
-            const float alpha = need ? ex2(m_used - mnew) : 1.f;
+            for (int j = 0; j < KT; ++j)
+              if (j < kv_t) mx4[j & 3] = fmaxf(mx4[j & 3], sv[j]);
+          }
+          float mraw = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          if constexpr (M64) mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
+          const float mnew = fmaxf(m_used, mraw == -INFINITY ? -INFINITY : mraw * a.qscale);
+          if (st == 0) {
+            m_used = mnew;
+          } else {
+            const bool need = mnew > m_used + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
+              // O_h must hold every earlier p.V product before it is rescaled
+              const int j = i - 1;
+              if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) return false;
+              tc_fence_after();
+              const float alpha = need ? ex2(m_used - mnew) : 1.f;
+              if constexpr (M64) {
+                // half-warp hw rescales columns [hw D/2, (hw + 1) D/2) of the row
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              float ov[32];
-              tmem_ld32(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
-              tmem_wait_ld();
+                for (int c = 0; c < D / 64; ++c) {
+                  float ov[32];
+                  tmem_ld16x2_x32<D / 2>(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
+                  tmem_wait_ld();
 #pragma unroll
-              for (int jj = 0; jj < 32; ++jj) ov[jj] *= alpha;
-              tmem_st32(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
-            }
-            tmem_wait_st();
-            if (need) {
-              l *= alpha;
-              m_used = mnew;
+                  for (int jj = 0; jj < 32; ++jj) ov[jj] *= alpha;
+                  tmem_st16x2_x32<D / 2>(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                  float ov[32];
+                  tmem_ld32(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int jj = 0; jj < 32; ++jj) ov[jj] *= alpha;
+                  tmem_st32(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
+                }
+              }
+              tmem_wait_st();
+              if (need) {
+                l *= alpha;
+                m_used = mnew;
+              }
             }
           }
-        }
-        const float ms = m_used == -INFINITY ? 0.f : m_used;
-        // p, and its split P_hi + P_lo: P_hi keeps the top 16 bits of p (a
-        // truncated bf16, so the remainder p - P_hi is exact in fp32), P_lo is
-        // that remainder rounded to the nearest bf16 (P_hi + P_lo is within
-        // 2^-16 p of p, with no one-sided bias).
-        // Each page of 16 keys is stored as soon as it is done (P_hi words, then
-        // P_lo words), so its store overlaps the next page's exponentials.
-        float pw[32];
-        float l4[4] = {0.f, 0.f, 0.f, 0.f};
-        auto page = [&](auto pg_tag, auto full_tag) {
-          constexpr int PG = decltype(pg_tag)::value;
-          constexpr bool FULL = decltype(full_tag)::value;
+          const float ms = m_used == -INFINITY ? 0.f : m_used;
+          // p, and its split P_hi + P_lo: P_hi keeps the top 16 bits of p (a
+          // truncated bf16, so the remainder p - P_hi is exact in fp32), P_lo is
+          // that remainder rounded to the nearest bf16 (P_hi + P_lo is within
+          // 2^-16 p of p, with no one-sided bias).  A page of 16 keys is 8 P_hi
+          // words then 8 P_lo words; each is stored as soon as it is done, so
+          // its store overlaps the next page's exponentials.
+          float pw[32];
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
+          auto page = [&](auto pg_tag, auto full_tag) {
+            constexpr int PG = decltype(pg_tag)::value;
+            constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = PG * 8 + jj;
-            float p0 = ex2(fmaf(sv[2 * j], a.qscale, -ms));
-            float p1 = ex2(fmaf(sv[2 * j + 1], a.qscale, -ms));
-            if (!FULL) {
-              p0 = 2 * j < kv_h ? p0 : 0.f;
-              p1 = 2 * j + 1 < kv_h ? p1 : 0.f;
+            for (int jj = 0; jj < 8; ++jj) {
+              const int j = PG * 8 + jj;
+              float p0 = ex2(fmaf(sv[2 * j], a.qscale, -ms));
+              float p1 = ex2(fmaf(sv[2 * j + 1], a.qscale, -ms));
+              if (!FULL) {
+                p0 = 2 * j < kv_t ? p0 : 0.f;
+                p1 = 2 * j + 1 < kv_t ? p1 : 0.f;
+              }
+              l4[jj & 3] += p0 + p1;
+              const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+              const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
+              pw[PG * 16 + jj] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
+              pw[PG * 16 + jj + 8] = __uint_as_float(pack_bf16x2(r0, r1));
             }
-            l4[jj & 3] += p0 + p1;
-            const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-            const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
-            pw[PG * 16 + jj] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
-            pw[PG * 16 + jj + 8] = __uint_as_float(pack_bf16x2(r0, r1));
+            // M = 64: the two half-warps' pages go to columns [0, 16) and
+            // [16, 32) of the key half in one store
+            if constexpr (M64) tmem_st16x2_x16<16>(t_s, pw);
+            else tmem_st16<PG * 16>(t_s + PG * 16, pw);
+          };
+          using I0 = std::integral_constant<int, 0>;
+          using I1 = std::integral_constant<int, 1>;
+          if (full) {
+            page(I0{}, std::true_type{});
+            if constexpr (!M64) page(I1{}, std::true_type{});
+          } else {
+            page(I0{}, std::false_type{});
+            if constexpr (!M64) page(I1{}, std::false_type{});
           }
-          tmem_st16<PG * 16>(t_s + PG * 16, pw);
-        };
-        using I0 = std::integral_constant<int, 0>;
-        using I1 = std::integral_constant<int, 1>;
-        if (kv_h == 32) {
-          page(I0{}, std::true_type{});
-          page(I1{}, std::true_type{});
-        } else {
-          page(I0{}, std::false_type{});
-          page(I1{}, std::false_type{});
-        }
-        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-        if (!last && __all_sync(0xffffffffu, mbar_test_wait(bar(S::B_SFULL + (i + 1) % kSBufs), ((i + 1) / kSBufs) & 1))) {
-          load_s(i + 1);
-          have_s = true;
-        }
+          l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+          if (!last &&
+              __all_sync(0xffffffffu, mbar_test_wait(bar(S::B_SFULL + (i + 1) % kSBufs), ((i + 1) / kSBufs) & 1))) {
+            load_s_tile(i + 1);
+            have_s = true;
+          }
         }  // act
         if (kvalid < np * 16) {
           // V rows past the last valid key may hold NaN; p = 0 there but 0 * NaN
           // would still poison the product, so those rows are zeroed (once the
           // V tile has landed)
-          if (!warp_wait(bar(S::B_VFULL + s), (i / NST) & 1, a.timeout_ns)) { ok = false; break; }
+          if (!warp_wait(bar(S::B_VFULL + s), (i / NST) & 1, a.timeout_ns)) return false;
           uint8_t* vst = smem + S::OFF_V + s * S::KSTAGE;
           const int nz = np * 16 - kvalid;
           for (int idx = tid; idx < nz * S::HALVES * 8; idx += kSmaxThreads) {
@@ -1124,13 +1169,14 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         tc_fence_before();
         mbar_arrive(bar(S::B_PFULL + b));
       }
-      if (!ok) break;
       // ---- epilogue: combine the two key halves of each row; this thread
-      // writes head dims [h * D/2, (h + 1) * D/2) of the row's partial result
+      // writes head dims [h D/2, (h + 1) D/2) of the row's partial result
+      // (M = 64: [h D/2 + hw D/4, h D/2 + (hw + 1) D/4))
       {
         const int j = i - 1;
-        if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) { ok = false; break; }
+        if (!warp_wait(bar(S::B_PV + j % kSBufs), (j / kSBufs) & 1, a.timeout_ns)) return false;
       }
+      if constexpr (M64) l += __shfl_xor_sync(0xffffffffu, l, 16);
       tc_fence_after();
       if (act) {
         const uint32_t mine[2] = {__float_as_uint(m_used), __float_as_uint(l)};
@@ -1139,44 +1185,68 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       }
       tc_fence_before();
       mbar_arrive(bar(S::B_XCH + quad));
-      if (!warp_wait(bar(S::B_XCH + quad), segord & 1, a.timeout_ns)) { ok = false; break; }
+      if (!warp_wait(bar(S::B_XCH + quad), segord & 1, a.timeout_ns)) return false;
       tc_fence_after();
       if (act) {
-      uint32_t other[2];
-      tmem_ld2(tmem + S::T_X + 2 * (1 - h) + lane_off, other);
-      tmem_wait_ld();
-      const float m0 = h == 0 ? m_used : __uint_as_float(other[0]), l0 = h == 0 ? l : __uint_as_float(other[1]);
-      const float m1 = h == 0 ? __uint_as_float(other[0]) : m_used, l1 = h == 0 ? __uint_as_float(other[1]) : l;
-      const float mm = fmaxf(m0, m1);
-      const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
-      const float L = w0 * l0 + w1 * l1;
-      const float c0 = w0 / L, c1 = w1 / L;
-      float* dst = nullptr;
-      if (r < R) {
-        const int prow = a.seg_prows[seg.prow + r / G];
-        dst = a.partial_o + ((size_t)prow * G + (r % G)) * D + h * (D / 2);
-        if (h == 0) a.partial_lse[(size_t)prow * G + (r % G)] = (mm + lg2(L)) * kLn2;
-      }
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const uint32_t col = h * (D / 2) + 32 * cc;
-        float o0[32], o1[32];
-        tmem_ld32(tmem + S::T_O + col + lane_off, o0);
-        tmem_ld32(tmem + S::T_O + D + col + lane_off, o1);
+        uint32_t other[2];
+        tmem_ld2(tmem + S::T_X + 2 * (1 - h) + lane_off, other);
         tmem_wait_ld();
-        if (dst) {
+        const float m0 = h == 0 ? m_used : __uint_as_float(other[0]), l0 = h == 0 ? l : __uint_as_float(other[1]);
+        const float m1 = h == 0 ? __uint_as_float(other[0]) : m_used, l1 = h == 0 ? __uint_as_float(other[1]) : l;
+        const float mm = fmaxf(m0, m1);
+        const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
+        const float L = w0 * l0 + w1 * l1;
+        const float c0 = w0 / L, c1 = w1 / L;
+        constexpr int NCOL = M64 ? D / 4 : D / 2;  // dims written by this thread
+        float* dst = nullptr;
+        if (r < R) {
+          const int prow = a.seg_prows[seg.prow + r / G];
+          dst = a.partial_o + ((size_t)prow * G + (r % G)) * D + h * (D / 2) + (M64 ? hw * NCOL : 0);
+          if (h == 0 && (!M64 || hw == 0)) a.partial_lse[(size_t)prow * G + (r % G)] = (mm + lg2(L)) * kLn2;
+        }
+        auto emit = [&](const float (&o0)[32], const float (&o1)[32], int n, float* d) {
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
+            if (4 * q4 >= n) break;
             float4 v;
             v.x = c0 * o0[4 * q4] + (w1 > 0.f ? c1 * o1[4 * q4] : 0.f);
             v.y = c0 * o0[4 * q4 + 1] + (w1 > 0.f ? c1 * o1[4 * q4 + 1] : 0.f);
             v.z = c0 * o0[4 * q4 + 2] + (w1 > 0.f ? c1 * o1[4 * q4 + 2] : 0.f);
             v.w = c0 * o0[4 * q4 + 3] + (w1 > 0.f ? c1 * o1[4 * q4 + 3] : 0.f);
-            *reinterpret_cast<float4*>(dst + 32 * cc + 4 * q4) = v;
+            *reinterpret_cast<float4*>(d + 4 * q4) = v;
+          }
+        };
+        if constexpr (M64) {
+          float o0[32], o1[32];
+          const uint32_t col = h * (D / 2);
+          if constexpr (NCOL == 32) {
+            tmem_ld16x2_x32<NCOL>(tmem + S::T_O + col + lane_off, o0);
+            tmem_ld16x2_x32<NCOL>(tmem + S::T_O + D + col + lane_off, o1);
+          } else {
+            tmem_ld16x2_x16<NCOL>(tmem + S::T_O + col + lane_off, o0);
+            tmem_ld16x2_x16<NCOL>(tmem + S::T_O + D + col + lane_off, o1);
+          }
+          tmem_wait_ld();
+          if (dst) emit(o0, o1, NCOL, dst);
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < D / 64; ++cc) {
+            const uint32_t col = h * (D / 2) + 32 * cc;
+            float o0[32], o1[32];
+            tmem_ld32(tmem + S::T_O + col + lane_off, o0);
+            tmem_ld32(tmem + S::T_O + D + col + lane_off, o1);
+            tmem_wait_ld();
+            if (dst) emit(o0, o1, 32, dst + 32 * cc);
           }
         }
-      }
       }  // act
+      return true;
+    };
+    while (si >= 0 && ok) {
+      const pa_seg seg = a.segs[si];
+      const int R = a.items[seg.item].n_queries * G;
+      ok = R <= 64 ? run_segment(std::true_type{}, seg, R) : run_segment(std::false_type{}, seg, R);
+      if (!ok) break;
       tc_fence_before();
       mbar_arrive(bar(S::B_OFREE));
       // these rows' pairs are merged by their last SIMT writer or the tail merge launch
