@@ -626,13 +626,15 @@ constexpr int kSegQConsumers = 11;   // V producer, S issuer, p.V issuer, 8 soft
 constexpr uint32_t kTmemCols = 512;  // the whole tensor memory of the SM (one CTA per SM)
 constexpr float kRescaleThreshold = kRescaleLog2;
 
-template <int D>
+// QR: rows of a Q buffer, 128, or 64 when no tile of the launch has more
+// (the smaller Q buffers leave room for a deeper K/V ring at D = 128)
+template <int D, int QR>
 struct MmaShape {
   static constexpr int HALVES = D / 64;
   static constexpr int KBLK = kMmaKT * 128;        // one 64-key x 64-dim swizzled block (8 KB)
   static constexpr int KSTAGE = HALVES * KBLK;     // K (or V) of one stage
   static constexpr int STAGE = 2 * KSTAGE;         // K and V of one stage
-  static constexpr int QBLK = 128 * 128;           // 128 rows x 64 dims (16 KB)
+  static constexpr int QBLK = QR * 128;            // QR rows x 64 dims
   static constexpr int QBUF = HALVES * QBLK;       // the Q rows of one segment
   static constexpr int FIXED = 2 * QBUF + 1024 + 1024;  // two Q buffers, barriers and queue, alignment slack
   static constexpr int NST_FIT = (kSmemMax - FIXED) / STAGE;
@@ -661,10 +663,10 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int G>
+template <int D, int G, int QR>
 __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk, const CUtensorMap* tv,
                                          uint8_t* smem_raw) {
-  using S = MmaShape<D>;
+  using S = MmaShape<D, QR>;
   constexpr int NST = S::NST;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -847,6 +849,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         if (si < 0) break;
         const pa_seg seg = a.segs[si];
         const bool m64 = a.items[seg.item].n_queries * G <= 64;
+        if (a.debug_checks && QR == 64 && !m64) record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -8);
         const uint32_t idesc_s = m64 ? idesc_s64 : idesc_s128, idesc_o = m64 ? idesc_o64 : idesc_o128;
         const int npages = (seg.n_tokens + 15) >> 4;
         for (int st = 0; st < npages; st += 4, ++i) {
@@ -923,7 +926,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     auto q_src = [&](int si) -> const uint16_t* {
       const pa_seg seg = a.segs[si];
       const pa_item item = a.items[seg.item];
-      if (rq >= item.n_queries * G) return nullptr;
+      if (rq >= item.n_queries * G || rq >= QR) return nullptr;
       int b = a.queries[item.query_off + rq / G];
       if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
         record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
@@ -942,7 +945,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       for (int cc = 0; cc < QCH; ++cc) {
         const int c = h * QCH + cc;
         const uint4 v = src ? *reinterpret_cast<const uint4*>(src + 8 * c) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(q_dst(0, c)) = v;
+        if (rq < QR) *reinterpret_cast<uint4*>(q_dst(0, c)) = v;
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(S::B_QFULL));
@@ -952,10 +955,12 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     // buffer's barrier a stage later
     auto prefetch_q = [&](int si, int qbuf) {
       const uint16_t* src = q_src(si);
+      if (rq < QR) {
 #pragma unroll
-      for (int cc = 0; cc < QCH; ++cc) {
-        const int c = h * QCH + cc;
-        cp_async16(smem_u32(q_dst(qbuf, c)), src ? src + 8 * c : a.q, src ? 16u : 0u);
+        for (int cc = 0; cc < QCH; ++cc) {
+          const int c = h * QCH + cc;
+          cp_async16(smem_u32(q_dst(qbuf, c)), src ? src + 8 * c : a.q, src ? 16u : 0u);
+        }
       }
       cp_async_commit();
     };
@@ -1266,12 +1271,12 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
 
 // Tensor-core class: CTA c runs MMA CTA list c.  It lets the CUDA-core launch
 // that follows it in the stream start at once (programmatic dependent launch).
-template <int D, int G>
+template <int D, int G, int QR>
 __global__ void __launch_bounds__(kMmaThreads, 1)
     mma_fwd_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
   griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem[];
-  mma_role<D, G>(a, &tk, &tv, smem);
+  mma_role<D, G, QR>(a, &tk, &tv, smem);
 }
 
 // CUDA-core class: block c runs SIMT warps [8c, 8c + 8).  When it runs beside
@@ -1420,14 +1425,22 @@ int set_smem_attr(K kernel, bool (&done)[64]) {
 // two occupy disjoint SMs (one CTA per SM each, n_mma + n_simt <= SMs).
 template <int D, int G>
 int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
-  static bool attr_mma[64] = {}, attr_simt[64] = {};
+  static bool attr_mma[64] = {}, attr_mma64[64] = {}, attr_simt[64] = {};
   const int n_simt_ctas = (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
   const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
   const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
   if (a.n_mma_ctas > 0) {
-    auto k = mma_fwd_kernel<D, G>;
-    if (int e = set_smem_attr(k, attr_mma)) return e;
-    k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D>::SMEM, st>>>(a, *tk, *tv);
+    // 64-row Q buffers buy a deeper K/V ring only at D = 128
+    constexpr bool kQ64 = MmaShape<D, 64>::NST > MmaShape<D, 128>::NST;
+    if (kQ64 && p.mma_max_rows <= 64) {
+      auto k = mma_fwd_kernel<D, G, kQ64 ? 64 : 128>;
+      if (int e = set_smem_attr(k, attr_mma64)) return e;
+      k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D, kQ64 ? 64 : 128>::SMEM, st>>>(a, *tk, *tv);
+    } else {
+      auto k = mma_fwd_kernel<D, G, 128>;
+      if (int e = set_smem_attr(k, attr_mma)) return e;
+      k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D, 128>::SMEM, st>>>(a, *tk, *tv);
+    }
     if (cudaError_t e = cudaGetLastError()) return (int)e;
   }
   if (n_simt_ctas > 0) {

@@ -306,7 +306,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   };
   const int64_t max_chunk_pages = cfg->max_chunk_tokens > 0 ? std::max(1, cfg->max_chunk_tokens / P) : 0;
   const double tile_bytes = 2.0 * 16 * D * 2;
-  int64_t simt_pages = 0, mma_pages = 0, mma_seg_total = 0;
+  int64_t simt_pages = 0, mma_pages = 0;
   double mma_cost = 0;  // SM-us
   for (const auto& it : items) {
     const int64_t np = ceil_div(it.n_tokens, P) * Hkv;
@@ -316,7 +316,6 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
       simt_pages += np + kSimtSegPages * Hkv;
     } else {
       mma_pages += np;
-      mma_seg_total += mma_seg_pages(it) * Hkv;
       // a tcgen05.mma costs the same for any rows up to 128, so a tile costs 128 rows
       const double rows = kMmaRowsPerCta;
       const double flops = 16.0 * rows * D * 6;  // per page: S (2rD per key) + split-p P.V (2 x 2rD per key)
@@ -352,34 +351,52 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   warp_segs.assign(1, 0);
   mma_cta_segs.assign(1, 0);
   if (mma_pages > 0) {
-    // Tensor-core work units: every (item, kv head) run cut into equal chunks
-    // of at most `chunk` pages, about kMmaChunksPerCta per CTA.  The CTAs take
-    // the chunks one after another from a counter in the image (the K producer
+    // Tensor-core work units, cut for guided self-scheduling: the CTAs take
+    // the units one after another from a counter in the image (the K producer
     // of each CTA fetches the next one), longest first, so an SM that runs
-    // faster takes more of them: the same stage of the same work was measured
-    // to take from 1.3k to 2.4k cycles on different SMs of one launch.
-    // A chunk is at least kMmaMinChunkPages long: each one pays an epilogue
-    // (≈3 us, during which its CTA's tensor pipe waits), so short chunks cost
-    // more than the balance they buy.  When that leaves about one chunk per
-    // CTA, each chunk gets a CTA of its own.
-    const int kMmaChunksPerCta = 2, kMmaMinChunkPages = 64;
-    int64_t chunk = ceil_div(mma_pages + mma_seg_total, (int64_t)n_mma * kMmaChunksPerCta);
-    if (chunk < kMmaMinChunkPages) chunk = kMmaMinChunkPages;
-    if (max_chunk_pages) chunk = std::min(chunk, max_chunk_pages);
+    // faster takes more of them (the same stage of the same work was measured
+    // to take from 0.79 to 1.17 us on different SMs of one launch).  Each cut
+    // takes about R / (kGuide * CTAs) pages, R being the tensor-core work not
+    // yet cut, from the run with the most pages left: the units shrink as the
+    // queue drains, so the last ones, whose end on a slow SM decides when the
+    // launch ends, are short, while most of the work still runs in long units.
+    // A unit is at least kMmaMinChunkPages long: each one pays an epilogue
+    // (about 3 us, during which its CTA's tensor pipe waits) and one more
+    // partial row per request and head.  When that leaves about one unit per
+    // CTA, each unit gets a CTA of its own.
+    const int kMmaMinChunkPages = 64;
+    const double kGuide = 2.0;
+    struct Run {
+      int64_t rem;  // pages not yet cut
+      int item, g, pb;
+    };
+    const auto fewer = [](const Run& x, const Run& y) { return x.rem < y.rem; };  // max-heap on rem
+    std::vector<Run> runs;
+    int64_t R = 0;
     for (size_t i = 0; i < items.size(); ++i) {
       const ItemRec& it = items[i];
       if (it.simt) continue;
-      const int npages = (int)ceil_div(it.n_tokens, P);
-      const int n = (int)ceil_div(npages, chunk);
-      for (int g = 0; g < Hkv; ++g) {
-        int pb = 0;
-        for (int c = 0; c < n; ++c) {
-          const int take = npages / n + (c < npages % n ? 1 : 0);
-          const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
-          mma_segs.push_back({(int)i, g, pb, tok, -1, queries[it.query_off]});
-          pb += take;
-        }
-      }
+      const int64_t npages = ceil_div(it.n_tokens, P);
+      for (int g = 0; g < Hkv; ++g) runs.push_back({npages, (int)i, g, 0});
+      R += npages * Hkv;
+    }
+    std::make_heap(runs.begin(), runs.end(), fewer);
+    while (!runs.empty()) {
+      std::pop_heap(runs.begin(), runs.end(), fewer);
+      Run& r = runs.back();
+      int64_t t = std::max<int64_t>(kMmaMinChunkPages, (int64_t)std::ceil((double)R / (kGuide * n_mma)));
+      if (max_chunk_pages) t = std::min(t, max_chunk_pages);
+      int64_t cut = std::min(t, r.rem);
+      // no sliver of less than half a minimum unit is left behind
+      if (!max_chunk_pages && r.rem - cut < kMmaMinChunkPages / 2) cut = r.rem;
+      const ItemRec& it = items[r.item];
+      const int tok = (int)(std::min<int64_t>(it.n_tokens, (r.pb + cut) * P) - (int64_t)r.pb * P);
+      mma_segs.push_back({r.item, r.g, r.pb, tok, -1, queries[it.query_off]});
+      r.pb += (int)cut;
+      r.rem -= cut;
+      R -= cut;
+      if (r.rem > 0) std::push_heap(runs.begin(), runs.end(), fewer);
+      else runs.pop_back();
     }
     std::stable_sort(mma_segs.begin(), mma_segs.end(),
                      [](const SegRec& x, const SegRec& y) { return x.n_tokens > y.n_tokens; });
@@ -500,6 +517,9 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   h.num_segments = h.num_segments_simt + h.num_segments_mma;
   h.simt_warps = (int32_t)warp_segs.size() - 1;
   h.mma_ctas = mma_segs.empty() ? 0 : n_mma;
+  plan->mma_max_rows = 0;
+  for (const auto& s : mma_segs)
+    plan->mma_max_rows = std::max(plan->mma_max_rows, std::min(kMmaRowsPerCta, items[s.item].n_queries * G));
   h.num_partial_rows = num_prows;
   h.num_tail_pairs = (int32_t)tail_pairs.size();
   uint64_t off = align256(sizeof(pa_image_header));

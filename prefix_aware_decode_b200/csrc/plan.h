@@ -47,6 +47,9 @@ struct pa_plan {
   int32_t wait_timeout_us = 0;
   pa_plan_stats stats{};
   pa_image_header hdr{};
+  // rows of the largest tensor-core tile (n_queries * G, at most 128): when
+  // it is at most 64 the launch holds 64-row Q buffers and a deeper K/V ring
+  int mma_max_rows = 0;
   HostBuf image;  // exactly what pa_plan_upload sends (image.size bytes)
   ~pa_plan() { hostbuf_release(image); }
   // cached TMA descriptors (encoded for the last pool pointers seen)

@@ -208,12 +208,12 @@ def tensor_core_units(w, flags=0):
 
 
 @pytest.mark.parametrize("config", [1, 2, 3, 5])
-def test_tensor_core_work_units_are_chunks_of_at_least_16_pages(config):
+def test_tensor_core_work_units_cover_each_run_in_pieces_of_at_least_32_pages(config):
     # at most one tensor-core CTA per 16 pages of tensor-core work (a small
     # shared prefix, config 1: 16 pages x 2 kv heads, is not spread over many
     # CTAs that each pay the segment's fixed cost); every (item, kv head) run
-    # is cut into equal chunks of at least 16 pages (or the whole run), and
-    # there are at least as many chunks as CTAs
+    # is covered by consecutive pieces of at least 32 pages (or the whole run),
+    # and there are at least as many pieces as CTAs
     w = wl.make_config(config, with_values=False)
     # config 1's small prefix is inlined by the profit model; shared on purpose here
     h, img, pages, runs = tensor_core_units(w, flags=pad.PA_PLAN_ALWAYS_SHARE if config == 1 else 0)
@@ -222,22 +222,33 @@ def test_tensor_core_work_units_are_chunks_of_at_least_16_pages(config):
     if config == 1:
         assert h.mma_ctas <= 2
     ns = h.num_segments_simt
-    for ids in runs.values():
-        sizes = [pages[i - ns] for i in ids]
-        total = sum(sizes)
-        assert max(sizes) - min(sizes) <= 1
-        assert len(sizes) == 1 or min(sizes) >= min(16, total)
+    for (item, g), ids in runs.items():
+        segs = sorted((int(img.segs[i][2]), pages[i - ns]) for i in ids)  # (page_begin, pages)
+        assert segs[0][0] == 0
+        for (b0, n0), (b1, _) in zip(segs, segs[1:]):
+            assert b1 == b0 + n0
+        total = sum(n for _, n in segs)
+        assert total == -(-int(img.items[item][1]) // 16)
+        assert len(segs) == 1 or min(n for _, n in segs) >= 32
 
 
-def test_tensor_core_work_units_longest_first_about_two_per_cta():
-    # config 3: root runs (256 pages per kv head and 128-row tile) and branch
-    # runs (64 pages): the CTAs take the units longest first from a shared
-    # counter, so a CTA that runs faster takes more of them; about two units
-    # per CTA (each unit pays an epilogue, so not many more)
-    w = wl.make_config(3, with_values=False)
+@pytest.mark.parametrize("config", [3, 5])
+def test_tensor_core_work_units_longest_first_and_short_at_the_end(config):
+    # guided self-scheduling: the CTAs take the units longest first from a
+    # shared counter, so a CTA that runs faster takes more of them; the units
+    # shrink as the queue drains, each cut about a 2 x CTAs-th of the work not
+    # yet cut, so the last units, which decide when the launch ends on a slow
+    # SM, are short, while most of the work still runs in long units (config 5:
+    # 256 runs of 2k-8k pages over 147 CTAs; config 3: 128-row root runs of 256
+    # pages and 64-page branch runs)
+    w = wl.make_config(config, with_values=False)
     h, img, pages, runs = tensor_core_units(w)
+    W, n = sum(pages), h.mma_ctas
     assert pages == sorted(pages, reverse=True)
-    assert h.mma_ctas <= len(pages) <= 4 * h.mma_ctas + len(runs)
+    assert pages[0] <= -(-W // (2 * n)) + 64
+    assert max(pages[-n:]) <= 64 and sum(pages[-n:]) <= W // 8
+    # about 2 ln(W / (2 n 64)) + 2 units per CTA, not many more
+    assert len(pages) <= n * (2 * np.log(max(2.0, W / (2 * n * 64))) + 4) + len(runs)
 
 
 # ------------------------------------------------------------- decode steps
