@@ -887,14 +887,19 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
             tc_fence_after();
             const uint32_t v_base = smem_u32(smem + S::OFF_V + s * S::KSTAGE);
             const int np = min(4, npages - st);
+            // 64-row launches: the whole stage goes to the accumulator of the
+            // group that owns it (stage j of the unit: group j % 2), whose first
+            // stage in the unit (j < 2) overwrites it
+            const int jst = st >> 2;
             for (int c = 0; c < np; ++c) {
               // 16-key chunk c (page c of the stage) belongs to key half c / 2.  P
               // chunk c: P_hi in columns [16c, 16c + 8), P_lo in [16c + 8, 16c + 16)
               // of the buffer; V: MN-major (64-dim atoms at +KBLK, 8-key groups at +1 KB)
-              const uint32_t d_o = tmem + S::T_O + (c >> 1) * D;
+              const uint32_t d_o = tmem + S::T_O + (QR == 64 ? (jst & 1) : (c >> 1)) * D;
+              const bool init = QR == 64 ? (jst < 2 && c == 0) : (first && (c & 1) == 0);
               const uint32_t a_p = tmem + S::T_S + b * kMmaKT + 16 * c;
               const uint64_t bd = umma_sdesc_sw128(v_base + c * 2048, S::KBLK >> 4, 64);
-              umma_bf16_ts(d_o, a_p, bd, idesc_o, (first && (c & 1) == 0) ? 0u : 1u);
+              umma_bf16_ts(d_o, a_p, bd, idesc_o, init ? 0u : 1u);
               umma_bf16_ts(d_o, a_p + 8, bd, idesc_o, 1u);
             }
             umma_commit(bar(S::B_PV + b));
@@ -1247,10 +1252,231 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       }  // act
       return true;
     };
+    // 64-row launches (QR = 64): the two warp groups take alternate stages of a
+    // work unit instead of alternate key halves of every stage.  Group g (warps
+    // 2-5: g = 0, 6-9: g = 1) owns stages j = g, g + 2, ... of the unit, with
+    // its own running maximum, sum and accumulator O_g; thread (row, hw = lane /
+    // 16) holds keys [32 hw, 32 hw + 32) of an owned stage, the two half-warps
+    // of a row combining their maxima with one shuffle.  Each group then has
+    // two stage periods for the chain S load -> exponentials -> P store of
+    // one stage, so the chains of two stages overlap.  A group arrives on the
+    // P barrier of a stage it does not own once S of that stage is there (so
+    // the barrier's previous phase is complete).  Returns false if a wait
+    // gave up.
+    auto run_segment_il = [&](auto, const pa_seg& seg, const int R) -> bool {
+      constexpr int KT = 32;
+      const int r = quad * 16 + (lane & 15);
+      const int kt0 = 32 * hw;
+      const bool act = quad * 16 < R;
+      const int npages = (seg.n_tokens + 15) >> 4;
+      float m_used = -INFINITY, l = 0.f;
+      bool mine_seen = false;  // this group has run a stage of the unit
+      bool q_known = false;
+      int q_at = 0;
+      for (int st = 0, j = 0; st < npages; st += 4, ++i, ++j) {
+        const int s = i % NST, b = i % kSBufs;
+        const int np = min(4, npages - st);
+        const int kvalid = min(kMmaKT, seg.n_tokens - st * 16);
+        const bool last = st + 4 >= npages;
+        const bool mine = (j & 1) == h;
+        // next work unit's Q rows (as in run_segment)
+        if (!q_known) {
+          int nsi = -1;
+          bool seen = seg_peek(qn, nsi);
+          if (!seen && last) {
+            if (!mbar_wait_bounded(bar(S::B_QF + qn % kSegQ), (qn / kSegQ) & 1, a.timeout_ns)) return false;
+            seen = seg_peek(qn, nsi);
+          }
+          if (seen) {
+            q_known = true;
+            q_at = st;
+            if (nsi >= 0) {
+              prefetch_q(nsi, (segord + 1) & 1);
+              q_pending = true;
+            }
+          }
+        }
+        if (q_pending && (st > q_at || last)) {
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(bar(S::B_QFULL + ((segord + 1) & 1)));
+          q_pending = false;
+        }
+        if (!mine) {
+          // S(i) issued means p.V(i - 3), and with it the previous phase of
+          // this P barrier, is complete; only then is the arrival counted for
+          // stage i
+          if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) return false;
+          mbar_arrive(bar(S::B_PFULL + b));
+          continue;
+        }
+        if (!warp_wait(bar(S::B_SFULL + b), (i / kSBufs) & 1, a.timeout_ns)) return false;
+        const uint32_t t_s = tmem + S::T_S + b * kMmaKT + lane_off;
+        if (act) {
+          tc_fence_after();
+          tmem_ld16x2_x32<32>(t_s, sv);
+          tmem_wait_ld_into(sv);
+          const int kv_t = max(0, min(KT, kvalid - kt0));
+          const bool full = __all_sync(0xffffffffu, kv_t == KT);
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (full) {
+#pragma unroll
+            for (int jj = 0; jj < KT; ++jj) mx4[jj & 3] = fmaxf(mx4[jj & 3], sv[jj]);
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < KT; ++jj)
+              if (jj < kv_t) mx4[jj & 3] = fmaxf(mx4[jj & 3], sv[jj]);
+          }
+          float mraw = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
+          const float mnew = fmaxf(m_used, mraw == -INFINITY ? -INFINITY : mraw * a.qscale);
+          if (!mine_seen) {
+            m_used = mnew;
+          } else {
+            const bool need = mnew > m_used + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
+              // O_g must hold every earlier p.V product of the group (stage i - 2)
+              const int jp = i - 2;
+              if (!warp_wait(bar(S::B_PV + jp % kSBufs), (jp / kSBufs) & 1, a.timeout_ns)) return false;
+              tc_fence_after();
+              const float alpha = need ? ex2(m_used - mnew) : 1.f;
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c) {
+                float ov[32];
+                tmem_ld16x2_x32<D / 2>(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) ov[jj] *= alpha;
+                tmem_st16x2_x32<D / 2>(tmem + S::T_O + h * D + lane_off + 32 * c, ov);
+              }
+              tmem_wait_st();
+              if (need) {
+                l *= alpha;
+                m_used = mnew;
+              }
+            }
+          }
+          const float ms = m_used == -INFINITY ? 0.f : m_used;
+          // P_hi / P_lo of the thread's two 16-key chunks (2 hw and 2 hw + 1):
+          // pw[16 c' + 0..7] = P_hi words, pw[16 c' + 8..15] = P_lo words
+          float pw[32];
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
+          auto chunk = [&](auto pg_tag, auto full_tag) {
+            constexpr int PG = decltype(pg_tag)::value;
+            constexpr bool FULL = decltype(full_tag)::value;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              const int k2 = PG * 8 + jj;
+              float p0 = ex2(fmaf(sv[2 * k2], a.qscale, -ms));
+              float p1 = ex2(fmaf(sv[2 * k2 + 1], a.qscale, -ms));
+              if (!FULL) {
+                p0 = 2 * k2 < kv_t ? p0 : 0.f;
+                p1 = 2 * k2 + 1 < kv_t ? p1 : 0.f;
+              }
+              l4[jj & 3] += p0 + p1;
+              const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+              const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
+              pw[PG * 16 + jj] = __uint_as_float(__byte_perm(u0, u1, 0x7632));
+              pw[PG * 16 + jj + 8] = __uint_as_float(pack_bf16x2(r0, r1));
+            }
+          };
+          using I0 = std::integral_constant<int, 0>;
+          using I1 = std::integral_constant<int, 1>;
+          if (full) {
+            chunk(I0{}, std::true_type{});
+            chunk(I1{}, std::true_type{});
+          } else {
+            chunk(I0{}, std::false_type{});
+            chunk(I1{}, std::false_type{});
+          }
+          // lanes 0-15: columns [0, 32) of the stage, lanes 16-31: [32, 64)
+          tmem_st16x2_x32<32>(t_s, pw);
+          l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        }  // act
+        mine_seen = true;
+        if (kvalid < np * 16) {
+          // V rows past the last valid key may hold NaN (see run_segment);
+          // zeroed by the owning group once the V tile has landed
+          if (!warp_wait(bar(S::B_VFULL + s), (i / NST) & 1, a.timeout_ns)) return false;
+          uint8_t* vst = smem + S::OFF_V + s * S::KSTAGE;
+          const int nz = np * 16 - kvalid;
+          const int gt = tid & 127;  // thread within the group
+          for (int idx = gt; idx < nz * S::HALVES * 8; idx += 128) {
+            const int row = kvalid + idx / (S::HALVES * 8);
+            const int hh = (idx >> 3) % S::HALVES, c = idx & 7;
+            *reinterpret_cast<uint4*>(vst + hh * S::KBLK + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(S::B_PFULL + b));
+      }
+      // ---- epilogue: combine the two groups' partial results of each row;
+      // thread (row, g, hw) writes head dims [g D/2 + hw D/4, g D/2 + (hw + 1) D/4)
+      {
+        const int jl = i - 1;
+        if (!warp_wait(bar(S::B_PV + jl % kSBufs), (jl / kSBufs) & 1, a.timeout_ns)) return false;
+      }
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      tc_fence_after();
+      if (act) {
+        const uint32_t mine2[2] = {__float_as_uint(m_used), __float_as_uint(l)};
+        tmem_st2(tmem + S::T_X + 2 * h + lane_off, mine2);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(S::B_XCH + quad));
+      if (!warp_wait(bar(S::B_XCH + quad), segord & 1, a.timeout_ns)) return false;
+      tc_fence_after();
+      if (act) {
+        uint32_t other[2];
+        tmem_ld2(tmem + S::T_X + 2 * (1 - h) + lane_off, other);
+        tmem_wait_ld();
+        const float m0 = h == 0 ? m_used : __uint_as_float(other[0]), l0 = h == 0 ? l : __uint_as_float(other[1]);
+        const float m1 = h == 0 ? __uint_as_float(other[0]) : m_used, l1 = h == 0 ? __uint_as_float(other[1]) : l;
+        const float mm = fmaxf(m0, m1);
+        const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
+        const float L = w0 * l0 + w1 * l1;
+        const float c0 = w0 / L, c1 = w1 / L;
+        constexpr int NCOL = D / 4;
+        float* dst = nullptr;
+        if (r < R) {
+          const int prow = a.seg_prows[seg.prow + r / G];
+          dst = a.partial_o + ((size_t)prow * G + (r % G)) * D + h * (D / 2) + hw * NCOL;
+          if (h == 0 && hw == 0) a.partial_lse[(size_t)prow * G + (r % G)] = (mm + lg2(L)) * kLn2;
+        }
+        float o0[32], o1[32];
+        const uint32_t col = h * (D / 2);
+        if constexpr (NCOL == 32) {
+          tmem_ld16x2_x32<NCOL>(tmem + S::T_O + col + lane_off, o0);
+          tmem_ld16x2_x32<NCOL>(tmem + S::T_O + D + col + lane_off, o1);
+        } else {
+          tmem_ld16x2_x16<NCOL>(tmem + S::T_O + col + lane_off, o0);
+          tmem_ld16x2_x16<NCOL>(tmem + S::T_O + D + col + lane_off, o1);
+        }
+        tmem_wait_ld();
+        if (dst) {
+          // a group that ran no stage of the unit (a one-stage unit) left its
+          // accumulator unwritten: its weight is 0 and its values are not read
+#pragma unroll
+          for (int q4 = 0; q4 < NCOL / 4; ++q4) {
+            float4 v;
+            v.x = (w0 > 0.f ? c0 * o0[4 * q4] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4] : 0.f);
+            v.y = (w0 > 0.f ? c0 * o0[4 * q4 + 1] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4 + 1] : 0.f);
+            v.z = (w0 > 0.f ? c0 * o0[4 * q4 + 2] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4 + 2] : 0.f);
+            v.w = (w0 > 0.f ? c0 * o0[4 * q4 + 3] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4 + 3] : 0.f);
+            *reinterpret_cast<float4*>(dst + 4 * q4) = v;
+          }
+        }
+      }  // act
+      return true;
+    };
     while (si >= 0 && ok) {
       const pa_seg seg = a.segs[si];
       const int R = a.items[seg.item].n_queries * G;
-      ok = R <= 64 ? run_segment(std::true_type{}, seg, R) : run_segment(std::false_type{}, seg, R);
+      if constexpr (QR == 64) ok = run_segment_il(0, seg, R);
+      else ok = R <= 64 ? run_segment(std::true_type{}, seg, R) : run_segment(std::false_type{}, seg, R);
       if (!ok) break;
       tc_fence_before();
       mbar_arrive(bar(S::B_OFREE));
@@ -1430,12 +1656,12 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
   const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
   const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
   if (a.n_mma_ctas > 0) {
-    // 64-row Q buffers buy a deeper K/V ring only at D = 128
-    constexpr bool kQ64 = MmaShape<D, 64>::NST > MmaShape<D, 128>::NST;
-    if (kQ64 && p.mma_max_rows <= 64) {
-      auto k = mma_fwd_kernel<D, G, kQ64 ? 64 : 128>;
+    // launches whose tiles all have at most 64 rows: 64-row Q buffers (a
+    // deeper K/V ring at D = 128) and the stage-interleaved softmax
+    if (p.mma_max_rows <= 64) {
+      auto k = mma_fwd_kernel<D, G, 64>;
       if (int e = set_smem_attr(k, attr_mma64)) return e;
-      k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D, kQ64 ? 64 : 128>::SMEM, st>>>(a, *tk, *tv);
+      k<<<a.n_mma_ctas, kMmaThreads, MmaShape<D, 64>::SMEM, st>>>(a, *tk, *tv);
     } else {
       auto k = mma_fwd_kernel<D, G, 128>;
       if (int e = set_smem_attr(k, attr_mma)) return e;
