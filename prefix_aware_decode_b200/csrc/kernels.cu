@@ -1214,16 +1214,15 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           dst = a.partial_o + ((size_t)prow * G + (r % G)) * D + h * (D / 2) + (M64 ? hw * NCOL : 0);
           if (h == 0 && (!M64 || hw == 0)) a.partial_lse[(size_t)prow * G + (r % G)] = (mm + lg2(L)) * kLn2;
         }
+        // n dims from column 0 of o0 / o1 to d (32-byte aligned), 8 per store
         auto emit = [&](const float (&o0)[32], const float (&o1)[32], int n, float* d) {
+          auto cmb = [&](int j) { return c0 * o0[j] + (w1 > 0.f ? c1 * o1[j] : 0.f); };
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            if (4 * q4 >= n) break;
-            float4 v;
-            v.x = c0 * o0[4 * q4] + (w1 > 0.f ? c1 * o1[4 * q4] : 0.f);
-            v.y = c0 * o0[4 * q4 + 1] + (w1 > 0.f ? c1 * o1[4 * q4 + 1] : 0.f);
-            v.z = c0 * o0[4 * q4 + 2] + (w1 > 0.f ? c1 * o1[4 * q4 + 2] : 0.f);
-            v.w = c0 * o0[4 * q4 + 3] + (w1 > 0.f ? c1 * o1[4 * q4 + 3] : 0.f);
-            *reinterpret_cast<float4*>(d + 4 * q4) = v;
+          for (int q8 = 0; q8 < 4; ++q8) {
+            if (8 * q8 >= n) break;
+            const int j = 8 * q8;
+            st_global_v8(d + j, cmb(j), cmb(j + 1), cmb(j + 2), cmb(j + 3), cmb(j + 4), cmb(j + 5), cmb(j + 6),
+                         cmb(j + 7));
           }
         };
         if constexpr (M64) {
@@ -1459,14 +1458,12 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         if (dst) {
           // a group that ran no stage of the unit (a one-stage unit) left its
           // accumulator unwritten: its weight is 0 and its values are not read
+          auto cmb = [&](int j) { return (w0 > 0.f ? c0 * o0[j] : 0.f) + (w1 > 0.f ? c1 * o1[j] : 0.f); };
 #pragma unroll
-          for (int q4 = 0; q4 < NCOL / 4; ++q4) {
-            float4 v;
-            v.x = (w0 > 0.f ? c0 * o0[4 * q4] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4] : 0.f);
-            v.y = (w0 > 0.f ? c0 * o0[4 * q4 + 1] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4 + 1] : 0.f);
-            v.z = (w0 > 0.f ? c0 * o0[4 * q4 + 2] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4 + 2] : 0.f);
-            v.w = (w0 > 0.f ? c0 * o0[4 * q4 + 3] : 0.f) + (w1 > 0.f ? c1 * o1[4 * q4 + 3] : 0.f);
-            *reinterpret_cast<float4*>(dst + 4 * q4) = v;
+          for (int q8 = 0; q8 < NCOL / 8; ++q8) {
+            const int j = 8 * q8;
+            st_global_v8(dst + j, cmb(j), cmb(j + 1), cmb(j + 2), cmb(j + 3), cmb(j + 4), cmb(j + 5), cmb(j + 6),
+                         cmb(j + 7));
           }
         }
       }  // act

@@ -355,6 +355,15 @@ __device__ __forceinline__ void tmem_st16x2_x32(uint32_t taddr, const float (&v)
       "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
+// 32-byte global store of 8 floats (p 32-byte aligned): a lane fills a whole
+// sector, where a 16-byte store leaves half of it for a second instruction.
+__device__ __forceinline__ void st_global_v8(float* p, float a0, float a1, float a2, float a3, float a4, float a5,
+                                             float a6, float a7) {
+  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(a0), "f"(a1), "f"(a2), "f"(a3),
+               "f"(a4), "f"(a5), "f"(a6), "f"(a7)
+               : "memory");
+}
+
 // Waits for this thread's tensor-memory loads, with v tied to the wait: v was
 // the destination of a load issued earlier, and its values are read only after
 // this point.
