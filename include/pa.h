@@ -377,6 +377,11 @@ const char *pa_status_string(pa_status s);
  *                                             [prow_off[b*Hkv+g], prow_off[b*Hkv+g+1])
  *   tail_pairs  int32[num_tail_pairs]         b*Hkv+g of every pair merged by the tail merge
  *                                             launch (tensor-core rows only, or mode 3), ascending
+ *   mix_pairs   int32[num_mix_pairs][2]       {b*Hkv+g, its number of SIMT rows} of the pairs
+ *                                             with both SIMT and tensor-core rows (mode 2); entry
+ *                                             k is SIMT warp (k mod simt_warps)'s to count once
+ *                                             the tensor-core launch has finished; {-1, -1}:
+ *                                             no pair
  *   partial_lse fp32[num_partial_rows][G]     (workspace only, not uploaded)
  *   partial_o   fp32[num_partial_rows][G][D]  (workspace only, not uploaded)
  */
@@ -397,11 +402,13 @@ typedef struct {
   int32_t sole;       /* SIMT: how the fused path combines this partial row of (query, kv_head).
                        * Bits 0-1, the mode: 0: arrival counter, the last of the pair's SIMT
                        * rows merges the pair; 1: it is the pair's only partial row and goes
-                       * straight to the output; 2: as 0, but the pair also has tensor-core
-                       * rows, so the merging warp first waits for the tensor-core launch;
-                       * 3: the pair also has tensor-core rows and is merged by the tail
-                       * merge launch (plans where a warp would otherwise defer more than
-                       * 16 such merges).  Bits 2-31: the pair's number of SIMT partial
+                       * straight to the output; 2: the pair also has tensor-core rows: its
+                       * counter also takes one arrival from the SIMT warp that the pair's
+                       * mix_pairs entry names, made after that warp's own work once the
+                       * tensor-core launch has finished, and whichever arrival is the last
+                       * merges the pair; 3: the pair also has tensor-core rows and is
+                       * merged by the tail merge launch (plans with more than 3 such pairs
+                       * per SIMT warp).  Bits 2-31: the pair's number of SIMT partial
                        * rows.  MMA segments: 0. */
   int32_t page_start; /* index into pages of the run's first page (item page_off + page_begin) */
 } pa_seg;
@@ -418,8 +425,10 @@ typedef struct {
   int32_t mma_next;       /* tensor-core work units taken so far in the running launch: 0 after
                              upload, and back at 0 after every launch that completes (after a
                              device-side error, upload the plan again) */
+  int32_t num_mix_pairs;  /* entries of mix_pairs */
+  int32_t reserved;       /* 0 */
   uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_mma_segs, off_counters, off_warp_segs,
-      off_prow_off, off_tail_pairs;
+      off_prow_off, off_tail_pairs, off_mix_pairs;
   uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;
 } pa_image_header;
 

@@ -29,6 +29,7 @@ PaDevPtrs dev_ptrs(const pa_plan& p, void* ws) {
   d.warp_segs = reinterpret_cast<const int32_t*>(b + h.off_warp_segs);
   d.prow_off = reinterpret_cast<const int32_t*>(b + h.off_prow_off);
   d.tail_pairs = reinterpret_cast<const int32_t*>(b + h.off_tail_pairs);
+  d.mix_pairs = reinterpret_cast<const int32_t*>(b + h.off_mix_pairs);
   d.partial_lse = reinterpret_cast<float*>(w + h.off_partial_lse);
   d.partial_o = reinterpret_cast<float*>(w + h.off_partial_o);
   d.status = reinterpret_cast<int32_t*>(b + offsetof(pa_image_header, status));

@@ -69,6 +69,8 @@ struct FwdArgs {
   int num_pages, B;
   int n_segs_mma;
   int32_t* mma_next;  // the counter of tensor-core work units taken (image header)
+  const int32_t* mix_pairs;  // {pair, SIMT rows} of the pairs with both classes' rows
+  int n_mix_pairs;
 };
 
 // ---------------------------------------------------------------- merge of one (request, kv head)
@@ -144,8 +146,9 @@ __device__ __forceinline__ void merge_pair(const float* partial_lse, const float
   if (lse && lane % LPR == 0) lse[(size_t)b * Hq + g * G + r] = m + logf(z);
 }
 
-// Called by a whole SIMT warp after it wrote a partial row of pair bg = b*Hkv+g:
-// counts the arrival; true if this was the last of the pair's n_simt SIMT rows.
+// Called by a whole SIMT warp after it wrote a partial row of pair bg = b*Hkv+g
+// (or, for a pair that also has tensor-core rows, once that launch has
+// finished): counts the arrival; true if this was the last of the pair's n.
 __device__ __forceinline__ bool simt_arrive(const FwdArgs& a, int bg, int n_simt, int lane) {
   __threadfence();
   __syncwarp();
@@ -468,11 +471,6 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, const CUtensorMap* t
     inflight |= 1u << (NST + slot);
   };
 
-  // pairs this warp merges once the tensor-core launch has completed
-  constexpr int kMaxDeferred = 16;
-  int deferred[kMaxDeferred];
-  int n_def = 0;
-
   SegInfo cur = load_seg(a.segs, seg_begin, seg_end);
   SegInfo nx = load_seg(a.segs, seg_begin + 1, seg_end);
   SegInfo nxx = load_seg(a.segs, seg_begin + 2, seg_end);
@@ -565,25 +563,26 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, const CUtensorMap* t
       }
     }
     if (a.out && (cur.mode == 0 || cur.mode == 2)) {
+      // a mixed pair (mode 2) counts one more arrival, made once the
+      // tensor-core launch has finished (below): if that one came first, this
+      // warp's is the last and the tensor-core rows are there
       const int bg = cur.query * a.Hkv + cur.kv_head;
-      if (simt_arrive(a, bg, cur.n_simt, lane)) {
-        if (cur.mode == 0) {
-          merge_and_reset<D, G>(a, bg, lane);
-        } else if (n_def < kMaxDeferred) {
-          deferred[n_def++] = bg;  // also has tensor-core rows: merged after this warp's own work
-        } else {
-          griddep_wait();
-          merge_and_reset<D, G>(a, bg, lane);
-        }
-      }
+      if (simt_arrive(a, bg, cur.n_simt + (cur.mode == 2 ? 1 : 0), lane)) merge_and_reset<D, G>(a, bg, lane);
     }
     cur = nx;
     nx = nxx;
     nxx = load_seg(a.segs, si + 3, seg_end);
   }
-  if (n_def > 0 && !failed) {
+  // after its own work, warp gw makes the tensor-core-side arrival of the
+  // mixed pairs in entries gw, gw + W, ... (W SIMT warps; at most a few per
+  // warp); whichever arrival is a pair's last merges it
+  if (a.out && a.n_mix_pairs > 0 && !failed) {
     griddep_wait();
-    for (int j = 0; j < n_def; ++j) merge_and_reset<D, G>(a, deferred[j], lane);
+    for (int k = gw; k < a.n_mix_pairs; k += a.n_simt_warps) {
+      const int bg = a.mix_pairs[2 * k], n_simt = a.mix_pairs[2 * k + 1];
+      if (bg < 0) continue;  // an entry no pair takes
+      if (simt_arrive(a, bg, n_simt + 1, lane)) merge_and_reset<D, G>(a, bg, lane);
+    }
   }
   if (failed) {
     // wait (bounded) for this warp's copies still in flight before leaving
@@ -1477,7 +1476,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
       if (!ok) break;
       tc_fence_before();
       mbar_arrive(bar(S::B_OFREE));
-      // these rows' pairs are merged by their last SIMT writer or the tail merge launch
+      // these rows' pairs are merged by their last arrival (fused merge) or the tail merge launch
       ++segord;
       si = take();
       if (si == -2) ok = false;
@@ -1625,6 +1624,8 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.tile_maps = p.tma_tiles ? 1 : 0;
   a.n_segs_mma = p.hdr.num_segments_mma;
   a.mma_next = d.mma_next;
+  a.mix_pairs = d.mix_pairs;
+  a.n_mix_pairs = p.hdr.num_mix_pairs;
   a.num_pages = p.num_pages_in_pool;
   a.B = p.B;
   return a;

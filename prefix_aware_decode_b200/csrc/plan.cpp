@@ -208,7 +208,7 @@ struct Planner {
 struct Scratch {
   std::vector<int> order, npg, qbuf;
   std::vector<ItemRec> items;
-  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows, tail_pairs;
+  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows, tail_pairs, mix_pairs;
   std::vector<SegRec> simt_segs, mma_segs;
   std::vector<int32_t> n_mma_rows;
 };
@@ -465,29 +465,52 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     for (int j = 0; j < it.n_queries; ++j) prow_off[(size_t)queries[it.query_off + j] * Hkv + s.kv_head + 1]++;
   }
   // fused merge: the last SIMT partial row of a pair to be written merges the
-  // pair (after the tensor-core launch has finished if the pair also has
-  // tensor-core rows); pairs with tensor-core rows only are merged by the
-  // tail merge launch
+  // pair; pairs with tensor-core rows only are merged by the tail merge
+  // launch.  A pair with both (mixed) also counts one arrival from a SIMT warp
+  // that makes it after its own work, once the tensor-core launch has
+  // finished: whichever arrival is the last merges the pair, so it is merged
+  // as soon as both classes' rows are there.  Entry k of mix_pairs takes that
+  // arrival from warp k mod W (W SIMT warps); the t-th mixed pair goes to the
+  // t-th warp of an order that visits every CTA before the second warp of
+  // any, so the merges after the tensor-core launch spread over all the
+  // class's SMs (entries no pair takes hold -1).  A warp merges its pairs one
+  // after another, ≈2.5 us each once the tensor-core launch has finished, so
+  // plans with more than kMixPerWarp mixed pairs per warp send them to the
+  // tail merge launch instead (config 5: 4096 pairs, 8 warps).
+  constexpr int kMixPerWarp = 3;
   std::vector<int32_t>& n_mma_rows = sc.n_mma_rows;
   n_mma_rows.assign(prow_off.begin() + 1, prow_off.end());
   for (const auto& s : simt_segs) prow_off[(size_t)s.query * Hkv + s.kv_head + 1]++;
-  // a SIMT warp defers the merges of its mixed pairs to the end of its work;
-  // if some warp would defer more than kSimtMaxDeferred, every mixed pair
-  // goes to the tail merge launch instead
-  bool mixed_to_tail = false;
-  if (!mma_segs.empty()) {
-    for (size_t w = 0; w + 1 < warp_segs.size() && !mixed_to_tail; ++w) {
-      int n = 0;
-      for (int si = warp_segs[w]; si < warp_segs[w + 1]; ++si)
-        n += n_mma_rows[(size_t)simt_segs[si].query * Hkv + simt_segs[si].kv_head] > 0;
-      mixed_to_tail = n > kSimtMaxDeferred;
-    }
-  }
-  std::vector<int32_t>& tail_pairs = sc.tail_pairs;
-  tail_pairs.clear();
+  const int W = (int)warp_segs.size() - 1;
+  int64_t n_mixed = 0;
   for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg)
-    if (n_mma_rows[bg] > 0 && (mixed_to_tail || prow_off[bg + 1] == n_mma_rows[bg]))
+    n_mixed += n_mma_rows[bg] > 0 && prow_off[bg + 1] > n_mma_rows[bg];
+  const bool mixed_to_tail = n_mixed > (int64_t)kMixPerWarp * W;
+  std::vector<int32_t>& tail_pairs = sc.tail_pairs;
+  std::vector<int32_t>& mix_pairs = sc.mix_pairs;
+  tail_pairs.clear();
+  mix_pairs.clear();
+  std::vector<int32_t> warp_order;
+  if (n_mixed > 0 && !mixed_to_tail) {
+    const int n_ctas = (W + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
+    for (int slot = 0; slot < kSimtWarpsPerCta; ++slot)
+      for (int c = 0; c < n_ctas; ++c)
+        if (c * kSimtWarpsPerCta + slot < W) warp_order.push_back(c * kSimtWarpsPerCta + slot);
+  }
+  int64_t t = 0;
+  for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg) {
+    if (n_mma_rows[bg] == 0) continue;
+    const int n_simt = prow_off[bg + 1] - n_mma_rows[bg];
+    if (n_simt == 0 || mixed_to_tail) {
       tail_pairs.push_back((int32_t)bg);
+      continue;
+    }
+    const size_t k = (size_t)(t / W) * W + warp_order[(size_t)(t % W)];
+    ++t;
+    if (mix_pairs.size() < 2 * (k + 1)) mix_pairs.resize(2 * (k + 1), -1);
+    mix_pairs[2 * k] = (int32_t)bg;
+    mix_pairs[2 * k + 1] = n_simt;
+  }
   for (size_t i = 1; i < prow_off.size(); ++i) prow_off[i] += prow_off[i - 1];
   std::vector<int32_t>& cursor = sc.cursor;
   cursor.assign(prow_off.begin(), prow_off.end() - 1);
@@ -522,6 +545,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     plan->mma_max_rows = std::max(plan->mma_max_rows, std::min(kMmaRowsPerCta, items[s.item].n_queries * G));
   h.num_partial_rows = num_prows;
   h.num_tail_pairs = (int32_t)tail_pairs.size();
+  h.num_mix_pairs = (int32_t)(mix_pairs.size() / 2);
   uint64_t off = align256(sizeof(pa_image_header));
   h.off_nodes = off; off = align256(off + items.size() * sizeof(pa_item));
   h.off_segs = off; off = align256(off + (size_t)h.num_segments * sizeof(pa_seg));
@@ -533,6 +557,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   h.off_warp_segs = off; off = align256(off + warp_segs.size() * 4);
   h.off_prow_off = off; off = align256(off + prow_off.size() * 4);
   h.off_tail_pairs = off; off = align256(off + tail_pairs.size() * 4);
+  h.off_mix_pairs = off; off = align256(off + mix_pairs.size() * 4);
   h.image_bytes = off;
   h.off_partial_lse = off; off = align256(off + (uint64_t)num_prows * G * 4);
   h.off_partial_o = off; off = align256(off + (uint64_t)num_prows * G * D * 4);
@@ -574,6 +599,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   put(h.off_warp_segs, warp_segs);
   put(h.off_prow_off, prow_off);
   put(h.off_tail_pairs, tail_pairs);
+  put(h.off_mix_pairs, mix_pairs);
   // the alignment gaps after the regions are zeroed: the image depends on the inputs only
   const uint64_t region_end[] = {sizeof(h),
                                  h.off_nodes + items.size() * sizeof(pa_item),
@@ -585,7 +611,8 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
                                  h.off_counters + (uint64_t)batch * Hkv * 4,
                                  h.off_warp_segs + warp_segs.size() * 4,
                                  h.off_prow_off + prow_off.size() * 4,
-                                 h.off_tail_pairs + tail_pairs.size() * 4};
+                                 h.off_tail_pairs + tail_pairs.size() * 4,
+                                 h.off_mix_pairs + mix_pairs.size() * 4};
   for (const uint64_t e : region_end) std::memset(img + e, 0, align256(e) - e);
 
   pa_plan_stats& st = plan->stats;

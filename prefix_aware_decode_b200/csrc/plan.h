@@ -14,10 +14,6 @@ static_assert(sizeof(pa_item) == 16, "pa_item must be 16 bytes");
 // to 128 rows with 6 warps (TMA producer, tcgen05 issuer, 4 softmax warps).
 constexpr int kSimtWarpsPerCta = 8;
 constexpr int kMmaRowsPerCta = 128;
-// A SIMT warp merges at most this many pairs that also have tensor-core rows
-// at the end of its work; plans that would need more send those pairs to the
-// tail merge launch instead.
-constexpr int kSimtMaxDeferred = 16;
 
 // Host buffer for plan images, taken from and returned to a small process-wide
 // pool so that building a plan does not page-fault fresh memory every time.
@@ -95,6 +91,7 @@ struct PaDevPtrs {
   const int32_t* warp_segs;
   const int32_t* prow_off;
   const int32_t* tail_pairs;
+  const int32_t* mix_pairs;
   float* partial_lse;
   float* partial_o;
   int32_t* status;

@@ -40,6 +40,7 @@ class Image:
         self.warp_segs = arr(h.off_warp_segs, h.simt_warps + 1)
         self.prow_off = arr(h.off_prow_off, h.batch * h.num_kv_heads + 1)
         self.tail_pairs = arr(h.off_tail_pairs, h.num_tail_pairs)
+        self.mix_pairs = arr(h.off_mix_pairs, h.num_mix_pairs, cols=2)
 
 
 def check_structure(img: Image, kv_lens, block_table, P=16):
@@ -71,11 +72,20 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
     modes = {int(m) & 3 for m in img.seg_sole[:nseg_simt]}
     mixed_to_tail = 3 in modes
     assert not (mixed_to_tail and 2 in modes)
+    mixed = sorted(bg for bg in mma_pairs if bg in simt_rows)
     assert list(img.tail_pairs) == sorted(bg for bg in mma_pairs if mixed_to_tail or bg not in simt_rows)
-    # a warp defers at most 16 mixed-pair merges
-    for w in range(len(img.warp_segs) - 1):
-        segs = range(img.warp_segs[w], img.warp_segs[w + 1])
-        assert sum(int(img.seg_sole[s]) & 3 == 2 for s in segs) <= 16
+    # the mixed pairs (both classes' rows) not sent to the tail launch: each in
+    # exactly one mix_pairs entry with its SIMT row count, at most 3 per warp
+    # (entry k belongs to warp k mod W), other entries empty
+    if mixed_to_tail:
+        assert h.num_mix_pairs == 0 and len(mixed) > 3 * h.simt_warps
+    else:
+        got = [(int(bg), int(n)) for bg, n in img.mix_pairs if bg >= 0]
+        assert sorted(got) == [(bg, simt_rows[bg]) for bg in mixed]
+        assert all(int(bg) == -1 and int(n) == -1 for bg, n in img.mix_pairs if bg < 0)
+        per_warp = np.bincount([k % max(1, h.simt_warps) for k in range(h.num_mix_pairs) if img.mix_pairs[k, 0] >= 0],
+                               minlength=max(1, h.simt_warps))
+        assert per_warp.max(initial=0) <= 3
     # warp lists partition the SIMT segments, in order; page_start and the
     # combine mode (tail merge, sole row or arrival counted) are consistent
     assert img.warp_segs[0] == 0 and img.warp_segs[-1] == nseg_simt
