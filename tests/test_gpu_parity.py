@@ -49,9 +49,18 @@ def test_large_configs_full_parity(config):
     dw = dev_config(config)
     w = dw.w
     ref_o, ref_l = oracle.attend_paged(w.q, w.k_pool, w.v_pool, w.block_table, w.kv_lens)
+    res = {}
     for fused in (False, True):
         out, lse, st, _ = run(dw, fused=fused)
         assert_close(compare(out, lse, ref_o, ref_l), f"config {config} fused={fused}")
+        res[fused] = (out, lse)
+    # the fused merge combines a pair's partial rows in the same fixed order
+    # whichever arrival merges it (config 3: 2048 mixed pairs, each counted by
+    # a designated small-row warp once the tensor-core launch has finished)
+    assert torch.equal(res[True][0].view(torch.int16), res[False][0].view(torch.int16))
+    assert torch.equal(res[True][1], res[False][1])
+    if config == 3:
+        assert st["num_segments_mma"] > 0 and st["num_tail_pairs"] == 0
 
 
 def test_config5_every_session_parity():
