@@ -22,6 +22,7 @@
 #include <new>
 #include <numeric>
 #include <stdexcept>
+#include <thread>
 #include <vector>
 
 #include "plan.h"
@@ -69,6 +70,9 @@ struct Planner {
   int64_t unique_tokens = 0, read_tokens = 0;
   int num_nodes = 0, num_shared = 0, num_kept = 0;
   bool invalid = false;
+  // set for the first call of the walk: its subtrees may be walked on several
+  // threads (walk_kids)
+  bool split_top = false;
 
   const int32_t* row(int b) const { return bt + (size_t)b * max_pages; }
 
@@ -122,6 +126,8 @@ struct Planner {
   // read again by this subtree's items).
   void walk(int lo, int hi, int depth, int eff_lo) {
     if (invalid) return;
+    const bool top = split_top;
+    split_top = false;
     if (hi - lo == 1) {
       const int b = order[lo];
       if (npg[b] > depth) {
@@ -194,11 +200,94 @@ struct Planner {
       return pa != pb ? pa < pb : a < b;
     });
     int start = e;
+    std::vector<std::pair<int, int>> kids;  // the first call's subtrees
     for (int i = e + 1; i <= hi; ++i) {
       if (i == hi || row(order[i])[l] != row(order[start])[l]) {
-        walk(start, i, l, next_eff);
+        if (top) kids.emplace_back(start, i);
+        else walk(start, i, l, next_eff);
         start = i;
       }
+    }
+    if (top) walk_kids(kids, l, next_eff);
+  }
+
+  // The subtrees of the first call, in order.  The walk reads the block table
+  // once (each row is compared with its group's first row), ≈10 MB for a
+  // batch like config 5's, so large batches walk contiguous runs of subtrees
+  // of about equal work on up to kWalkThreads threads: each thread writes its
+  // own items, pages and queries (the subtrees own disjoint ranges of `order`
+  // and read the inputs only), and the outputs are appended in subtree order,
+  // so the plan is the one the serial walk gives.
+  void walk_kids(const std::vector<std::pair<int, int>>& kids, int depth, int eff) {
+    constexpr int kWalkThreads = 8;
+    constexpr int64_t kMinWalkPagesPerThread = 32768;
+    std::vector<int64_t> work(kids.size(), 0);
+    int64_t total = 0;
+    for (size_t k = 0; k < kids.size(); ++k) {
+      for (int i = kids[k].first; i < kids[k].second; ++i) work[k] += std::max(0, npg[order[i]] - depth);
+      total += work[k];
+    }
+    const unsigned hw = std::thread::hardware_concurrency();
+    int T = (int)std::min<int64_t>({(int64_t)kWalkThreads, (int64_t)std::max(1u, hw), (int64_t)kids.size(),
+                                    total / kMinWalkPagesPerThread});
+    if (T < 2) {
+      for (const auto& k : kids) walk(k.first, k.second, depth, eff);
+      return;
+    }
+    // contiguous runs of subtrees, about total / T pages each
+    std::vector<size_t> cut(1, 0);
+    int64_t acc = 0;
+    for (size_t k = 0; k < kids.size(); ++k) {
+      acc += work[k];
+      if ((int)cut.size() < T && acc * T >= total * (int64_t)cut.size() && k + 1 < kids.size()) cut.push_back(k + 1);
+    }
+    cut.push_back(kids.size());
+    const int n = (int)cut.size() - 1;
+    struct Part {
+      std::vector<ItemRec> items;
+      std::vector<int32_t> pages, queries;
+      std::vector<int> qbuf;
+    };
+    std::vector<Part> parts(n);
+    std::vector<Planner> subs;
+    subs.reserve(n);
+    for (int t = 0; t < n; ++t)
+      subs.push_back(Planner{kv_lens, bt, max_pages, P, G, Hq, Hkv, D, flags, num_pages_in_pool, order, npg,
+                             parts[t].items, parts[t].pages, parts[t].queries, parts[t].qbuf});
+    auto run = [&](int t) {
+      try {
+        for (size_t k = cut[t]; k < cut[t + 1]; ++k) subs[t].walk(kids[k].first, kids[k].second, depth, eff);
+      } catch (...) {
+        subs[t].invalid = true;
+      }
+    };
+    std::vector<std::thread> th;
+    th.reserve(n);
+    int started = 0;
+    try {
+      for (int t = 1; t < n; ++t, ++started) th.emplace_back(run, t);
+    } catch (...) {
+      // a thread could not start: the rest of the runs are walked here
+    }
+    run(0);
+    for (int t = 1 + started; t < n; ++t) run(t);
+    for (auto& x : th) x.join();
+    for (int t = 0; t < n; ++t) {
+      const Planner& sp = subs[t];
+      const int base_p = (int)pages.size(), base_q = (int)queries.size();
+      for (ItemRec it : parts[t].items) {
+        it.page_off += base_p;
+        it.query_off += base_q;
+        items.push_back(it);
+      }
+      pages.insert(pages.end(), parts[t].pages.begin(), parts[t].pages.end());
+      queries.insert(queries.end(), parts[t].queries.begin(), parts[t].queries.end());
+      unique_tokens += sp.unique_tokens;
+      read_tokens += sp.read_tokens;
+      num_nodes += sp.num_nodes;
+      num_shared += sp.num_shared;
+      num_kept += sp.num_kept;
+      invalid = invalid || sp.invalid;
     }
   }
 };
@@ -737,6 +826,7 @@ extern "C" pa_status pa_plan_create(const pa_config* cfg, int32_t batch, const i
     pl.items.reserve(batch + 64);
     pl.pages.reserve(total_pages);
     pl.queries.reserve(2 * batch);
+    pl.split_top = true;
     pl.walk(0, batch, 0, 0);
     if (pl.invalid) { delete plan; return PA_ERR_INVALID; }
     const std::vector<ItemRec>& items = pl.items;
