@@ -58,9 +58,9 @@ class ClockSampler:
     """nvidia-smi clocks and throttle reasons, sampled during a timed region.
 
     Samples carry nvidia-smi's own timestamps; only those inside the timed
-    region (marked by mark_start / mark_end, plus 100 ms for the lag of the
-    driver's counters) are summarised, so idle samples taken before and after
-    it do not enter the median."""
+    regions (each marked by mark_start / mark_end, plus 100 ms for the lag of
+    the driver's counters) are summarised, so idle samples taken before, after
+    and between them do not enter the median."""
 
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -72,6 +72,7 @@ class ClockSampler:
         self.samples = []
         self.proc = None
         self.t0 = self.t1 = None
+        self.windows = []  # [start, end] of each timed region
 
     def start(self):
         try:
@@ -84,10 +85,10 @@ class ClockSampler:
             self.proc = None
 
     def mark_start(self):
-        self.t0 = time.time()
+        self.windows.append([time.time(), None])
 
     def mark_end(self):
-        self.t1 = time.time()
+        self.windows[-1][1] = time.time()
 
     def _read(self):
         for line in self.proc.stdout:
@@ -110,11 +111,18 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         rows = [s for s in self.samples if len(s) >= 10 and s[2].replace(".", "").isdigit()]
-        t0, t1 = self.t0, (self.t1 or time.time()) + 0.1
-        inside = [s for s in rows if t0 is None or (self._when(s[0]) or 0.0) >= t0 and (self._when(s[0]) or 0.0) <= t1]
-        if not inside and t0 is not None:  # a region shorter than the sampling period: the next sample
-            later = [s for s in rows if (self._when(s[0]) or 0.0) >= t0]
-            inside = later[:1]
+        wins = self.windows or ([[self.t0, self.t1]] if self.t0 is not None else [])
+        wins = [(a, (b or time.time()) + 0.1) for a, b in wins]
+
+        def within(s):
+            t = self._when(s[0]) or 0.0
+            return any(a <= t <= b for a, b in wins)
+
+        inside = [s for s in rows if not wins or within(s)]
+        for a, b in wins:
+            if not any(a <= (self._when(s[0]) or 0.0) <= b for s in inside):
+                # a region shorter than the sampling period: the next sample
+                inside += [s for s in rows if (self._when(s[0]) or 0.0) >= a][:1]
         sm = [float(s[2]) for s in inside]
         smax = [float(s[3]) for s in rows if s[3].replace(".", "").isdigit()]
         power = [float(s[4]) for s in inside if s[4].replace(".", "").isdigit()]
@@ -126,7 +134,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_min_mhz": min(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "power_w_max": max(power) if power else None,
                 "reasons": sorted(reasons), "samples": len(inside),
-                "note": "samples inside the timed region only (nvidia-smi timestamps, 20 ms period)"}
+                "note": "samples inside the timed regions only (nvidia-smi timestamps, 20 ms period)"}
 
 
 def kernels_hash() -> str:
@@ -284,12 +292,15 @@ class Bench:
         prof_every = 4  # profiling events on every 4th step of the timed region
         step_events = [mk_events(4) if i % prof_every == 0 else None for i in range(nsteps)]
         host_us = []
+        # one stepper per pool copy (their arguments are marshalled once), all
+        # on the same image buffer
         stepper = pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, q, k0, v0, ws, out, lse, stream=stream)
+        steppers = [stepper] + [pad.DecodeStep(w.num_pages, w.Hq, w.Hkv, w.D, q, kc, vc, ws, out, lse, stream=stream,
+                                               images=stepper.images) for kc, vc in pools[1:]]
 
         def step(i):
             t = time.perf_counter()
-            stepper.set_pools(*pools[i % copies])
-            stepper(kv_lens, block_table, events=step_events[i])
+            steppers[i % copies](kv_lens, block_table, events=step_events[i])
             host_us.append((time.perf_counter() - t) * 1e6)
 
         for i in range(args.warmup):
@@ -316,11 +327,38 @@ class Bench:
         ev1.record(stream)
         torch.cuda.synchronize()
         clocks.mark_end()
+        # forward + merge on the device: the step's plan, uploaded once, attended
+        # K times back to back over the rotated pools (the host stays ahead, so
+        # nothing but the launches is timed)
+        dplan = pad.Plan(kv_lens, block_table, w.num_pages, w.Hq, w.Hkv, w.D)
+        dplan.upload(ws, stream)
+        for i in range(args.warmup):
+            dplan.attend(q, *pools[i % copies], ws, out, lse, stream)
+        torch.cuda.synchronize()
+        time.sleep(0.3)  # the same start as the decode loop's: clocks not yet held down by the power cap
+        self.barrier()
+        clocks.mark_start()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(2):  # queued ahead of the first event, so the device is busy when it fires
+            dplan.attend(q, *pools[i % copies], ws, out, lse, stream)
+        d0.record(stream)
+        for i in range(args.steps):
+            dplan.attend(q, *pools[(i + 2) % copies], ws, out, lse, stream)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        fwd_ms = self.max_over_ranks(d0.elapsed_time(d1)) / args.steps
+        dstatus = dplan.device_status(ws, stream)
+        dplan.close()
+        assert dstatus == pad.PA_OK, dstatus
+        clocks.mark_end()
         self.barrier()
         clk = clocks.stop()
         ms_step = self.max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
-        fwd_ms = statistics.mean(step_events[i][0].elapsed_time(step_events[i][1])
-                                 for i in range(args.warmup, nsteps) if step_events[i] is not None)
+        # forward + merge inside the decode steps: when the device has caught
+        # up with the host, the first event also counts the host's submission
+        # of the launches
+        fwd_in_step_ms = statistics.mean(step_events[i][0].elapsed_time(step_events[i][1])
+                                         for i in range(args.warmup, nsteps) if step_events[i] is not None)
         launches = (pst["mma_ctas"] > 0) + (pst["simt_warps"] > 0) + (pst["num_tail_pairs"] > 0)
         achieved = algo["total"] / (fwd_ms * 1e-3) / 1e9
         hbm = self.hbm_peak
@@ -332,13 +370,15 @@ class Bench:
             "ms_per_step": ms_step, "queries_per_s": w.B * self.world / (ms_step * 1e-3),
             "unique_kv_frac_of_hbm": w.unique_kv_bytes / (ms_step * 1e-3) / 1e9 / hbm,
             "forward_merge_us": fwd_ms * 1e3,
+            "forward_merge_us_in_step": fwd_in_step_ms * 1e3,
             "forward_queries_per_s": w.B / (fwd_ms * 1e-3),
             "forward_unique_kv_frac_of_hbm": w.unique_kv_bytes / (fwd_ms * 1e-3) / 1e9 / hbm,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": measured_traffic(config),
                          "algorithmic_bytes": algo,
                          "kernel": "forward launches of both tile classes with the merge fused, plus the tail "
-                                   "merge launch when the plan has one, timed together with CUDA events",
+                                   "merge launch when the plan has one, timed together with CUDA events over "
+                                   "K back-to-back calls of the step's plan",
                          "launches_per_step": launches,
                          "peak_kind": f"{self.peak_kind} hbm_gbs (copy, burst)"},
             "plan_us": pst["plan_us"], "host_us_per_step_median": statistics.median(host_us),
@@ -346,6 +386,7 @@ class Bench:
                                          "num_tail_pairs", "num_partial_rows", "read_kv_bytes",
                                          "workspace_bytes", "image_bytes")},
             "clocks": clk, "gpu_launches": args.steps * launches,
+            "gpu_launches_device_loop": args.steps * launches,
         }
 
         if config == 1 and args.amortise > 0:
@@ -371,7 +412,7 @@ class Bench:
             dt = time.perf_counter() - t0
             res["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
                                    "sample": f"first {n} of {w.B} queries of the same workload, one pass"}
-        del pools, q, k0, v0, out, lse, ws, stepper
+        del pools, q, k0, v0, out, lse, ws, stepper, steppers
         torch.cuda.empty_cache()
         return res
 
