@@ -369,8 +369,9 @@ const char *pa_status_string(pa_status s);
  *   queries     int32[num_query_entries]      request ids, per item
  *   seg_prows   int32[num_query_entries_mma]  partial row of each (MMA seg, query)
  *   mma_segs    int32[2]                      {0, num_segments_mma}: the tensor-core work units,
- *                                             longest first; the tensor-core CTAs take them one
- *                                             at a time from the counter mma_next of the header
+ *                                             longest first; CTA c starts with unit c, and the
+ *                                             CTAs take the rest one at a time from the counter
+ *                                             mma_next of the header
  *   counters    int32[B * Hkv]                arrival counters of the fused merge (zero)
  *   warp_segs   int32[simt_warps + 1]         SIMT warp w runs segs [warp_segs[w], warp_segs[w+1])
  *   prow_off    int32[B * Hkv + 1]            partial rows of (b, g) are
@@ -398,7 +399,8 @@ typedef struct {
   int32_t page_begin; /* first page of the run, index within the item's pages */
   int32_t n_tokens;   /* valid tokens of the run (its pages are ceil(n_tokens / P)) */
   int32_t prow;       /* SIMT: the partial row written; MMA: index into seg_prows */
-  int32_t query;      /* SIMT: the request; MMA: first request of the item */
+  int32_t query;      /* SIMT: the request; MMA: the item's query_off (its requests are
+                       * queries[query .. query + sole)) */
   int32_t sole;       /* SIMT: how the fused path combines this partial row of (query, kv_head).
                        * Bits 0-1, the mode: 0: arrival counter, the last of the pair's SIMT
                        * rows merges the pair; 1: it is the pair's only partial row and goes
@@ -409,7 +411,8 @@ typedef struct {
                        * merges the pair; 3: the pair also has tensor-core rows and is
                        * merged by the tail merge launch (plans with more than 3 such pairs
                        * per SIMT warp).  Bits 2-31: the pair's number of SIMT partial
-                       * rows.  MMA segments: 0. */
+                       * rows.  MMA segments: the item's n_queries (the tile has sole * G
+                       * rows). */
   int32_t page_start; /* index into pages of the run's first page (item page_off + page_begin) */
 } pa_seg;
 
@@ -422,8 +425,9 @@ typedef struct {
   int32_t num_items, num_segments, num_segments_simt, num_segments_mma, simt_warps;
   int32_t num_partial_rows, mma_ctas;
   int32_t num_tail_pairs; /* pairs merged by the tail launch of pa_attend / pa_decode_step */
-  int32_t mma_next;       /* tensor-core work units taken so far in the running launch: 0 after
-                             upload, and back at 0 after every launch that completes (after a
+  int32_t mma_next;       /* takes of tensor-core work units from the counter so far in the
+                             running launch (units past each CTA's first): 0 after upload,
+                             and back at 0 after every launch that completes (after a
                              device-side error, upload the plan again) */
   int32_t num_mix_pairs;  /* entries of mix_pairs */
   int32_t reserved;       /* 0 */

@@ -751,11 +751,21 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
           ok = false;
           break;
         }
+        // CTA c's first unit is unit c (no atomic on the way to its first
+        // load); the later ones come from the counter, after the first
+        // min(grid, units) units.  Every CTA that had a first unit makes one
+        // take that finds the list empty, so the takes return 0 .. units - 1
+        // and the last of them puts the counter back to zero.
         int v = -1;
         if (lane == 0) {
-          const int idx = atomicAdd(a.mma_next, 1);
-          if (idx < a.n_segs_mma) v = idx;
-          else if (idx == a.n_segs_mma + (int)gridDim.x - 1) *a.mma_next = 0;  // the launch's last take
+          const int n_first = min((int)gridDim.x, a.n_segs_mma);
+          if (qn == 0) {
+            v = (int)blockIdx.x < n_first ? (int)blockIdx.x : -1;
+          } else {
+            const int t = atomicAdd(a.mma_next, 1);
+            if (n_first + t < a.n_segs_mma) v = n_first + t;
+            if (t == a.n_segs_mma - 1) *a.mma_next = 0;  // the launch's last take
+          }
           segq[j] = v;
           mbar_arrive(bar(S::B_QF + j));
         }
@@ -777,7 +787,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         si = v;
       }
       const pa_seg seg = a.segs[si];
-      const int32_t* pg = a.pages + a.items[seg.item].page_off + seg.page_begin;
+      const int32_t* pg = a.pages + seg.page_start;
       const int npages = (seg.n_tokens + 15) >> 4;
       auto page_at = [&](int x) -> int {
         if (x >= npages) return 0;
@@ -847,7 +857,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
         if (si == -2) ok = false;
         if (si < 0) break;
         const pa_seg seg = a.segs[si];
-        const bool m64 = a.items[seg.item].n_queries * G <= 64;
+        const bool m64 = seg.sole * G <= 64;  // a tensor-core unit's sole: its requests
         if (a.debug_checks && QR == 64 && !m64) record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -8);
         const uint32_t idesc_s = m64 ? idesc_s64 : idesc_s128, idesc_o = m64 ? idesc_o64 : idesc_o128;
         const int npages = (seg.n_tokens + 15) >> 4;
@@ -928,10 +938,9 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     int i = 0, segord = 0;
     // The q row this thread copies for segment si (nullptr: a row past the tile's)
     auto q_src = [&](int si) -> const uint16_t* {
-      const pa_seg seg = a.segs[si];
-      const pa_item item = a.items[seg.item];
-      if (rq >= item.n_queries * G || rq >= QR) return nullptr;
-      int b = a.queries[item.query_off + rq / G];
+      const pa_seg seg = a.segs[si];  // query: the unit's first index into queries; sole: its requests
+      if (rq >= seg.sole * G || rq >= QR) return nullptr;
+      int b = a.queries[seg.query + rq / G];
       if (a.debug_checks && (uint32_t)b >= (uint32_t)a.B) {
         record_status(a.status, PA_ERR_DEVICE, blockIdx.x, -1 - b);
         b = 0;
@@ -1470,7 +1479,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const CUtensorMap* tk
     };
     while (si >= 0 && ok) {
       const pa_seg seg = a.segs[si];
-      const int R = a.items[seg.item].n_queries * G;
+      const int R = seg.sole * G;
       if constexpr (QR == 64) ok = run_segment_il(0, seg, R);
       else ok = R <= 64 ? run_segment(std::true_type{}, seg, R) : run_segment(std::false_type{}, seg, R);
       if (!ok) break;

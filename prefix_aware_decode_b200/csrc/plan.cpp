@@ -227,9 +227,12 @@ struct Planner {
       for (int i = kids[k].first; i < kids[k].second; ++i) work[k] += std::max(0, npg[order[i]] - depth);
       total += work[k];
     }
-    const unsigned hw = std::thread::hardware_concurrency();
-    int T = (int)std::min<int64_t>({(int64_t)kWalkThreads, (int64_t)std::max(1u, hw), (int64_t)kids.size(),
-                                    total / kMinWalkPagesPerThread});
+    int T = (int)std::min<int64_t>({(int64_t)kWalkThreads, (int64_t)kids.size(), total / kMinWalkPagesPerThread});
+    if (T >= 2) {
+      // the host's thread count, asked once (a system call of a few us)
+      static const unsigned hw = std::max(1u, std::thread::hardware_concurrency());
+      T = std::min<int>(T, (int)hw);
+    }
     if (T < 2) {
       for (const auto& k : kids) walk(k.first, k.second, depth, eff);
       return;
@@ -676,8 +679,13 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
                items[s.item].page_off + s.page_begin};
   }
-  for (const auto& s : mma_segs)
-    ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, 0, items[s.item].page_off + s.page_begin};
+  // a tensor-core unit carries its item's request list (query_off, n_queries)
+  // itself, so the kernel reaches its pages and Q rows without the item
+  for (const auto& s : mma_segs) {
+    const ItemRec& it = items[s.item];
+    ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, it.query_off, it.n_queries,
+               it.page_off + s.page_begin};
+  }
   auto put = [&](uint64_t o, const std::vector<int32_t>& v) {
     if (!v.empty()) std::memcpy(img + o, v.data(), v.size() * 4);
   };

@@ -100,7 +100,8 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
             assert img.seg_sole[si] & 3 == want
             assert img.seg_sole[si] >> 2 == simt_rows[bg]
         else:
-            assert img.seg_sole[si] == 0
+            # a tensor-core unit names its item's request list itself
+            assert q == img.items[item][3] and img.seg_sole[si] == img.items[item][2]
     # coverage: each (request, kv head) reads each token (page, slot) exactly once
     seen = {}
     prows_written = np.zeros(h.num_partial_rows, dtype=np.int64)
