@@ -430,7 +430,8 @@ typedef struct {
                              and back at 0 after every launch that completes (after a
                              device-side error, upload the plan again) */
   int32_t num_mix_pairs;  /* entries of mix_pairs */
-  int32_t reserved;       /* 0 */
+  int32_t simt_warps_per_cta; /* SIMT warps of a CTA of the small-row launch (6 or 8): warp w runs
+                                 in CTA w / simt_warps_per_cta */
   uint64_t off_nodes, off_segs, off_pages, off_queries, off_seg_prows, off_mma_segs, off_counters, off_warp_segs,
       off_prow_off, off_tail_pairs, off_mix_pairs;
   uint64_t off_partial_lse, off_partial_o, image_bytes, workspace_bytes;

@@ -54,7 +54,7 @@ class PaImageHeader(ctypes.Structure):
                 + [(n, ctypes.c_int32) for n in ("batch", "num_q_heads", "num_kv_heads", "head_dim", "page_size",
                                                  "num_items", "num_segments", "num_segments_simt", "num_segments_mma",
                                                  "simt_warps", "num_partial_rows", "mma_ctas", "num_tail_pairs",
-                                                 "mma_next", "num_mix_pairs", "reserved")]
+                                                 "mma_next", "num_mix_pairs", "simt_warps_per_cta")]
                 + [(n, ctypes.c_uint64) for n in ("off_nodes", "off_segs", "off_pages", "off_queries",
                                                   "off_seg_prows", "off_mma_segs", "off_counters", "off_warp_segs",
                                                   "off_prow_off", "off_tail_pairs", "off_mix_pairs", "off_partial_lse",

@@ -61,6 +61,7 @@ struct FwdArgs {
   __nv_bfloat16* out;  // non-null: fused merge
   float* lse;
   int Hq, Hkv, G, n_simt_warps, n_segs_simt, n_mma_ctas;
+  int simt_wpc;  // SIMT warps per CTA of the small-row launch
   float qscale;  // softmax scale * log2(e): scores are kept in base-2 units
   uint64_t timeout_ns;
   int fault_drop;
@@ -193,7 +194,10 @@ struct SimtShape {
   static constexpr int KT = D / 16;         // k steps of K.Q^T, d tiles of V^T.P^T
   static constexpr int FIXED = W * 2 * QT + 1024 + W * 8 * 8;  // q slots, alignment slack, barriers
   static constexpr int NST_FIT = (kSmemMax - FIXED) / (W * STAGE);
-  static constexpr int NST = NST_FIT < (D == 128 ? 3 : 6) ? NST_FIT : (D == 128 ? 3 : 6);  // ring stages
+  // ring stages: two D = 128 tiles or three D = 64 tiles per warp (16 and 12 KB
+  // in flight); deeper rings (3 and 6) were measured slower: config 3 232 ->
+  // 211 us, config 4 275 -> 272 us, config 2 47.4 -> 45.6 us at 8 warps
+  static constexpr int NST = NST_FIT < (D == 128 ? 2 : 3) ? NST_FIT : (D == 128 ? 2 : 3);
   static constexpr int RING = NST * STAGE;  // one warp's ring (a multiple of 1 KB: swizzle atoms stay aligned)
   static constexpr int OFF_Q = W * RING;
   static constexpr int OFF_BAR = OFF_Q + W * 2 * QT;
@@ -338,7 +342,7 @@ __device__ __forceinline__ void simt_role(const FwdArgs& a, const CUtensorMap* t
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp >= kSimtWarpsPerCta) return;
-  const int gw = blockIdx.x * kSimtWarpsPerCta + warp;
+  const int gw = blockIdx.x * a.simt_wpc + warp;
   if (gw >= a.n_simt_warps) return;  // no block-wide barrier in this role
   const uint32_t ring = smem_u32(smem + warp * S::RING);
   uint8_t* qslot = smem + S::OFF_Q + warp * 2 * S::QT;  // two q-row slots
@@ -1624,6 +1628,8 @@ FwdArgs make_fwd_args(const pa_plan& p, const PaDevPtrs& d, void* out, float* ls
   a.Hkv = p.Hkv;
   a.G = p.G;
   a.n_simt_warps = p.hdr.simt_warps;
+  a.simt_wpc = p.hdr.simt_warps_per_cta >= 1 && p.hdr.simt_warps_per_cta <= kSimtWarpsPerCta
+                   ? p.hdr.simt_warps_per_cta : kSimtWarpsPerCta;
   a.n_segs_simt = p.hdr.num_segments_simt;
   a.n_mma_ctas = p.hdr.mma_ctas;
   a.qscale = p.scale * kLog2e;
@@ -1659,7 +1665,7 @@ int set_smem_attr(K kernel, bool (&done)[64]) {
 template <int D, int G>
 int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
   static bool attr_mma[64] = {}, attr_mma64[64] = {}, attr_simt[64] = {};
-  const int n_simt_ctas = (a.n_simt_warps + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
+  const int n_simt_ctas = (a.n_simt_warps + a.simt_wpc - 1) / a.simt_wpc;
   const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(p.tma_k);
   const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(p.tma_v);
   if (a.n_mma_ctas > 0) {
@@ -1683,7 +1689,7 @@ int launch_fwd_t(const pa_plan& p, const FwdArgs& a, cudaStream_t st) {
     if (int e = set_smem_attr(k, attr_simt)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(n_simt_ctas);
-    cfg.blockDim = dim3(kSimtWarpsPerCta * 32);
+    cfg.blockDim = dim3(a.simt_wpc * 32);
     cfg.dynamicSmemBytes = SimtShape<D, G>::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

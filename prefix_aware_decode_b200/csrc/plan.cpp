@@ -498,8 +498,21 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     mma_cta_segs.push_back((int32_t)mma_segs.size());
   }
 
+  // SIMT warps per CTA.  Each warp keeps two D = 128 tiles (16 KB) or three
+  // D = 64 tiles (12 KB) in flight; when every warp streams a long run of
+  // D = 128 tiles (kSimtLongSpan or more at 8 warps), 6 warps per SM (96 KB in
+  // flight) moved the bytes faster than 8 (128 KB) or 10: config 4 262.5
+  // against 271.8 and 274.8 us, config 3 208.4 against 211.5 us; with short
+  // runs the warps' fixed costs dominate and 8 are faster (config 2 45.6
+  // against 47.6 us, 1024 config-1 problems at D = 64 105 against 129 us).
+  // The rule is about the HBM traffic of many SMs: a class of a few CTAs
+  // beside a long tensor-core launch (config 5) keeps its 8 warps.
+  int simt_wpc = kSimtWarpsPerCta;
+  if (simt_pages > 0 && D == 128 && 2 * (S - n_mma) >= S &&
+      ceil_div(simt_pages, (int64_t)std::max(1, S - n_mma) * kSimtWarpsPerCta) >= kSimtLongSpan)
+    simt_wpc = kSimtWarpsPerCtaLong;
   if (simt_pages > 0) {
-    const int64_t W = (int64_t)std::max(1, S - n_mma) * kSimtWarpsPerCta;
+    const int64_t W = (int64_t)std::max(1, S - n_mma) * simt_wpc;
     int64_t span = ceil_div(simt_pages, W);
     if (span < 4) span = 4;
     if (max_chunk_pages) span = std::min(span, max_chunk_pages);
@@ -584,10 +597,10 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   mix_pairs.clear();
   std::vector<int32_t> warp_order;
   if (n_mixed > 0 && !mixed_to_tail) {
-    const int n_ctas = (W + kSimtWarpsPerCta - 1) / kSimtWarpsPerCta;
-    for (int slot = 0; slot < kSimtWarpsPerCta; ++slot)
+    const int n_ctas = (W + simt_wpc - 1) / simt_wpc;
+    for (int slot = 0; slot < simt_wpc; ++slot)
       for (int c = 0; c < n_ctas; ++c)
-        if (c * kSimtWarpsPerCta + slot < W) warp_order.push_back(c * kSimtWarpsPerCta + slot);
+        if (c * simt_wpc + slot < W) warp_order.push_back(c * simt_wpc + slot);
   }
   int64_t t = 0;
   for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg) {
@@ -631,6 +644,7 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   h.num_segments_mma = (int32_t)mma_segs.size();
   h.num_segments = h.num_segments_simt + h.num_segments_mma;
   h.simt_warps = (int32_t)warp_segs.size() - 1;
+  h.simt_warps_per_cta = simt_wpc;
   h.mma_ctas = mma_segs.empty() ? 0 : n_mma;
   plan->mma_max_rows = 0;
   for (const auto& s : mma_segs)

@@ -9,10 +9,15 @@
 static_assert(sizeof(pa_seg) == 32, "pa_seg must be 32 bytes (vector loads)");
 static_assert(sizeof(pa_item) == 16, "pa_item must be 16 bytes");
 
-// Forward launch shape: 8 warps per CTA, one CTA per SM.  A CUDA-core (SIMT)
-// CTA runs 8 independent warps; a tensor-core (MMA) CTA works on tiles of up
-// to 128 rows with 6 warps (TMA producer, tcgen05 issuer, 4 softmax warps).
+// Forward launch shape: one CTA per SM.  A CUDA-core (SIMT) CTA runs up to 8
+// independent warps (6 when every warp streams long runs of D = 128 tiles:
+// kSimtLongSpan tiles or more; fewer bytes in flight per SM measured faster
+// there, see the planner); a tensor-core (MMA) CTA works on tiles of up to
+// 128 rows with 12 warps (two TMA producers, two tcgen05 issuers, 8 softmax
+// warps).
 constexpr int kSimtWarpsPerCta = 8;
+constexpr int kSimtWarpsPerCtaLong = 6;
+constexpr int kSimtLongSpan = 64;
 constexpr int kMmaRowsPerCta = 128;
 
 // Host buffer for plan images, taken from and returned to a small process-wide

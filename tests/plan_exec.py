@@ -59,6 +59,8 @@ def check_structure(img: Image, kv_lens, block_table, P=16):
         assert h.mma_ctas == 0
     assert h.mma_next == 0
     assert np.all(img.counters == 0)
+    # small-row launch: 8 warps per CTA, or 6 when its warps stream long runs
+    assert h.simt_warps_per_cta in (6, 8)
     # pairs with tensor-core rows; the tail list holds those without SIMT rows, ascending
     mma_pairs, simt_rows = set(), {}
     for si in range(nseg_simt, h.num_segments):

@@ -42,7 +42,7 @@ def test_small_configs_full_parity(config, fused):
     assert_close(m, f"config {config}")
 
 
-@pytest.mark.parametrize("config", [3, 4])
+@pytest.mark.parametrize("config", [2, 3, 4])
 def test_large_configs_full_parity(config):
     # every request of the workload, both the two-launch path (pa_forward +
     # pa_merge) and the fused one (pa_attend)
@@ -55,12 +55,16 @@ def test_large_configs_full_parity(config):
         assert_close(compare(out, lse, ref_o, ref_l), f"config {config} fused={fused}")
         res[fused] = (out, lse)
     # the fused merge combines a pair's partial rows in the same fixed order
-    # whichever arrival merges it (config 3: 2048 mixed pairs, each counted by
-    # a designated small-row warp once the tensor-core launch has finished)
+    # whichever arrival merges it (config 2: 512 mixed pairs, each counted by
+    # a designated small-row warp once the tensor-core launch has finished;
+    # config 3: 2048 mixed pairs, more than 3 per small-row warp, merged by the
+    # tail merge launch)
     assert torch.equal(res[True][0].view(torch.int16), res[False][0].view(torch.int16))
     assert torch.equal(res[True][1], res[False][1])
-    if config == 3:
+    if config == 2:
         assert st["num_segments_mma"] > 0 and st["num_tail_pairs"] == 0
+    if config == 3:
+        assert st["num_segments_mma"] > 0 and st["num_tail_pairs"] > 0
 
 
 def test_config5_every_session_parity():

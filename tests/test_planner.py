@@ -45,7 +45,7 @@ def test_config2_tree_and_classes():
     assert st["num_nodes"] == 65 and st["num_shared_nodes"] == 1 and st["num_kept_shared"] == 1
     # 256 rows of the shared root -> 2 query tiles of 128 rows on the tensor-core class
     assert st["num_items"] == 64 + 2
-    assert 0 < st["mma_ctas"] < 148 and st["simt_warps"] <= (148 - st["mma_ctas"]) * 8
+    assert 0 < st["mma_ctas"] < 148 and st["simt_warps"] <= (148 - st["mma_ctas"]) * 8  # at most 8 per CTA
     assert st["num_segments_mma"] > 0 and st["num_segments_simt"] > 0
 
 
@@ -392,8 +392,9 @@ def test_plans_for_very_few_sms(num_sms):
     p = make_plan(w, num_sms=num_sms)
     st = p.stats()
     assert st["mma_ctas"] >= 1 and st["simt_warps"] >= 1
-    assert st["mma_ctas"] + -(-st["simt_warps"] // 8) <= max(2, num_sms)
     img = Image(p.host_image())
+    wpc = img.h.simt_warps_per_cta
+    assert st["mma_ctas"] + -(-st["simt_warps"] // wpc) <= max(2, num_sms)
     check_structure(img, w.kv_lens, w.block_table)
     out, lse = execute(img, w.q, w.k_pool, w.v_pool)
     np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
@@ -492,3 +493,21 @@ def test_append_plan_rejects_bad_chunks():
         pad.Plan.append([10], [0], bt, 4, 8, 2, 64)
     with pytest.raises(pad.PaError):
         pad.Plan.append([60], [5], bt, 4, 8, 2, 64)  # 65 tokens > 4 pages
+
+
+def test_small_row_warps_per_cta():
+    # 6 warps per CTA when the small-row class streams long runs of D = 128
+    # tiles on most SMs (configs 3 and 4), else 8: short runs (config 2), a
+    # class of one CTA beside the tensor-core launch (config 5), D = 64
+    want = {2: 8, 3: 6, 4: 6, 5: 8}
+    for c, wpc in want.items():
+        w = wl.make_config(c, with_values=False)
+        img = Image(make_plan(w).host_image())
+        assert img.h.simt_warps_per_cta == wpc, c
+        # the warp lists cover whole CTAs of that many warps at most
+        assert img.h.simt_warps <= (148 - img.h.mma_ctas) * wpc
+    # long independent requests: 6 warps at D = 128, 8 at D = 64
+    roots = wl.random_tree(seed=5, n_queries=128, depth=0, leaf_tokens=(4000, 6000))
+    for D, wpc in ((128, 6), (64, 8)):
+        wd = wl.build_workload("long", roots, Hq=32, Hkv=8, D=D, seed=5, with_values=False)
+        assert Image(make_plan(wd).host_image()).h.simt_warps_per_cta == wpc, D
