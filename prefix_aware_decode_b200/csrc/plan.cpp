@@ -52,6 +52,10 @@ struct ItemRec {
 
 struct SegRec {
   int item, kv_head, page_begin, n_tokens, prow, query;
+  // a resized list is overwritten before it is read: no zero fill
+  SegRec() {}
+  SegRec(int it, int g, int pb, int nt, int pr, int q)
+      : item(it), kv_head(g), page_begin(pb), n_tokens(nt), prow(pr), query(q) {}
 };
 
 struct Planner {
@@ -300,7 +304,8 @@ struct Planner {
 struct Scratch {
   std::vector<int> order, npg, qbuf;
   std::vector<ItemRec> items;
-  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows, tail_pairs, mix_pairs;
+  std::vector<int32_t> pages, queries, warp_segs, mma_cta_segs, prow_off, cursor, seg_prows, tail_pairs, mix_pairs,
+      warp_order;
   std::vector<SegRec> simt_segs, mma_segs;
   std::vector<int32_t> n_mma_rows;
 };
@@ -526,9 +531,10 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     warp_segs.resize((size_t)W + 2);
     SegRec* sp = simt_segs.data();
     int32_t* wp = warp_segs.data() + 1;
-    int32_t n_seg = 0;
-    int64_t n_warp = 1;
-    int64_t used = 0;  // pages in the current warp's span
+    int32_t n_seg = 0, cap = (int32_t)simt_segs.size();
+    const int span_i = (int)std::min<int64_t>(span, INT32_MAX / 4), W_i = (int)W;
+    int n_warp = 1;
+    int used = 0;  // pages in the current warp's span
     for (size_t i = 0; i < items.size(); ++i) {
       const ItemRec& it = items[i];
       if (!it.simt) continue;
@@ -538,16 +544,17 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
         int pb = 0;
         used += kSimtSegPages;  // the unit's fixed cost
         while (pb < npages) {
-          const int take = (int)std::max<int64_t>(1, std::min<int64_t>(npages - pb, span - used));
+          const int take = std::max(1, std::min(npages - pb, span_i - used));
           const int tok = std::min(it.n_tokens, (pb + take) * P) - pb * P;
-          if ((size_t)n_seg == simt_segs.size()) {
-            simt_segs.resize(2 * simt_segs.size());
+          if (n_seg == cap) {
+            simt_segs.resize(2 * (size_t)cap);
             sp = simt_segs.data();
+            cap = (int32_t)simt_segs.size();
           }
-          sp[n_seg++] = {(int)i, g, pb, tok, -1, b};
+          sp[n_seg++] = SegRec{(int)i, g, pb, tok, -1, b};
           pb += take;
           used += take;
-          if (used >= span && n_warp < W) {  // never more than W warps
+          if (used >= span_i && n_warp < W_i) {  // never more than W warps
             *wp++ = n_seg;
             ++n_warp;
             used = 0;
@@ -595,14 +602,22 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
   std::vector<int32_t>& mix_pairs = sc.mix_pairs;
   tail_pairs.clear();
   mix_pairs.clear();
-  std::vector<int32_t> warp_order;
+  std::vector<int32_t>& warp_order = sc.warp_order;
+  warp_order.clear();
   if (n_mixed > 0 && !mixed_to_tail) {
     const int n_ctas = (W + simt_wpc - 1) / simt_wpc;
     for (int slot = 0; slot < simt_wpc; ++slot)
       for (int c = 0; c < n_ctas; ++c)
         if (c * simt_wpc + slot < W) warp_order.push_back(c * simt_wpc + slot);
+    // the t-th mixed pair takes entry (t / W) W + warp_order[t % W]; the list
+    // ends after the last entry taken
+    const int64_t last = n_mixed - 1, base = last / W * W;
+    int32_t top = 0;
+    for (int64_t r = 0; r <= last % W; ++r) top = std::max(top, warp_order[(size_t)r]);
+    mix_pairs.assign((size_t)(2 * (base + top + 1)), -1);
   }
-  int64_t t = 0;
+  int64_t round = 0;  // (t / W) W for the t-th mixed pair
+  int pos = 0;        // t % W
   for (size_t bg = 0; bg + 1 < prow_off.size(); ++bg) {
     if (n_mma_rows[bg] == 0) continue;
     const int n_simt = prow_off[bg + 1] - n_mma_rows[bg];
@@ -610,9 +625,11 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
       tail_pairs.push_back((int32_t)bg);
       continue;
     }
-    const size_t k = (size_t)(t / W) * W + warp_order[(size_t)(t % W)];
-    ++t;
-    if (mix_pairs.size() < 2 * (k + 1)) mix_pairs.resize(2 * (k + 1), -1);
+    const size_t k = (size_t)(round + warp_order[(size_t)pos]);
+    if (++pos == W) {
+      pos = 0;
+      round += W;
+    }
     mix_pairs[2 * k] = (int32_t)bg;
     mix_pairs[2 * k + 1] = n_simt;
   }
@@ -685,13 +702,20 @@ static void finish_plan(pa_plan* plan, Scratch& sc, const std::vector<ItemRec>& 
     di[i] = {items[i].page_off, items[i].n_tokens, items[i].n_queries, items[i].query_off};
   pa_seg* ds = reinterpret_cast<pa_seg*>(img + h.off_segs);
   size_t k = 0;
-  for (const auto& s : simt_segs) {
-    const size_t bg = (size_t)s.query * Hkv + s.kv_head;
-    const int n_rows = prow_off[bg + 1] - prow_off[bg], n_simt = n_rows - n_mma_rows[bg];
-    const int mode = n_mma_rows[bg] > 0 ? (mixed_to_tail ? 3 : 2) : n_rows == 1 ? 1 : 0;
-    const int sole = mode | (n_simt << 2);
-    ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
-               items[s.item].page_off + s.page_begin};
+  {
+    size_t pbg = SIZE_MAX;
+    int sole = 0;
+    for (const auto& s : simt_segs) {
+      const size_t bg = (size_t)s.query * Hkv + s.kv_head;
+      if (bg != pbg) {  // a pair's segments are consecutive
+        pbg = bg;
+        const int n_rows = prow_off[bg + 1] - prow_off[bg], n_simt = n_rows - n_mma_rows[bg];
+        const int mode = n_mma_rows[bg] > 0 ? (mixed_to_tail ? 3 : 2) : n_rows == 1 ? 1 : 0;
+        sole = mode | (n_simt << 2);
+      }
+      ds[k++] = {s.item, s.kv_head, s.page_begin, s.n_tokens, s.prow, s.query, sole,
+                 items[s.item].page_off + s.page_begin};
+    }
   }
   // a tensor-core unit carries its item's request list (query_off, n_queries)
   // itself, so the kernel reaches its pages and Q rows without the item
