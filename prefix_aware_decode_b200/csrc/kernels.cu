@@ -9,13 +9,14 @@
 // are two launches of one CTA per SM that run side by side (the pages'
 // multi-stream execution, done here with programmatic dependent launch):
 //   - MMA class: work units with two or more requests, up to 128 rows, on the
-//     5th-generation tensor cores: a producer warp streams 64-key stages with
-//     2-D TMA copies (128-byte swizzle), one thread issues tcgen05.mma with S,
-//     P and the accumulators in tensor memory, and 8 warps run the softmax.
-//   - SIMT class: work units of one request (G <= 8 rows).  Each of 8 warps
-//     streams its own run of (page, kv head) tiles with 1-D bulk copies into a
-//     private shared-memory ring and computes on the CUDA cores with packed
-//     fp32x2 FMAs.
+//     5th-generation tensor cores: two producer warps stream the K and the V
+//     of 64-key stages with 2-D TMA copies (128-byte swizzle), one thread
+//     issues the S products and another the p.V products (tcgen05.mma, S, P
+//     and the accumulators in tensor memory), and 8 warps run the softmax.
+//   - SIMT class: work units of one request (G <= 8 rows).  Each warp of a
+//     CTA streams its own run of (page, kv head) tiles with 3-D TMA copies
+//     into a private shared-memory ring and computes with warp-level
+//     tensor-core products (mma.sync), the request's rows held in registers.
 // Both emit, per (request, kv head, key range), the normalised partial output
 // o = sum_t e^{s_t - m} v_t / l and lse = m + ln l in fp32.
 //
@@ -169,8 +170,9 @@ __device__ __forceinline__ void merge_and_reset(const FwdArgs& a, int bg, int la
 
 // ---------------------------------------------------------------- small-row class (one request, G rows)
 //
-// Each of 8 warps streams its own run of (page, kv head) tiles through a
-// private ring in shared memory: per tile, K and V arrive as D/64 boxes of 16
+// Each of the CTA's warps (8, or 6 for long runs: the plan's choice) streams
+// its own run of (page, kv head) tiles through a private ring in shared
+// memory: per tile, K and V arrive as D/64 boxes of 16
 // keys x 64 dims each (2-D TMA, 128-byte swizzle, completed on the stage's
 // mbarrier).  The G query rows of the request stay in registers as the B
 // operand of warp-level tensor-core products (mma.sync m16n8k16, bf16 in,
