@@ -138,9 +138,17 @@ class ClockSampler:
 
 
 def kernels_hash() -> str:
+    """sha256 prefix of kernels.cu's code: its lines with // comments and
+    surrounding blanks removed, so an edit of the comments alone keeps a
+    capture of the same code valid."""
     import hashlib
-    src = open(os.path.join(_ROOT, "prefix_aware_decode_b200", "csrc", "kernels.cu"), "rb").read()
-    return hashlib.sha256(src).hexdigest()[:16]
+    src = open(os.path.join(_ROOT, "prefix_aware_decode_b200", "csrc", "kernels.cu"), encoding="utf-8").read()
+    code = []
+    for line in src.splitlines():
+        line = line.split("//", 1)[0].strip()
+        if line:
+            code.append(line)
+    return hashlib.sha256("\n".join(code).encode()).hexdigest()[:16]
 
 
 def measured_traffic(config: int):
