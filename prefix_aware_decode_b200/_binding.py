@@ -136,6 +136,24 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
+def _host_ptr(a: np.ndarray) -> int:
+    """Address of a host array's data (the buffer protocol: a fraction of the
+    cost of ndarray.ctypes per call)."""
+    try:
+        return ctypes.addressof(ctypes.c_char.from_buffer(a))
+    except (TypeError, ValueError, BufferError):  # read-only or empty arrays
+        return a.ctypes.data
+
+
+def _host_i32(a, ndim: int) -> np.ndarray:
+    """a as a C-contiguous int32 array of `ndim` dimensions (no copy when it is one)."""
+    if not (isinstance(a, np.ndarray) and a.dtype == np.int32 and a.flags.c_contiguous):
+        a = np.ascontiguousarray(a, dtype=np.int32)
+    if a.ndim != ndim:
+        raise ValueError(f"expected a {ndim}-d host array, got {a.ndim}-d")
+    return a
+
+
 def _dptr(t, name: str, align: int = 16) -> int:
     p = t.data_ptr()
     if not t.is_cuda:
@@ -162,7 +180,7 @@ class Plan:
         cfg = PaConfig(num_q_heads, num_kv_heads, head_dim, page_size, softmax_scale, num_sms, max_chunk_tokens,
                        flags, wait_timeout_us)
         h = ctypes.c_void_p()
-        _check(self._lib.pa_plan_create(ctypes.byref(cfg), kv.shape[0], kv.ctypes.data, bt.ctypes.data,
+        _check(self._lib.pa_plan_create(ctypes.byref(cfg), kv.shape[0], _host_ptr(kv), _host_ptr(bt),
                                         bt.shape[1], int(num_pages), ctypes.byref(h)), "pa_plan_create")
         self._h = h
         self.B, self.Hq, self.Hkv, self.D = int(kv.shape[0]), num_q_heads, num_kv_heads, head_dim
@@ -200,7 +218,7 @@ class Plan:
         if bt.ndim != 2 or kv.ndim != 1 or bt.shape[0] != kv.shape[0] or kv.shape[0] != self.B:
             raise ValueError("block_table must be [B][max_pages] and kv_lens [B], B as before")
         h = ctypes.c_void_p()
-        _check(self._lib.pa_plan_advance(self._h, kv.ctypes.data, bt.ctypes.data, bt.shape[1], int(num_pages),
+        _check(self._lib.pa_plan_advance(self._h, _host_ptr(kv), _host_ptr(bt), bt.shape[1], int(num_pages),
                                          ctypes.byref(h)), "pa_plan_advance")
         nxt = Plan.__new__(Plan)
         nxt._lib, nxt._h = self._lib, h
@@ -370,6 +388,9 @@ class DecodeStep:
             self._events = (ctypes.c_void_p * 4)(*[e.cuda_event if e is not None else None for e in events])
             ev = self._events
         q, k, v, ws, wsb, im, imb, out, lse = self.args
-        _check(self._lib.pa_decode_step(ctypes.byref(self.cfg), kv_lens.shape[0], kv_lens.ctypes.data,
-                                        block_table.ctypes.data, block_table.shape[1], self.num_pages, q, k, v,
+        kv_lens, block_table = _host_i32(kv_lens, 1), _host_i32(block_table, 2)
+        if block_table.shape[0] != kv_lens.shape[0]:
+            raise ValueError("block_table must be [B][max_pages] and kv_lens [B]")
+        _check(self._lib.pa_decode_step(ctypes.byref(self.cfg), kv_lens.shape[0], _host_ptr(kv_lens),
+                                        _host_ptr(block_table), block_table.shape[1], self.num_pages, q, k, v,
                                         ws, wsb, im, imb, out, lse, ev, self.stream, None), "pa_decode_step")

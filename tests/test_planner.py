@@ -511,3 +511,21 @@ def test_small_row_warps_per_cta():
     for D, wpc in ((128, 6), (64, 8)):
         wd = wl.build_workload("long", roots, Hq=32, Hkv=8, D=D, seed=5, with_values=False)
         assert Image(make_plan(wd).host_image()).h.simt_warps_per_cta == wpc, D
+
+
+def test_binding_host_arrays():
+    # host arrays reach the library by address: the buffer-protocol address is
+    # the array's data, other dtypes and layouts are converted, read-only
+    # arrays still work, and a wrong rank is refused
+    from prefix_aware_decode_b200 import _binding as B
+
+    a = np.arange(64, dtype=np.int32)
+    assert B._host_ptr(a) == a.ctypes.data
+    assert B._host_i32(a, 1) is a
+    b = B._host_i32(np.arange(12, dtype=np.int64).reshape(3, 4)[:, ::2], 2)
+    assert b.dtype == np.int32 and b.flags.c_contiguous and b.tolist() == [[0, 2], [4, 6], [8, 10]]
+    ro = np.arange(8, dtype=np.int32)
+    ro.flags.writeable = False
+    assert B._host_ptr(ro) == ro.ctypes.data
+    with pytest.raises(ValueError):
+        B._host_i32(a, 2)
