@@ -310,8 +310,10 @@ pa_status pa_plan_set_profile_events(pa_plan *plan, void *const *events, int32_t
  * The image is copied into the next half on a stream of the library's own (the
  * library keeps one copy stream and four events per device, and no device
  * memory): the copy for step k+1 runs while the kernels of step k do, and
- * `stream` waits for it (an event) before its launches.  A half is refilled
- * only after the launches that read it have completed.  The device status word
+ * `stream` waits for it (an event) before its launches.  An image of at most
+ * 16 KiB is copied on `stream` itself instead (in stream order, with fewer
+ * host calls).  A half is refilled only after the launches that read it have
+ * completed.  The device status word
  * of the step is in its half: read it with pa_get_device_status on the plan
  * returned through plan_out, before two more pa_decode_step calls refill that
  * half.  pa_plan_upload (or pa_attend_noalloc) of that plan makes it refer to
