@@ -289,8 +289,10 @@ def test_advanced_plan_on_the_device_matches_the_oracle():
 
 def test_decode_steps_alternating_batches_and_one_plan_over_several_pools():
     # pa_decode_step uploads each step's plan into one of two device slots on a
-    # copy stream of its own; alternating two different batches through the
-    # same stepper must give each batch its own result every time
+    # copy stream of its own (config 1's 3.8 KB image on the compute stream
+    # itself, config 2's on the copy stream, so the slots switch between the
+    # two ways); alternating two different batches must give each batch its
+    # own result every time
     wa = wl.make_config(1)
     wb = wl.make_config(2, scale=0.25)
     da, db = DevWorkload(wa), DevWorkload(wb)
